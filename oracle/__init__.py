@@ -1,0 +1,345 @@
+"""fp64 CPU oracle for the lightning indexer and its MISA / HISA variants.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may use it. The CUDA path never imports it, and
+it imports nothing from the CUDA path. It reads the same rounded host buffers
+that the GPU reads (built by ``sparse_attention_token_score_b200.workloads``),
+widens them exactly to fp64 and follows the pages' steps in order:
+
+* dense indexer + top-k ("MISA: Mixture of Indexer Sparse Attention for
+  Long-Context LLM Inference", section "Problem statement"): score every
+  causal-prefix token with all H_I heads, keep the k best.
+* MISA (same page, section "Methodology"): split the prefix into
+  M = ceil(L/B) blocks, mean-pool the keys of each block, compute a per-head
+  affinity from the pooled keys, keep the top-h heads per query, score all
+  tokens with those heads only, keep the top-k.
+* MISA-dagger (same page, "Hierarchical variant"): the routed pass keeps k'
+  candidates, the full H_I-head indexer re-scores them, keep the top-k.
+* HISA ("HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse
+  Attention" review, section 3): score pooled block keys, keep the top-m
+  blocks, score the tokens of the surviving blocks, keep the top-k.
+
+Readings where the pages are silent (each is listed in the design notes):
+* Ties in any selection go to the lower index; a selection over fewer
+  candidates than asked returns all of them, padded with -1; selected indices
+  are returned in ascending order.
+* A query at absolute position p sees keys s <= p; a pooled block m is visible
+  when its first token is (m*B <= p). Pooled keys are the bf16-rounded fp64
+  mean of all tokens of the block (fewer in a partial last block).
+* Routed scoring uses the chosen heads' original signed weights, with no
+  renormalisation.
+* FP8 inputs are dequantised exactly (scale * decoded byte) and scored in the
+  unfactored form.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "indexer_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C core with gcc (-O2, no fast-math: sums stay sequential)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _core():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        lib.or_score_pairs.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
+                                       P, P, P, P]
+        lib.or_score_pairs.restype = None
+        lib.or_router.argtypes = [P, P, P, ctypes.c_longlong, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_longlong, P, P]
+        lib.or_router.restype = None
+        lib.or_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_core().or_num_threads())
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ------------------------------------------------------------ number formats
+def widen_bf16(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> fp64 (exact): the pattern is the top half of an fp32."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _e4m3_value(code: int) -> float:
+    """Value of an OCP FP8 E4M3 code: 1 sign, 4 exponent (bias 7), 3 mantissa
+    bits; exponent 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN; no infinities."""
+    s = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 0xF and m == 0x7:
+        return float("nan")
+    if e == 0:
+        return s * (m / 8.0) * 2.0 ** -6
+    return s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+E4M3_TABLE = np.array([_e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+def decode_e4m3(codes: np.ndarray) -> np.ndarray:
+    """FP8 e4m3 bytes -> fp64 (exact)."""
+    return E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
+
+
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp64 to bf16 directly (nearest, ties to even), no intermediate fp32.
+
+    bf16 keeps 7 of fp64's 52 fraction bits; rounding adds half an ulp minus one
+    plus the kept lsb to the 45 dropped bits, then truncates. Valid for zero and
+    for normal values inside the bf16 exponent range (all the pooled keys here)."""
+    x = np.asarray(x, dtype=np.float64)
+    ax = np.abs(x)
+    if np.any((ax != 0) & ((ax < 2.0 ** -126) | (ax >= 2.0 ** 127))):
+        raise ValueError("f64_to_bf16_bits: value outside the normal bf16 range")
+    u = x.view(np.uint64)
+    lsb = (u >> np.uint64(45)) & np.uint64(1)
+    u = (u + np.uint64((1 << 44) - 1) + lsb) & ~np.uint64((1 << 45) - 1)
+    f32 = u.view(np.float64).astype(np.float32)  # exact: 8 significant bits, in range
+    return (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+# ------------------------------------------------------------ inputs -> fp64
+def dequant(inp, b: int = 0):
+    """fp64 (q [T,H,d], k [L,d], w [T,H]) of sequence ``b``."""
+    if inp.dtype == "bf16":
+        q = widen_bf16(inp.q[b])
+        k = widen_bf16(inp.k[b])
+    else:
+        q = decode_e4m3(inp.q[b]) * inp.q_scale[b].astype(np.float64)[..., None]
+        k = decode_e4m3(inp.k[b]) * inp.k_scale[b].astype(np.float64)[:, None]
+    return q, k, inp.w[b].astype(np.float64)
+
+
+# ------------------------------------------------------------ primitives
+def score_pairs(q: np.ndarray, k: np.ndarray, w: np.ndarray, pq: np.ndarray, pk: np.ndarray,
+                hmask: Optional[np.ndarray] = None):
+    """Indexer score of pairs (pq[i], pk[i]): returns (score, cond), fp64.
+
+    score = sum_h w[t,h] ReLU(q[t,h].k[s]);  cond = sum_h |w[t,h]| ReLU(q[t,h].k[s]).
+    ``hmask`` [T,H] (uint8) restricts the sum to the marked heads."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    T, H, d = q.shape
+    assert k.shape[1] == d and w.shape == (T, H)
+    pq = np.ascontiguousarray(pq, dtype=np.int64)
+    pk = np.ascontiguousarray(pk, dtype=np.int64)
+    assert pq.shape == pk.shape
+    if pq.size:
+        assert pq.min() >= 0 and pq.max() < T and pk.min() >= 0 and pk.max() < k.shape[0]
+    hm = None if hmask is None else np.ascontiguousarray(hmask, dtype=np.uint8)
+    if hm is not None:
+        assert hm.shape == (T, H)
+    out = np.empty(pq.shape, dtype=np.float64)
+    cond = np.empty(pq.shape, dtype=np.float64)
+    _core().or_score_pairs(_ptr(q), _ptr(k), _ptr(w), _ptr(hm), H, d, pq.size, _ptr(pq), _ptr(pk),
+                           _ptr(out), _ptr(cond))
+    return out, cond
+
+
+def select_topk(scores: np.ndarray, k: int, index: Optional[np.ndarray] = None) -> np.ndarray:
+    """The k best candidates by (score descending, index ascending).
+
+    NaN scores mark candidates that do not exist. Returns their indices
+    (``index[j]`` if given, else j) in ascending order, padded with -1 to k."""
+    scores = np.asarray(scores, dtype=np.float64)
+    idx = np.arange(scores.size, dtype=np.int64) if index is None else np.asarray(index, dtype=np.int64)
+    ok = ~np.isnan(scores)
+    s, ix = scores[ok], idx[ok]
+    order = np.lexsort((ix, -s))  # primary: -score ascending; secondary: index ascending
+    chosen = np.sort(ix[order[:k]])
+    out = np.full(k, -1, dtype=np.int64)
+    out[:chosen.size] = chosen
+    return out
+
+
+def kth_score(scores: np.ndarray, k: int, index: Optional[np.ndarray] = None) -> float:
+    """Score of the k-th best candidate (NaN if there are fewer than k)."""
+    s = np.asarray(scores, dtype=np.float64)
+    s = s[~np.isnan(s)]
+    if s.size < k or k <= 0:
+        return float("nan")
+    return float(np.sort(s)[::-1][k - 1])
+
+
+def visible_count(p: np.ndarray, L: int) -> np.ndarray:
+    """Keys visible to queries at absolute positions p: s <= p and s < L."""
+    return np.clip(np.asarray(p, dtype=np.int64) + 1, 0, L)
+
+
+def meanpool_bf16(k_bits: np.ndarray, B: int) -> np.ndarray:
+    """Pooled keys kbar[m] = bf16(mean of k[mB : min((m+1)B, L)]) from bf16 keys
+    [L, d] (MISA page, "Methodology", step 1: M = ceil(L/B) blocks, mean-pooled
+    indexing keys). The mean is taken in fp64 and rounded once."""
+    k = widen_bf16(k_bits)
+    L, d = k.shape
+    M = -(-L // B)
+    out = np.empty((M, d), dtype=np.float64)
+    for m in range(M):
+        blk = k[m * B:min((m + 1) * B, L)]
+        out[m] = blk.sum(axis=0) / blk.shape[0]
+    return f64_to_bf16_bits(out)
+
+
+# ------------------------------------------------------------ dense indexer
+def dense_scores_row(q, k, w, t: int, p: int, keys: Optional[np.ndarray] = None):
+    """Scores of query t (absolute position p) on ``keys`` (default: the whole
+    visible prefix). Returns (keys, score, cond)."""
+    L = k.shape[0]
+    if keys is None:
+        keys = np.arange(int(visible_count(p, L)), dtype=np.int64)
+    pq = np.full(keys.shape, t, dtype=np.int64)
+    s, c = score_pairs(q, k, w, pq, keys)
+    return keys, s, c
+
+
+def dense_topk(inp, topk: int, queries: Optional[Sequence[int]] = None, b: int = 0):
+    """Dense lightning indexer + top-k for queries of sequence b.
+
+    Returns dict with 'idx' [nq, topk] (ascending, -1 padded) and per query
+    'scores' / 'cond' over the visible prefix."""
+    q, k, w = dequant(inp, b)
+    if queries is None:
+        queries = range(q.shape[0])
+    res = {"idx": [], "scores": [], "cond": [], "queries": list(queries)}
+    for t in queries:
+        keys, s, c = dense_scores_row(q, k, w, t, inp.q_offset + t)
+        res["idx"].append(select_topk(s, topk))
+        res["scores"].append(s)
+        res["cond"].append(c)
+    res["idx"] = np.array(res["idx"], dtype=np.int64).reshape(len(res["queries"]), topk)
+    return res
+
+
+# ------------------------------------------------------------ MISA
+def router_affinity(q: np.ndarray, kbar: np.ndarray, w: np.ndarray, nvis_blocks: np.ndarray):
+    """a[t,h] = |w[t,h]| * sum_{m < nvis[t]} ReLU(q[t,h].kbar[m]) (fp64)."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    kbar = np.ascontiguousarray(kbar, dtype=np.float64)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    T, H, d = q.shape
+    nv = np.ascontiguousarray(nvis_blocks, dtype=np.int64)
+    assert nv.shape == (T,)
+    a = np.empty((T, H), dtype=np.float64)
+    _core().or_router(_ptr(q), _ptr(kbar), _ptr(w), T, H, d, kbar.shape[0], _ptr(nv), _ptr(a))
+    return a
+
+
+def visible_blocks(p: np.ndarray, B: int, M: int) -> np.ndarray:
+    """Blocks whose first token is visible: m*B <= p, m < M."""
+    return np.clip(np.asarray(p, dtype=np.int64) // B + 1, 0, M)
+
+
+def misa(inp, block: int, h: int, topk: int, kprime: int = 0,
+         queries: Optional[Sequence[int]] = None, b: int = 0,
+         heads_given: Optional[np.ndarray] = None, cand_given: Optional[np.ndarray] = None):
+    """MISA routed indexer (kprime == 0) or MISA-dagger (kprime > 0).
+
+    heads_given [nq, h] / cand_given [nq, kprime]: run the later stages on these
+    choices instead of the oracle's own (lets a test condition each stage on
+    the GPU's previous discrete choice). Returns a dict with every stage."""
+    assert inp.dtype == "bf16"
+    q, k, w = dequant(inp, b)
+    T, H, d = q.shape
+    L = k.shape[0]
+    if queries is None:
+        queries = np.arange(T)
+    queries = np.asarray(queries, dtype=np.int64)
+    kbar_bits = meanpool_bf16(inp.k[b], block)
+    kbar = widen_bf16(kbar_bits)
+    M = kbar.shape[0]
+    p = inp.q_offset + queries
+    a = router_affinity(q[queries], kbar, w[queries], visible_blocks(p, block, M))
+    heads = np.stack([select_topk(a[i], h) for i in range(len(queries))]) if heads_given is None \
+        else np.asarray(heads_given, dtype=np.int64)
+    out = {"kbar_bits": kbar_bits, "affinity": a, "heads": heads, "queries": queries,
+           "routed_scores": [], "routed_cond": [], "idx": [], "cand": [], "scores": [], "cond": []}
+    for i, t in enumerate(queries):
+        hm = np.zeros((T, H), dtype=np.uint8)
+        hm[t, heads[i][heads[i] >= 0]] = 1
+        V = int(visible_count(p[i], L))
+        keys = np.arange(V, dtype=np.int64)
+        sr, cr = score_pairs(q, k, w, np.full(V, t, dtype=np.int64), keys, hmask=hm)
+        out["routed_scores"].append(sr)
+        out["routed_cond"].append(cr)
+        if kprime <= 0:
+            out["idx"].append(select_topk(sr, topk))
+            continue
+        cand = select_topk(sr, kprime) if cand_given is None else np.asarray(cand_given[i], dtype=np.int64)
+        out["cand"].append(cand)
+        cv = cand[cand >= 0]
+        _, s, c = dense_scores_row(q, k, w, int(t), int(p[i]), keys=cv)
+        out["scores"].append(s)
+        out["cond"].append(c)
+        out["idx"].append(select_topk(s, topk, index=cv))
+    out["idx"] = np.array(out["idx"], dtype=np.int64).reshape(len(queries), topk)
+    return out
+
+
+# ------------------------------------------------------------ HISA
+def hisa(inp, block: int, m: int, topk: int, queries: Optional[Sequence[int]] = None, b: int = 0,
+         blocks_given: Optional[np.ndarray] = None):
+    """HISA: block-level coarse filter on pooled keys (top-m blocks), then
+    token-level scoring inside the surviving blocks (top-k).
+
+    blocks_given [nq, m]: run the token stage on these blocks instead of the
+    oracle's own choice."""
+    assert inp.dtype == "bf16"
+    q, k, w = dequant(inp, b)
+    T, H, d = q.shape
+    L = k.shape[0]
+    if queries is None:
+        queries = np.arange(T)
+    queries = np.asarray(queries, dtype=np.int64)
+    kbar_bits = meanpool_bf16(inp.k[b], block)
+    kbar = widen_bf16(kbar_bits)
+    M = kbar.shape[0]
+    p = inp.q_offset + queries
+    nvb = visible_blocks(p, block, M)
+    out = {"kbar_bits": kbar_bits, "queries": queries, "block_scores": [], "block_cond": [],
+           "blocks": [], "idx": [], "tokens": [], "scores": [], "cond": []}
+    for i, t in enumerate(queries):
+        bidx = np.arange(nvb[i], dtype=np.int64)
+        sb, cb = score_pairs(q[t][None], kbar, w[t][None], np.zeros(bidx.size, dtype=np.int64), bidx)
+        out["block_scores"].append(sb)
+        out["block_cond"].append(cb)
+        blocks = select_topk(sb, m) if blocks_given is None else np.asarray(blocks_given[i], dtype=np.int64)
+        out["blocks"].append(blocks)
+        bv = blocks[blocks >= 0]
+        toks = (bv[:, None] * block + np.arange(block, dtype=np.int64)[None, :]).reshape(-1)
+        toks = np.sort(toks[toks < visible_count(p[i], L)])
+        _, s, c = dense_scores_row(q, k, w, int(t), int(p[i]), keys=toks)
+        out["tokens"].append(toks)
+        out["scores"].append(s)
+        out["cond"].append(c)
+        out["idx"].append(select_topk(s, topk, index=toks))
+    out["blocks"] = np.array(out["blocks"], dtype=np.int64).reshape(len(queries), m)
+    out["idx"] = np.array(out["idx"], dtype=np.int64).reshape(len(queries), topk)
+    return out
