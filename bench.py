@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 lightning indexer (score + top-k) on synthetic inputs.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the indexer hot path over one batch of resident inputs:
+for the default workload (the DeepSeek-V3.2-shaped prefill chunk: T=4096
+queries at the end of a 32768-token prefix, H_I=64, d=128, top-k=2048) that is
+tcgen05 scoring of every visible (query, key) pair followed by the per-query
+radix top-k, both through the C-ABI entry point indexer_score_topk.
+Other workloads: tiny, decode (FP8), misa (MISA-dagger), hisa.
+
+The metric is scored query-key pairs per second (visible pairs of the dense
+problem, so routed / filtered variants show their speed-up in the same unit).
+Timing: W warm-up steps, then K steps, each preceded by a 256 MiB L2 flush
+and timed with CUDA events on the launching stream; a barrier + synchronize
+bracket the timed region; the max over ranks is reported. With N > 1 every
+rank runs an independent replica on its own GPU (the path has no exchange
+step), so the aggregate is weak scaling.
+
+Extra keys: roofline of the dominant kernel (timed alone, same inputs),
+cpu_baseline (the fp64 oracle on a bounded sample, host cores), e2e (host
+buffers, H2D + call + D2H inside the timed region), clocks sampled during the
+timed region, gpu_launches.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DSA indexer score+top-k: Gpairs/s and % roofline (prefill TC, decode HBM)"
+UNIT = "Gpairs/s"
+FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ workloads
+def workload_desc(name):
+    from sparse_attention_token_score_b200 import workloads as wl
+    c = dict(wl.CONFIGS[name])
+    batch = c.get("batch", 1)
+    off = c.get("q_offset", c["L"] - 1)
+    pairs = wl.visible_pairs(c["T"], c["L"], off, batch)
+    tag = {"tiny": "tiny_prefill", "dsa": "dsa_chunk", "decode": "decode_fp8",
+           "misa": "misa_dagger", "hisa": "hisa"}[name]
+    label = f"{tag}_B{batch}_T{c['T']}_L{c['L']}_H{c['H']}_d{c['d']}_k{c['topk']}"
+    if name == "misa":
+        label += f"_blk{c['block']}_h{c['h']}_kp{c['kprime']}"
+    if name == "hisa":
+        label += f"_blk{c['block']}_m{c['m']}"
+    return c, batch, off, pairs, label
+
+
+class Runner:
+    """Device-resident inputs + the C-ABI call of one workload."""
+
+    def __init__(self, name, inp, torch):
+        from sparse_attention_token_score_b200 import binding as B
+        self.B, self.torch, self.name = B, torch, name
+        self.c, self.batch, self.off, self.pairs, self.label = workload_desc(name)
+        self.inp = inp
+        q, k, w, qs, ks = B.to_device(inp)
+        self.dev = (q, k, w, qs, ks)
+        self.ix = B.Indexer(q, k, w, inp.q_offset, qs, ks)
+        c = self.c
+        self.topk = c["topk"]
+        self.idx = torch.empty((self.batch, c["T"], self.topk), dtype=torch.int32, device="cuda")
+        a = self.ix.args
+        if name in ("tiny", "dsa", "decode"):
+            self.ws = B.alloc_workspace(B.indexer_workspace_size(a, self.topk))
+            self.launches = 2
+        elif name == "misa":
+            self.ws = B.alloc_workspace(B.misa_workspace_size(a, c["block"], c["h"], self.topk, c["kprime"]))
+            self.launches = 7  # meanpool, router, select_heads, routed score, top-k', gather score, top-k
+        else:
+            self.ws = B.alloc_workspace(B.hisa_workspace_size(a, c["block"], c["m"], self.topk))
+            self.launches = 5  # meanpool, block score, top-m, gather score, top-k
+        self.dtype = "e4m3" if inp.dtype != "bf16" else "bf16"
+
+    def step(self, args=None, out=None):
+        B, c = self.B, self.c
+        a = self.ix.args if args is None else args
+        o = self.idx if out is None else out
+        if self.name in ("tiny", "dsa", "decode"):
+            B.indexer_score_topk(a, self.topk, o, None, self.ws)
+        elif self.name == "misa":
+            B.misa_route_score_topk(a, c["block"], c["h"], self.topk, c["kprime"], o, None, None,
+                                    None, self.ws)
+        else:
+            B.hisa_block_filter_topk(a, c["block"], c["m"], self.topk, o, None, None, self.ws)
+
+    # dominant kernel, launched alone through the score-stage entry point
+    def dominant(self):
+        """(callable, algorithmic units per launch, bound, name)."""
+        B, torch, c = self.B, self.torch, self.c
+        if self.name in ("tiny", "dsa", "decode"):
+            out = torch.empty((self.batch, c["T"], c["L"]), dtype=torch.float32, device="cuda")
+            ws = B.alloc_workspace(256)
+            fn = lambda: B.indexer_scores(self.ix.args, out, c["L"], ws)
+            if self.name == "decode":
+                # bytes the scorer must read per visible pair: one FP8 key row + its fp32 scale
+                return fn, self.pairs * (c["d"] + 4), "hbm", "score_tc<fp8>"
+            return fn, self.pairs * 2.0 * c["d"] * c["H"], "tensor", "score_tc<bf16>"
+        if self.name == "misa":
+            # the routed scoring pass: the same kernel on h gathered heads per query
+            q, k, w, _, _ = self.dev
+            h = c["h"]
+            qh = q[:, :, :h].contiguous()
+            wh = w[:, :, :h].contiguous()
+            a = B.make_args(qh, k, wh, self.inp.q_offset)
+            out = torch.empty((self.batch, c["T"], c["L"]), dtype=torch.float32, device="cuda")
+            ws = B.alloc_workspace(256)
+            self._keep = (qh, wh, a, out, ws)
+            return (lambda: B.indexer_scores(a, out, c["L"], ws)), self.pairs * 2.0 * c["d"] * h, \
+                "tensor", "score_tc<bf16,h=8> (routed)"
+        return None, None, None, None
+
+
+def l2_flush(buf):
+    buf.add_(1)
+
+
+def time_steps(fn, n, torch, flush):
+    """Per-launch CUDA-event times (ms) on the current stream, L2 flushed before each."""
+    st = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for e0, e1 in ev:
+        l2_flush(flush)
+        e0.record(st)
+        fn()
+        e1.record(st)
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-i", str(gpu_index), "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.p.terminate()
+        self.p.wait(timeout=10)
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.count(",") >= 8]
+        os.unlink(self.f.name)
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v and "Not" not in v})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+def oracle_sample(name, inp, budget_s=12.0, max_q=4096):
+    """Time the fp64 oracle, as it stands, on a bounded sample of this workload's
+    queries (the same computation as one GPU step, restricted to the sample)."""
+    import oracle
+    from sparse_attention_token_score_b200 import workloads as wl
+    c = wl.CONFIGS[name]
+    T = c["T"]
+    rng = np.random.default_rng(1)
+
+    def run(qs, b=0):
+        t0 = time.perf_counter()
+        if name == "misa":
+            oracle.misa(inp, c["block"], c["h"], c["topk"], kprime=c["kprime"], queries=qs, b=b)
+        elif name == "hisa":
+            oracle.hisa(inp, c["block"], c["m"], c["topk"], queries=qs, b=b)
+        else:
+            oracle.dense_topk(inp, c["topk"], queries=qs, b=b)
+        return time.perf_counter() - t0
+
+    def pairs(qs, b=0):
+        off = inp.q_offset
+        return int(sum(min(off + int(t) + 1, inp.L) for t in qs))
+
+    if name == "decode":
+        # one unit = one sequence's query
+        t1 = run([0], b=0)
+        nb = max(1, min(inp.batch, int(budget_s / max(t1, 1e-3))))
+        t = 0.0
+        for b in range(1, nb + 1):
+            t += run([0], b=b % inp.batch)
+        return nb * inp.L / t / 1e9, f"{nb} of {inp.batch} sequences (all {inp.L} keys each)", nb, t
+    q1 = rng.choice(T, 2, replace=False)
+    t1 = run(q1) / 2
+    n = int(max(2, min(max_q, budget_s / max(t1, 1e-4))))
+    qs = np.sort(rng.choice(T, n, replace=False)) if n < T else np.arange(T)
+    t = run(qs)
+    return pairs(qs) / t / 1e9, f"{len(qs)} of {T} queries (uniform sample)", len(qs), t
+
+
+def run_reference(args):
+    """The oracle arm: fp64 CPU oracle on host cores, bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from sparse_attention_token_score_b200 import workloads as wl
+    c, batch, off, pairs, label = workload_desc(args.workload)
+    inp = wl.make_inputs(args.workload, seed=0)
+    per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    vals, samples = [], None
+    for i in range(args.warmup + args.steps):
+        v, samples, _, _ = oracle_sample(args.workload, inp, budget_s=per_step / 2)
+        if i >= args.warmup:
+            vals.append(v)
+    value = float(np.mean(vals))
+    cores = oracle.num_threads()
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": pairs / (value * 1e9) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": label, "pairs_per_step": pairs, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": samples},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="dsa", choices=["tiny", "dsa", "decode", "misa", "hisa"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from sparse_attention_token_score_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    inp = wl.make_inputs(args.workload, seed=rank)
+    r = Runner(args.workload, inp, torch)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    for _ in range(args.warmup):
+        r.step()
+    torch.cuda.synchronize()
+
+    # ---- timed region
+    sampler = ClockSampler(local) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    times = time_steps(r.step, args.steps, torch, flush)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms = float(sum(times))
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * r.pairs * args.steps / (total_ms / 1e3) / 1e9
+    assert r.ix.device_status() == 0, "device wait timed out"
+
+    # ---- dominant kernel alone (roofline)
+    peaks, peak_src = load_peaks()
+    fn, units, bound, kname = r.dominant()
+    roof = None
+    if fn is not None:
+        for _ in range(3):
+            fn()
+        kt = time_steps(fn, args.steps, torch, flush)
+        kms = statistics.mean(kt)
+        if bound == "tensor":
+            achieved = units / (kms / 1e3) / 1e12
+            peak = peaks["bf16_tflops"]
+            unit = "TFLOP/s"
+        else:
+            achieved = units / (kms / 1e3) / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+        roof = {"bound": bound, "kernel": kname, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "peak_source": f"{peak_src} ({'bf16 burst' if bound == 'tensor' else 'HBM copy'})",
+                "kernel_ms": kms, "algorithmic_units_per_launch": units, "traffic": None}
+
+    # ---- end to end: host buffers, H2D + call + D2H per step
+    q, k, w, qs, ks = r.dev
+    host = [t.cpu().pin_memory() if t is not None else None for t in (q, k, w, qs, ks)]
+    dev2 = [torch.empty_like(t) if t is not None else None for t in (q, k, w, qs, ks)]
+    from sparse_attention_token_score_b200 import binding as B
+    a2 = B.make_args(dev2[0], dev2[1], dev2[2], inp.q_offset, dev2[3], dev2[4])
+    out_host = torch.empty(r.idx.shape, dtype=torch.int32, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host if t is not None)
+    d2h = out_host.numel() * 4
+
+    def e2e_step():
+        for hsrc, ddst in zip(host, dev2):
+            if hsrc is not None:
+                ddst.copy_(hsrc, non_blocking=True)
+        r.step(args=a2)
+        out_host.copy_(r.idx, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    et = time_steps(e2e_step, args.steps, torch, flush)
+    e_ms = float(sum(et))
+    if world > 1:
+        t = torch.tensor([e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e_value = world * r.pairs * args.steps / (e_ms / 1e3) / 1e9
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        v, sample, _, secs = oracle_sample(args.workload, inp)
+        cpu = {"value": v, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": sample, "seconds": round(secs, 2)}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    c = r.c
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": r.dtype, "data": "synthetic",
+        "config": {"workload": r.label, "batch": r.batch, "T": c["T"], "L": c["L"], "H": c["H"],
+                   "d": c["d"], "topk": c["topk"], "q_offset": inp.q_offset,
+                   "pairs_per_step": r.pairs, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "256 MiB buffer written before every timed step"},
+        "queries_per_s": world * r.batch * c["T"] * args.steps / (total_ms / 1e3),
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e_ms / args.steps},
+        "gpu_launches": r.launches * args.steps,
+        "clocks": clocks,
+        "step_ms": {"min": min(times), "median": statistics.median(times), "max": max(times)},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

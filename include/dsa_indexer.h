@@ -1,0 +1,167 @@
+/*
+ * dsa_indexer.h - C ABI of the B200 (sm_100a) DeepSeek-Sparse-Attention
+ * lightning indexer: dense scoring + top-k, MISA head routing, HISA
+ * block-then-token filtering.
+ *
+ * The method (sources: "MISA: Mixture of Indexer Sparse Attention for
+ * Long-Context LLM Inference", sections "Problem statement", "Methodology",
+ * "Hierarchical variant (MISA-dagger)"; "HISA: Efficient Hierarchical Indexing
+ * for Fine-Grained Sparse Attention" review, section 3; "DoSA: Dots Sparse
+ * Attention" review, section 3, for the signed head weights):
+ *
+ *   For query t at absolute position p_t = q_offset + t, every key s <= p_t
+ *   (s < L) is scored by H indexer heads,
+ *       I[t,s] = sum_h w[t,h] * ReLU(q[t,h,:] . k[s,:]),
+ *   and the top-k keys are kept for the downstream sparse attention.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, row-major, owned by the caller.
+ *     The library allocates nothing; scratch lives in a caller-provided
+ *     workspace whose size the *_workspace_size functions return.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Arguments are validated on the host before any launch;
+ *     a failed validation returns an error and launches nothing.
+ *   - Selection: the k best candidates by (score descending, index ascending);
+ *     fewer candidates than k -> all of them. Each output row lists the chosen
+ *     indices in ascending order, padded with -1 (and score -inf).
+ *   - The first 256 bytes of every workspace hold a device status word. Each
+ *     call clears it; kernels set it if a bounded wait gave up.
+ *     dsa_device_status() synchronises the stream and reports it.
+ *   - The workspace must be 256-byte aligned; q and k 16-byte aligned; w and
+ *     scales 4-byte aligned.
+ *   - Calls that share a workspace must not overlap in time (use one stream).
+ *
+ * Supported shapes: d in {64, 128}; bf16 H in {8, 16, 32, 64};
+ * FP8 e4m3 (decode): d = 128, H in {32, 64}. Other shapes return
+ * DSA_ERR_UNSUPPORTED.
+ */
+#ifndef DSA_INDEXER_H
+#define DSA_INDEXER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_EXPORT __attribute__((visibility("default")))
+#else
+#define DSA_EXPORT
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { DSA_BF16 = 0, DSA_FP8_E4M3 = 1 } dsa_dtype;
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_ARG = -1,         /* null pointer, bad size, misaligned pointer            */
+  DSA_ERR_UNSUPPORTED = -2, /* valid but not built: head count, head dim, dtype      */
+  DSA_ERR_WORKSPACE = -3,   /* ws_bytes smaller than the *_workspace_size result     */
+  DSA_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed           */
+  DSA_ERR_TIMEOUT = -5      /* a device-side bounded wait gave up (dsa_device_status) */
+} dsa_status;
+
+/* One indexer problem: `batch` independent sequences, each with T queries at
+ * positions q_offset .. q_offset+T-1 and a prefix of L keys. */
+typedef struct {
+  int batch;          /* independent sequences (decode: one query each)          */
+  int T;              /* queries per sequence                                    */
+  int L;              /* keys per sequence                                       */
+  int H;              /* indexer heads                                           */
+  int d;              /* head dimension                                          */
+  long long q_offset; /* absolute position of query 0 (>= 0); key s is visible to
+                         query t iff s <= q_offset + t                           */
+  dsa_dtype qk_dtype; /* DSA_BF16: q, k bf16; DSA_FP8_E4M3: q, k e4m3 bytes       */
+  const void* q;      /* [batch, T, H, d]                                        */
+  const float* q_scale; /* [batch, T, H] per-(query, head) dequant scale (FP8), else NULL */
+  const void* k;      /* [batch, L, d]                                           */
+  const float* k_scale; /* [batch, L] per-token dequant scale (FP8), else NULL    */
+  const float* w;     /* [batch, T, H] signed head weights, fp32                 */
+} dsa_indexer_args;
+
+/* Human-readable name of a status code (static storage). */
+DSA_EXPORT const char* dsa_status_string(dsa_status s);
+
+/* Synchronise `stream`, then report and clear the device status word of
+ * `workspace`: DSA_ERR_TIMEOUT if a kernel's bounded wait gave up since the
+ * last call that used this workspace, DSA_ERR_CUDA on a CUDA error, else OK. */
+DSA_EXPORT dsa_status dsa_device_status(void* workspace, void* stream);
+
+/* ------------------------------------------------------------ dense indexer
+ * indexer_score_topk: for every query of every sequence, score all visible
+ * keys with all H heads and keep the top `topk`.
+ *   out_idx   [batch, T, topk] int32 key indices (ascending, -1 padded)
+ *   out_score [batch, T, topk] fp32 scores of those keys, or NULL
+ * bf16 inputs score on tcgen05 bf16 MMAs; FP8 inputs use FP8 MMAs with
+ *   I[t,s] = k_scale[s] * sum_h (w[t,h] * q_scale[t,h]) * ReLU(q8[t,h,:] . k8[s,:]).
+ * Workspace: [batch*T*L] fp32 scores plus the 256-byte header. */
+DSA_EXPORT size_t indexer_workspace_size(const dsa_indexer_args* a, int topk);
+DSA_EXPORT dsa_status indexer_score_topk(const dsa_indexer_args* a, int topk, int32_t* out_idx,
+                              float* out_score, void* workspace, size_t ws_bytes, void* stream);
+
+/* Stage 1 alone: write the scores I[t,s] of all visible keys into
+ * out_scores[(b*T + t) * ld + s] (ld >= L). Entries with s > q_offset + t are
+ * left untouched. Workspace: the 256-byte header only. */
+DSA_EXPORT dsa_status indexer_scores(const dsa_indexer_args* a, float* out_scores, long long ld,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* Stage 2 alone: per-row top-k of fp32 scores [rows, ld]. Row r belongs to
+ * query t = r % T; its candidates are positions 0 .. n_r - 1 with
+ *   n_r = clamp((q_offset + t) / pstride + 1, 0, row_len)   if pstride > 0,
+ *   n_r = row_len                                           if pstride == 0.
+ * -inf marks an absent candidate. Selected positions j are written as
+ *   cand[r * n_slots + j / blk] * blk + j % blk   if cand != NULL, else j.
+ * Workspace: the 256-byte header only. */
+DSA_EXPORT dsa_status indexer_topk_rows(const float* scores, long long rows, long long ld, int T,
+                             long long q_offset, int pstride, int row_len, int topk,
+                             const int32_t* cand, int n_slots, int blk, int32_t* out_idx,
+                             float* out_score, void* workspace, size_t ws_bytes, void* stream);
+
+/* Pooled keys: kbar[b, m, :] = bf16(mean of k[b, m*block : min((m+1)*block, L), :]),
+ * m < M = ceil(L / block); mean in fp64, rounded once (nearest even). bf16 only.
+ *   k [batch, L, d] bf16 -> kbar [batch, M, d] bf16. */
+DSA_EXPORT dsa_status dsa_meanpool_keys(const void* k, int batch, int L, int d, int block, void* kbar,
+                             void* stream);
+
+/* ------------------------------------------------------------ MISA
+ * misa_route_score_topk (MISA page, "Methodology"): split the prefix into
+ * M = ceil(L / block) blocks of mean-pooled keys kbar; per query and head the
+ * router affinity
+ *     a[t,h] = |w[t,h]| * sum over blocks m with m*block <= p_t of ReLU(q[t,h,:] . kbar[m,:]);
+ * keep the top-h heads per query (ties -> lower head); score every visible
+ * token with those heads only (their original signed weights); keep the top
+ * `topk` (kprime == 0), or, MISA-dagger (kprime > 0), keep the top `kprime`
+ * candidates, re-score them with all H heads and keep the top `topk`.
+ *   out_idx   [batch, T, topk] int32 token indices
+ *   out_score [batch, T, topk] fp32 (routed scores; full-H scores for MISA-dagger) or NULL
+ *   out_heads [batch, T, h] int32 chosen heads (ascending) or NULL
+ *   out_cand  [batch, T, kprime] int32 MISA-dagger candidates (ascending, -1 padded) or NULL
+ * bf16 only; h in {8, 16, 32, 64}, h <= H; MISA-dagger needs d = 128 and
+ * H in {32, 64}. */
+DSA_EXPORT size_t misa_workspace_size(const dsa_indexer_args* a, int block, int h, int topk, int kprime);
+DSA_EXPORT dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, int topk,
+                                 int kprime, int32_t* out_idx, float* out_score,
+                                 int32_t* out_heads, int32_t* out_cand, void* workspace,
+                                 size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------ HISA
+ * hisa_block_filter_topk (HISA review, section 3): block-level coarse filter,
+ * then token-level refinement. Pooled keys kbar as for MISA; block score
+ *     S_b[t,m] = sum_h w[t,h] * ReLU(q[t,h,:] . kbar[m,:]) for blocks with m*block <= p_t;
+ * keep the top-m blocks (ties -> lower block); score the visible tokens of the
+ * kept blocks with the full indexer; keep the top `topk`.
+ *   out_idx    [batch, T, topk] int32 token indices
+ *   out_score  [batch, T, topk] fp32 token scores or NULL
+ *   out_blocks [batch, T, m] int32 kept blocks (ascending, -1 padded) or NULL
+ * bf16 only; token refinement needs d = 128 and H in {32, 64}. */
+DSA_EXPORT size_t hisa_workspace_size(const dsa_indexer_args* a, int block, int m, int topk);
+DSA_EXPORT dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, int topk,
+                                  int32_t* out_idx, float* out_score, int32_t* out_blocks,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_INDEXER_H */

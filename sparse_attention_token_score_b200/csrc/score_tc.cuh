@@ -1,0 +1,474 @@
+// Lightning-indexer scoring on the 5th-generation tensor cores (tcgen05).
+//
+// Score (DeepSeek Sparse Attention lightning indexer; "MISA: Mixture of
+// Indexer Sparse Attention for Long-Context LLM Inference", section "Problem
+// statement"; signed head weights: "DoSA: Dots Sparse Attention", section 3):
+//     I[t,s] = sum_h w[t,h] * ReLU(q[t,h,:] . k[s,:])
+// FP8 inputs carry a per-token key scale and a per-(query, head) scale, and
+// since ReLU(a*x) = a*ReLU(x) for a > 0 the kernel computes
+//     I[t,s] = ks[s] * sum_h (w[t,h] * qs[t,h]) * ReLU(q8[t,h,:] . k8[s,:]).
+//
+// One persistent CTA per SM, warp-specialised:
+//   producer warp(s) -> shared-memory ring of key tiles (TMA, or cp.async
+//                       gathers of arbitrary key rows), plus the stationary
+//                       query tile of the current query group (TMA)
+//   MMA warp         -> one thread issues tcgen05.mma into a double-buffered
+//                       TMEM accumulator
+//   8 epilogue warps -> tcgen05.ld, ReLU, head-weighted sum, causal mask,
+//                       fp32 store. The [T, H, L] head logits never leave TMEM.
+//
+// Orientation (score modes): keys on the MMA M dimension (128 TMEM lanes, one
+// key per epilogue thread), QPT queries x H heads on N, so each thread reduces
+// over heads inside its own registers. Router mode swaps the roles: QPT*H =
+// 128 (query, head) rows on M, 256 pooled keys on N, and each thread reduces
+// ReLU over the pooled keys (MISA page, section "Methodology", step 1).
+//
+// Work split: the (query group, key tile) pairs of the whole launch are
+// flattened and every CTA takes one contiguous range, so causal imbalance
+// between groups evens out; the query tile is reloaded only when the group
+// changes. Router mode assigns whole groups round-robin (its per-row sums
+// must not be split across CTAs).
+#pragma once
+#include "common.cuh"
+
+namespace dsa {
+
+enum class ScoreMode : int { kTma = 0, kGather = 1, kRouter = 2 };
+
+struct ScoreParams {
+  int batch;            // independent sequences
+  int T;                // queries per sequence
+  int Lk;               // key rows per sequence (tokens, or pooled blocks)
+  int L_tok;            // gather mode: tokens per sequence (rows of kg per sequence)
+  long long q_offset;   // absolute position of query 0
+  int pstride;          // key row s sits at position s * pstride (1 = tokens, B = blocks)
+  const float* w;       // [batch*T, H] signed head weights
+  const float* q_scale; // [batch*T, H] (FP8) or nullptr
+  const float* k_scale; // [batch*Lk]   (FP8) or nullptr
+  float* out;           // score: [batch*T, ldo]; router: 2 x [batch*T*H] partial sums
+  long long ldo;
+  const __nv_bfloat16* kg;  // gather mode: keys [batch*L_tok, D]
+  const int* cand;          // gather mode: [batch*T, n_slots] block / token ids, -1 = none
+  int n_slots, blk, n_compact;  // compact position c -> cand[c / blk] * blk + c % blk
+  unsigned* err;            // device error word
+};
+
+template <int ELEM_, int D_, int H_, int QPT_, ScoreMode MODE_, int NSTAGE_>
+struct ScoreCfg {
+  static constexpr int ELEM = ELEM_;  // bytes per element: 2 = bf16, 1 = e4m3
+  static constexpr int D = D_, H = H_, QPT = QPT_, NSTAGE = NSTAGE_;
+  static constexpr ScoreMode MODE = MODE_;
+  static constexpr bool ROUTER = MODE_ == ScoreMode::kRouter;
+  static constexpr bool GATHER = MODE_ == ScoreMode::kGather;
+  static constexpr int ROW_BYTES = D * ELEM;
+  static_assert(ROW_BYTES == 128 || ROW_BYTES == 256, "rows must be 1 or 2 swizzle atoms wide");
+  static constexpr int KBLK = ROW_BYTES / 128;          // 128-byte column blocks per row
+  static constexpr int QROWS = QPT * H;                 // stationary query tile rows
+  static constexpr int KROWS = ROUTER ? 256 : 128;      // streaming key tile rows
+  static constexpr int MMA_N = ROUTER ? KROWS : QROWS;
+  static_assert(ROUTER ? QROWS == 128 : (QROWS % 16 == 0 && QROWS >= 32 && QROWS <= 256),
+                "bad tile shape");
+  static_assert(!GATHER || (QPT == 1 && ELEM == 2 && ROW_BYTES == 256),
+                "gather mode: one bf16 query per group, d = 128");
+  // Each producer warp owns the stages s with s % NPROD == its index, so every
+  // stage is refilled by one warp in order and a parity wait is never more
+  // than one phase behind.
+  static_assert(NSTAGE % (MODE_ == ScoreMode::kGather ? 4 : 1) == 0, "stages per producer warp");
+  static constexpr int Q_BYTES = QROWS * ROW_BYTES;
+  static constexpr int K_BYTES = KROWS * ROW_BYTES;
+  static constexpr int NKSTEP = ROW_BYTES / 32;         // one MMA consumes 32 bytes of K
+  static constexpr int TMEM_COLS = (2 * MMA_N <= 32) ? 32 : (2 * MMA_N <= 64) ? 64
+                                 : (2 * MMA_N <= 128) ? 128 : (2 * MMA_N <= 256) ? 256 : 512;
+  static constexpr int NPROD = GATHER ? 4 : 1;          // producer warps
+  static constexpr int MMA_WARP = NPROD;
+  static constexpr int EPI_WARP0 = NPROD + 1;
+  static constexpr int NTHREADS = (EPI_WARP0 + 8) * 32;
+  // Tile split between the two epilogue warp sets: alternate tiles (router,
+  // and one-query groups) or the two halves of the queries of every tile.
+  static constexpr bool SPLIT_TILES = ROUTER || QPT == 1;
+  static constexpr int TEMPTY_ARRIVALS = SPLIT_TILES ? 4 : 8;
+  static constexpr uint32_t IDESC = umma_idesc(ELEM == 2 ? 1u : 0u, 128, MMA_N);
+  // shared memory layout (offsets from a 1024-aligned base)
+  static constexpr int SMEM_Q = 0;
+  static constexpr int SMEM_K = Q_BYTES;
+  static constexpr int SMEM_BAR = SMEM_K + NSTAGE * K_BYTES;
+  static constexpr int NBAR = 2 * NSTAGE + 7;
+  static constexpr int SMEM_USED = SMEM_BAR + NBAR * 8 + 16;
+  // Pad to more than half an SM so two CTAs never share an SM's TMEM.
+  static constexpr int SMEM_BYTES = (SMEM_USED + 1024 < 120 * 1024) ? 120 * 1024 : SMEM_USED + 1024;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+// Iterates this CTA's (group, tile) pairs. Every thread runs its own copy;
+// all copies visit the same sequence.
+template <class C>
+struct TileSched {
+  int gpb, G;
+  int g, j, nt;
+  long long left;   // tiles left (flat split)
+  bool first, last, done;
+
+  __device__ __forceinline__ int ntile(const ScoreParams& p, int grp) const {
+    const int tg = grp % gpb;
+    if (C::GATHER) return (p.n_compact + C::KROWS - 1) / C::KROWS;
+    const int t_last = min(p.T, (tg + 1) * C::QPT) - 1;
+    const long long pos = p.q_offset + t_last;
+    long long nk = pos / p.pstride + 1;
+    if (nk > p.Lk) nk = p.Lk;
+    return static_cast<int>((nk + C::KROWS - 1) / C::KROWS);
+  }
+
+  __device__ __forceinline__ void init(const ScoreParams& p) {
+    gpb = (p.T + C::QPT - 1) / C::QPT;
+    G = p.batch * gpb;
+    done = false;
+    if (C::ROUTER) {
+      left = 0;
+      g = blockIdx.x;
+      while (g < G && (nt = ntile(p, g)) == 0) g += gridDim.x;
+      if (g >= G) { done = true; return; }
+      j = 0;
+    } else {
+      long long W = 0;
+      for (int q = 0; q < G; ++q) W += ntile(p, q);
+      const long long b0 = W * blockIdx.x / gridDim.x;
+      const long long b1 = W * (blockIdx.x + 1) / gridDim.x;
+      left = b1 - b0;
+      if (left <= 0) { done = true; return; }
+      long long acc = 0;
+      g = 0;
+      for (;; ++g) {
+        nt = ntile(p, g);
+        if (acc + nt > b0) break;
+        acc += nt;
+      }
+      j = static_cast<int>(b0 - acc);
+    }
+    first = true;
+    last = (j == nt - 1) || (!C::ROUTER && left == 1);
+  }
+
+  __device__ __forceinline__ void next(const ScoreParams& p) {
+    if (C::ROUTER) {
+      if (++j == nt) {
+        g += gridDim.x;
+        while (g < G && (nt = ntile(p, g)) == 0) g += gridDim.x;
+        if (g >= G) { done = true; return; }
+        j = 0;
+        first = true;
+      } else {
+        first = false;
+      }
+      last = (j == nt - 1);
+    } else {
+      if (--left == 0) { done = true; return; }
+      if (++j == nt) {
+        do { ++g; nt = ntile(p, g); } while (nt == 0);
+        j = 0;
+        first = true;
+      } else {
+        first = false;
+      }
+      last = (j == nt - 1) || (left == 1);
+    }
+  }
+};
+
+// Token behind compact position c of gathered row r; -1 if there is none or it
+// is not visible to the query (position q_pos).
+__device__ __forceinline__ long long gathered_token(const ScoreParams& p, long long r, int c,
+                                                    long long q_pos) {
+  if (c >= p.n_compact) return -1;
+  const int slot = c / p.blk;
+  const int cb = __ldg(p.cand + r * p.n_slots + slot);
+  if (cb < 0) return -1;
+  const long long tok = static_cast<long long>(cb) * p.blk + (c - slot * p.blk);
+  if (tok >= p.L_tok || tok > q_pos) return -1;
+  return tok;
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::NTHREADS, 1)
+score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const ScoreParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t s_q = s_base + C::SMEM_Q;
+  const uint32_t s_k = s_base + C::SMEM_K;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
+  auto full = [&](int i) { return smem_u32(&bars[i]); };
+  auto empty = [&](int i) { return smem_u32(&bars[C::NSTAGE + i]); };
+  const uint32_t qfull = smem_u32(&bars[2 * C::NSTAGE]);
+  const uint32_t qempty = smem_u32(&bars[2 * C::NSTAGE + 1]);
+  auto tfull = [&](int b) { return smem_u32(&bars[2 * C::NSTAGE + 2 + b]); };
+  auto tempty = [&](int b) { return smem_u32(&bars[2 * C::NSTAGE + 4 + b]); };
+  const uint32_t mdone = smem_u32(&bars[2 * C::NSTAGE + 6]);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      mbar_init(full(i), C::GATHER ? 32 : 1);
+      mbar_init(empty(i), 1);
+    }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull(b), 1);
+      mbar_init(tempty(b), C::TEMPTY_ARRIVALS);
+    }
+    mbar_init(mdone, 1);
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32 * C::MMA_WARP + 1) {
+    tma_prefetch_desc(&tm_q);
+    if (!C::GATHER) tma_prefetch_desc(&tm_k);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  TileSched<C> s;
+  s.init(p);
+
+  if (warp < C::NPROD) {
+    // ------------------------------------------------------------ producer
+    const int pw = warp;
+    uint32_t it = 0, gq = 0;
+    bool ok = true;
+    for (; !s.done; s.next(p), ++it) {
+      const int b = s.g / s.gpb;
+      const int tg = s.g % s.gpb;
+      const bool mine = C::GATHER ? (static_cast<int>(it % C::NPROD) == pw) : true;
+      if (s.first) {
+        // The query tile is always loaded by warp 0, group by group in order.
+        if (pw == 0 && lane == 0) {
+          if (!mbar_wait(qempty, (gq & 1u) ^ 1u, p.err)) { ok = false; }
+          else {
+            mbar_arrive_expect_tx(qfull, C::Q_BYTES);
+            const int row0 = (b * p.T + tg * C::QPT) * C::H;
+#pragma unroll
+            for (int kb = 0; kb < C::KBLK; ++kb)
+              tma_load_2d(s_q + kb * C::QROWS * 128, &tm_q, qfull, kb * (128 / C::ELEM), row0);
+          }
+        }
+        ++gq;
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      if (!mine) continue;
+      const int stage = static_cast<int>(it % C::NSTAGE);
+      const uint32_t ph = (it / C::NSTAGE) & 1u;
+      if (!C::GATHER) {
+        if (lane == 0) {
+          if (!mbar_wait(empty(stage), ph ^ 1u, p.err)) { ok = false; }
+          else {
+            mbar_arrive_expect_tx(full(stage), C::K_BYTES);
+            const int krow0 = b * p.Lk + s.j * C::KROWS;
+#pragma unroll
+            for (int kb = 0; kb < C::KBLK; ++kb)
+              tma_load_2d(s_k + stage * C::K_BYTES + kb * C::KROWS * 128, &tm_k, full(stage),
+                          kb * (128 / C::ELEM), krow0);
+          }
+        }
+      } else {
+        // Gather 128 key rows (one per compact position) with 16-byte cp.async:
+        // a half-warp copies one 256-byte row, chunk c of row r lands at its
+        // 128-byte-swizzle slot (c ^ (r & 7)) so the tensor core sees the same
+        // layout a TMA load would have written.
+        if (!mbar_wait(empty(stage), ph ^ 1u, p.err)) ok = false;
+        if (ok) {
+          const long long r = static_cast<long long>(b) * p.T + tg;
+          const long long q_pos = p.q_offset + tg;
+          const int ch = lane & 15;
+          const uint32_t tile = s_k + stage * C::K_BYTES;
+          for (int i = 0; i < C::KROWS / 2; ++i) {
+            const int row = 2 * i + (lane >> 4);
+            const long long tok = gathered_token(p, r, s.j * C::KROWS + row, q_pos);
+            const int kb = ch >> 3;
+            const uint32_t dst = tile + kb * C::KROWS * 128 + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+            if (tok >= 0) {
+              const __nv_bfloat16* src = p.kg + (static_cast<long long>(b) * p.L_tok + tok) * C::D + ch * 8;
+              cp_async_16(dst, src);
+            } else {
+              asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+            }
+          }
+          cp_async_commit_wait_all();
+          fence_proxy_async_smem();
+          mbar_arrive(full(stage));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+    }
+    if (!ok && lane == 0) {
+      // Error path: wait (bounded) for the TMA loads that may still be in
+      // flight before the CTA releases its shared memory. cp.async gathers
+      // were already waited for before their arrive.
+      if (pw == 0 && gq > 0) mbar_drain(qfull, (gq - 1) & 1u);
+      if (!C::GATHER) {
+        const uint32_t lo = it > C::NSTAGE ? it - C::NSTAGE : 0;
+        for (uint32_t i = lo; i < it; ++i) mbar_drain(full(i % C::NSTAGE), (i / C::NSTAGE) & 1u);
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, gq = 0;
+      bool ok = true;
+      for (; !s.done; s.next(p), ++it) {
+        if (s.first && !mbar_wait(qfull, gq & 1u, p.err)) { ok = false; break; }
+        const int stage = static_cast<int>(it % C::NSTAGE);
+        const uint32_t ph = (it / C::NSTAGE) & 1u;
+        const int buf = static_cast<int>(it & 1u);
+        const uint32_t tph = (it >> 1) & 1u;
+        if (!mbar_wait(tempty(buf), tph ^ 1u, p.err)) { ok = false; break; }
+        if (!mbar_wait(full(stage), ph, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::MMA_N);
+        const uint32_t k_tile = s_k + stage * C::K_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < C::NKSTEP; ++ks) {
+          const int kb = (ks * 32) / 128;
+          const int inner = (ks * 32) % 128;
+          const uint64_t kdesc = umma_desc_sw128(k_tile + kb * C::KROWS * 128 + inner);
+          const uint64_t qdesc = umma_desc_sw128(s_q + kb * C::QROWS * 128 + inner);
+          const uint64_t adesc = C::ROUTER ? qdesc : kdesc;
+          const uint64_t bdesc = C::ROUTER ? kdesc : qdesc;
+          if (C::ELEM == 2) mma_bf16(d_tmem, adesc, bdesc, C::IDESC, ks > 0 ? 1u : 0u);
+          else mma_f8(d_tmem, adesc, bdesc, C::IDESC, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(empty(stage));
+        tc_commit(tfull(buf));
+        if (s.last) { tc_commit(qempty); ++gq; }
+      }
+      if (!ok) {
+        // Error path: let every MMA already issued finish before TMEM is freed.
+        tc_commit(mdone);
+        mbar_drain(mdone, 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - C::EPI_WARP0;        // 0..7
+    const int quarter = warp & 3;              // TMEM lanes this warp may read
+    const int set = e >> 2;                    // 0 or 1
+    const int row = quarter * 32 + lane;       // accumulator row = TMEM lane
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    float racc = 0.f;                          // router partial sum
+    uint32_t it = 0;
+    for (; !s.done; s.next(p), ++it) {
+      const int b = s.g / s.gpb;
+      const int tg = s.g % s.gpb;
+      const int buf = static_cast<int>(it & 1u);
+      const bool mine = C::SPLIT_TILES ? (buf == set) : true;
+      if (mine) {
+        if (!mbar_wait(tfull(buf), (it >> 1) & 1u, p.err)) break;
+        tc_fence_after();
+        const uint32_t taddr = lane_addr + static_cast<uint32_t>(buf * C::MMA_N);
+        if (C::ROUTER) {
+          // rows: (query, head) pairs; columns: pooled keys j*256 + c
+          const int t = tg * C::QPT + row / C::H;
+          const long long pos = p.q_offset + (t < p.T ? t : p.T - 1);
+          long long mv = pos / p.pstride + 1;
+          if (mv > p.Lk) mv = p.Lk;
+          const long long m0 = static_cast<long long>(s.j) * C::KROWS;
+          float part = 0.f;
+#pragma unroll 1
+          for (int cc = 0; cc < C::KROWS; cc += 32) {
+            float v[32];
+            tmem_ld32(taddr + cc, v);
+            if (m0 + cc + 32 <= mv) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) part += fmaxf(v[i], 0.f);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) part += (m0 + cc + i < mv) ? fmaxf(v[i], 0.f) : 0.f;
+            }
+          }
+          racc += part;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty(buf));
+        } else {
+          constexpr int QH = C::SPLIT_TILES ? 1 : C::QPT / 2;   // queries per thread
+          constexpr int NC = QH * C::H;                          // columns per thread
+          const int q0 = C::SPLIT_TILES ? 0 : set * QH;          // first query (in group)
+          const int key = s.j * C::KROWS + row;                  // key row / compact position
+          const long long rbase = static_cast<long long>(b) * p.T + tg * C::QPT + q0;
+          float acc[QH];
+#pragma unroll
+          for (int i = 0; i < QH; ++i) acc[i] = 0.f;
+#pragma unroll
+          for (int cc = 0; cc < NC; cc += 32) {
+            float coef[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int ql = (cc + i) / C::H;
+              const int h = (cc + i) % C::H;
+              const int tq = tg * C::QPT + q0 + ql;
+              const long long ci = (rbase + ql - (tq < p.T ? 0 : tq - p.T + 1)) * C::H + h;
+              float c = __ldg(p.w + ci);
+              if (C::ELEM == 1) c *= __ldg(p.q_scale + ci);
+              coef[i] = c;
+            }
+            float v[32];
+            tmem_ld32(taddr + q0 * C::H + cc, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int ql = (cc + i) / C::H;
+              acc[ql] = fmaf(coef[i], fmaxf(v[i], 0.f), acc[ql]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty(buf));
+          if (C::GATHER) {
+            const long long r = static_cast<long long>(b) * p.T + tg;
+            if (key < p.n_compact) {
+              const long long tok = gathered_token(p, r, key, p.q_offset + tg);
+              p.out[r * p.ldo + key] = tok >= 0 ? acc[0] : -INFINITY;
+            }
+          } else if (key < p.Lk) {
+            const float ks = (C::ELEM == 1) ? __ldg(p.k_scale + static_cast<long long>(b) * p.Lk + key) : 1.f;
+#pragma unroll
+            for (int ql = 0; ql < QH; ++ql) {
+              const int t = tg * C::QPT + q0 + ql;
+              if (t < p.T && static_cast<long long>(key) * p.pstride <= p.q_offset + t)
+                p.out[(rbase + ql) * p.ldo + key] = ks * acc[ql];
+            }
+          }
+        }
+      }
+      if (C::ROUTER && s.last) {
+        // End of a query group: each set writes its partial sums (possibly 0).
+        const int t = tg * C::QPT + row / C::H;
+        if (t < p.T) {
+          const long long ix = (static_cast<long long>(b) * p.T + t) * C::H + (row % C::H);
+          p.out[static_cast<long long>(set) * p.batch * p.T * C::H + ix] = racc;
+        }
+        racc = 0.f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace dsa

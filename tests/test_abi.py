@@ -1,0 +1,96 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function
+include/dsa_indexer.h declares, and its host-side validation rejects bad
+arguments before any CUDA call (so these run on CPU)."""
+import ctypes
+
+import pytest
+
+from sparse_attention_token_score_b200 import binding as B
+from sparse_attention_token_score_b200 import build as build_mod
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = B.header_symbols()
+    assert len(names) == 11
+    assert set(names) == set(B._SIGS)
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def test_status_strings(lib):
+    assert lib.dsa_status_string(0) == b"ok"
+    assert lib.dsa_status_string(-3) == b"workspace too small"
+    assert lib.dsa_status_string(-5) == b"device wait timed out"
+
+
+def _args(**kw):
+    a = B.IndexerArgs(batch=1, T=4, L=256, H=64, d=128, q_offset=252, qk_dtype=B.DSA_BF16)
+    a.q, a.k, a.w = 0x10000, 0x20000, 0x30000  # never dereferenced: validation fails first
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_workspace_sizes(lib):
+    a = _args()
+    assert lib.indexer_workspace_size(ctypes.byref(a), 16) == 256 + 4 * 256 * 4
+    assert lib.indexer_workspace_size(None, 16) == 0
+    m = lib.misa_workspace_size(ctypes.byref(a), 64, 8, 16, 0)
+    m2 = lib.misa_workspace_size(ctypes.byref(a), 64, 8, 16, 128)
+    assert m2 == m + 2 * 256 * 4 * 2  # candidates + their scores, [T, kprime] each
+    assert lib.hisa_workspace_size(ctypes.byref(a), 128, 2, 16) > 256
+
+
+@pytest.mark.parametrize("bad", [
+    dict(batch=0), dict(T=0), dict(L=0), dict(q_offset=-1), dict(q=None), dict(w=None),
+    dict(q=0x10008),  # q not 16-byte aligned
+    dict(qk_dtype=7),
+    dict(qk_dtype=B.DSA_FP8_E4M3),  # FP8 without scales
+])
+def test_invalid_arguments_rejected(lib, bad):
+    a = _args(**bad)
+    st = lib.indexer_score_topk(ctypes.byref(a), 16, ctypes.c_void_p(0x40000), None,
+                                ctypes.c_void_p(0x50000), 1 << 30, None)
+    assert st == -1
+
+
+@pytest.mark.parametrize("shape", [dict(H=48), dict(d=96), dict(H=128)])
+def test_unsupported_shapes(lib, shape):
+    a = _args(**shape)
+    st = lib.indexer_score_topk(ctypes.byref(a), 16, ctypes.c_void_p(0x40000), None,
+                                ctypes.c_void_p(0x50000), 1 << 30, None)
+    assert st == -2
+
+
+def test_workspace_checks(lib):
+    a = _args()
+    out = ctypes.c_void_p(0x40000)
+    assert lib.indexer_score_topk(ctypes.byref(a), 16, out, None, None, 1 << 30, None) == -3
+    assert lib.indexer_score_topk(ctypes.byref(a), 16, out, None, ctypes.c_void_p(0x50000), 100, None) == -3
+    assert lib.indexer_score_topk(ctypes.byref(a), 16, out, None, ctypes.c_void_p(0x50010), 1 << 30, None) == -1
+    assert lib.indexer_score_topk(ctypes.byref(a), 0, out, None, ctypes.c_void_p(0x50000), 1 << 30, None) == -1
+
+
+def test_variant_argument_checks(lib):
+    a = _args()
+    out = ctypes.c_void_p(0x40000)
+    ws = ctypes.c_void_p(0x50000)
+    big = 1 << 40
+    # h > H, unsupported h, bad block
+    assert lib.misa_route_score_topk(ctypes.byref(a), 64, 65, 16, 0, out, None, None, None, ws, big, None) == -1
+    assert lib.misa_route_score_topk(ctypes.byref(a), 64, 12, 16, 0, out, None, None, None, ws, big, None) == -2
+    assert lib.misa_route_score_topk(ctypes.byref(a), 0, 8, 16, 0, out, None, None, None, ws, big, None) == -1
+    # MISA is bf16 only
+    f = _args(qk_dtype=B.DSA_FP8_E4M3, q_scale=0x60000, k_scale=0x70000)
+    assert lib.misa_route_score_topk(ctypes.byref(f), 64, 8, 16, 0, out, None, None, None, ws, big, None) == -2
+    assert lib.hisa_block_filter_topk(ctypes.byref(a), 128, 0, 16, out, None, None, ws, big, None) == -1
+    h8 = _args(H=8)
+    assert lib.hisa_block_filter_topk(ctypes.byref(h8), 128, 2, 16, out, None, None, ws, big, None) == -2
+    assert lib.indexer_topk_rows(None, 4, 256, 4, 0, 1, 256, 16, None, 0, 1, out, None, ws, big, None) == -1
+    assert lib.dsa_meanpool_keys(None, 1, 256, 128, 64, ws, None) == -1

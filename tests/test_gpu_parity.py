@@ -1,0 +1,307 @@
+"""CUDA path (through the C-ABI) against the fp64 oracle, on the same seeded
+inputs: element-by-element at sizes the oracle finishes in seconds (several
+tiles plus ragged tails), and on sampled queries at the full workload sizes
+the benchmark times. Every discrete stage of MISA / HISA is compared on its
+own, and the next stage's oracle is then run on the GPU's choice."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_token_score_b200 import binding as B
+from sparse_attention_token_score_b200 import workloads as wl
+from tests.parity_util import RTOL_BF16, RTOL_FP8, check_scores, check_selection
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    B.lib()
+
+
+def _indexer(inp):
+    q, k, w, qs, ks = B.to_device(inp)
+    return B.Indexer(q, k, w, inp.q_offset, qs, ks)
+
+
+def _dense_check(inp, topk, queries=None, batches=None, rtol=RTOL_BF16, what=""):
+    ix = _indexer(inp)
+    idx, sc = ix.dense(topk, with_score=True)
+    assert ix.device_status() == 0
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    ties = 0
+    for b in (range(inp.batch) if batches is None else batches):
+        qs = range(inp.T) if queries is None else queries
+        res = oracle.dense_topk(inp, topk, queries=qs, b=b)
+        for i, t in enumerate(res["queries"]):
+            s, c = res["scores"][i], res["cond"][i]
+            cand = np.arange(s.size)
+            ties += check_selection(idx[b, t], cand, s, c, topk, what=f"{what} b={b} t={t}")
+            n = min(topk, s.size)
+            sel = idx[b, t, :n]
+            check_scores(sc[b, t, :n], s[sel], c[sel], rtol, what=f"{what} scores b={b} t={t}")
+            assert np.all(np.isneginf(sc[b, t, n:]))
+    return ties
+
+
+# ------------------------------------------------------------------ dense scores
+SHAPES = [  # batch, T, L, H, d, q_offset
+    (2, 37, 300, 64, 128, 263),
+    (1, 70, 515, 8, 64, 445),
+    (1, 33, 200, 16, 128, 0),
+    (1, 20, 700, 32, 64, 680),
+    (3, 9, 129, 64, 64, 500),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_dense_scores_elementwise(shape):
+    b, T, L, H, d, off = shape
+    inp = wl.prefill_inputs(T, L, H, d, q_offset=off, seed=11, batch=b)
+    ix = _indexer(inp)
+    out = torch.full((b, T, L), float("nan"), device="cuda")
+    ws = B.alloc_workspace(256)
+    B.indexer_scores(ix.args, out, L, ws)
+    assert B.dsa_device_status(ws) == 0
+    out = out.cpu().numpy()
+    for bb in range(b):
+        res = oracle.dense_topk(inp, 1, b=bb)
+        for t in range(T):
+            V = min(off + t + 1, L)
+            check_scores(out[bb, t, :V], res["scores"][t], res["cond"][t], RTOL_BF16,
+                         what=f"b={bb} t={t}")
+            assert np.all(np.isnan(out[bb, t, V:])), "invisible entries must be left untouched"
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("topk", [1, 7, 130, 1000])
+def test_dense_topk_ragged(shape, topk):
+    b, T, L, H, d, off = shape
+    inp = wl.prefill_inputs(T, L, H, d, q_offset=off, seed=12, batch=b)
+    _dense_check(inp, topk, what=str(shape))
+
+
+def test_dense_tiny_config_full():
+    c = wl.CONFIGS["tiny"]
+    inp = wl.make_inputs("tiny", seed=0)
+    _dense_check(inp, c["topk"], what="tiny")
+
+
+def test_dense_all_negative_weights_ties_to_lowest():
+    inp = wl.prefill_inputs(6, 600, 8, 64, q_offset=590, seed=5)
+    inp.w[:] = -np.abs(inp.w)
+    inp.k[0, ::3] = 0  # zero keys score exactly 0 (the maximum) on every head
+    ix = _indexer(inp)
+    idx, sc = ix.dense(40, with_score=True)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    res = oracle.dense_topk(inp, 40)
+    for t in range(6):
+        s = res["scores"][t]
+        zeros = np.flatnonzero(s == 0.0)
+        assert zeros.size >= 40
+        assert idx[0, t].tolist() == zeros[:40].tolist()
+        assert np.all(sc[0, t] == 0.0)
+
+
+def test_dense_duplicate_keys_exact_ties():
+    inp = wl.prefill_inputs(5, 400, 16, 128, q_offset=395, seed=6)
+    inp.k[0, 200:400] = inp.k[0, 0:200]  # every key appears twice
+    assert _dense_check(inp, 33, what="dup") == 0
+
+
+def test_dense_single_key_and_query():
+    inp = wl.prefill_inputs(1, 1, 64, 128, q_offset=0, seed=7)
+    _dense_check(inp, 4, what="1x1")
+
+
+def test_dsa_config_sampled():
+    c = wl.CONFIGS["dsa"]
+    inp = wl.make_inputs("dsa", seed=0)
+    qs = [0, 1, 2, 3, 4, 1023, 2047, 2048, 3071, 4094, 4095] + list(
+        np.random.default_rng(0).choice(c["T"], 5, replace=False))
+    _dense_check(inp, c["topk"], queries=qs, what="dsa")
+
+
+# ------------------------------------------------------------------ FP8 decode
+@pytest.mark.parametrize("H", [32, 64])
+def test_fp8_decode_small(H):
+    inp = wl.decode_inputs(batch=3, L=1000, H=H, d=128, seed=8, cluster_frac=0.05)
+    _dense_check(inp, 77, rtol=RTOL_FP8, what=f"fp8 H={H}")
+
+
+def test_fp8_scores_elementwise():
+    inp = wl.decode_inputs(batch=2, L=777, H=64, d=128, seed=9, cluster_frac=0.05)
+    ix = _indexer(inp)
+    out = torch.full((2, 1, 777), float("nan"), device="cuda")
+    ws = B.alloc_workspace(256)
+    B.indexer_scores(ix.args, out, 777, ws)
+    out = out.cpu().numpy()
+    for b in range(2):
+        res = oracle.dense_topk(inp, 1, b=b)
+        check_scores(out[b, 0], res["scores"][0], res["cond"][0], RTOL_FP8, what=f"fp8 b={b}")
+
+
+def test_decode_config_sampled():
+    c = wl.CONFIGS["decode"]
+    inp = wl.make_inputs("decode", seed=0)
+    _dense_check(inp, c["topk"], batches=[0, 17, 63], rtol=RTOL_FP8, what="decode")
+
+
+# ------------------------------------------------------------------ meanpool
+@pytest.mark.parametrize("L,B_", [(1000, 64), (777, 128), (64, 64), (130, 1)])
+def test_meanpool_bit_exact(L, B_):
+    inp = wl.prefill_inputs(1, L, 8, 128, seed=10, batch=2)
+    _, k, _, _, _ = B.to_device(inp)
+    M = -(-L // B_)
+    kbar = torch.empty((2, M, 128), dtype=torch.bfloat16, device="cuda")
+    B.dsa_meanpool_keys(k, B_, kbar)
+    got = kbar.view(torch.int16).cpu().numpy().view(np.uint16)
+    for b in range(2):
+        assert np.array_equal(got[b], oracle.meanpool_bf16(inp.k[b], B_))
+
+
+# ------------------------------------------------------------------ MISA
+def _heads_check(gpu_heads, aff, h, what):
+    for i in range(aff.shape[0]):
+        check_selection(gpu_heads[i], np.arange(aff.shape[1]), aff[i], aff[i], h, what=f"{what} heads {i}")
+
+
+def _misa_check(inp, block, h, topk, kprime, queries, what):
+    ix = _indexer(inp)
+    idx, sc, heads, cand = ix.misa(block, h, topk, kprime, with_score=True, with_heads=True,
+                                   with_cand=True)
+    assert ix.device_status() == 0
+    idx, sc, heads = idx.cpu().numpy()[0], sc.cpu().numpy()[0], heads.cpu().numpy()[0]
+    cand = cand.cpu().numpy()[0] if cand is not None else None
+    qs = np.asarray(queries)
+    free = oracle.misa(inp, block, h, topk, kprime=0, queries=qs)
+    _heads_check(heads[qs], free["affinity"], h, what)
+    # conditioned on the GPU's heads (and candidates)
+    cond = oracle.misa(inp, block, h, topk, kprime=kprime, queries=qs, heads_given=heads[qs],
+                       cand_given=None if cand is None else cand[qs])
+    for i, t in enumerate(qs):
+        V = min(inp.q_offset + t + 1, inp.L)
+        if kprime == 0:
+            s, c = cond["routed_scores"][i], cond["routed_cond"][i]
+            check_selection(idx[t], np.arange(V), s, c, topk, what=f"{what} t={t}")
+            n = min(topk, V)
+            check_scores(sc[t, :n], s[idx[t, :n]], c[idx[t, :n]], RTOL_BF16, what=f"{what} t={t}")
+        else:
+            check_selection(cand[t], np.arange(V), cond["routed_scores"][i], cond["routed_cond"][i],
+                            kprime, what=f"{what} cand t={t}")
+            cv = cand[t][cand[t] >= 0]
+            s, c = cond["scores"][i], cond["cond"][i]
+            check_selection(idx[t], cv, s, c, topk, what=f"{what} t={t}")
+            n = min(topk, cv.size)
+            where = np.searchsorted(cv, idx[t, :n])
+            check_scores(sc[t, :n], s[where], c[where], RTOL_BF16, what=f"{what} scores t={t}")
+
+
+@pytest.mark.parametrize("kprime", [0, 400])
+def test_misa_small(kprime):
+    inp = wl.prefill_inputs(40, 3000, 64, 128, q_offset=2960, seed=13, w_std=0.125)
+    _misa_check(inp, block=64, h=8, topk=100, kprime=kprime, queries=range(40), what=f"misa k'={kprime}")
+
+
+def test_misa_ragged_blocks():
+    # L not a multiple of the block, queries near the start (few visible blocks)
+    inp = wl.prefill_inputs(50, 1000, 32, 128, q_offset=30, seed=14)
+    _misa_check(inp, block=48, h=16, topk=64, kprime=200, queries=range(50), what="misa ragged")
+
+
+def test_misa_all_heads_equals_dense_gpu():
+    inp = wl.prefill_inputs(24, 2000, 64, 128, q_offset=1976, seed=15)
+    ix = _indexer(inp)
+    d_idx, d_sc = ix.dense(64, with_score=True)
+    m_idx, m_sc, heads, _ = ix.misa(64, 64, 64, 0, with_score=True, with_heads=True)
+    assert torch.equal(heads[0], torch.arange(64, dtype=torch.int32, device="cuda").expand(24, 64))
+    assert torch.equal(d_idx, m_idx)
+    assert torch.equal(d_sc, m_sc)
+
+
+def test_misa_dagger_all_candidates_equals_dense():
+    inp = wl.prefill_inputs(16, 900, 64, 128, q_offset=880, seed=16)
+    ix = _indexer(inp)
+    d_idx, d_sc = ix.dense(50, with_score=True)
+    m_idx, m_sc, _, _ = ix.misa(64, 8, 50, kprime=900, with_score=True)
+    res = oracle.dense_topk(inp, 50)
+    m_idx, m_sc = m_idx.cpu().numpy()[0], m_sc.cpu().numpy()[0]
+    for t in range(16):
+        check_selection(m_idx[t], np.arange(res["scores"][t].size), res["scores"][t], res["cond"][t], 50)
+
+
+def test_misa_config_sampled():
+    c = wl.CONFIGS["misa"]
+    inp = wl.make_inputs("misa", seed=0)
+    qs = [0, 1, 1000, 2046, 2047]
+    _misa_check(inp, c["block"], c["h"], c["topk"], c["kprime"], qs, what="misa cfg")
+
+
+def test_misa_plain_config_sampled():
+    c = wl.CONFIGS["misa"]
+    inp = wl.make_inputs("misa", seed=0)
+    _misa_check(inp, c["block"], c["h"], c["topk"], 0, [3, 777, 2047], what="misa plain cfg")
+
+
+# ------------------------------------------------------------------ HISA
+def _hisa_check(inp, block, m, topk, queries, what):
+    ix = _indexer(inp)
+    idx, sc, blocks = ix.hisa(block, m, topk, with_score=True, with_blocks=True)
+    assert ix.device_status() == 0
+    idx, sc, blocks = idx.cpu().numpy()[0], sc.cpu().numpy()[0], blocks.cpu().numpy()[0]
+    qs = np.asarray(queries)
+    free = oracle.hisa(inp, block, m, topk, queries=qs)
+    for i, t in enumerate(qs):
+        s, c = free["block_scores"][i], free["block_cond"][i]
+        check_selection(blocks[t], np.arange(s.size), s, c, m, what=f"{what} blocks t={t}")
+    cond = oracle.hisa(inp, block, m, topk, queries=qs, blocks_given=blocks[qs])
+    for i, t in enumerate(qs):
+        toks, s, c = cond["tokens"][i], cond["scores"][i], cond["cond"][i]
+        check_selection(idx[t], toks, s, c, topk, what=f"{what} t={t}")
+        n = min(topk, toks.size)
+        where = np.searchsorted(toks, idx[t, :n])
+        check_scores(sc[t, :n], s[where], c[where], RTOL_BF16, what=f"{what} scores t={t}")
+
+
+def test_hisa_small():
+    inp = wl.prefill_inputs(30, 5000, 32, 128, q_offset=4970, seed=17, recency=0.1)
+    _hisa_check(inp, block=128, m=8, topk=300, queries=range(30), what="hisa")
+
+
+def test_hisa_ragged():
+    inp = wl.prefill_inputs(40, 1100, 64, 128, q_offset=100, seed=18)
+    _hisa_check(inp, block=96, m=5, topk=200, queries=range(40), what="hisa ragged")
+
+
+def test_hisa_all_blocks_equals_dense():
+    inp = wl.prefill_inputs(12, 1500, 32, 128, q_offset=1488, seed=19)
+    ix = _indexer(inp)
+    h_idx, _, _ = ix.hisa(128, 12, 80)
+    res = oracle.dense_topk(inp, 80)
+    h_idx = h_idx.cpu().numpy()[0]
+    for t in range(12):
+        check_selection(h_idx[t], np.arange(res["scores"][t].size), res["scores"][t], res["cond"][t], 80)
+
+
+def test_hisa_config_sampled():
+    c = wl.CONFIGS["hisa"]
+    inp = wl.make_inputs("hisa", seed=0)
+    _hisa_check(inp, c["block"], c["m"], c["topk"], [0, 511, 1023], what="hisa cfg")
+
+
+# ------------------------------------------------------------------ boundary on the GPU
+def test_errors_are_reported_not_launched():
+    inp = wl.prefill_inputs(4, 256, 64, 128, seed=20)
+    ix = _indexer(inp)
+    idx = torch.empty((1, 4, 8), dtype=torch.int32, device="cuda")
+    small = B.alloc_workspace(256)
+    with pytest.raises(B.DsaError) as e:
+        B.indexer_score_topk(ix.args, 8, idx, None, small)
+    assert e.value.status == -3
+    with pytest.raises(B.DsaError) as e:
+        ix.misa(64, 12, 8)
+    assert e.value.status == -2
+    assert B.dsa_device_status(small) == 0
