@@ -55,9 +55,13 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ workloads
-def workload_desc(name):
+def workload_desc(name, queries=None):
     from sparse_attention_token_score_b200 import workloads as wl
     c = dict(wl.CONFIGS[name])
+    if queries:  # a smaller chunk at the end of the same prefix (profiling cases)
+        c["T"] = int(queries)
+        if "q_offset" in c:
+            c["q_offset"] = c["L"] - c["T"]
     batch = c.get("batch", 1)
     off = c.get("q_offset", c["L"] - 1)
     pairs = wl.visible_pairs(c["T"], c["L"], off, batch)
@@ -74,10 +78,10 @@ def workload_desc(name):
 class Runner:
     """Device-resident inputs + the C-ABI call of one workload."""
 
-    def __init__(self, name, inp, torch):
+    def __init__(self, name, inp, torch, queries=None):
         from sparse_attention_token_score_b200 import binding as B
         self.B, self.torch, self.name = B, torch, name
-        self.c, self.batch, self.off, self.pairs, self.label = workload_desc(name)
+        self.c, self.batch, self.off, self.pairs, self.label = workload_desc(name, queries)
         self.inp = inp
         q, k, w, qs, ks = B.to_device(inp)
         self.dev = (q, k, w, qs, ks)
@@ -186,7 +190,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle (CPU) timing
-def oracle_sample(name, inp, budget_s=12.0, max_q=4096):
+def oracle_sample(name, inp, budget_s=10.0, max_q=4096):
     """Time the fp64 oracle, as it stands, on a bounded sample of this workload's
     queries (the same computation as one GPU step, restricted to the sample)."""
     import oracle
@@ -210,18 +214,21 @@ def oracle_sample(name, inp, budget_s=12.0, max_q=4096):
         return int(sum(min(off + int(t) + 1, inp.L) for t in qs))
 
     if name == "decode":
-        # one unit = one sequence's query
-        t1 = run([0], b=0)
-        nb = max(1, min(inp.batch, int(budget_s / max(t1, 1e-3))))
-        t = 0.0
-        for b in range(1, nb + 1):
-            t += run([0], b=b % inp.batch)
+        # one unit = one sequence's query; add sequences until budget_s is spent
+        t, nb = 0.0, 0
+        while t < budget_s and nb < inp.batch:
+            t += run([0], b=nb)
+            nb += 1
         return nb * inp.L / t / 1e9, f"{nb} of {inp.batch} sequences (all {inp.L} keys each)", nb, t
-    q1 = rng.choice(T, 2, replace=False)
-    t1 = run(q1) / 2
-    n = int(max(2, min(max_q, budget_s / max(t1, 1e-4))))
-    qs = np.sort(rng.choice(T, n, replace=False)) if n < T else np.arange(T)
-    t = run(qs)
+    # grow the sample until one run takes at least budget_s (or covers every query)
+    n = 8
+    while True:
+        n = min(n, T, max_q)
+        qs = np.sort(rng.choice(T, n, replace=False)) if n < T else np.arange(T)
+        t = run(qs)
+        if t >= budget_s or n >= min(T, max_q):
+            break
+        n = int(n * min(8.0, max(2.0, 1.2 * budget_s / max(t, 1e-3))))
     return pairs(qs) / t / 1e9, f"{len(qs)} of {T} queries (uniform sample)", len(qs), t
 
 
@@ -254,6 +261,21 @@ def run_reference(args):
     return 0
 
 
+def make_inputs(name, seed, queries=0):
+    """The workload's inputs; with `queries`, only the last `queries` queries
+    of the chunk (same prefix, same distributions)."""
+    from sparse_attention_token_score_b200 import workloads as wl
+    inp = wl.make_inputs(name, seed=seed)
+    if queries and queries < inp.T:
+        T0 = inp.T - queries
+        inp.q = inp.q[:, T0:].copy()
+        inp.w = inp.w[:, T0:].copy()
+        if inp.q_scale is not None:
+            inp.q_scale = inp.q_scale[:, T0:].copy()
+        inp.q_offset += T0
+    return inp
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -263,6 +285,10 @@ def main():
     ap.add_argument("--workload", default="dsa", choices=["tiny", "dsa", "decode", "misa", "hisa"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--queries", type=int, default=0,
+                    help="profiling: use only the last N queries of the chunk")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="profiling: launch only the dominant kernel (W + K times)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -288,9 +314,14 @@ def main():
         if world > 1:
             dist.barrier()
 
-    inp = wl.make_inputs(args.workload, seed=rank)
-    r = Runner(args.workload, inp, torch)
+    inp = make_inputs(args.workload, rank, args.queries)
+    r = Runner(args.workload, inp, torch, args.queries)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    if args.kernel_only:
+        fn, _, _, kname = r.dominant()
+        kt = time_steps(fn, args.warmup + args.steps, torch, flush)[args.warmup:]
+        print(json.dumps({"kernel": kname, "workload": r.label, "kernel_ms": kt}), flush=True)
+        return 0
     for _ in range(args.warmup):
         r.step()
     torch.cuda.synchronize()

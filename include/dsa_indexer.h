@@ -25,10 +25,11 @@
  *     fewer candidates than k -> all of them. Each output row lists the chosen
  *     indices in ascending order, padded with -1 (and score -inf).
  *   - The first 256 bytes of every workspace hold a device status word. Each
- *     call clears it; kernels set it if a bounded wait gave up.
- *     dsa_device_status() synchronises the stream and reports it.
- *   - The workspace must be 256-byte aligned; q and k 16-byte aligned; w and
- *     scales 4-byte aligned.
+ *     call that passes validation clears it (stream-ordered); kernels set it
+ *     if a bounded wait gave up. dsa_device_status() synchronises the stream
+ *     and reports it. Zero a new workspace once before its first status read.
+ *   - The workspace must be 256-byte aligned; q, k, w and q_scale 16-byte
+ *     aligned; k_scale 4-byte aligned.
  *   - Calls that share a workspace must not overlap in time (use one stream).
  *
  * Supported shapes: d in {64, 128}; bf16 H in {8, 16, 32, 64};

@@ -125,8 +125,10 @@ def make_args(q: torch.Tensor, k: torch.Tensor, w: torch.Tensor, q_offset: int,
 
 
 def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
-    """A 256-byte aligned device buffer of at least nbytes (torch's allocator aligns to 512)."""
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8,
+    """A zeroed, 256-byte aligned device buffer of at least nbytes (torch's
+    allocator aligns to 512). Zeroing makes the status word of a workspace that
+    no call has used yet read as "ok"."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8,
                        device=device if device is not None else "cuda")
 
 

@@ -109,9 +109,13 @@ dsa_status launch_score(const ScoreParams& p, const void* q, long long q_rows, c
 // Dense / routed / block scoring, bf16: N = 256 columns = (256 / H) queries x H heads.
 dsa_status run_scores_bf16(int D, int H, const ScoreParams& p, const void* q, long long q_rows,
                            const void* k, long long k_rows, cudaStream_t st) {
+#ifndef DSA_EPIW
+#define DSA_EPIW 8
+#endif
 #define DSA_CASE(DD, HH)                                                                          \
   if (D == DD && H == HH)                                                                         \
-    return launch_score<ScoreCfg<2, DD, HH, 256 / HH, ScoreMode::kTma, (DD == 128 ? 4 : 8)>>(    \
+    return launch_score<                                                                          \
+        ScoreCfg<2, DD, HH, 256 / HH, ScoreMode::kTma, (DD == 128 ? 4 : 8), DSA_EPIW>>(          \
         p, q, q_rows, k, k_rows, st);
   DSA_CASE(64, 8) DSA_CASE(64, 16) DSA_CASE(64, 32) DSA_CASE(64, 64)
   DSA_CASE(128, 8) DSA_CASE(128, 16) DSA_CASE(128, 32) DSA_CASE(128, 64)
@@ -174,11 +178,11 @@ dsa_status validate(const dsa_indexer_args* a, bool bf16_only) {
   if (a->batch < 1 || a->T < 1 || a->L < 1 || a->H < 1 || a->d < 1 || a->q_offset < 0)
     return DSA_ERR_ARG;
   if (a->qk_dtype != DSA_BF16 && a->qk_dtype != DSA_FP8_E4M3) return DSA_ERR_ARG;
-  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->w, 4)) return DSA_ERR_ARG;
+  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->w, 16)) return DSA_ERR_ARG;
   const bool fp8 = a->qk_dtype == DSA_FP8_E4M3;
   if (fp8) {
     if (!a->q_scale || !a->k_scale) return DSA_ERR_ARG;
-    if (!aligned(a->q_scale, 4) || !aligned(a->k_scale, 4)) return DSA_ERR_ARG;
+    if (!aligned(a->q_scale, 16) || !aligned(a->k_scale, 4)) return DSA_ERR_ARG;
   }
   if (a->q_offset > (1LL << 40)) return DSA_ERR_ARG;
   if (static_cast<long long>(a->batch) * a->T * a->H > INT_MAX ||

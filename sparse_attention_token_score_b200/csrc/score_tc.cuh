@@ -31,6 +31,7 @@
 #pragma once
 #include "common.cuh"
 
+
 namespace dsa {
 
 enum class ScoreMode : int { kTma = 0, kGather = 1, kRouter = 2 };
@@ -53,7 +54,7 @@ struct ScoreParams {
   unsigned* err;            // device error word
 };
 
-template <int ELEM_, int D_, int H_, int QPT_, ScoreMode MODE_, int NSTAGE_>
+template <int ELEM_, int D_, int H_, int QPT_, ScoreMode MODE_, int NSTAGE_, int EPIW_ = 8>
 struct ScoreCfg {
   static constexpr int ELEM = ELEM_;  // bytes per element: 2 = bf16, 1 = e4m3
   static constexpr int D = D_, H = H_, QPT = QPT_, NSTAGE = NSTAGE_;
@@ -82,11 +83,15 @@ struct ScoreCfg {
   static constexpr int NPROD = GATHER ? 4 : 1;          // producer warps
   static constexpr int MMA_WARP = NPROD;
   static constexpr int EPI_WARP0 = NPROD + 1;
-  static constexpr int NTHREADS = (EPI_WARP0 + 8) * 32;
-  // Tile split between the two epilogue warp sets: alternate tiles (router,
-  // and one-query groups) or the two halves of the queries of every tile.
+  // Epilogue warps: EPIW = 4 * NSETS; each set of 4 warps covers the 128
+  // TMEM lanes. Sets take alternate tiles (router and one-query groups, 2
+  // sets), or split the queries of every tile between them.
+  static constexpr int EPIW = EPIW_;
+  static constexpr int NSETS = EPIW / 4;
   static constexpr bool SPLIT_TILES = ROUTER || QPT == 1;
-  static constexpr int TEMPTY_ARRIVALS = SPLIT_TILES ? 4 : 8;
+  static_assert(EPIW == 8 || (EPIW == 16 && !SPLIT_TILES && QPT % 4 == 0), "epilogue warps");
+  static constexpr int NTHREADS = (EPI_WARP0 + EPIW) * 32;
+  static constexpr int TEMPTY_ARRIVALS = SPLIT_TILES ? 4 : EPIW;
   static constexpr uint32_t IDESC = umma_idesc(ELEM == 2 ? 1u : 0u, 128, MMA_N);
   // shared memory layout (offsets from a 1024-aligned base)
   static constexpr int SMEM_Q = 0;
@@ -361,9 +366,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - C::EPI_WARP0;        // 0..7
+    const int e = warp - C::EPI_WARP0;        // 0 .. EPIW-1
     const int quarter = warp & 3;              // TMEM lanes this warp may read
-    const int set = e >> 2;                    // 0 or 1
+    const int set = e >> 2;                    // 0 .. NSETS-1
     const int row = quarter * 32 + lane;       // accumulator row = TMEM lane
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     float racc = 0.f;                          // router partial sum
@@ -377,7 +382,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!mbar_wait(tfull(buf), (it >> 1) & 1u, p.err)) break;
         tc_fence_after();
         const uint32_t taddr = lane_addr + static_cast<uint32_t>(buf * C::MMA_N);
-        if (C::ROUTER) {
+        if constexpr (C::ROUTER) {
           // rows: (query, head) pairs; columns: pooled keys j*256 + c
           const int t = tg * C::QPT + row / C::H;
           const long long pos = p.q_offset + (t < p.T ? t : p.T - 1);
@@ -402,43 +407,130 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           __syncwarp();
           if (lane == 0) mbar_arrive(tempty(buf));
         } else {
-          constexpr int QH = C::SPLIT_TILES ? 1 : C::QPT / 2;   // queries per thread
+          constexpr int QH = C::SPLIT_TILES ? 1 : C::QPT / C::NSETS;   // queries per thread
           constexpr int NC = QH * C::H;                          // columns per thread
+          constexpr int NCH = NC / 32;                           // 32-column chunks
+          // independent partial sums per query (breaks the FMA dependency chain)
+#if defined(DSA_NO_FFMA2)
+          constexpr int NP = C::H >= 32 ? 4 : (C::H == 16 ? 2 : 1);
+#else
+          constexpr int NP = C::H >= 32 ? 2 : 1;   // packed pairs: 2 x 2 lanes
+#endif
           const int q0 = C::SPLIT_TILES ? 0 : set * QH;          // first query (in group)
           const int key = s.j * C::KROWS + row;                  // key row / compact position
           const long long rbase = static_cast<long long>(b) * p.T + tg * C::QPT + q0;
-          float acc[QH];
+          // head weights of this thread's columns are contiguous in w when every
+          // query of the half-group exists
+          const bool full_group = tg * C::QPT + q0 + QH <= p.T;
+          const float* wrow = p.w + rbase * C::H;
+          const float* srow = (C::ELEM == 1) ? p.q_scale + rbase * C::H : nullptr;
+          float acc[QH][NP];
 #pragma unroll
-          for (int i = 0; i < QH; ++i) acc[i] = 0.f;
+          for (int i = 0; i < QH; ++i)
 #pragma unroll
-          for (int cc = 0; cc < NC; cc += 32) {
-            float coef[32];
+            for (int j = 0; j < NP; ++j) acc[i][j] = 0.f;
+#if !defined(DSA_NO_FFMA2)
+          unsigned long long acc2[QH][NP];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int ql = (cc + i) / C::H;
-              const int h = (cc + i) % C::H;
-              const int tq = tg * C::QPT + q0 + ql;
-              const long long ci = (rbase + ql - (tq < p.T ? 0 : tq - p.T + 1)) * C::H + h;
-              float c = __ldg(p.w + ci);
-              if (C::ELEM == 1) c *= __ldg(p.q_scale + ci);
-              coef[i] = c;
+          for (int i = 0; i < QH; ++i)
+#pragma unroll
+            for (int j = 0; j < NP; ++j) acc2[i][j] = 0ull;
+#endif
+          // TMEM -> registers one 32-column chunk at a time: the next chunk's
+          // load is issued before this chunk's arithmetic, and the buffer goes
+          // back to the MMA warp as soon as the last chunk has landed, so the
+          // next tile's MMAs overlap the remaining math.
+          constexpr int PH = 1;  // chunks per phase (more would exceed the register budget)
+          constexpr int NPHASE = NCH / PH;
+          uint32_t vb[2][PH][32];
+#pragma unroll
+          for (int c = 0; c < PH; ++c) tmem_ld32_issue(taddr + q0 * C::H + c * 32, vb[0][c]);
+#pragma unroll
+          for (int c = 0; c < PH; ++c) tmem_ld_wait(vb[0][c]);
+#pragma unroll
+          for (int ph = 0; ph < NPHASE; ++ph) {
+            if (ph + 1 < NPHASE) {
+#pragma unroll
+              for (int c = 0; c < PH; ++c)
+                tmem_ld32_issue(taddr + q0 * C::H + ((ph + 1) * PH + c) * 32, vb[(ph + 1) & 1][c]);
+            } else {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(tempty(buf));
             }
-            float v[32];
-            tmem_ld32(taddr + q0 * C::H + cc, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int ql = (cc + i) / C::H;
-              acc[ql] = fmaf(coef[i], fmaxf(v[i], 0.f), acc[ql]);
+            for (int c = 0; c < PH; ++c) {
+              const int cc = (ph * PH + c) * 32;
+              const uint32_t (&v)[32] = vb[ph & 1][c];
+              float coef[32];
+              if (full_group) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                  float4 c4 = __ldg(reinterpret_cast<const float4*>(wrow + cc + i));
+                  if (C::ELEM == 1) {
+                    const float4 s4 = __ldg(reinterpret_cast<const float4*>(srow + cc + i));
+                    c4.x *= s4.x; c4.y *= s4.y; c4.z *= s4.z; c4.w *= s4.w;
+                  }
+                  coef[i] = c4.x; coef[i + 1] = c4.y; coef[i + 2] = c4.z; coef[i + 3] = c4.w;
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  const int ql = (cc + i) / C::H;
+                  const int h = (cc + i) % C::H;
+                  const int tq = tg * C::QPT + q0 + ql;
+                  const long long ci = (rbase + ql - (tq < p.T ? 0 : tq - p.T + 1)) * C::H + h;
+                  float c = __ldg(p.w + ci);
+                  if (C::ELEM == 1) c *= __ldg(p.q_scale + ci);
+                  coef[i] = c;
+                }
+              }
+#if defined(DSA_NO_FFMA2)
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int ql = (cc + i) / C::H;
+                const int pp = i % NP;
+                acc[ql][pp] = fmaf(coef[i], fmaxf(__uint_as_float(v[i]), 0.f), acc[ql][pp]);
+              }
+#else
+#pragma unroll
+              for (int i = 0; i < 32; i += 2) {
+                const int ql = (cc + i) / C::H;
+                const int pp = (i / 2) % NP;
+                acc2[ql][pp] = ffma2(pack2(coef[i], coef[i + 1]),
+                                     pack2(fmaxf(__uint_as_float(v[i]), 0.f),
+                                           fmaxf(__uint_as_float(v[i + 1]), 0.f)),
+                                     acc2[ql][pp]);
+              }
+#endif
+            }
+            if (ph + 1 < NPHASE) {
+#pragma unroll
+              for (int c = 0; c < PH; ++c) tmem_ld_wait(vb[(ph + 1) & 1][c]);
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tempty(buf));
+#if !defined(DSA_NO_FFMA2)
+#pragma unroll
+          for (int i = 0; i < QH; ++i)
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+              const float2 f = unpack2(acc2[i][j]);
+              acc[i][j] = f.x + f.y;
+            }
+#endif
+          float accq[QH];
+#pragma unroll
+          for (int i = 0; i < QH; ++i) {
+            float a = acc[i][0];
+            if (NP == 2) a = acc[i][0] + acc[i][1];
+            if (NP == 4) a = (acc[i][0] + acc[i][1]) + (acc[i][2] + acc[i][3]);
+            accq[i] = a;
+          }
           if (C::GATHER) {
             const long long r = static_cast<long long>(b) * p.T + tg;
             if (key < p.n_compact) {
               const long long tok = gathered_token(p, r, key, p.q_offset + tg);
-              p.out[r * p.ldo + key] = tok >= 0 ? acc[0] : -INFINITY;
+              p.out[r * p.ldo + key] = tok >= 0 ? accq[0] : -INFINITY;
             }
           } else if (key < p.Lk) {
             const float ks = (C::ELEM == 1) ? __ldg(p.k_scale + static_cast<long long>(b) * p.Lk + key) : 1.f;
@@ -446,7 +538,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int ql = 0; ql < QH; ++ql) {
               const int t = tg * C::QPT + q0 + ql;
               if (t < p.T && static_cast<long long>(key) * p.pstride <= p.q_offset + t)
-                p.out[(rbase + ql) * p.ldo + key] = ks * acc[ql];
+                p.out[(rbase + ql) * p.ldo + key] = ks * accq[ql];
             }
           }
         }

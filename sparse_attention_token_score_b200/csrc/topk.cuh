@@ -7,14 +7,20 @@
 // return all of them. Output: selected positions in ascending order (mapped
 // through an optional index map), padded with -1 (score -inf).
 //
-// Method: scores map to order-preserving 32-bit keys (-0 folded onto +0,
-// absent -> 0). A three-digit radix select (11 + 11 + 10 bits, shared-memory
-// histograms with warp-aggregated atomics) finds the k-th key tau and how many
-// keys equal to tau to take; a final ordered pass writes the keys above tau and
-// the first keys equal to tau, in position order, through a block-wide scan.
+// Scores map to order-preserving 32-bit keys (-0 folded onto +0, absent -> 0).
+// The k-th key tau and the number of keys equal to tau to take are found in
+// two steps:
+//   1. coarse: a 2048-bin histogram over *values* (bins evenly spaced between
+//      the row's min and max, a monotone map, so contention stays low even
+//      though the scores crowd a few exponents) locates the bin holding the
+//      k-th value; the bin's elements are compacted into a small buffer;
+//   2. exact: a three-digit radix select (11 + 11 + 10 bits) over that buffer.
+// If the bin is too large for the buffer (mass ties), the exact radix select
+// runs over the whole row instead. The write-out gives each warp a contiguous
+// segment: count, one block-wide exclusive scan of the 32 warp counts, then
+// ballot-ordered stores, so positions come out in ascending order.
 // Rows up to TK_SMEM_ROW entries are staged once in shared memory; longer rows
-// are streamed from global memory (L2) with a candidate cache for the third
-// digit.
+// are re-read from global memory (L2) on each pass.
 #pragma once
 #include "common.cuh"
 
@@ -36,10 +42,13 @@ struct TopkParams {
 };
 
 constexpr int TK_THREADS = 1024;
+constexpr int TK_WARPS = TK_THREADS / 32;
+constexpr int TK_BINS = 2048;
 constexpr int TK_SMEM_ROW = 40960;   // rows up to this length are staged in shared memory
-constexpr int TK_CAND_CAP = 20480;   // (key, position) pairs cached for long rows
-constexpr int TK_SMEM_WORDS = 2048 + 64 + 16 + (TK_SMEM_ROW > 2 * TK_CAND_CAP ? TK_SMEM_ROW : 2 * TK_CAND_CAP);
+constexpr int TK_CAND_CAP = 8192;    // keys of the threshold bin
+constexpr int TK_SMEM_WORDS = TK_BINS + 128 + TK_CAND_CAP + TK_SMEM_ROW;
 constexpr int TK_SMEM_BYTES = TK_SMEM_WORDS * 4;
+constexpr int TK_UNROLL = 8;        // float4 loads in flight per thread in the row load
 
 __device__ __forceinline__ uint32_t score_key(float x) {
   if (!(x > -INFINITY)) return 0u;  // -inf (absent) and NaN
@@ -80,16 +89,8 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* ws, ui
   return r;
 }
 
-// Add one to hist[digit] for every lane with `has`, one atomic per distinct digit.
-__device__ __forceinline__ void hist_add(uint32_t* hist, bool has, uint32_t digit) {
-  const uint32_t m = __match_any_sync(0xffffffffu, has ? digit : 0xFFFFFFFFu);
-  if (has && (threadIdx.x & 31) == static_cast<unsigned>(__ffs(m) - 1))
-    atomicAdd(&hist[digit], static_cast<uint32_t>(__popc(m)));
-}
-
-// Given a histogram of NB bins (NB = 1024 * BPT) and a 1-based rank `need`
-// counted from the largest digit, find the digit holding that rank and the
-// rank inside it. Writes vars[0] = digit, vars[1] = new need.
+// Histogram of NB = 1024 * BPT bins, 1-based rank `need` counted from the top:
+// find the bin holding that rank and the rank inside it -> vars[0], vars[1].
 template <int BPT>
 __device__ __forceinline__ void radix_pick(const uint32_t* hist, uint32_t need, uint32_t* ws,
                                            uint32_t* vars) {
@@ -111,13 +112,67 @@ __device__ __forceinline__ void radix_pick(const uint32_t* hist, uint32_t need, 
   __syncthreads();
 }
 
+// Source of the keys of one row: shared-memory stage, candidate buffer, or global.
+struct RowSrc {
+  const uint32_t* smem;  // staged keys (or nullptr)
+  const float* g;        // global row
+  __device__ __forceinline__ uint32_t get(int i) const {
+    return smem ? smem[i] : score_key(__ldcg(g + i));
+  }
+};
+
+// Exact radix select over the keys of positions [0, n) (shared-memory keys, or
+// the global row when keys == nullptr); keys equal to 0 (absent) are ignored.
+// Leaves vars[0] = tau, the need-th largest key, and vars[1] = how many keys
+// equal to tau rank within the top `need`.
+__device__ void exact_select(const uint32_t* keys, const float* g, int n, uint32_t need,
+                             uint32_t* hist, uint32_t* ws, uint32_t* vars) {
+  const RowSrc src{keys, g};
+  uint32_t prefix = 0;
+  const int shifts[3] = {21, 10, 0};
+  const uint32_t widths[3] = {11, 11, 10};
+#pragma unroll 1
+  for (int d = 0; d < 3; ++d) {
+    for (int i = threadIdx.x; i < TK_BINS; i += TK_THREADS) hist[i] = 0;
+    __syncthreads();
+    const int sh = shifts[d];
+    const uint32_t hi_sh = sh + widths[d];
+    #pragma unroll 4
+    for (int i = threadIdx.x; i < n; i += TK_THREADS) {
+      const uint32_t key = src.get(i);
+      if (key != 0u && (hi_sh >= 32 || (key >> hi_sh) == prefix))
+        atomicAdd(&hist[(key >> sh) & ((1u << widths[d]) - 1u)], 1u);
+    }
+    __syncthreads();
+    if (d < 2) radix_pick<2>(hist, need, ws, vars);
+    else radix_pick<1>(hist, need, ws, vars);
+    prefix = (prefix << widths[d]) | vars[0];
+    need = vars[1];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    vars[0] = prefix;
+    vars[1] = need;
+  }
+  __syncthreads();
+}
+
+// Value bin of a present key: 2048 evenly spaced bins over [lo, lo + 2048/scale].
+__device__ __forceinline__ int value_bin(uint32_t key, float lo, float scale) {
+  const float v = (key_score(key) - lo) * scale;
+  int b = static_cast<int>(v);
+  return b < 0 ? 0 : (b > TK_BINS - 1 ? TK_BINS - 1 : b);
+}
+
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkParams p) {
   extern __shared__ uint32_t tk_smem[];
-  uint32_t* hist = tk_smem;          // 2048
-  uint32_t* ws = hist + 2048;        // 64
-  uint32_t* vars = ws + 64;          // 16
-  uint32_t* cache = vars + 16;       // row keys, or (key, position) pairs
-  const int tid = threadIdx.x;
+  uint32_t* hist = tk_smem;                  // TK_BINS
+  uint32_t* ws = hist + TK_BINS;             // 64
+  uint32_t* vars = ws + 64;                  // 64
+  uint32_t* cbuf = vars + 64;                // TK_CAND_CAP keys of the threshold bin
+  uint32_t* stage = cbuf + TK_CAND_CAP;      // TK_SMEM_ROW
+  float* fvars = reinterpret_cast<float*>(vars + 32);
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
   for (long long r = blockIdx.x; r < p.rows; r += gridDim.x) {
     const int t = static_cast<int>(r % p.T);
@@ -130,90 +185,165 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
     const int n = static_cast<int>(nl);
     const float* row = p.scores + r * p.ld;
     const bool staged = n <= TK_SMEM_ROW;
+    const uint32_t* skeys = staged ? stage : nullptr;
+    const RowSrc src{skeys, row};
     const int k = p.k;
 
-    // ---- digit 1 (bits 31..21) + count of present candidates
-    for (int i = tid; i < 2048; i += TK_THREADS) hist[i] = 0;
-    __syncthreads();
+    // ---- pass 1: stage keys; count present; min / max of present values
     uint32_t nv = 0;
-    for (int base = 0; base < n; base += TK_THREADS) {
-      const int i = base + tid;
-      const uint32_t key = i < n ? score_key(__ldcg(row + i)) : 0u;
-      if (staged && i < n) cache[i] = key;
-      nv += key != 0u;
-      hist_add(hist, key != 0u, key >> 21);
+    float vmin = INFINITY, vmax = -INFINITY;
+    const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15u) == 0);
+    if (vec) {
+      // TK_UNROLL float4 loads per thread are in flight before any is used
+      // (128 KB per SM for a 32K-entry row), so the row streams at HBM rate.
+      const int n4 = n >> 2;
+      for (int base = 0; base < n4; base += TK_THREADS * TK_UNROLL) {
+        float4 x[TK_UNROLL];
+#pragma unroll
+        for (int u = 0; u < TK_UNROLL; ++u) {
+          const int i = base + u * TK_THREADS + tid;
+          x[u] = i < n4 ? __ldcg(reinterpret_cast<const float4*>(row) + i)
+                        : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        }
+#pragma unroll
+        for (int u = 0; u < TK_UNROLL; ++u) {
+          const int i = base + u * TK_THREADS + tid;
+          if (i >= n4) continue;
+          const float xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t key = score_key(xs[j]);
+            if (staged) stage[4 * i + j] = key;
+            if (key) { ++nv; const float v = key_score(key); vmin = fminf(vmin, v); vmax = fmaxf(vmax, v); }
+          }
+        }
+      }
+      for (int i = 4 * n4 + tid; i < n; i += TK_THREADS) {
+        const uint32_t key = score_key(__ldcg(row + i));
+        if (staged) stage[i] = key;
+        if (key) { ++nv; const float v = key_score(key); vmin = fminf(vmin, v); vmax = fmaxf(vmax, v); }
+      }
+    } else {
+      for (int i = tid; i < n; i += TK_THREADS) {
+        const uint32_t key = score_key(__ldcg(row + i));
+        if (staged) stage[i] = key;
+        if (key) { ++nv; const float v = key_score(key); vmin = fminf(vmin, v); vmax = fmaxf(vmax, v); }
+      }
     }
-    uint32_t nvalid;
-    block_excl_scan(nv, ws, nvalid);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      nv += __shfl_xor_sync(0xffffffffu, nv, o);
+      vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    }
+    if (lane == 0) {
+      ws[wid] = nv;
+      fvars[wid] = vmin;
+      reinterpret_cast<float*>(ws)[32 + wid] = vmax;
+    }
+    __syncthreads();
+    if (wid == 0) {
+      uint32_t a = ws[lane];
+      float mn = fvars[lane], mx = reinterpret_cast<float*>(ws)[32 + lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      if (lane == 0) {
+        vars[8] = a;
+        reinterpret_cast<float*>(vars)[16] = mn;
+        reinterpret_cast<float*>(vars)[17] = mx;
+      }
+    }
+    __syncthreads();
+    const uint32_t nvalid = vars[8];
+    const float lo = reinterpret_cast<float*>(vars)[16], hi = reinterpret_cast<float*>(vars)[17];
     const uint32_t keff = min(static_cast<uint32_t>(k), nvalid);
+    __syncthreads();
 
     uint32_t thr = 0, take_eq = 0;  // select key > thr, plus the first take_eq keys == thr
     if (keff < nvalid) {
+      // ---- coarse: value-binned histogram
+      const float span = hi - lo;
+      const float scale = span > 0.f ? static_cast<float>(TK_BINS) / span : 0.f;
+      for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[i] = 0;
+      if (tid == 0) vars[10] = 0;
+      __syncthreads();
+      #pragma unroll 4
+      for (int i = tid; i < n; i += TK_THREADS) {
+        const uint32_t key = src.get(i);
+        if (key) atomicAdd(&hist[value_bin(key, lo, scale)], 1u);
+      }
+      __syncthreads();
       radix_pick<2>(hist, keff, ws, vars);
-      const uint32_t d1 = vars[0];
-      const uint32_t need1 = vars[1];
-      const uint32_t cnt1 = hist[d1];
-      const bool use_cache = !staged && cnt1 <= TK_CAND_CAP;
+      const int b = static_cast<int>(vars[0]);
+      const uint32_t need = vars[1];
+      const uint32_t cnt = hist[b];
       __syncthreads();
-      // ---- digit 2 (bits 20..10) among keys with digit 1 == d1
-      for (int i = tid; i < 2048; i += TK_THREADS) hist[i] = 0;
-      if (tid == 0) vars[2] = 0;
-      __syncthreads();
-      for (int base = 0; base < n; base += TK_THREADS) {
-        const int i = base + tid;
-        const uint32_t key = i < n ? (staged ? cache[i] : score_key(__ldcg(row + i))) : 0u;
-        const bool in = key != 0u && (key >> 21) == d1;
-        hist_add(hist, in, (key >> 10) & 0x7FFu);
-        if (use_cache && in) {
-          const uint32_t slot = atomicAdd(&vars[2], 1u);
-          cache[2 * slot] = key;
-          cache[2 * slot + 1] = static_cast<uint32_t>(i);
+      if (cnt <= TK_CAND_CAP) {
+        #pragma unroll 4
+        for (int i = tid; i < n; i += TK_THREADS) {
+          const uint32_t key = src.get(i);
+          if (key && value_bin(key, lo, scale) == b) cbuf[atomicAdd(&vars[10], 1u)] = key;
         }
-      }
-      __syncthreads();
-      radix_pick<2>(hist, need1, ws, vars);
-      const uint32_t d2 = vars[0];
-      const uint32_t need2 = vars[1];
-      const uint32_t ncache = vars[2];
-      const uint32_t pre = (d1 << 11) | d2;
-      __syncthreads();
-      // ---- digit 3 (bits 9..0) among keys with digits 1-2 == pre
-      for (int i = tid; i < 2048; i += TK_THREADS) hist[i] = 0;
-      __syncthreads();
-      if (use_cache) {
-        for (int base = 0; base < static_cast<int>(ncache); base += TK_THREADS) {
-          const int i = base + tid;
-          const uint32_t key = i < static_cast<int>(ncache) ? cache[2 * i] : 0u;
-          hist_add(hist, key != 0u && (key >> 10) == pre, key & 0x3FFu);
-        }
+        __syncthreads();
+        exact_select(cbuf, nullptr, static_cast<int>(cnt), need, hist, ws, vars);
       } else {
-        for (int base = 0; base < n; base += TK_THREADS) {
-          const int i = base + tid;
-          const uint32_t key = i < n ? (staged ? cache[i] : score_key(__ldcg(row + i))) : 0u;
-          hist_add(hist, key != 0u && (key >> 10) == pre, key & 0x3FFu);
-        }
+        exact_select(skeys, row, n, keff, hist, ws, vars);
       }
-      __syncthreads();
-      radix_pick<1>(hist, need2, ws, vars);
-      thr = (pre << 10) | vars[0];
+      thr = vars[0];
       take_eq = vars[1];
       __syncthreads();
     }
 
     // ---- ordered write-out: keys > thr, then the first take_eq keys == thr
+    const int seg = ((n + TK_WARPS * 32 - 1) / (TK_WARPS * 32)) * 32;  // per-warp segment
+    const int s0 = wid * seg;
+    const int s1 = min(n, s0 + seg);
+    uint32_t cgt = 0, ceq = 0;
+    #pragma unroll 4
+    for (int i = s0 + lane; i < s1; i += 32) {
+      const uint32_t key = src.get(i);
+      cgt += key > thr;
+      ceq += (key == thr) && key != 0u;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      cgt += __shfl_xor_sync(0xffffffffu, cgt, o);
+      ceq += __shfl_xor_sync(0xffffffffu, ceq, o);
+    }
+    if (lane == 0) { ws[wid] = cgt; ws[32 + wid] = ceq; }
+    __syncthreads();
+    if (wid == 0) {
+      const uint32_t g = ws[lane], e = ws[32 + lane];
+      uint32_t gi = g, ei = e;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, gi, o);
+        const uint32_t z = __shfl_up_sync(0xffffffffu, ei, o);
+        if (lane >= o) { gi += y; ei += z; }
+      }
+      ws[lane] = gi - g;
+      ws[32 + lane] = ei - e;
+    }
+    __syncthreads();
+    uint32_t run_gt = ws[wid], run_eq = ws[32 + wid];
+    __syncthreads();
     int32_t* oi = p.out_idx + r * p.k;
     float* os = p.out_score ? p.out_score + r * p.k : nullptr;
-    uint32_t run_gt = 0, run_eq = 0;
-    for (int base = 0; base < n; base += TK_THREADS) {
-      const int i = base + tid;
-      const uint32_t key = i < n ? (staged ? cache[i] : score_key(__ldcg(row + i))) : 0u;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int base = s0; base < s1; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = i < s1 ? src.get(i) : 0u;
       const bool gt = key > thr;
       const bool eq = (key == thr) && key != 0u;
-      uint32_t tot;
-      const uint32_t ex = block_excl_scan((gt ? 0x10000u : 0u) | (eq ? 1u : 0u), ws, tot);
-      const uint32_t eq_before = run_eq + (ex & 0xFFFFu);
+      const uint32_t bg = __ballot_sync(0xffffffffu, gt);
+      const uint32_t be = __ballot_sync(0xffffffffu, eq);
+      const uint32_t eq_before = run_eq + __popc(be & below);
       if (gt || (eq && eq_before < take_eq)) {
-        const uint32_t pos = run_gt + (ex >> 16) + min(eq_before, take_eq);
+        const uint32_t pos = run_gt + __popc(bg & below) + min(eq_before, take_eq);
         int idx = i;
         if (p.cand) {
           const int slot = i / p.blk;
@@ -222,9 +352,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
         oi[pos] = idx;
         if (os) os[pos] = key_score(key);
       }
-      run_gt += tot >> 16;
-      run_eq += tot & 0xFFFFu;
-      if (run_gt + min(run_eq, take_eq) >= keff) break;
+      run_gt += __popc(bg);
+      run_eq += __popc(be);
     }
     for (int j = static_cast<int>(keff) + tid; j < k; j += TK_THREADS) {
       oi[j] = -1;
