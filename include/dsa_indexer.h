@@ -101,6 +101,27 @@ DSA_EXPORT size_t indexer_workspace_size(const dsa_indexer_args* a, int topk);
 DSA_EXPORT dsa_status indexer_score_topk(const dsa_indexer_args* a, int topk, int32_t* out_idx,
                               float* out_score, void* workspace, size_t ws_bytes, void* stream);
 
+/* indexer_score_topk_noalloc: the same dense score + top-k as
+ * indexer_score_topk, for callers that cannot allocate device memory: code
+ * running inside a stream capture whose graph must not contain allocations,
+ * plugins handed a fixed memory arena by a host runtime that owns every
+ * device allocation, and callers with no allocator at all (no torch, no
+ * cudaMalloc permission). It takes no workspace: its scores scratch is a
+ * 64 MiB array in the library's own device memory (reserved on every GPU
+ * that loads the library, until the process exits), so it accepts problems
+ * with 256 + 4 * batch * T * L <= 64 MiB (e.g. 64 decode sequences of
+ * 131072 keys) and returns DSA_ERR_WORKSPACE for larger ones.
+ * It allocates nothing and calls no allocating routine. The first call on a
+ * device looks the scratch's device address up (cudaGetSymbolAddress, with
+ * that device current) and caches it; make that first call before any stream
+ * capture. Every call on a device shares the one scratch array: calls that
+ * may overlap on the GPU (different streams, no ordering between them) race
+ * and must not be issued. The status word at the start of the scratch is
+ * cleared by each call. No method page has a counterpart of this entry
+ * point; it is plumbing. */
+DSA_EXPORT dsa_status indexer_score_topk_noalloc(const dsa_indexer_args* a, int topk,
+                                                 int32_t* out_idx, float* out_score, void* stream);
+
 /* Stage 1 alone: write the scores I[t,s] of all visible keys into
  * out_scores[(b*T + t) * ld + s] (ld >= L). Entries with s > q_offset + t are
  * left untouched. Workspace: the 256-byte header only. */

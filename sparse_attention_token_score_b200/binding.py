@@ -44,6 +44,7 @@ _SIGS = {
     "dsa_device_status": (ctypes.c_int, [_P, _P]),
     "indexer_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int]),
     "indexer_score_topk": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
+    "indexer_score_topk_noalloc": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P]),
     "indexer_scores": (ctypes.c_int, [_P, _P, ctypes.c_longlong, _P, ctypes.c_size_t, _P]),
     "indexer_topk_rows": (ctypes.c_int, [_P, ctypes.c_longlong, ctypes.c_longlong, ctypes.c_int,
                                          ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -142,6 +143,14 @@ def indexer_score_topk(args: IndexerArgs, topk: int, out_idx: torch.Tensor,
     _check("indexer_score_topk",
            lib().indexer_score_topk(ctypes.byref(args), topk, _ptr(out_idx), _ptr(out_score),
                                     _ptr(workspace), workspace.numel(), _stream_ptr(stream)))
+
+
+def indexer_score_topk_noalloc(args: IndexerArgs, topk: int, out_idx: torch.Tensor,
+                               out_score: Optional[torch.Tensor], stream=None):
+    """indexer_score_topk without a workspace (the library's static scratch)."""
+    _check("indexer_score_topk_noalloc",
+           lib().indexer_score_topk_noalloc(ctypes.byref(args), topk, _ptr(out_idx),
+                                            _ptr(out_score), _stream_ptr(stream)))
 
 
 def indexer_scores(args: IndexerArgs, out_scores: torch.Tensor, ld: int, workspace: torch.Tensor,

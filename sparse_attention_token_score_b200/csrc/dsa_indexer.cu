@@ -509,3 +509,48 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ no-allocation variant
+// Dense score + top-k for callers that cannot allocate device memory. The
+// scores scratch lives in a file-scope __device__ array that every device
+// loading this library reserves until exit. Host code must not pass
+// `g_noalloc_scratch` itself to a kernel: on the host that name is only a
+// stand-in for the device symbol. The device address is looked up once per
+// device with cudaGetSymbolAddress (the first call on a device, with that
+// device current) and cached.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDev] = {nullptr};
+
+dsa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDev) return DSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" dsa_status indexer_score_topk_noalloc(const dsa_indexer_args* a, int topk,
+                                                 int32_t* out_idx, float* out_score,
+                                                 void* stream) {
+  DSA_TRY(validate(a, false));
+  if (!out_idx || topk < 1 || topk > (1 << 24)) return DSA_ERR_ARG;
+  if (indexer_workspace_size(a, topk) > kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  DSA_TRY(noalloc_scratch(&scratch));
+  // Same launches as indexer_score_topk; its status word (first 4 bytes of
+  // the scratch) is cleared on the stream before the kernels run.
+  return indexer_score_topk(a, topk, out_idx, out_score, scratch, kNoAllocScratchBytes, stream);
+}
