@@ -55,13 +55,15 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ workloads
-def workload_desc(name, queries=None):
+def workload_desc(name, queries=None, batch=None):
     from sparse_attention_token_score_b200 import workloads as wl
     c = dict(wl.CONFIGS[name])
     if queries:  # a smaller chunk at the end of the same prefix (profiling cases)
         c["T"] = int(queries)
         if "q_offset" in c:
             c["q_offset"] = c["L"] - c["T"]
+    if batch and "batch" in c:  # fewer sequences (profiling cases)
+        c["batch"] = int(batch)
     batch = c.get("batch", 1)
     off = c.get("q_offset", c["L"] - 1)
     pairs = wl.visible_pairs(c["T"], c["L"], off, batch)
@@ -78,10 +80,10 @@ def workload_desc(name, queries=None):
 class Runner:
     """Device-resident inputs + the C-ABI call of one workload."""
 
-    def __init__(self, name, inp, torch, queries=None):
+    def __init__(self, name, inp, torch, queries=None, batch=None):
         from sparse_attention_token_score_b200 import binding as B
         self.B, self.torch, self.name = B, torch, name
-        self.c, self.batch, self.off, self.pairs, self.label = workload_desc(name, queries)
+        self.c, self.batch, self.off, self.pairs, self.label = workload_desc(name, queries, batch)
         self.inp = inp
         q, k, w, qs, ks = B.to_device(inp)
         self.dev = (q, k, w, qs, ks)
@@ -261,10 +263,14 @@ def run_reference(args):
     return 0
 
 
-def make_inputs(name, seed, queries=0):
+def make_inputs(name, seed, queries=0, batch=0):
     """The workload's inputs; with `queries`, only the last `queries` queries
-    of the chunk (same prefix, same distributions)."""
+    of the chunk (same prefix, same distributions); with `batch`, only the
+    first `batch` sequences."""
     from sparse_attention_token_score_b200 import workloads as wl
+    if batch and name == "decode":
+        c = wl.CONFIGS[name]
+        return wl.decode_inputs(batch, c["L"], c["H"], c["d"], seed=seed)
     inp = wl.make_inputs(name, seed=seed)
     if queries and queries < inp.T:
         T0 = inp.T - queries
@@ -287,6 +293,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--queries", type=int, default=0,
                     help="profiling: use only the last N queries of the chunk")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="profiling: use only the first N sequences (decode)")
     ap.add_argument("--kernel-only", action="store_true",
                     help="profiling: launch only the dominant kernel (W + K times)")
     args = ap.parse_args()
@@ -314,8 +322,8 @@ def main():
         if world > 1:
             dist.barrier()
 
-    inp = make_inputs(args.workload, rank, args.queries)
-    r = Runner(args.workload, inp, torch, args.queries)
+    inp = make_inputs(args.workload, rank, args.queries, args.batch)
+    r = Runner(args.workload, inp, torch, args.queries, args.batch)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     if args.kernel_only:
         fn, _, _, kname = r.dominant()

@@ -46,7 +46,7 @@ constexpr int TK_WARPS = TK_THREADS / 32;
 constexpr int TK_BINS = 2048;
 constexpr int TK_SMEM_ROW = 40960;   // rows up to this length are staged in shared memory
 constexpr int TK_CAND_CAP = 8192;    // keys of the threshold bin
-constexpr int TK_SMEM_WORDS = TK_BINS + 128 + TK_CAND_CAP + TK_SMEM_ROW;
+constexpr int TK_SMEM_WORDS = TK_BINS + 128 + TK_CAND_CAP + TK_SMEM_ROW + 4;
 constexpr int TK_SMEM_BYTES = TK_SMEM_WORDS * 4;
 constexpr int TK_UNROLL = 8;        // float4 loads in flight per thread in the row load
 
@@ -112,41 +112,43 @@ __device__ __forceinline__ void radix_pick(const uint32_t* hist, uint32_t need, 
   __syncthreads();
 }
 
-// Source of the keys of one row: shared-memory stage, candidate buffer, or global.
+// Source of one row's scores: the shared-memory stage, or the global row.
 struct RowSrc {
-  const uint32_t* smem;  // staged keys (or nullptr)
-  const float* g;        // global row
-  __device__ __forceinline__ uint32_t get(int i) const {
-    return smem ? smem[i] : score_key(__ldcg(g + i));
+  const float* smem;  // staged scores (or nullptr)
+  const float* g;     // global row
+  __device__ __forceinline__ float get(int i) const { return smem ? smem[i] : __ldcg(g + i); }
+  __device__ __forceinline__ float4 get4(int i4) const {
+    return smem ? reinterpret_cast<const float4*>(smem)[i4]
+                : __ldcg(reinterpret_cast<const float4*>(g) + i4);
   }
 };
 
-// Exact radix select over the keys of positions [0, n) (shared-memory keys, or
-// the global row when keys == nullptr); keys equal to 0 (absent) are ignored.
-// Leaves vars[0] = tau, the need-th largest key, and vars[1] = how many keys
-// equal to tau rank within the top `need`.
-__device__ void exact_select(const uint32_t* keys, const float* g, int n, uint32_t need,
+__device__ __forceinline__ bool present(float x) { return x > -INFINITY; }  // false for -inf, NaN
+
+// Exact radix select over keys (score_key) of a key buffer (cbuf != nullptr,
+// n keys) or of positions [0, n) of a row; keys equal to 0 (absent) are
+// ignored. Leaves vars[0] = tau, the need-th largest key, and vars[1] = how
+// many keys equal to tau rank within the top `need`.
+__device__ void exact_select(const uint32_t* cbuf, const RowSrc& src, int n, uint32_t need,
                              uint32_t* hist, uint32_t* ws, uint32_t* vars) {
-  const RowSrc src{keys, g};
   uint32_t prefix = 0;
-  const int shifts[3] = {21, 10, 0};
-  const uint32_t widths[3] = {11, 11, 10};
 #pragma unroll 1
   for (int d = 0; d < 3; ++d) {
+    const int sh = d == 0 ? 21 : (d == 1 ? 10 : 0);
+    const uint32_t width = d == 2 ? 10u : 11u;
+    const uint32_t hi_sh = sh + width;
     for (int i = threadIdx.x; i < TK_BINS; i += TK_THREADS) hist[i] = 0;
     __syncthreads();
-    const int sh = shifts[d];
-    const uint32_t hi_sh = sh + widths[d];
-    #pragma unroll 4
+#pragma unroll 4
     for (int i = threadIdx.x; i < n; i += TK_THREADS) {
-      const uint32_t key = src.get(i);
+      const uint32_t key = cbuf ? cbuf[i] : score_key(src.get(i));
       if (key != 0u && (hi_sh >= 32 || (key >> hi_sh) == prefix))
-        atomicAdd(&hist[(key >> sh) & ((1u << widths[d]) - 1u)], 1u);
+        atomicAdd(&hist[(key >> sh) & ((1u << width) - 1u)], 1u);
     }
     __syncthreads();
     if (d < 2) radix_pick<2>(hist, need, ws, vars);
     else radix_pick<1>(hist, need, ws, vars);
-    prefix = (prefix << widths[d]) | vars[0];
+    prefix = (prefix << width) | vars[0];
     need = vars[1];
     __syncthreads();
   }
@@ -157,11 +159,14 @@ __device__ void exact_select(const uint32_t* keys, const float* g, int n, uint32
   __syncthreads();
 }
 
-// Value bin of a present key: 2048 evenly spaced bins over [lo, lo + 2048/scale].
-__device__ __forceinline__ int value_bin(uint32_t key, float lo, float scale) {
-  const float v = (key_score(key) - lo) * scale;
-  int b = static_cast<int>(v);
-  return b < 0 ? 0 : (b > TK_BINS - 1 ? TK_BINS - 1 : b);
+// Value bin of a present score: TK_BINS evenly spaced bins over [lo, lo + TK_BINS/scale].
+// (x - lo) * scale >= 0; adding 1.5 * 2^23 leaves round-to-nearest(v) in the low
+// mantissa bits (a monotone map, no float-to-int conversion instruction).
+// scale == 0 (all scores equal, or a span that overflows) puts everything in bin 0.
+__device__ __forceinline__ int value_bin(float x, float lo, float scale) {
+  const float v = (scale > 0.f ? (x - lo) * scale : 0.f) + 12582912.0f;
+  const int b = __float_as_int(v) - 0x4B400000;
+  return min(b, TK_BINS - 1);
 }
 
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkParams p) {
@@ -170,7 +175,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
   uint32_t* ws = hist + TK_BINS;             // 64
   uint32_t* vars = ws + 64;                  // 64
   uint32_t* cbuf = vars + 64;                // TK_CAND_CAP keys of the threshold bin
-  uint32_t* stage = cbuf + TK_CAND_CAP;      // TK_SMEM_ROW
+  float* stage = reinterpret_cast<float*>(cbuf + TK_CAND_CAP);  // TK_SMEM_ROW scores
   float* fvars = reinterpret_cast<float*>(vars + 32);
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
@@ -184,51 +189,44 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
     }
     const int n = static_cast<int>(nl);
     const float* row = p.scores + r * p.ld;
-    const bool staged = n <= TK_SMEM_ROW;
-    const uint32_t* skeys = staged ? stage : nullptr;
-    const RowSrc src{skeys, row};
+    const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15u) == 0);
+    const bool staged = n <= TK_SMEM_ROW && vec;
+    const RowSrc src{staged ? stage : nullptr, row};
+    const int n4 = vec ? (n >> 2) : 0;     // float4 part [0, 4*n4), scalar tail [4*n4, n)
     const int k = p.k;
 
-    // ---- pass 1: stage keys; count present; min / max of present values
+    // ---- pass 1: (stage) count present scores, min / max
     uint32_t nv = 0;
     float vmin = INFINITY, vmax = -INFINITY;
-    const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15u) == 0);
-    if (vec) {
-      // TK_UNROLL float4 loads per thread are in flight before any is used
-      // (128 KB per SM for a 32K-entry row), so the row streams at HBM rate.
-      const int n4 = n >> 2;
-      for (int base = 0; base < n4; base += TK_THREADS * TK_UNROLL) {
-        float4 x[TK_UNROLL];
+    for (int base = 0; base < n4; base += TK_THREADS * TK_UNROLL) {
+      float4 x[TK_UNROLL];
 #pragma unroll
-        for (int u = 0; u < TK_UNROLL; ++u) {
-          const int i = base + u * TK_THREADS + tid;
-          x[u] = i < n4 ? __ldcg(reinterpret_cast<const float4*>(row) + i)
-                        : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-        }
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int i = base + u * TK_THREADS + tid;
+        x[u] = i < n4 ? __ldcg(reinterpret_cast<const float4*>(row) + i)
+                      : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
 #pragma unroll
-        for (int u = 0; u < TK_UNROLL; ++u) {
-          const int i = base + u * TK_THREADS + tid;
-          if (i >= n4) continue;
-          const float xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int i = base + u * TK_THREADS + tid;
+        if (staged && i < n4) reinterpret_cast<float4*>(stage)[i] = x[u];
+        const float xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t key = score_key(xs[j]);
-            if (staged) stage[4 * i + j] = key;
-            if (key) { ++nv; const float v = key_score(key); vmin = fminf(vmin, v); vmax = fmaxf(vmax, v); }
-          }
+        for (int j = 0; j < 4; ++j) {
+          const bool pr = present(xs[j]);
+          nv += pr;
+          vmin = fminf(vmin, pr ? xs[j] : INFINITY);
+          vmax = fmaxf(vmax, xs[j]);
         }
       }
-      for (int i = 4 * n4 + tid; i < n; i += TK_THREADS) {
-        const uint32_t key = score_key(__ldcg(row + i));
-        if (staged) stage[i] = key;
-        if (key) { ++nv; const float v = key_score(key); vmin = fminf(vmin, v); vmax = fmaxf(vmax, v); }
-      }
-    } else {
-      for (int i = tid; i < n; i += TK_THREADS) {
-        const uint32_t key = score_key(__ldcg(row + i));
-        if (staged) stage[i] = key;
-        if (key) { ++nv; const float v = key_score(key); vmin = fminf(vmin, v); vmax = fmaxf(vmax, v); }
-      }
+    }
+    for (int i = 4 * n4 + tid; i < n; i += TK_THREADS) {
+      const float x = __ldcg(row + i);
+      if (staged) stage[i] = x;
+      const bool pr = present(x);
+      nv += pr;
+      vmin = fminf(vmin, pr ? x : INFINITY);
+      vmax = fmaxf(vmax, x);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -263,18 +261,27 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
     const uint32_t keff = min(static_cast<uint32_t>(k), nvalid);
     __syncthreads();
 
-    uint32_t thr = 0, take_eq = 0;  // select key > thr, plus the first take_eq keys == thr
+    // select score > thr, plus the first take_eq scores == thr (-0 == +0 as floats)
+    float thr = -INFINITY;
+    uint32_t take_eq = 0;
     if (keff < nvalid) {
       // ---- coarse: value-binned histogram
       const float span = hi - lo;
-      const float scale = span > 0.f ? static_cast<float>(TK_BINS) / span : 0.f;
+      const float scale = (span > 0.f && span < INFINITY) ? static_cast<float>(TK_BINS - 1) / span : 0.f;
       for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[i] = 0;
       if (tid == 0) vars[10] = 0;
       __syncthreads();
-      #pragma unroll 4
-      for (int i = tid; i < n; i += TK_THREADS) {
-        const uint32_t key = src.get(i);
-        if (key) atomicAdd(&hist[value_bin(key, lo, scale)], 1u);
+#pragma unroll 2
+      for (int i = tid; i < n4; i += TK_THREADS) {
+        const float4 x = src.get4(i);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (present(xs[j])) atomicAdd(&hist[value_bin(xs[j], lo, scale)], 1u);
+      }
+      for (int i = 4 * n4 + tid; i < n; i += TK_THREADS) {
+        const float x = src.get(i);
+        if (present(x)) atomicAdd(&hist[value_bin(x, lo, scale)], 1u);
       }
       __syncthreads();
       radix_pick<2>(hist, keff, ws, vars);
@@ -283,31 +290,54 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
       const uint32_t cnt = hist[b];
       __syncthreads();
       if (cnt <= TK_CAND_CAP) {
-        #pragma unroll 4
-        for (int i = tid; i < n; i += TK_THREADS) {
-          const uint32_t key = src.get(i);
-          if (key && value_bin(key, lo, scale) == b) cbuf[atomicAdd(&vars[10], 1u)] = key;
+#pragma unroll 2
+        for (int i = tid; i < n4; i += TK_THREADS) {
+          const float4 x = src.get4(i);
+          const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (present(xs[j]) && value_bin(xs[j], lo, scale) == b)
+              cbuf[atomicAdd(&vars[10], 1u)] = score_key(xs[j]);
+        }
+        for (int i = 4 * n4 + tid; i < n; i += TK_THREADS) {
+          const float x = src.get(i);
+          if (present(x) && value_bin(x, lo, scale) == b) cbuf[atomicAdd(&vars[10], 1u)] = score_key(x);
         }
         __syncthreads();
-        exact_select(cbuf, nullptr, static_cast<int>(cnt), need, hist, ws, vars);
+        exact_select(cbuf, src, static_cast<int>(cnt), need, hist, ws, vars);
       } else {
-        exact_select(skeys, row, n, keff, hist, ws, vars);
+        exact_select(nullptr, src, n, keff, hist, ws, vars);
       }
-      thr = vars[0];
+      thr = key_score(vars[0]);
       take_eq = vars[1];
       __syncthreads();
     }
 
-    // ---- ordered write-out: keys > thr, then the first take_eq keys == thr
-    const int seg = ((n + TK_WARPS * 32 - 1) / (TK_WARPS * 32)) * 32;  // per-warp segment
-    const int s0 = wid * seg;
+    // ---- ordered write-out. Warp w owns the contiguous segment [s0, s1);
+    // lane l of a 128-entry chunk owns entries 4l .. 4l+3 (one float4).
+    const int seg = ((n + TK_WARPS * 128 - 1) / (TK_WARPS * 128)) * 128;
+    const int s0 = min(n, wid * seg);
     const int s1 = min(n, s0 + seg);
+    const bool v4 = vec;  // 16-byte aligned row: float4 chunks
+    auto load4 = [&](int i, float (&x)[4]) {
+      if (v4 && i + 3 < s1) {
+        const float4 f = src.get4(i >> 2);
+        x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x[j] = (i + j < s1) ? src.get(i + j) : -INFINITY;
+      }
+    };
     uint32_t cgt = 0, ceq = 0;
-    #pragma unroll 4
-    for (int i = s0 + lane; i < s1; i += 32) {
-      const uint32_t key = src.get(i);
-      cgt += key > thr;
-      ceq += (key == thr) && key != 0u;
+#pragma unroll 2
+    for (int base = s0; base < s1; base += 128) {
+      float x[4];
+      load4(base + 4 * lane, x);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        cgt += x[j] > thr;
+        ceq += x[j] == thr && present(x[j]);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -333,27 +363,45 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
     __syncthreads();
     int32_t* oi = p.out_idx + r * p.k;
     float* os = p.out_score ? p.out_score + r * p.k : nullptr;
-    const uint32_t below = (1u << lane) - 1u;
-    for (int base = s0; base < s1; base += 32) {
-      const int i = base + lane;
-      const uint32_t key = i < s1 ? src.get(i) : 0u;
-      const bool gt = key > thr;
-      const bool eq = (key == thr) && key != 0u;
-      const uint32_t bg = __ballot_sync(0xffffffffu, gt);
-      const uint32_t be = __ballot_sync(0xffffffffu, eq);
-      const uint32_t eq_before = run_eq + __popc(be & below);
-      if (gt || (eq && eq_before < take_eq)) {
-        const uint32_t pos = run_gt + __popc(bg & below) + min(eq_before, take_eq);
-        int idx = i;
-        if (p.cand) {
-          const int slot = i / p.blk;
-          idx = __ldg(p.cand + r * p.n_slots + slot) * p.blk + (i - slot * p.blk);
-        }
-        oi[pos] = idx;
-        if (os) os[pos] = key_score(key);
+    for (int base = s0; base < s1; base += 128) {
+      const int i0 = base + 4 * lane;
+      float x[4];
+      load4(i0, x);
+      uint32_t ng = 0, ne = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        ng += x[j] > thr;
+        ne += x[j] == thr && present(x[j]);
       }
-      run_gt += __popc(bg);
-      run_eq += __popc(be);
+      // exclusive prefix over the lanes (entries of lower lanes come first)
+      uint32_t pg = ng, pe = ne;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, pg, o);
+        const uint32_t z = __shfl_up_sync(0xffffffffu, pe, o);
+        if (lane >= o) { pg += y; pe += z; }
+      }
+      uint32_t gb = run_gt + pg - ng, eb = run_eq + pe - ne;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const bool gt = x[j] > thr;
+        const bool eq = x[j] == thr && present(x[j]);
+        if (gt || (eq && eb < take_eq)) {
+          const uint32_t pos = gb + min(eb, take_eq);
+          const int i = i0 + j;
+          int idx = i;
+          if (p.cand) {
+            const int slot = i / p.blk;
+            idx = __ldg(p.cand + r * p.n_slots + slot) * p.blk + (i - slot * p.blk);
+          }
+          oi[pos] = idx;
+          if (os) os[pos] = x[j] == 0.f ? 0.f : x[j];
+        }
+        gb += gt;
+        eb += eq;
+      }
+      run_gt += __shfl_sync(0xffffffffu, pg, 31);
+      run_eq += __shfl_sync(0xffffffffu, pe, 31);
     }
     for (int j = static_cast<int>(keff) + tid; j < k; j += TK_THREADS) {
       oi[j] = -1;
