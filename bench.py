@@ -115,6 +115,20 @@ class Runner:
         else:
             B.hisa_block_filter_topk(a, c["block"], c["m"], self.topk, o, None, None, self.ws)
 
+    # second stage alone: top-k over the rows the scoring stage just wrote
+    def topk_stage(self):
+        B, torch, c = self.B, self.torch, self.c
+        if self.name not in ("tiny", "dsa", "decode"):
+            return None
+        out = torch.empty((self.batch, c["T"], c["L"]), dtype=torch.float32, device="cuda")
+        ws = B.alloc_workspace(256)
+        B.indexer_scores(self.ix.args, out, c["L"], ws)
+        idx = torch.empty((self.batch, c["T"], self.topk), dtype=torch.int32, device="cuda")
+        rows = self.batch * c["T"]
+        self._keep_topk = (out, ws, idx)
+        return lambda: B.indexer_topk_rows(out, rows, c["L"], c["T"], self.inp.q_offset, 1, c["L"],
+                                           self.topk, None, 0, 1, idx, None, ws)
+
     # dominant kernel, launched alone through the score-stage entry point
     def dominant(self):
         """(callable, algorithmic units per launch, bound, name)."""
@@ -368,9 +382,12 @@ def main():
             achieved = units / (kms / 1e3) / 1e9
             peak = peaks["hbm_gbs"]
             unit = "GB/s"
+        tk = r.topk_stage()
+        topk_ms = statistics.mean(time_steps(tk, args.steps, torch, flush)) if tk else None
         roof = {"bound": bound, "kernel": kname, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "peak_source": f"{peak_src} ({'bf16 burst' if bound == 'tensor' else 'HBM copy'})",
-                "kernel_ms": kms, "algorithmic_units_per_launch": units, "traffic": None}
+                "kernel_ms": kms, "algorithmic_units_per_launch": units, "traffic": None,
+                "topk_stage_ms": topk_ms}
 
     # ---- end to end: host buffers, H2D + call + D2H per step
     q, k, w, qs, ks = r.dev

@@ -165,7 +165,7 @@ dsa_status launch_topk(const TopkParams& tp, cudaStream_t st) {
       return DSA_ERR_CUDA;
     attr[dev] = true;
   }
-  long long grid = num_sms();
+  long long grid = static_cast<long long>(num_sms()) * TK_CTAS_PER_SM;
   if (tp.rows < grid) grid = tp.rows;
   topk_rows_kernel<<<static_cast<int>(grid), TK_THREADS, TK_SMEM_BYTES, st>>>(tp);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;

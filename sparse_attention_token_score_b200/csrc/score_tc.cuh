@@ -290,15 +290,23 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // a half-warp copies one 256-byte row, chunk c of row r lands at its
         // 128-byte-swizzle slot (c ^ (r & 7)) so the tensor core sees the same
         // layout a TMA load would have written.
+        // The tile's 128 token ids are resolved first (lane l owns rows l,
+        // l+32, l+64, l+96: four independent loads), then handed to the
+        // copying lanes with shuffles, so no copy waits on a dependent load.
+        const long long r = static_cast<long long>(b) * p.T + tg;
+        const long long q_pos = p.q_offset + tg;
+        long long toks[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) toks[u] = gathered_token(p, r, s.j * C::KROWS + 32 * u + lane, q_pos);
         if (!mbar_wait(empty(stage), ph ^ 1u, p.err)) ok = false;
         if (ok) {
-          const long long r = static_cast<long long>(b) * p.T + tg;
-          const long long q_pos = p.q_offset + tg;
           const int ch = lane & 15;
           const uint32_t tile = s_k + stage * C::K_BYTES;
+#pragma unroll 8
           for (int i = 0; i < C::KROWS / 2; ++i) {
             const int row = 2 * i + (lane >> 4);
-            const long long tok = gathered_token(p, r, s.j * C::KROWS + row, q_pos);
+            // row r lives in lane (r & 31) of toks[r >> 5]; rows 2i and 2i+1 share r >> 5
+            const long long tok = __shfl_sync(0xffffffffu, toks[(2 * i) >> 5], row & 31);
             const int kb = ch >> 3;
             const uint32_t dst = tile + kb * C::KROWS * 128 + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
             if (tok >= 0) {

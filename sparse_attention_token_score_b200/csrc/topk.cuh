@@ -7,20 +7,30 @@
 // return all of them. Output: selected positions in ascending order (mapped
 // through an optional index map), padded with -1 (score -inf).
 //
-// Scores map to order-preserving 32-bit keys (-0 folded onto +0, absent -> 0).
-// The k-th key tau and the number of keys equal to tau to take are found in
-// two steps:
-//   1. coarse: a 2048-bin histogram over *values* (bins evenly spaced between
-//      the row's min and max, a monotone map, so contention stays low even
-//      though the scores crowd a few exponents) locates the bin holding the
-//      k-th value; the bin's elements are compacted into a small buffer;
-//   2. exact: a three-digit radix select (11 + 11 + 10 bits) over that buffer.
-// If the bin is too large for the buffer (mass ties), the exact radix select
-// runs over the whole row instead. The write-out gives each warp a contiguous
-// segment: count, one block-wide exclusive scan of the 32 warp counts, then
-// ballot-ordered stores, so positions come out in ascending order.
-// Rows up to TK_SMEM_ROW entries are staged once in shared memory; longer rows
-// are re-read from global memory (L2) on each pass.
+// Scores map to order-preserving 32-bit keys (-0 folded onto +0, absent -> 0)
+// where integer order is needed; elsewhere scores are compared as floats
+// (which already treat -0 and +0 as equal). Per row:
+//   1. stage the row in shared memory when it fits (one full-rate read),
+//      and take every S-th score as a sample (S a power of two, at most 4096
+//      samples; a longer row stays in global memory / L2 and only its sample
+//      is read here);
+//   2. a 2048-bin value histogram of the sample (bins evenly spaced between
+//      the sample's min and max) brackets the k-th score in a band
+//      [t_lo, t_hi] wide enough (4 standard deviations of the sample rank on
+//      each side) that the k-th score lies inside with near certainty;
+//   3. one pass over the row: each warp owns a contiguous segment; for every
+//      32 consecutive positions the warp's ballot of "score > t_hi" is stored
+//      as that word of a selection bitmap, and the band's scores go to the
+//      warp's candidate list (key, position), in position order;
+//   4. an exact three-digit radix select (11 + 11 + 10 bits) over the
+//      candidates gives tau and how many scores equal to tau to take; the
+//      selected candidates are OR-ed into the bitmap;
+//   5. the bitmap is emitted in position order (per-warp popcounts, one
+//      prefix sum over the warps, each lane writes its set bits).
+// If a check fails (unlucky sample, mass ties, a full candidate list, fewer
+// present scores than k), the row falls back to a full value histogram, an
+// exact select over the k-th value's bin (or the whole row), a counting pass
+// and an ordered write pass.
 #pragma once
 #include "common.cuh"
 
@@ -41,14 +51,21 @@ struct TopkParams {
   int n_slots, blk;
 };
 
-constexpr int TK_THREADS = 1024;
+constexpr int TK_THREADS = 1024;     // one row per CTA, one CTA per SM
+constexpr int TK_CTAS_PER_SM = 1;
 constexpr int TK_WARPS = TK_THREADS / 32;
 constexpr int TK_BINS = 2048;
-constexpr int TK_SMEM_ROW = 40960;   // rows up to this length are staged in shared memory
-constexpr int TK_CAND_CAP = 8192;    // keys of the threshold bin
-constexpr int TK_SMEM_WORDS = TK_BINS + 128 + TK_CAND_CAP + TK_SMEM_ROW + 4;
+constexpr int TK_SMEM_ROW = 32768;   // rows up to this length are staged in shared memory
+constexpr int TK_LIST = 128;         // band candidates per warp segment
+constexpr int TK_CAND_CAP = TK_WARPS * TK_LIST;
+constexpr int TK_SAMPLE_MAX = 4096;  // sampled scores per row
+constexpr int TK_BITMAP_WORDS = 4096;
+// longer rows take the fallback path (their selection bitmap would not fit)
+constexpr long long TK_MAX_BITMAP_ROW = 32LL * TK_BITMAP_WORDS;
+constexpr int TK_SMEM_WORDS =
+    TK_BINS + 128 + TK_SAMPLE_MAX + 2 * TK_CAND_CAP + TK_BITMAP_WORDS + TK_SMEM_ROW;
 constexpr int TK_SMEM_BYTES = TK_SMEM_WORDS * 4;
-constexpr int TK_UNROLL = 8;        // float4 loads in flight per thread in the row load
+constexpr int TK_UNROLL = 8;         // float4 loads in flight per thread when staging a row
 
 __device__ __forceinline__ uint32_t score_key(float x) {
   if (!(x > -INFINITY)) return 0u;  // -inf (absent) and NaN
@@ -72,7 +89,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* ws, ui
   if (lane == 31) ws[wid] = x;
   __syncthreads();
   if (wid == 0) {
-    const uint32_t s = ws[lane];
+    const uint32_t s = lane < TK_THREADS / 32 ? ws[lane] : 0u;
     uint32_t inc = s;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -112,14 +129,38 @@ __device__ __forceinline__ void radix_pick(const uint32_t* hist, uint32_t need, 
   __syncthreads();
 }
 
-// Source of one row's scores: the shared-memory stage, or the global row.
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 lds_f32x4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts_f32x4(uint32_t a, float4 v) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+
+// Source of one row's scores: the shared-memory stage (explicit shared-window
+// loads) or the global row, chosen at compile time so the passes carry no
+// per-access branch.
+template <bool STAGED>
 struct RowSrc {
-  const float* smem;  // staged scores (or nullptr)
-  const float* g;     // global row
-  __device__ __forceinline__ float get(int i) const { return smem ? smem[i] : __ldcg(g + i); }
-  __device__ __forceinline__ float4 get4(int i4) const {
-    return smem ? reinterpret_cast<const float4*>(smem)[i4]
-                : __ldcg(reinterpret_cast<const float4*>(g) + i4);
+  uint32_t sbase;   // shared address of the staged row
+  const float* g;   // global row
+  __device__ __forceinline__ float get(int i) const {
+    if constexpr (STAGED) return lds_f32(sbase + 4u * static_cast<uint32_t>(i));
+    else return __ldcg(g + i);
   }
 };
 
@@ -129,7 +170,8 @@ __device__ __forceinline__ bool present(float x) { return x > -INFINITY; }  // f
 // n keys) or of positions [0, n) of a row; keys equal to 0 (absent) are
 // ignored. Leaves vars[0] = tau, the need-th largest key, and vars[1] = how
 // many keys equal to tau rank within the top `need`.
-__device__ void exact_select(const uint32_t* cbuf, const RowSrc& src, int n, uint32_t need,
+template <class Src>
+__device__ void exact_select(const uint32_t* cbuf, const Src& src, int n, uint32_t need,
                              uint32_t* hist, uint32_t* ws, uint32_t* vars) {
   uint32_t prefix = 0;
 #pragma unroll 1
@@ -146,8 +188,8 @@ __device__ void exact_select(const uint32_t* cbuf, const RowSrc& src, int n, uin
         atomicAdd(&hist[(key >> sh) & ((1u << width) - 1u)], 1u);
     }
     __syncthreads();
-    if (d < 2) radix_pick<2>(hist, need, ws, vars);
-    else radix_pick<1>(hist, need, ws, vars);
+    if (d < 2) radix_pick<2048 / TK_THREADS>(hist, need, ws, vars);
+    else radix_pick<1024 / TK_THREADS>(hist, need, ws, vars);
     prefix = (prefix << width) | vars[0];
     need = vars[1];
     __syncthreads();
@@ -160,44 +202,53 @@ __device__ void exact_select(const uint32_t* cbuf, const RowSrc& src, int n, uin
 }
 
 // Value bin of a present score: TK_BINS evenly spaced bins over [lo, lo + TK_BINS/scale].
-// (x - lo) * scale >= 0; adding 1.5 * 2^23 leaves round-to-nearest(v) in the low
+// For x in [lo, hi], (x - lo) * scale >= 0; adding 1.5 * 2^23 leaves round-to-nearest(v) in the low
 // mantissa bits (a monotone map, no float-to-int conversion instruction).
 // scale == 0 (all scores equal, or a span that overflows) puts everything in bin 0.
 __device__ __forceinline__ int value_bin(float x, float lo, float scale) {
   const float v = (scale > 0.f ? (x - lo) * scale : 0.f) + 12582912.0f;
   const int b = __float_as_int(v) - 0x4B400000;
-  return min(b, TK_BINS - 1);
+  return min(max(b, 0), TK_BINS - 1);  // scores outside [lo, hi] land in the end bins
 }
 
-__global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkParams p) {
-  extern __shared__ uint32_t tk_smem[];
-  uint32_t* hist = tk_smem;                  // TK_BINS
-  uint32_t* ws = hist + TK_BINS;             // 64
-  uint32_t* vars = ws + 64;                  // 64
-  uint32_t* cbuf = vars + 64;                // TK_CAND_CAP keys of the threshold bin
-  float* stage = reinterpret_cast<float*>(cbuf + TK_CAND_CAP);  // TK_SMEM_ROW scores
+// One row of the selection (see the file comment). STAGED: the row fits in
+// shared memory and starts on a 16-byte boundary.
+template <bool STAGED>
+__device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem, long long r, int n,
+                                         const float* row) {
+  uint32_t* hist = tk_smem;                      // TK_BINS
+  uint32_t* ws = hist + TK_BINS;                 // 64
+  uint32_t* vars = ws + 64;                      // 64
+  uint32_t* samp = vars + 64;                    // TK_SAMPLE_MAX sampled scores (as floats)
+  uint32_t* ckey = samp + TK_SAMPLE_MAX;         // TK_CAND_CAP keys (warp w: [w*TK_LIST, +TK_LIST))
+  uint32_t* cpos = ckey + TK_CAND_CAP;           // TK_CAND_CAP positions
+  uint32_t* bmap = cpos + TK_CAND_CAP;           // TK_BITMAP_WORDS selection bitmap
+  float* stage = reinterpret_cast<float*>(bmap + TK_BITMAP_WORDS);  // TK_SMEM_ROW scores
   float* fvars = reinterpret_cast<float*>(vars + 32);
+  float* fsamp = reinterpret_cast<float*>(samp);
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const uint32_t s_stage = smem_u32(stage);
+  const RowSrc<STAGED> src{s_stage, row};
+  const int k = p.k;
+  // warp segments (multiples of 128 entries)
+  const int seg = ((n + TK_WARPS * 128 - 1) / (TK_WARPS * 128)) * 128;
+  const int s0 = min(n, wid * seg);
+  const int s1 = min(n, s0 + seg);
+  const bool fast = n > k && n <= TK_MAX_BITMAP_ROW;
+  // sample stride: a power of two >= 4 so that samples sit at float4 starts
+  int S = 4;
+  while (static_cast<long long>(S) * TK_SAMPLE_MAX < n) S <<= 1;
+  const int ns = (n + S - 1) / S;
 
-  for (long long r = blockIdx.x; r < p.rows; r += gridDim.x) {
-    const int t = static_cast<int>(r % p.T);
-    long long nl = p.Lrow;
-    if (p.pstride > 0) {
-      nl = (p.q_offset + t) / p.pstride + 1;
-      if (nl > p.Lrow) nl = p.Lrow;
-      if (nl < 0) nl = 0;
-    }
-    const int n = static_cast<int>(nl);
-    const float* row = p.scores + r * p.ld;
-    const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15u) == 0);
-    const bool staged = n <= TK_SMEM_ROW && vec;
-    const RowSrc src{staged ? stage : nullptr, row};
-    const int n4 = vec ? (n >> 2) : 0;     // float4 part [0, 4*n4), scalar tail [4*n4, n)
-    const int k = p.k;
+  float thr = -INFINITY;  // select score > thr, plus the first take_eq scores == thr
+  uint32_t take_eq = 0;
+  uint32_t keff = 0;
+  bool done = false;      // row written by the bitmap path
 
-    // ---- pass 1: (stage) count present scores, min / max
-    uint32_t nv = 0;
-    float vmin = INFINITY, vmax = -INFINITY;
+  // ---- 1. stage (or sample only)
+  if constexpr (STAGED) {
+    const int n4 = n >> 2;
     for (int base = 0; base < n4; base += TK_THREADS * TK_UNROLL) {
       float4 x[TK_UNROLL];
 #pragma unroll
@@ -209,24 +260,231 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
 #pragma unroll
       for (int u = 0; u < TK_UNROLL; ++u) {
         const int i = base + u * TK_THREADS + tid;
-        if (staged && i < n4) reinterpret_cast<float4*>(stage)[i] = x[u];
-        const float xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const bool pr = present(xs[j]);
-          nv += pr;
-          vmin = fminf(vmin, pr ? xs[j] : INFINITY);
-          vmax = fmaxf(vmax, xs[j]);
+        if (i < n4) {
+          sts_f32x4(s_stage + 16u * static_cast<uint32_t>(i), x[u]);
+          if (((4 * i) & (S - 1)) == 0) fsamp[(4 * i) / S] = x[u].x;
         }
       }
     }
     for (int i = 4 * n4 + tid; i < n; i += TK_THREADS) {
       const float x = __ldcg(row + i);
-      if (staged) stage[i] = x;
-      const bool pr = present(x);
-      nv += pr;
-      vmin = fminf(vmin, pr ? x : INFINITY);
-      vmax = fmaxf(vmax, x);
+      sts_f32(s_stage + 4u * static_cast<uint32_t>(i), x);
+      if ((i & (S - 1)) == 0) fsamp[i / S] = x;
+    }
+  } else if (fast) {
+#pragma unroll 8
+    for (int m = tid; m < ns; m += TK_THREADS) fsamp[m] = __ldcg(row + static_cast<long long>(m) * S);
+  }
+  __syncthreads();
+
+  if (fast) {
+    // ---- 2. sample: present count, min / max, value histogram -> band
+    uint32_t nsv = 0;
+    float vmin = INFINITY, vmax = -INFINITY;
+    for (int m = tid; m < ns; m += TK_THREADS) {
+      const float x = fsamp[m];
+      if (present(x)) { ++nsv; vmin = fminf(vmin, x); vmax = fmaxf(vmax, x); }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      nsv += __shfl_xor_sync(0xffffffffu, nsv, o);
+      vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    }
+    if (lane == 0) { ws[wid] = nsv; fvars[wid] = vmin; reinterpret_cast<float*>(ws)[32 + wid] = vmax; }
+    for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[i] = 0;
+    __syncthreads();
+    if (wid == 0) {
+      const bool has = lane < TK_WARPS;  // one partial per warp
+      uint32_t a = has ? ws[lane] : 0u;
+      float mn = has ? fvars[lane] : INFINITY;
+      float mx = has ? reinterpret_cast<float*>(ws)[32 + lane] : -INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      if (lane == 0) {
+        vars[8] = a;
+        reinterpret_cast<float*>(vars)[16] = mn;
+        reinterpret_cast<float*>(vars)[17] = mx;
+      }
+    }
+    __syncthreads();
+    const uint32_t nsvu = vars[8];
+    const float lo = reinterpret_cast<float*>(vars)[16], hi = reinterpret_cast<float*>(vars)[17];
+    const float span = hi - lo;
+    const float scale = (span > 0.f && span < INFINITY) ? static_cast<float>(TK_BINS - 1) / span : 0.f;
+    for (int m = tid; m < ns; m += TK_THREADS) {
+      const float x = fsamp[m];
+      if (present(x)) atomicAdd(&hist[value_bin(x, lo, scale)], 1u);
+    }
+    __syncthreads();
+    // expected rank of the k-th score inside the sample
+    const float nsvf = static_cast<float>(nsvu);
+    const float pr = fminf(1.f, static_cast<float>(k) / fmaxf(1.f, nsvf * static_cast<float>(S)));
+    const float center = pr * nsvf;
+    const float delta = 4.f * sqrtf(nsvf * pr * (1.f - pr)) + 4.f;
+    const int r_hi = static_cast<int>(floorf(center - delta));
+    const int r_lo = static_cast<int>(ceilf(center + delta));
+    {
+      constexpr int BPT = TK_BINS / TK_THREADS;
+      const int u = TK_THREADS - 1 - tid;  // owner of bins [u*BPT, (u+1)*BPT)
+      uint32_t loc = 0;
+#pragma unroll
+      for (int q = 0; q < BPT; ++q) loc += hist[u * BPT + q];
+      uint32_t tot;
+      long long above = block_excl_scan(loc, ws, tot);
+      if (tid == 0) { vars[12] = TK_BINS; vars[13] = 0; }
+      __syncthreads();
+#pragma unroll
+      for (int q = BPT - 1; q >= 0; --q) {
+        const long long c = hist[u * BPT + q];
+        if (r_hi >= 1 && above < r_hi && r_hi <= above + c) vars[12] = u * BPT + q;
+        if (r_lo <= static_cast<int>(tot) && above < r_lo && r_lo <= above + c) vars[13] = u * BPT + q;
+        above += c;
+      }
+      __syncthreads();
+    }
+    const int b_hi = static_cast<int>(vars[12]);
+    const int b_lo = static_cast<int>(vars[13]);
+    const float t_hi = (b_hi >= TK_BINS - 1 || scale == 0.f) ? INFINITY
+                                                            : lo + (static_cast<float>(b_hi) + 0.5f) / scale;
+    const float t_lo = (b_lo <= 0 || scale == 0.f) ? -INFINITY
+                                                   : lo + (static_cast<float>(b_lo) - 0.5f) / scale;
+    __syncthreads();
+
+    // ---- 3. band pass: bitmap words of "> t_hi", per-warp candidate lists.
+    // Above / present counts are per lane and reduced once after the pass.
+    uint32_t c_above = 0, c_band = 0, c_present = 0;
+    uint32_t* my_key = ckey + wid * TK_LIST;
+    uint32_t* my_pos = cpos + wid * TK_LIST;
+    for (int base = s0; base < s1; base += 128) {
+      // the chunk's four loads are issued before any of their uses
+      float xv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = base + 32 * j + lane;
+        xv[j] = i < s1 ? src.get(i) : -INFINITY;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = base + 32 * j + lane;
+        const float x = xv[j];
+        const bool up = x > t_hi;
+        const bool band = x >= t_lo && x <= t_hi && present(x);
+        c_above += up;
+        c_present += present(x);
+        const uint32_t ma = __ballot_sync(0xffffffffu, up);
+        if (lane == 0 && base + 32 * j < s1) bmap[(base + 32 * j) >> 5] = ma;
+        const uint32_t mb = __ballot_sync(0xffffffffu, band);
+        if (mb) {
+          if (band) {
+            const uint32_t slot = c_band + __popc(mb & lt_mask);
+            if (slot < TK_LIST) { my_key[slot] = score_key(x); my_pos[slot] = static_cast<uint32_t>(i); }
+          }
+          c_band += __popc(mb);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      c_above += __shfl_xor_sync(0xffffffffu, c_above, o);
+      c_present += __shfl_xor_sync(0xffffffffu, c_present, o);
+    }
+    for (int sl = static_cast<int>(c_band) + lane; sl < TK_LIST; sl += 32) my_key[sl] = 0u;  // empty slots
+    if (lane == 0) { ws[wid] = c_above; ws[32 + wid] = c_present; samp[wid] = c_band; }
+    __syncthreads();
+    uint32_t above_all = 0, nvalid = 0, nc = 0, cmax = 0;
+    for (int w = 0; w < TK_WARPS; ++w) {
+      above_all += ws[w];
+      nvalid += ws[32 + w];
+      nc += samp[w];
+      cmax = max(cmax, samp[w]);
+    }
+    keff = min(static_cast<uint32_t>(k), nvalid);
+    const bool band_ok = keff < nvalid && cmax <= TK_LIST && above_all < keff && keff <= above_all + nc;
+    __syncthreads();
+    if (band_ok) {
+      // ---- 4. exact select among the candidates
+      exact_select(ckey, src, TK_CAND_CAP, keff - above_all, hist, ws, vars);
+      const uint32_t tau = vars[0];
+      const uint32_t teq = vars[1];
+      // eq counts per warp list -> prefix (lists are in position order)
+      const uint32_t cb = samp[wid];
+      uint32_t ceq = 0;
+      for (int sl = lane; sl < static_cast<int>(cb); sl += 32) ceq += my_key[sl] == tau;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ceq += __shfl_xor_sync(0xffffffffu, ceq, o);
+      if (lane == 0) ws[wid] = ceq;
+      __syncthreads();
+      uint32_t eq_before = 0;
+      for (int w = 0; w < wid; ++w) eq_before += ws[w];
+      for (int base = 0; base < static_cast<int>(cb); base += 32) {
+        const int sl = base + lane;
+        const uint32_t key = sl < static_cast<int>(cb) ? my_key[sl] : 0u;
+        const bool eq = key == tau && key != 0u;
+        const uint32_t me = __ballot_sync(0xffffffffu, eq);
+        const uint32_t rank = eq_before + __popc(me & lt_mask);
+        if (key > tau || (eq && rank < teq)) {
+          const uint32_t pos = my_pos[sl];
+          atomicOr(&bmap[pos >> 5], 1u << (pos & 31u));
+        }
+        eq_before += __popc(me);
+      }
+      __syncthreads();
+      // ---- 5. emit the bitmap in position order
+      const int w0 = s0 >> 5;                              // this warp's words
+      const int w1 = s1 > s0 ? (s1 + 31) >> 5 : w0;      // (none for an empty segment)
+      const int per = (w1 - w0 + 31) / 32;                 // words per lane (contiguous)
+      const int l0 = min(w1, w0 + lane * per), l1 = min(w1, l0 + per);
+      uint32_t cnt = 0;
+      for (int wd = l0; wd < l1; ++wd) cnt += __popc(bmap[wd]);
+      uint32_t inc = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      if (lane == 31) ws[32 + wid] = inc;
+      __syncthreads();
+      uint32_t wbase = 0;
+      for (int w = 0; w < wid; ++w) wbase += ws[32 + w];
+      uint32_t out = wbase + inc - cnt;
+      int32_t* oi = p.out_idx + r * p.k;
+      float* os = p.out_score ? p.out_score + r * p.k : nullptr;
+      for (int wd = l0; wd < l1; ++wd) {
+        uint32_t bits = bmap[wd];
+        while (bits) {
+          const int b = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          const int i = wd * 32 + b;
+          int idx = i;
+          if (p.cand) {
+            const int slot = i / p.blk;
+            idx = __ldg(p.cand + r * p.n_slots + slot) * p.blk + (i - slot * p.blk);
+          }
+          if (out < static_cast<uint32_t>(k)) {  // holds by construction; guards the row
+            oi[out] = idx;
+            if (os) { const float x = src.get(i); os[out] = x == 0.f ? 0.f : x; }
+          }
+          ++out;
+        }
+      }
+      done = true;
+    }
+    __syncthreads();
+  }
+
+  if (!done) {
+    // ---- fallback: min / max and present count over the row, full value
+    // histogram, exact select, counting pass, ordered write pass
+    uint32_t nv = 0;
+    float vmin = INFINITY, vmax = -INFINITY;
+    for (int i = tid; i < n; i += TK_THREADS) {
+      const float x = src.get(i);
+      if (present(x)) { ++nv; vmin = fminf(vmin, x); vmax = fmaxf(vmax, x); }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -234,15 +492,13 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
       vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
       vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
     }
-    if (lane == 0) {
-      ws[wid] = nv;
-      fvars[wid] = vmin;
-      reinterpret_cast<float*>(ws)[32 + wid] = vmax;
-    }
+    if (lane == 0) { ws[wid] = nv; fvars[wid] = vmin; reinterpret_cast<float*>(ws)[32 + wid] = vmax; }
     __syncthreads();
     if (wid == 0) {
-      uint32_t a = ws[lane];
-      float mn = fvars[lane], mx = reinterpret_cast<float*>(ws)[32 + lane];
+      const bool has = lane < TK_WARPS;  // one partial per warp
+      uint32_t a = has ? ws[lane] : 0u;
+      float mn = has ? fvars[lane] : INFINITY;
+      float mx = has ? reinterpret_cast<float*>(ws)[32 + lane] : -INFINITY;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         a += __shfl_xor_sync(0xffffffffu, a, o);
@@ -258,53 +514,31 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
     __syncthreads();
     const uint32_t nvalid = vars[8];
     const float lo = reinterpret_cast<float*>(vars)[16], hi = reinterpret_cast<float*>(vars)[17];
-    const uint32_t keff = min(static_cast<uint32_t>(k), nvalid);
+    keff = min(static_cast<uint32_t>(k), nvalid);
     __syncthreads();
-
-    // select score > thr, plus the first take_eq scores == thr (-0 == +0 as floats)
-    float thr = -INFINITY;
-    uint32_t take_eq = 0;
     if (keff < nvalid) {
-      // ---- coarse: value-binned histogram
       const float span = hi - lo;
       const float scale = (span > 0.f && span < INFINITY) ? static_cast<float>(TK_BINS - 1) / span : 0.f;
       for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[i] = 0;
       if (tid == 0) vars[10] = 0;
       __syncthreads();
-#pragma unroll 2
-      for (int i = tid; i < n4; i += TK_THREADS) {
-        const float4 x = src.get4(i);
-        const float xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (present(xs[j])) atomicAdd(&hist[value_bin(xs[j], lo, scale)], 1u);
-      }
-      for (int i = 4 * n4 + tid; i < n; i += TK_THREADS) {
+      for (int i = tid; i < n; i += TK_THREADS) {
         const float x = src.get(i);
         if (present(x)) atomicAdd(&hist[value_bin(x, lo, scale)], 1u);
       }
       __syncthreads();
-      radix_pick<2>(hist, keff, ws, vars);
+      radix_pick<TK_BINS / TK_THREADS>(hist, keff, ws, vars);
       const int b = static_cast<int>(vars[0]);
       const uint32_t need = vars[1];
       const uint32_t cnt = hist[b];
       __syncthreads();
       if (cnt <= TK_CAND_CAP) {
-#pragma unroll 2
-        for (int i = tid; i < n4; i += TK_THREADS) {
-          const float4 x = src.get4(i);
-          const float xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (present(xs[j]) && value_bin(xs[j], lo, scale) == b)
-              cbuf[atomicAdd(&vars[10], 1u)] = score_key(xs[j]);
-        }
-        for (int i = 4 * n4 + tid; i < n; i += TK_THREADS) {
+        for (int i = tid; i < n; i += TK_THREADS) {
           const float x = src.get(i);
-          if (present(x) && value_bin(x, lo, scale) == b) cbuf[atomicAdd(&vars[10], 1u)] = score_key(x);
+          if (present(x) && value_bin(x, lo, scale) == b) ckey[atomicAdd(&vars[10], 1u)] = score_key(x);
         }
         __syncthreads();
-        exact_select(cbuf, src, static_cast<int>(cnt), need, hist, ws, vars);
+        exact_select(ckey, src, static_cast<int>(cnt), need, hist, ws, vars);
       } else {
         exact_select(nullptr, src, n, keff, hist, ws, vars);
       }
@@ -312,31 +546,15 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
       take_eq = vars[1];
       __syncthreads();
     }
-
-    // ---- ordered write-out. Warp w owns the contiguous segment [s0, s1);
-    // lane l of a 128-entry chunk owns entries 4l .. 4l+3 (one float4).
-    const int seg = ((n + TK_WARPS * 128 - 1) / (TK_WARPS * 128)) * 128;
-    const int s0 = min(n, wid * seg);
-    const int s1 = min(n, s0 + seg);
-    const bool v4 = vec;  // 16-byte aligned row: float4 chunks
-    auto load4 = [&](int i, float (&x)[4]) {
-      if (v4 && i + 3 < s1) {
-        const float4 f = src.get4(i >> 2);
-        x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
-      } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) x[j] = (i + j < s1) ? src.get(i + j) : -INFINITY;
-      }
-    };
+    // counting pass (per warp segment), prefix over the warps, ordered write
     uint32_t cgt = 0, ceq = 0;
-#pragma unroll 2
     for (int base = s0; base < s1; base += 128) {
-      float x[4];
-      load4(base + 4 * lane, x);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        cgt += x[j] > thr;
-        ceq += x[j] == thr && present(x[j]);
+        const int i = base + 32 * j + lane;
+        const float x = i < s1 ? src.get(i) : -INFINITY;
+        cgt += x > thr;
+        ceq += x == thr && present(x);
       }
     }
 #pragma unroll
@@ -346,67 +564,60 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_rows_kernel(const TopkPara
     }
     if (lane == 0) { ws[wid] = cgt; ws[32 + wid] = ceq; }
     __syncthreads();
-    if (wid == 0) {
-      const uint32_t g = ws[lane], e = ws[32 + lane];
-      uint32_t gi = g, ei = e;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, gi, o);
-        const uint32_t z = __shfl_up_sync(0xffffffffu, ei, o);
-        if (lane >= o) { gi += y; ei += z; }
-      }
-      ws[lane] = gi - g;
-      ws[32 + lane] = ei - e;
-    }
-    __syncthreads();
-    uint32_t run_gt = ws[wid], run_eq = ws[32 + wid];
+    uint32_t run_gt = 0, run_eq = 0;
+    for (int w = 0; w < wid; ++w) { run_gt += ws[w]; run_eq += ws[32 + w]; }
     __syncthreads();
     int32_t* oi = p.out_idx + r * p.k;
     float* os = p.out_score ? p.out_score + r * p.k : nullptr;
     for (int base = s0; base < s1; base += 128) {
-      const int i0 = base + 4 * lane;
-      float x[4];
-      load4(i0, x);
-      uint32_t ng = 0, ne = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        ng += x[j] > thr;
-        ne += x[j] == thr && present(x[j]);
-      }
-      // exclusive prefix over the lanes (entries of lower lanes come first)
-      uint32_t pg = ng, pe = ne;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, pg, o);
-        const uint32_t z = __shfl_up_sync(0xffffffffu, pe, o);
-        if (lane >= o) { pg += y; pe += z; }
-      }
-      uint32_t gb = run_gt + pg - ng, eb = run_eq + pe - ne;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const bool gt = x[j] > thr;
-        const bool eq = x[j] == thr && present(x[j]);
-        if (gt || (eq && eb < take_eq)) {
+        const int i = base + 32 * j + lane;
+        const float x = i < s1 ? src.get(i) : -INFINITY;
+        const bool gt = x > thr;
+        const bool eq = x == thr && present(x);
+        const uint32_t mg = __ballot_sync(0xffffffffu, gt);
+        const uint32_t me = __ballot_sync(0xffffffffu, eq);
+        const uint32_t gb = run_gt + __popc(mg & lt_mask);
+        const uint32_t eb = run_eq + __popc(me & lt_mask);
+        if ((gt || (eq && eb < take_eq)) && gb + min(eb, take_eq) < static_cast<uint32_t>(k)) {
           const uint32_t pos = gb + min(eb, take_eq);
-          const int i = i0 + j;
           int idx = i;
           if (p.cand) {
             const int slot = i / p.blk;
             idx = __ldg(p.cand + r * p.n_slots + slot) * p.blk + (i - slot * p.blk);
           }
           oi[pos] = idx;
-          if (os) os[pos] = x[j] == 0.f ? 0.f : x[j];
+          if (os) os[pos] = x == 0.f ? 0.f : x;
         }
-        gb += gt;
-        eb += eq;
+        run_gt += __popc(mg);
+        run_eq += __popc(me);
       }
-      run_gt += __shfl_sync(0xffffffffu, pg, 31);
-      run_eq += __shfl_sync(0xffffffffu, pe, 31);
     }
-    for (int j = static_cast<int>(keff) + tid; j < k; j += TK_THREADS) {
-      oi[j] = -1;
-      if (os) os[j] = -INFINITY;
+  }
+  int32_t* oi = p.out_idx + r * p.k;
+  float* os = p.out_score ? p.out_score + r * p.k : nullptr;
+  for (int j = static_cast<int>(keff) + tid; j < k; j += TK_THREADS) {
+    oi[j] = -1;
+    if (os) os[j] = -INFINITY;
+  }
+}
+
+__global__ void __launch_bounds__(TK_THREADS, TK_CTAS_PER_SM) topk_rows_kernel(const TopkParams p) {
+  extern __shared__ uint32_t tk_smem[];
+  for (long long r = blockIdx.x; r < p.rows; r += gridDim.x) {
+    const int t = static_cast<int>(r % p.T);
+    long long nl = p.Lrow;
+    if (p.pstride > 0) {
+      nl = (p.q_offset + t) / p.pstride + 1;
+      if (nl > p.Lrow) nl = p.Lrow;
+      if (nl < 0) nl = 0;
     }
+    const int n = static_cast<int>(nl);
+    const float* row = p.scores + r * p.ld;
+    const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15u) == 0);
+    if (n <= TK_SMEM_ROW && vec) topk_row<true>(p, tk_smem, r, n, row);
+    else topk_row<false>(p, tk_smem, r, n, row);
     __syncthreads();
   }
 }
