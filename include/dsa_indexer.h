@@ -28,13 +28,13 @@
  *     call that passes validation clears it (stream-ordered); kernels set it
  *     if a bounded wait gave up. dsa_device_status() synchronises the stream
  *     and reports it. Zero a new workspace once before its first status read.
- *   - The workspace must be 256-byte aligned; q, k, w and q_scale 16-byte
- *     aligned; k_scale 4-byte aligned.
+ *   - The workspace must be 256-byte aligned; q, k, w, q_scale and k_scale
+ *     16-byte aligned.
  *   - Calls that share a workspace must not overlap in time (use one stream).
  *
  * Supported shapes: d in {64, 128}; bf16 H in {8, 16, 32, 64};
- * FP8 e4m3 (decode): d = 128, H in {32, 64}. Other shapes return
- * DSA_ERR_UNSUPPORTED.
+ * FP8 e4m3 (decode): d = 128, H in {32, 64}, L a multiple of 4. Other shapes
+ * return DSA_ERR_UNSUPPORTED.
  */
 #ifndef DSA_INDEXER_H
 #define DSA_INDEXER_H

@@ -182,7 +182,8 @@ dsa_status validate(const dsa_indexer_args* a, bool bf16_only) {
   const bool fp8 = a->qk_dtype == DSA_FP8_E4M3;
   if (fp8) {
     if (!a->q_scale || !a->k_scale) return DSA_ERR_ARG;
-    if (!aligned(a->q_scale, 16) || !aligned(a->k_scale, 4)) return DSA_ERR_ARG;
+    if (!aligned(a->q_scale, 16) || !aligned(a->k_scale, 16)) return DSA_ERR_ARG;
+    if (a->L % 4 != 0) return DSA_ERR_UNSUPPORTED;  // key-scale rows are copied in 16-byte units
   }
   if (a->q_offset > (1LL << 40)) return DSA_ERR_ARG;
   if (static_cast<long long>(a->batch) * a->T * a->H > INT_MAX ||

@@ -96,12 +96,16 @@ struct ScoreCfg {
   // shared memory layout (offsets from a 1024-aligned base)
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_K = Q_BYTES;
-  static constexpr int SMEM_BAR = SMEM_K + NSTAGE * K_BYTES;
+  // FP8: the per-key dequant scales of each stage's 128 keys ride with the tile
+  static constexpr int KSC_BYTES = (ELEM == 1 && !ROUTER && !GATHER) ? KROWS * 4 : 0;
+  static constexpr int SMEM_KSC = SMEM_K + NSTAGE * K_BYTES;
+  static constexpr int SMEM_BAR = SMEM_KSC + NSTAGE * KSC_BYTES;
   static constexpr int NBAR = 2 * NSTAGE + 7;
   static constexpr int SMEM_USED = SMEM_BAR + NBAR * 8 + 16;
   // Pad to more than half an SM so two CTAs never share an SM's TMEM.
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024 < 120 * 1024) ? 120 * 1024 : SMEM_USED + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static_assert(!KSC_BYTES || SPLIT_TILES, "key scales are read by one 4-warp set per tile");
 };
 
 // Iterates this CTA's (group, tile) pairs. Every thread runs its own copy;
@@ -110,23 +114,32 @@ template <class C>
 struct TileSched {
   int gpb, G;
   int g, j, nt;
+  int b, tg;        // sequence and query group within it (kept incrementally)
   long long left;   // tiles left (flat split)
   bool first, last, done;
 
-  __device__ __forceinline__ int ntile(const ScoreParams& p, int grp) const {
-    const int tg = grp % gpb;
+  // key tiles of query group tg (the same for every sequence)
+  __device__ __forceinline__ int ntile_tg(const ScoreParams& p, int tgi) const {
     if (C::GATHER) return (p.n_compact + C::KROWS - 1) / C::KROWS;
-    const int t_last = min(p.T, (tg + 1) * C::QPT) - 1;
+    const int t_last = min(p.T, (tgi + 1) * C::QPT) - 1;
     const long long pos = p.q_offset + t_last;
-    long long nk = pos / p.pstride + 1;
+    long long nk;
+    if (p.pstride == 1) nk = pos + 1;
+    else if (pos < 0x7fffffffLL) nk = static_cast<unsigned>(pos) / static_cast<unsigned>(p.pstride) + 1;
+    else nk = pos / p.pstride + 1;
     if (nk > p.Lk) nk = p.Lk;
     return static_cast<int>((nk + C::KROWS - 1) / C::KROWS);
   }
+  __device__ __forceinline__ int ntile(const ScoreParams& p, int grp) const {
+    return ntile_tg(p, grp % gpb);
+  }
 
+  // All 32 lanes of the warp call init together (warp-cooperative scans).
   __device__ __forceinline__ void init(const ScoreParams& p) {
     gpb = (p.T + C::QPT - 1) / C::QPT;
     G = p.batch * gpb;
     done = false;
+    const int lane = threadIdx.x & 31;
     if (C::ROUTER) {
       left = 0;
       g = blockIdx.x;
@@ -134,21 +147,42 @@ struct TileSched {
       if (g >= G) { done = true; return; }
       j = 0;
     } else {
+      // total tiles: lane l sums groups l, l+32, ...
       long long W = 0;
-      for (int q = 0; q < G; ++q) W += ntile(p, q);
+      for (int q = lane; q < G; q += 32) W += ntile(p, q);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
       const long long b0 = W * blockIdx.x / gridDim.x;
       const long long b1 = W * (blockIdx.x + 1) / gridDim.x;
       left = b1 - b0;
       if (left <= 0) { done = true; return; }
+      // first group whose tiles reach past b0: scan 32 groups at a time
       long long acc = 0;
-      g = 0;
-      for (;; ++g) {
-        nt = ntile(p, g);
-        if (acc + nt > b0) break;
-        acc += nt;
+      for (int base = 0;; base += 32) {
+        const int q = base + lane;
+        const long long nq = q < G ? ntile(p, q) : 0;
+        long long inc = nq;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const long long y = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += y;
+        }
+        const long long tot = __shfl_sync(0xffffffffu, inc, 31);
+        if (acc + tot > b0) {
+          const uint32_t m = __ballot_sync(0xffffffffu, acc + inc > b0);
+          const int src = __ffs(m) - 1;
+          const long long inc_s = __shfl_sync(0xffffffffu, inc, src);
+          const long long nq_s = __shfl_sync(0xffffffffu, nq, src);
+          g = base + src;
+          j = static_cast<int>(b0 - (acc + inc_s - nq_s));
+          nt = static_cast<int>(nq_s);
+          break;
+        }
+        acc += tot;
       }
-      j = static_cast<int>(b0 - acc);
     }
+    b = g / gpb;
+    tg = g - b * gpb;
     first = true;
     last = (j == nt - 1) || (!C::ROUTER && left == 1);
   }
@@ -159,6 +193,8 @@ struct TileSched {
         g += gridDim.x;
         while (g < G && (nt = ntile(p, g)) == 0) g += gridDim.x;
         if (g >= G) { done = true; return; }
+        b = g / gpb;
+        tg = g - b * gpb;
         j = 0;
         first = true;
       } else {
@@ -168,7 +204,11 @@ struct TileSched {
     } else {
       if (--left == 0) { done = true; return; }
       if (++j == nt) {
-        do { ++g; nt = ntile(p, g); } while (nt == 0);
+        do {
+          ++g;
+          if (++tg == gpb) { tg = 0; ++b; }
+          nt = ntile_tg(p, tg);
+        } while (nt == 0);
         j = 0;
         first = true;
       } else {
@@ -218,7 +258,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NSTAGE; ++i) {
       mbar_init(full(i), C::GATHER ? 32 : 1);
-      mbar_init(empty(i), 1);
+      // FP8: a stage is free once its MMAs are done and the epilogue warps of
+      // its tile have read the stage's key scales
+      mbar_init(empty(i), C::KSC_BYTES ? 1 + 4 : 1);
     }
     mbar_init(qfull, 1);
     mbar_init(qempty, 1);
@@ -251,8 +293,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint32_t it = 0, gq = 0;
     bool ok = true;
     for (; !s.done; s.next(p), ++it) {
-      const int b = s.g / s.gpb;
-      const int tg = s.g % s.gpb;
+      const int b = s.b;
+      const int tg = s.tg;
       const bool mine = C::GATHER ? (static_cast<int>(it % C::NPROD) == pw) : true;
       if (s.first) {
         // The query tile is always loaded by warp 0, group by group in order.
@@ -277,12 +319,18 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (lane == 0) {
           if (!mbar_wait(empty(stage), ph ^ 1u, p.err)) { ok = false; }
           else {
-            mbar_arrive_expect_tx(full(stage), C::K_BYTES);
             const int krow0 = b * p.Lk + s.j * C::KROWS;
+            // scales of the tile's keys that exist (Lk % 4 == 0: 16-byte multiples)
+            const uint32_t ksc_bytes =
+                C::KSC_BYTES ? static_cast<uint32_t>(min(C::KROWS, p.Lk - s.j * C::KROWS)) * 4u : 0u;
+            mbar_arrive_expect_tx(full(stage), C::K_BYTES + ksc_bytes);
 #pragma unroll
             for (int kb = 0; kb < C::KBLK; ++kb)
               tma_load_2d(s_k + stage * C::K_BYTES + kb * C::KROWS * 128, &tm_k, full(stage),
                           kb * (128 / C::ELEM), krow0);
+            if (C::KSC_BYTES)
+              bulk_load(s_base + C::SMEM_KSC + stage * C::KSC_BYTES, p.k_scale + krow0, ksc_bytes,
+                        full(stage));
           }
         }
       } else {
@@ -382,8 +430,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float racc = 0.f;                          // router partial sum
     uint32_t it = 0;
     for (; !s.done; s.next(p), ++it) {
-      const int b = s.g / s.gpb;
-      const int tg = s.g % s.gpb;
+      const int b = s.b;
+      const int tg = s.tg;
       const int buf = static_cast<int>(it & 1u);
       const bool mine = C::SPLIT_TILES ? (buf == set) : true;
       if (mine) {
@@ -426,6 +474,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #endif
           const int q0 = C::SPLIT_TILES ? 0 : set * QH;          // first query (in group)
           const int key = s.j * C::KROWS + row;                  // key row / compact position
+          float ks = 1.f;                                        // FP8 key dequant scale
+          if constexpr (C::KSC_BYTES != 0) {
+            const int stage = static_cast<int>(it % C::NSTAGE);
+            ks = reinterpret_cast<const float*>(smem + C::SMEM_KSC + stage * C::KSC_BYTES)[row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty(stage));
+          }
           const long long rbase = static_cast<long long>(b) * p.T + tg * C::QPT + q0;
           // head weights of this thread's columns are contiguous in w when every
           // query of the half-group exists
@@ -541,12 +596,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               p.out[r * p.ldo + key] = tok >= 0 ? accq[0] : -INFINITY;
             }
           } else if (key < p.Lk) {
-            const float ks = (C::ELEM == 1) ? __ldg(p.k_scale + static_cast<long long>(b) * p.Lk + key) : 1.f;
+            // query q0+ql sees this key iff key * pstride <= q_offset + t0 + ql
+            const int t0 = tg * C::QPT + q0;
+            const long long e = static_cast<long long>(key) * p.pstride - (p.q_offset + t0);
+            float* orow = p.out + rbase * p.ldo + key;
 #pragma unroll
             for (int ql = 0; ql < QH; ++ql) {
-              const int t = tg * C::QPT + q0 + ql;
-              if (t < p.T && static_cast<long long>(key) * p.pstride <= p.q_offset + t)
-                p.out[(rbase + ql) * p.ldo + key] = ks * accq[ql];
+              if (t0 + ql < p.T && e <= ql) orow[ql * p.ldo] = ks * accq[ql];
             }
           }
         }
