@@ -95,7 +95,7 @@ dsa_status launch_score(const ScoreParams& p, const void* q, long long q_rows, c
   }
   CUtensorMap tq, tk;
   if (!make_tmap(&tq, q, C::ELEM == 1, C::D, q_rows, C::QROWS)) return DSA_ERR_CUDA;
-  if (C::GATHER) tk = tq;
+  if (C::GATHER && !p.blk_tma) tk = tq;
   else if (!make_tmap(&tk, k, C::ELEM == 1, C::D, k_rows, C::KROWS)) return DSA_ERR_CUDA;
   int grid = num_sms();
   if (C::ROUTER) {
@@ -147,12 +147,16 @@ dsa_status run_router(int D, int H, const ScoreParams& p, const void* q, long lo
 }
 
 // Gathered re-scoring (MISA-dagger candidates, HISA surviving blocks).
-dsa_status run_gather(int D, int H, const ScoreParams& p, const void* q, long long q_rows,
+// When blk is a multiple of 128, every 128-row tile is one contiguous key
+// run and is fetched with TMA; otherwise rows are gathered with cp.async.
+dsa_status run_gather(int D, int H, ScoreParams p, const void* q, long long q_rows,
                       cudaStream_t st) {
+  p.blk_tma = (p.blk % 128 == 0) ? 1 : 0;
+  const long long k_rows = static_cast<long long>(p.batch) * p.L_tok;
   if (D == 128 && H == 64)
-    return launch_score<ScoreCfg<2, 128, 64, 1, ScoreMode::kGather, 4>>(p, q, q_rows, nullptr, 0, st);
+    return launch_score<ScoreCfg<2, 128, 64, 1, ScoreMode::kGather, 4>>(p, q, q_rows, p.kg, k_rows, st);
   if (D == 128 && H == 32)
-    return launch_score<ScoreCfg<2, 128, 32, 1, ScoreMode::kGather, 4>>(p, q, q_rows, nullptr, 0, st);
+    return launch_score<ScoreCfg<2, 128, 32, 1, ScoreMode::kGather, 4>>(p, q, q_rows, p.kg, k_rows, st);
   return DSA_ERR_UNSUPPORTED;
 }
 

@@ -51,6 +51,7 @@ struct ScoreParams {
   const __nv_bfloat16* kg;  // gather mode: keys [batch*L_tok, D]
   const int* cand;          // gather mode: [batch*T, n_slots] block / token ids, -1 = none
   int n_slots, blk, n_compact;  // compact position c -> cand[c / blk] * blk + c % blk
+  int blk_tma;              // gather mode, blk % 128 == 0: a tile is one contiguous key run (TMA)
   unsigned* err;            // device error word
 };
 
@@ -257,7 +258,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NSTAGE; ++i) {
-      mbar_init(full(i), C::GATHER ? 32 : 1);
+      mbar_init(full(i), (C::GATHER && !p.blk_tma) ? 32 : 1);
       // FP8: a stage is free once its MMAs are done and the epilogue warps of
       // its tile have read the stage's key scales
       mbar_init(empty(i), C::KSC_BYTES ? 1 + 4 : 1);
@@ -277,7 +278,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   }
   if (threadIdx.x == 32 * C::MMA_WARP + 1) {
     tma_prefetch_desc(&tm_q);
-    if (!C::GATHER) tma_prefetch_desc(&tm_k);
+    if (!C::GATHER || p.blk_tma) tma_prefetch_desc(&tm_k);
   }
   tc_fence_before();
   __syncthreads();
@@ -295,7 +296,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (; !s.done; s.next(p), ++it) {
       const int b = s.b;
       const int tg = s.tg;
-      const bool mine = C::GATHER ? (static_cast<int>(it % C::NPROD) == pw) : true;
+      // gathers: tiles round-robin over the producer warps (each owns its
+      // stages); contiguous block tiles (TMA): warp 0 loads every tile
+      const bool mine = C::GATHER ? (p.blk_tma ? pw == 0 : static_cast<int>(it % C::NPROD) == pw) : true;
       if (s.first) {
         // The query tile is always loaded by warp 0, group by group in order.
         if (pw == 0 && lane == 0) {
@@ -315,7 +318,28 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (!mine) continue;
       const int stage = static_cast<int>(it % C::NSTAGE);
       const uint32_t ph = (it / C::NSTAGE) & 1u;
-      if (!C::GATHER) {
+      if (C::GATHER && p.blk_tma) {
+        // the tile's 128 compact positions are tokens cand[slot] * blk + [c0 % blk, +128)
+        if (lane == 0) {
+          if (!mbar_wait(empty(stage), ph ^ 1u, p.err)) { ok = false; }
+          else {
+            const long long r = static_cast<long long>(b) * p.T + tg;
+            const int c0 = s.j * C::KROWS;
+            const int slot = c0 / p.blk;
+            const int cb = c0 < p.n_compact ? __ldg(p.cand + r * p.n_slots + slot) : -1;
+            if (cb >= 0) {
+              const long long tok0 = static_cast<long long>(cb) * p.blk + (c0 - slot * p.blk);
+              mbar_arrive_expect_tx(full(stage), C::K_BYTES);
+#pragma unroll
+              for (int kb = 0; kb < C::KBLK; ++kb)
+                tma_load_2d(s_k + stage * C::K_BYTES + kb * C::KROWS * 128, &tm_k, full(stage),
+                            kb * (128 / C::ELEM), static_cast<int>(b * p.L_tok + tok0));
+            } else {
+              mbar_arrive(full(stage));  // no keys: the epilogue writes -inf for the whole tile
+            }
+          }
+        }
+      } else if (!C::GATHER) {
         if (lane == 0) {
           if (!mbar_wait(empty(stage), ph ^ 1u, p.err)) { ok = false; }
           else {
@@ -377,7 +401,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // flight before the CTA releases its shared memory. cp.async gathers
       // were already waited for before their arrive.
       if (pw == 0 && gq > 0) mbar_drain(qfull, (gq - 1) & 1u);
-      if (!C::GATHER) {
+      if (!C::GATHER || p.blk_tma) {
         const uint32_t lo = it > C::NSTAGE ? it - C::NSTAGE : 0;
         for (uint32_t i = lo; i < it; ++i) mbar_drain(full(i % C::NSTAGE), (i / C::NSTAGE) & 1u);
       }

@@ -56,7 +56,9 @@ constexpr int TK_CTAS_PER_SM = 1;
 constexpr int TK_WARPS = TK_THREADS / 32;
 constexpr int TK_BINS = 2048;
 constexpr int TK_SMEM_ROW = 32768;   // rows up to this length are staged in shared memory
-constexpr int TK_LIST = 128;         // band candidates per warp segment
+constexpr int TK_LIST = 128;         // band candidates per warp segment (staged rows)
+// rows that are not staged keep their candidate lists in the unused stage area
+constexpr int TK_LIST_LONG = TK_SMEM_ROW / (2 * (TK_THREADS / 32));
 constexpr int TK_CAND_CAP = TK_WARPS * TK_LIST;
 constexpr int TK_SAMPLE_MAX = 4096;  // sampled scores per row
 constexpr int TK_BITMAP_WORDS = 4096;
@@ -230,6 +232,10 @@ __device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem,
   const uint32_t lt_mask = (1u << lane) - 1u;
   const uint32_t s_stage = smem_u32(stage);
   const RowSrc<STAGED> src{s_stage, row};
+  // per-warp band candidate lists (keys, positions)
+  constexpr int LIST = STAGED ? TK_LIST : TK_LIST_LONG;
+  uint32_t* lkey = STAGED ? ckey : reinterpret_cast<uint32_t*>(stage);
+  uint32_t* lpos = STAGED ? cpos : reinterpret_cast<uint32_t*>(stage) + TK_WARPS * TK_LIST_LONG;
   const int k = p.k;
   // warp segments (multiples of 128 entries)
   const int seg = ((n + TK_WARPS * 128 - 1) / (TK_WARPS * 128)) * 128;
@@ -358,18 +364,18 @@ __device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem,
     // ---- 3. band pass: bitmap words of "> t_hi", per-warp candidate lists.
     // Above / present counts are per lane and reduced once after the pass.
     uint32_t c_above = 0, c_band = 0, c_present = 0;
-    uint32_t* my_key = ckey + wid * TK_LIST;
-    uint32_t* my_pos = cpos + wid * TK_LIST;
-    for (int base = s0; base < s1; base += 128) {
-      // the chunk's four loads are issued before any of their uses
-      float xv[4];
+    uint32_t* my_key = lkey + wid * LIST;
+    uint32_t* my_pos = lpos + wid * LIST;
+    for (int base = s0; base < s1; base += 256) {
+      // the loads of two 128-entry chunks are issued before any of their uses
+      float xv[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const int i = base + 32 * j + lane;
         xv[j] = i < s1 ? src.get(i) : -INFINITY;
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const int i = base + 32 * j + lane;
         const float x = xv[j];
         const bool up = x > t_hi;
@@ -382,7 +388,7 @@ __device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem,
         if (mb) {
           if (band) {
             const uint32_t slot = c_band + __popc(mb & lt_mask);
-            if (slot < TK_LIST) { my_key[slot] = score_key(x); my_pos[slot] = static_cast<uint32_t>(i); }
+            if (slot < LIST) { my_key[slot] = score_key(x); my_pos[slot] = static_cast<uint32_t>(i); }
           }
           c_band += __popc(mb);
         }
@@ -393,7 +399,7 @@ __device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem,
       c_above += __shfl_xor_sync(0xffffffffu, c_above, o);
       c_present += __shfl_xor_sync(0xffffffffu, c_present, o);
     }
-    for (int sl = static_cast<int>(c_band) + lane; sl < TK_LIST; sl += 32) my_key[sl] = 0u;  // empty slots
+    for (int sl = static_cast<int>(c_band) + lane; sl < LIST; sl += 32) my_key[sl] = 0u;  // empty slots
     if (lane == 0) { ws[wid] = c_above; ws[32 + wid] = c_present; samp[wid] = c_band; }
     __syncthreads();
     uint32_t above_all = 0, nvalid = 0, nc = 0, cmax = 0;
@@ -404,11 +410,11 @@ __device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem,
       cmax = max(cmax, samp[w]);
     }
     keff = min(static_cast<uint32_t>(k), nvalid);
-    const bool band_ok = keff < nvalid && cmax <= TK_LIST && above_all < keff && keff <= above_all + nc;
+    const bool band_ok = keff < nvalid && cmax <= LIST && above_all < keff && keff <= above_all + nc;
     __syncthreads();
     if (band_ok) {
       // ---- 4. exact select among the candidates
-      exact_select(ckey, src, TK_CAND_CAP, keff - above_all, hist, ws, vars);
+      exact_select(lkey, src, TK_WARPS * LIST, keff - above_all, hist, ws, vars);
       const uint32_t tau = vars[0];
       const uint32_t teq = vars[1];
       // eq counts per warp list -> prefix (lists are in position order)
