@@ -156,6 +156,26 @@ class Runner:
         return None, None, None, None
 
 
+def aggregate_ranks(total_ms: float, units_per_rank_step: int, steps: int, world: int, reduce_max=None):
+    """Whole-job throughput of independent replicas: every rank processes
+    `units_per_rank_step` units per step; the job takes as long as its slowest
+    rank. reduce_max(x) returns the max of x over ranks (identity on one rank).
+    Returns (max total ms, aggregate units per second)."""
+    t = reduce_max(total_ms) if (reduce_max is not None and world > 1) else total_ms
+    return t, world * units_per_rank_step * steps / (t / 1e3)
+
+
+def dist_max(dist, device):
+    """reduce_max over the default process group (NCCL on GPUs, gloo on CPU)."""
+    import torch
+
+    def f(x):
+        v = torch.tensor([float(x)], dtype=torch.float64, device=device)
+        dist.all_reduce(v, op=dist.ReduceOp.MAX)
+        return float(v.item())
+    return f
+
+
 def l2_flush(buf):
     buf.add_(1)
 
@@ -356,13 +376,10 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop() if sampler else None
-    total_ms = float(sum(times))
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    rmax = dist_max(dist, "cuda") if world > 1 else None
+    total_ms, pairs_per_s = aggregate_ranks(float(sum(times)), r.pairs, args.steps, world, rmax)
     ms_per_step = total_ms / args.steps
-    value = world * r.pairs * args.steps / (total_ms / 1e3) / 1e9
+    value = pairs_per_s / 1e9
     assert r.ix.device_status() == 0, "device wait timed out"
 
     # ---- dominant kernel alone (roofline)
@@ -411,12 +428,8 @@ def main():
     torch.cuda.synchronize()
     barrier()
     et = time_steps(e2e_step, args.steps, torch, flush)
-    e_ms = float(sum(et))
-    if world > 1:
-        t = torch.tensor([e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
-    e2e_value = world * r.pairs * args.steps / (e_ms / 1e3) / 1e9
+    e_ms, e_pairs_per_s = aggregate_ranks(float(sum(et)), r.pairs, args.steps, world, rmax)
+    e2e_value = e_pairs_per_s / 1e9
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
     cpu = None

@@ -128,6 +128,19 @@ DSA_EXPORT dsa_status indexer_score_topk_noalloc(const dsa_indexer_args* a, int 
 DSA_EXPORT dsa_status indexer_scores(const dsa_indexer_args* a, float* out_scores, long long ld,
                           void* workspace, size_t ws_bytes, void* stream);
 
+/* Gathered re-scoring (the MISA-dagger re-score and HISA token stages alone):
+ * for every query (row r = b*T + t) and compact position c < n_slots * blk,
+ * with token s = cand[r * n_slots + c / blk] * blk + c % blk,
+ *     out[r * ld + c] = I[t, s]  (all H heads)  if cand[...] >= 0, s < L, s <= q_offset + t,
+ *     out[r * ld + c] = -inf                      otherwise.
+ * blk = 1: token candidates; blk = B: candidate blocks of B tokens (a block
+ * size that is a multiple of 128 fetches whole blocks with TMA).
+ *   cand [batch*T, n_slots] int32; out [batch*T, ld] fp32, ld >= n_slots * blk.
+ * bf16 only; d = 128, H in {32, 64}. Workspace: the 256-byte header only. */
+DSA_EXPORT dsa_status indexer_score_gathered(const dsa_indexer_args* a, const int32_t* cand,
+                                             int n_slots, int blk, float* out, long long ld,
+                                             void* workspace, size_t ws_bytes, void* stream);
+
 /* Stage 2 alone: per-row top-k of fp32 scores [rows, ld]. Row r belongs to
  * query t = r % T; its candidates are positions 0 .. n_r - 1 with
  *   n_r = clamp((q_offset + t) / pstride + 1, 0, row_len)   if pstride > 0,

@@ -46,6 +46,8 @@ _SIGS = {
     "indexer_score_topk": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "indexer_score_topk_noalloc": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P]),
     "indexer_scores": (ctypes.c_int, [_P, _P, ctypes.c_longlong, _P, ctypes.c_size_t, _P]),
+    "indexer_score_gathered": (ctypes.c_int, [_P, _P, ctypes.c_int, ctypes.c_int, _P,
+                                              ctypes.c_longlong, _P, ctypes.c_size_t, _P]),
     "indexer_topk_rows": (ctypes.c_int, [_P, ctypes.c_longlong, ctypes.c_longlong, ctypes.c_int,
                                          ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          _P, ctypes.c_int, ctypes.c_int, _P, _P, _P,
@@ -158,6 +160,13 @@ def indexer_scores(args: IndexerArgs, out_scores: torch.Tensor, ld: int, workspa
     _check("indexer_scores",
            lib().indexer_scores(ctypes.byref(args), _ptr(out_scores), ld, _ptr(workspace),
                                 workspace.numel(), _stream_ptr(stream)))
+
+
+def indexer_score_gathered(args: IndexerArgs, cand: torch.Tensor, n_slots: int, blk: int,
+                           out: torch.Tensor, ld: int, workspace: torch.Tensor, stream=None):
+    _check("indexer_score_gathered",
+           lib().indexer_score_gathered(ctypes.byref(args), _ptr(cand), n_slots, blk, _ptr(out), ld,
+                                        _ptr(workspace), workspace.numel(), _stream_ptr(stream)))
 
 
 def indexer_topk_rows(scores: torch.Tensor, rows: int, ld: int, T: int, q_offset: int, pstride: int,

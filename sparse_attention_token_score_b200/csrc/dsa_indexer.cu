@@ -306,6 +306,29 @@ dsa_status indexer_scores(const dsa_indexer_args* a, float* out, long long ld, v
   return run_scores_bf16(a->d, a->H, p, a->q, q_rows, a->k, k_rows, st);
 }
 
+dsa_status indexer_score_gathered(const dsa_indexer_args* a, const int32_t* cand, int n_slots,
+                                  int blk, float* out, long long ld, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  DSA_TRY(validate(a, true));
+  if (!cand || !out || n_slots < 1 || blk < 1 || !aligned(cand, 4) || !aligned(out, 4))
+    return DSA_ERR_ARG;
+  if (static_cast<long long>(n_slots) * blk > INT_MAX / 2) return DSA_ERR_UNSUPPORTED;
+  if (ld < static_cast<long long>(n_slots) * blk) return DSA_ERR_ARG;
+  if (a->d != 128 || (a->H != 32 && a->H != 64)) return DSA_ERR_UNSUPPORTED;
+  DSA_TRY(check_ws(ws, ws_bytes, kHdr));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DSA_TRY(clear_status(ws, st));
+  ScoreParams pg = base_params(a, static_cast<unsigned*>(ws));
+  pg.out = out;
+  pg.ldo = ld;
+  pg.kg = static_cast<const __nv_bfloat16*>(a->k);
+  pg.cand = cand;
+  pg.n_slots = n_slots;
+  pg.blk = blk;
+  pg.n_compact = n_slots * blk;
+  return run_gather(a->d, a->H, pg, a->q, static_cast<long long>(a->batch) * a->T * a->H, st);
+}
+
 dsa_status indexer_topk_rows(const float* scores, long long rows, long long ld, int T,
                              long long q_offset, int pstride, int row_len, int topk,
                              const int32_t* cand, int n_slots, int blk, int32_t* out_idx,

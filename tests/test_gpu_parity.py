@@ -177,19 +177,24 @@ def _heads_check(gpu_heads, aff, h, what):
         check_selection(gpu_heads[i], np.arange(aff.shape[1]), aff[i], aff[i], h, what=f"{what} heads {i}")
 
 
-def _misa_check(inp, block, h, topk, kprime, queries, what):
+def _misa_check(inp, block, h, topk, kprime, queries, what, batches=(0,)):
     ix = _indexer(inp)
-    idx, sc, heads, cand = ix.misa(block, h, topk, kprime, with_score=True, with_heads=True,
+    IDX, SC, HEADS, CAND = ix.misa(block, h, topk, kprime, with_score=True, with_heads=True,
                                    with_cand=True)
     assert ix.device_status() == 0
-    idx, sc, heads = idx.cpu().numpy()[0], sc.cpu().numpy()[0], heads.cpu().numpy()[0]
-    cand = cand.cpu().numpy()[0] if cand is not None else None
+    for b in batches:
+        _misa_check_one(inp, block, h, topk, kprime, queries, f"{what} b={b}", b,
+                        IDX.cpu().numpy()[b], SC.cpu().numpy()[b], HEADS.cpu().numpy()[b],
+                        CAND.cpu().numpy()[b] if CAND is not None else None)
+
+
+def _misa_check_one(inp, block, h, topk, kprime, queries, what, b, idx, sc, heads, cand):
     qs = np.asarray(queries)
-    free = oracle.misa(inp, block, h, topk, kprime=0, queries=qs)
+    free = oracle.misa(inp, block, h, topk, kprime=0, queries=qs, b=b)
     _heads_check(heads[qs], free["affinity"], h, what)
     # conditioned on the GPU's heads (and candidates)
     cond = oracle.misa(inp, block, h, topk, kprime=kprime, queries=qs, heads_given=heads[qs],
-                       cand_given=None if cand is None else cand[qs])
+                       cand_given=None if cand is None else cand[qs], b=b)
     for i, t in enumerate(qs):
         V = min(inp.q_offset + t + 1, inp.L)
         if kprime == 0:
@@ -218,6 +223,19 @@ def test_misa_ragged_blocks():
     # L not a multiple of the block, queries near the start (few visible blocks)
     inp = wl.prefill_inputs(50, 1000, 32, 128, q_offset=30, seed=14)
     _misa_check(inp, block=48, h=16, topk=64, kprime=200, queries=range(50), what="misa ragged")
+
+
+def test_misa_batched_h32_dagger():
+    # router with 4 queries x 32 heads per row tile, routed scoring with h = 16
+    inp = wl.prefill_inputs(20, 2000, 32, 128, q_offset=1980, seed=26, batch=2)
+    _misa_check(inp, block=64, h=16, topk=50, kprime=300, queries=range(20), what="misa b2",
+                batches=(0, 1))
+
+
+def test_misa_h8_head_dim_64():
+    # router with 16 queries x 8 heads per row tile, d = 64, plain MISA
+    inp = wl.prefill_inputs(40, 1500, 8, 64, q_offset=1460, seed=27)
+    _misa_check(inp, block=32, h=8, topk=64, kprime=0, queries=range(40), what="misa h8 d64")
 
 
 def test_misa_all_heads_equals_dense_gpu():
@@ -255,17 +273,22 @@ def test_misa_plain_config_sampled():
 
 
 # ------------------------------------------------------------------ HISA
-def _hisa_check(inp, block, m, topk, queries, what):
+def _hisa_check(inp, block, m, topk, queries, what, batches=(0,)):
     ix = _indexer(inp)
-    idx, sc, blocks = ix.hisa(block, m, topk, with_score=True, with_blocks=True)
+    IDX, SC, BLOCKS = ix.hisa(block, m, topk, with_score=True, with_blocks=True)
     assert ix.device_status() == 0
-    idx, sc, blocks = idx.cpu().numpy()[0], sc.cpu().numpy()[0], blocks.cpu().numpy()[0]
+    for b in batches:
+        _hisa_check_one(inp, block, m, topk, queries, f"{what} b={b}", b, IDX.cpu().numpy()[b],
+                        SC.cpu().numpy()[b], BLOCKS.cpu().numpy()[b])
+
+
+def _hisa_check_one(inp, block, m, topk, queries, what, b, idx, sc, blocks):
     qs = np.asarray(queries)
-    free = oracle.hisa(inp, block, m, topk, queries=qs)
+    free = oracle.hisa(inp, block, m, topk, queries=qs, b=b)
     for i, t in enumerate(qs):
         s, c = free["block_scores"][i], free["block_cond"][i]
         check_selection(blocks[t], np.arange(s.size), s, c, m, what=f"{what} blocks t={t}")
-    cond = oracle.hisa(inp, block, m, topk, queries=qs, blocks_given=blocks[qs])
+    cond = oracle.hisa(inp, block, m, topk, queries=qs, blocks_given=blocks[qs], b=b)
     for i, t in enumerate(qs):
         toks, s, c = cond["tokens"][i], cond["scores"][i], cond["cond"][i]
         check_selection(idx[t], toks, s, c, topk, what=f"{what} t={t}")
@@ -284,6 +307,11 @@ def test_hisa_ragged():
     _hisa_check(inp, block=96, m=5, topk=200, queries=range(40), what="hisa ragged")
 
 
+def test_hisa_batched_h64():
+    inp = wl.prefill_inputs(16, 3000, 64, 128, q_offset=2984, seed=28, batch=2, recency=0.1)
+    _hisa_check(inp, block=128, m=6, topk=100, queries=range(16), what="hisa b2", batches=(0, 1))
+
+
 def test_hisa_all_blocks_equals_dense():
     inp = wl.prefill_inputs(12, 1500, 32, 128, q_offset=1488, seed=19)
     ix = _indexer(inp)
@@ -298,6 +326,34 @@ def test_hisa_config_sampled():
     c = wl.CONFIGS["hisa"]
     inp = wl.make_inputs("hisa", seed=0)
     _hisa_check(inp, c["block"], c["m"], c["topk"], [0, 511, 1023], what="hisa cfg")
+
+
+# ------------------------------------------------------------------ gathered re-scoring alone
+@pytest.mark.parametrize("blk,n_slots", [(1, 700), (128, 9), (64, 5)])
+def test_gathered_scores_elementwise(blk, n_slots):
+    inp = wl.prefill_inputs(12, 1500, 64, 128, q_offset=1200, seed=29, batch=2)
+    rng = np.random.default_rng(blk)
+    nb = -(-1500 // blk)
+    cand = np.sort(np.stack([rng.choice(nb, n_slots, replace=False) for _ in range(24)]), axis=1)
+    cand[3, -2:] = -1  # padding slots
+    cand = cand.astype(np.int32)
+    ix = _indexer(inp)
+    out = torch.full((24, n_slots * blk), float("nan"), device="cuda")
+    ws = B.alloc_workspace(256)
+    B.indexer_score_gathered(ix.args, torch.from_numpy(cand).cuda(), n_slots, blk, out, n_slots * blk, ws)
+    assert B.dsa_device_status(ws) == 0
+    out = out.cpu().numpy()
+    for b in range(2):
+        q, k, w = oracle.dequant(inp, b)
+        for t in range(12):
+            r = b * 12 + t
+            pos = np.arange(n_slots * blk)
+            c = cand[r][pos // blk]
+            tok = c.astype(np.int64) * blk + pos % blk
+            ok = (c >= 0) & (tok < 1500) & (tok <= 1200 + t)
+            assert np.all(np.isneginf(out[r][~ok]))
+            s_, c_ = oracle.score_pairs(q, k, w, np.full(ok.sum(), t), tok[ok])
+            check_scores(out[r][ok], s_, c_, RTOL_BF16, what=f"gathered blk={blk} r={r}")
 
 
 # ------------------------------------------------------------------ boundary on the GPU
