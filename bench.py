@@ -18,7 +18,9 @@ bracket the timed region; the max over ranks is reported. With N > 1 every
 rank runs an independent replica on its own GPU (the path has no exchange
 step), so the aggregate is weak scaling.
 
-Extra keys: roofline of the dominant kernel (timed alone, same inputs),
+Extra keys: roofline of the dominant kernel (every kernel of the step timed
+alone on the inputs the step gives it; the slowest is the roofline's, all are
+listed under "kernels"),
 cpu_baseline (the fp64 oracle on a bounded sample, host cores), e2e (host
 buffers, H2D + call + D2H inside the timed region), clocks sampled during the
 timed region, gpu_launches.
@@ -115,45 +117,107 @@ class Runner:
         else:
             B.hisa_block_filter_topk(a, c["block"], c["m"], self.topk, o, None, None, self.ws)
 
-    # second stage alone: top-k over the rows the scoring stage just wrote
-    def topk_stage(self):
+    # ---- the step's kernels, each launched alone through the C-ABI on the
+    # inputs the step gives it (roofline and per-kernel shares)
+    def kernels(self):
+        """List of (name, callable, algorithmic units per launch, bound), in
+        the step's order. Units: FLOPs for tensor-bound kernels (2 * d per
+        head per scored pair), bytes for HBM-bound ones."""
         B, torch, c = self.B, self.torch, self.c
-        if self.name not in ("tiny", "dsa", "decode"):
-            return None
-        out = torch.empty((self.batch, c["T"], c["L"]), dtype=torch.float32, device="cuda")
+        T, L, H, d, k = c["T"], c["L"], c["H"], c["d"], self.topk
+        rows = self.batch * T
         ws = B.alloc_workspace(256)
-        B.indexer_scores(self.ix.args, out, c["L"], ws)
-        idx = torch.empty((self.batch, c["T"], self.topk), dtype=torch.int32, device="cuda")
-        rows = self.batch * c["T"]
-        self._keep_topk = (out, ws, idx)
-        return lambda: B.indexer_topk_rows(out, rows, c["L"], c["T"], self.inp.q_offset, 1, c["L"],
-                                           self.topk, None, 0, 1, idx, None, ws)
-
-    # dominant kernel, launched alone through the score-stage entry point
-    def dominant(self):
-        """(callable, algorithmic units per launch, bound, name)."""
-        B, torch, c = self.B, self.torch, self.c
+        keep = [ws]
+        out = []
         if self.name in ("tiny", "dsa", "decode"):
-            out = torch.empty((self.batch, c["T"], c["L"]), dtype=torch.float32, device="cuda")
-            ws = B.alloc_workspace(256)
-            fn = lambda: B.indexer_scores(self.ix.args, out, c["L"], ws)
+            sc = torch.empty((self.batch, T, L), dtype=torch.float32, device="cuda")
+            idx = torch.empty((self.batch, T, k), dtype=torch.int32, device="cuda")
+            keep += [sc, idx]
+            f_score = lambda: B.indexer_scores(self.ix.args, sc, L, ws)
+            f_score()
             if self.name == "decode":
-                # bytes the scorer must read per visible pair: one FP8 key row + its fp32 scale
-                return fn, self.pairs * (c["d"] + 4), "hbm", "score_tc<fp8>"
-            return fn, self.pairs * 2.0 * c["d"] * c["H"], "tensor", "score_tc<bf16>"
-        if self.name == "misa":
-            # the routed scoring pass: the same kernel on h gathered heads per query
-            q, k, w, _, _ = self.dev
-            h = c["h"]
-            qh = q[:, :, :h].contiguous()
-            wh = w[:, :, :h].contiguous()
-            a = B.make_args(qh, k, wh, self.inp.q_offset)
-            out = torch.empty((self.batch, c["T"], c["L"]), dtype=torch.float32, device="cuda")
-            ws = B.alloc_workspace(256)
-            self._keep = (qh, wh, a, out, ws)
-            return (lambda: B.indexer_scores(a, out, c["L"], ws)), self.pairs * 2.0 * c["d"] * h, \
-                "tensor", "score_tc<bf16,h=8> (routed)"
-        return None, None, None, None
+                # one FP8 key row + its fp32 scale per visible pair
+                out.append(("score_tc<fp8>", f_score, self.pairs * (d + 4), "hbm"))
+            else:
+                out.append(("score_tc<bf16>", f_score, self.pairs * 2.0 * d * H, "tensor"))
+            # every visible score read once, k indices written per row
+            out.append(("topk_rows", lambda: B.indexer_topk_rows(sc, rows, L, T, self.inp.q_offset, 1, L, k,
+                                                                 None, 0, 1, idx, None, ws),
+                        self.pairs * 4 + rows * k * 4, "hbm"))
+        elif self.name == "misa":
+            h, kp = c["h"], c["kprime"]
+            q, kk, w, _, _ = self.dev
+            # the routed pass scores with h heads per query: the same kernel on a
+            # query tensor of h heads (head choice does not change its cost)
+            qh, wh = q[:, :, :h].contiguous(), w[:, :, :h].contiguous()
+            ah = B.make_args(qh, kk, wh, self.inp.q_offset)
+            routed = torch.empty((self.batch, T, L), dtype=torch.float32, device="cuda")
+            cand = torch.empty((self.batch, T, kp), dtype=torch.int32, device="cuda")
+            comp = torch.empty((self.batch, T, kp), dtype=torch.float32, device="cuda")
+            idx = torch.empty((self.batch, T, k), dtype=torch.int32, device="cuda")
+            keep += [qh, wh, ah, routed, cand, comp, idx]
+            B.misa_route_score_topk(self.ix.args, c["block"], h, k, kp, idx, None, None, cand, self.ws)
+            f_routed = lambda: B.indexer_scores(ah, routed, L, ws)
+            f_routed()
+            out.append(("score_tc<bf16,h=%d> (routed)" % h, f_routed, self.pairs * 2.0 * d * h, "tensor"))
+            out.append(("topk_rows (k'=%d over routed rows)" % kp,
+                        lambda: B.indexer_topk_rows(routed, rows, L, T, self.inp.q_offset, 1, L, kp, None,
+                                                    0, 1, cand, None, ws),
+                        self.pairs * 4 + rows * kp * 4, "hbm"))
+            f_gather = lambda: B.indexer_score_gathered(self.ix.args, cand, kp, 1, comp, kp, ws)
+            f_gather()
+            out.append(("score_tc<bf16> gathered (MISA-dagger re-score)", f_gather,
+                        rows * kp * 2.0 * d * H, "tensor"))
+            out.append(("topk_rows (k=%d over k' candidates)" % k,
+                        lambda: B.indexer_topk_rows(comp, rows, kp, T, self.inp.q_offset, 0, kp, k, cand,
+                                                    kp, 1, idx, None, ws),
+                        rows * kp * 4 + rows * k * 8, "hbm"))
+        else:
+            m, blk = c["m"], c["block"]
+            nc = m * blk
+            blocks = torch.empty((self.batch, T, m), dtype=torch.int32, device="cuda")
+            comp = torch.empty((self.batch, T, nc), dtype=torch.float32, device="cuda")
+            idx = torch.empty((self.batch, T, k), dtype=torch.int32, device="cuda")
+            keep += [blocks, comp, idx]
+            B.hisa_block_filter_topk(self.ix.args, blk, m, k, idx, None, blocks, self.ws)
+            f_gather = lambda: B.indexer_score_gathered(self.ix.args, blocks, m, blk, comp, nc, ws)
+            f_gather()
+            out.append(("score_tc<bf16> gathered (HISA kept blocks)", f_gather,
+                        rows * nc * 2.0 * d * H, "tensor"))
+            out.append(("topk_rows (k=%d over m*block tokens)" % k,
+                        lambda: B.indexer_topk_rows(comp, rows, nc, T, self.inp.q_offset, 0, nc, k, blocks,
+                                                    m, blk, idx, None, ws),
+                        rows * nc * 4 + rows * k * 8, "hbm"))
+        self._keep = keep
+        return out
+
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture of the kernel named, valid only while its sources hash to
+# the value recorded with it (None otherwise). Full-size captures unless the
+# profile summary says it was scaled from a smaller case.
+TRAFFIC = {}
+KERNEL_SOURCES = {
+    "score_tc": ("score_tc.cuh", "common.cuh"),
+    "topk_rows": ("topk.cuh", "common.cuh"),
+}
+
+
+def source_hash(kernel_name):
+    import hashlib
+    fam = "topk_rows" if kernel_name.startswith("topk_rows") else "score_tc"
+    h = hashlib.sha1()
+    for f in KERNEL_SOURCES[fam]:
+        with open(os.path.join(ROOT, "sparse_attention_token_score_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def traffic_for(workload, kernel_name):
+    t = TRAFFIC.get((workload, kernel_name))
+    if t is None or t[1] != source_hash(kernel_name):
+        return None
+    return t[0]
 
 
 def aggregate_ranks(total_ms: float, units_per_rank_step: int, steps: int, world: int, reduce_max=None):
@@ -330,7 +394,9 @@ def main():
     ap.add_argument("--batch", type=int, default=0,
                     help="profiling: use only the first N sequences (decode)")
     ap.add_argument("--kernel-only", action="store_true",
-                    help="profiling: launch only the dominant kernel (W + K times)")
+                    help="profiling: launch only one kernel of the step (W + K times)")
+    ap.add_argument("--kernel", type=int, default=0,
+                    help="with --kernel-only: index into the step's kernel list (0 = first)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -360,7 +426,7 @@ def main():
     r = Runner(args.workload, inp, torch, args.queries, args.batch)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     if args.kernel_only:
-        fn, _, _, kname = r.dominant()
+        kname, fn, _, _ = r.kernels()[args.kernel]
         kt = time_steps(fn, args.warmup + args.steps, torch, flush)[args.warmup:]
         print(json.dumps({"kernel": kname, "workload": r.label, "kernel_ms": kt}), flush=True)
         return 0
@@ -382,29 +448,28 @@ def main():
     value = pairs_per_s / 1e9
     assert r.ix.device_status() == 0, "device wait timed out"
 
-    # ---- dominant kernel alone (roofline)
+    # ---- each kernel alone; the one with the largest time is the roofline's
     peaks, peak_src = load_peaks()
-    fn, units, bound, kname = r.dominant()
-    roof = None
-    if fn is not None:
+    per_kernel = []
+    for kname, fn, units, bound in r.kernels():
         for _ in range(3):
             fn()
-        kt = time_steps(fn, args.steps, torch, flush)
-        kms = statistics.mean(kt)
+        kms = statistics.mean(time_steps(fn, args.steps, torch, flush))
         if bound == "tensor":
-            achieved = units / (kms / 1e3) / 1e12
-            peak = peaks["bf16_tflops"]
-            unit = "TFLOP/s"
+            achieved, peak, unit = units / (kms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
         else:
-            achieved = units / (kms / 1e3) / 1e9
-            peak = peaks["hbm_gbs"]
-            unit = "GB/s"
-        tk = r.topk_stage()
-        topk_ms = statistics.mean(time_steps(tk, args.steps, torch, flush)) if tk else None
-        roof = {"bound": bound, "kernel": kname, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "peak_source": f"{peak_src} ({'bf16 burst' if bound == 'tensor' else 'HBM copy'})",
-                "kernel_ms": kms, "algorithmic_units_per_launch": units, "traffic": None,
-                "topk_stage_ms": topk_ms}
+            achieved, peak, unit = units / (kms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        per_kernel.append({"kernel": kname, "bound": bound, "ms": kms, "achieved": achieved, "peak": peak,
+                           "unit": unit, "frac": achieved / peak, "algorithmic_units_per_launch": units,
+                           "traffic": traffic_for(args.workload, kname)})
+    dom = max(per_kernel, key=lambda e: e["ms"])
+    kernel_sum = sum(e["ms"] for e in per_kernel)
+    for e in per_kernel:
+        e["share_of_listed"] = e["ms"] / kernel_sum
+    roof = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],
+            "frac": dom["frac"], "traffic": dom["traffic"], "kernel": dom["kernel"], "kernel_ms": dom["ms"],
+            "algorithmic_units_per_launch": dom["algorithmic_units_per_launch"],
+            "peak_source": f"{peak_src} ({'bf16 burst' if dom['bound'] == 'tensor' else 'HBM copy'})"}
 
     # ---- end to end: host buffers, H2D + call + D2H per step
     q, k, w, qs, ks = r.dev
@@ -454,6 +519,7 @@ def main():
                    "l2": "256 MiB buffer written before every timed step"},
         "queries_per_s": world * r.batch * c["T"] * args.steps / (total_ms / 1e3),
         "roofline": roof,
+        "kernels": per_kernel,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e_ms / args.steps},

@@ -33,8 +33,8 @@
  *   - Calls that share a workspace must not overlap in time (use one stream).
  *
  * Supported shapes: d in {64, 128}; bf16 H in {8, 16, 32, 64};
- * FP8 e4m3 (decode): d = 128, H in {32, 64}, L a multiple of 4. Other shapes
- * return DSA_ERR_UNSUPPORTED.
+ * FP8 e4m3 (decode): d = 128, H in {32, 64}. Other shapes return
+ * DSA_ERR_UNSUPPORTED.
  */
 #ifndef DSA_INDEXER_H
 #define DSA_INDEXER_H

@@ -95,7 +95,7 @@ dsa_status launch_score(const ScoreParams& p, const void* q, long long q_rows, c
   }
   CUtensorMap tq, tk;
   if (!make_tmap(&tq, q, C::ELEM == 1, C::D, q_rows, C::QROWS)) return DSA_ERR_CUDA;
-  if (C::GATHER && !p.blk_tma) tk = tq;
+  if (C::GATHER && !p.blk_tma) tk = tq;  // token gathers copy rows with cp.async (no key map)
   else if (!make_tmap(&tk, k, C::ELEM == 1, C::D, k_rows, C::KROWS)) return DSA_ERR_CUDA;
   int grid = num_sms();
   if (C::ROUTER) {
@@ -124,12 +124,15 @@ dsa_status run_scores_bf16(int D, int H, const ScoreParams& p, const void* q, lo
 }
 
 // FP8 decode scoring: one query per group, N = H.
+#ifndef DSA_FP8_NSTAGE
+#define DSA_FP8_NSTAGE 8
+#endif
 dsa_status run_scores_fp8(int D, int H, const ScoreParams& p, const void* q, long long q_rows,
                           const void* k, long long k_rows, cudaStream_t st) {
   if (D == 128 && H == 64)
-    return launch_score<ScoreCfg<1, 128, 64, 1, ScoreMode::kTma, 8>>(p, q, q_rows, k, k_rows, st);
+    return launch_score<ScoreCfg<1, 128, 64, 1, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
   if (D == 128 && H == 32)
-    return launch_score<ScoreCfg<1, 128, 32, 1, ScoreMode::kTma, 8>>(p, q, q_rows, k, k_rows, st);
+    return launch_score<ScoreCfg<1, 128, 32, 1, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
   return DSA_ERR_UNSUPPORTED;
 }
 
@@ -154,13 +157,16 @@ dsa_status run_gather(int D, int H, ScoreParams p, const void* q, long long q_ro
   p.blk_tma = (p.blk % 128 == 0) ? 1 : 0;
   const long long k_rows = static_cast<long long>(p.batch) * p.L_tok;
   if (D == 128 && H == 64)
-    return launch_score<ScoreCfg<2, 128, 64, 1, ScoreMode::kGather, 4>>(p, q, q_rows, p.kg, k_rows, st);
+    return launch_score<ScoreCfg<2, 128, 64, 1, ScoreMode::kGather, 6>>(p, q, q_rows, p.kg, k_rows, st);
   if (D == 128 && H == 32)
-    return launch_score<ScoreCfg<2, 128, 32, 1, ScoreMode::kGather, 4>>(p, q, q_rows, p.kg, k_rows, st);
+    return launch_score<ScoreCfg<2, 128, 32, 1, ScoreMode::kGather, 6>>(p, q, q_rows, p.kg, k_rows, st);
   return DSA_ERR_UNSUPPORTED;
 }
 
-dsa_status launch_topk(const TopkParams& tp, cudaStream_t st) {
+// ws: the call's workspace; its first word is the device status the
+// kernel's bounded waits report to.
+dsa_status launch_topk(void* ws, TopkParams tp, cudaStream_t st) {
+  tp.err = static_cast<unsigned*>(ws);
   static bool attr[kMaxDev] = {false};
   const int dev = current_device();
   if (!attr[dev]) {
@@ -187,7 +193,6 @@ dsa_status validate(const dsa_indexer_args* a, bool bf16_only) {
   if (fp8) {
     if (!a->q_scale || !a->k_scale) return DSA_ERR_ARG;
     if (!aligned(a->q_scale, 16) || !aligned(a->k_scale, 16)) return DSA_ERR_ARG;
-    if (a->L % 4 != 0) return DSA_ERR_UNSUPPORTED;  // key-scale rows are copied in 16-byte units
   }
   if (a->q_offset > (1LL << 40)) return DSA_ERR_ARG;
   if (static_cast<long long>(a->batch) * a->T * a->H > INT_MAX ||
@@ -243,6 +248,7 @@ TopkParams topk_params(const float* scores, long long rows, long long ld, int T,
   t.cand = cand;
   t.n_slots = n_slots;
   t.blk = blk;
+  t.err = nullptr;
   return t;
 }
 
@@ -341,7 +347,7 @@ dsa_status indexer_topk_rows(const float* scores, long long rows, long long ld, 
   DSA_TRY(check_ws(ws, ws_bytes, kHdr));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DSA_TRY(clear_status(ws, st));
-  return launch_topk(topk_params(scores, rows, ld, T, q_offset, pstride, row_len, topk, out_idx,
+  return launch_topk(ws, topk_params(scores, rows, ld, T, q_offset, pstride, row_len, topk, out_idx,
                                  out_score, cand, cand ? n_slots : 0, cand ? blk : 1),
                      st);
 }
@@ -364,7 +370,7 @@ dsa_status indexer_score_topk(const dsa_indexer_args* a, int topk, int32_t* out_
     DSA_TRY(run_scores_fp8(a->d, a->H, p, a->q, q_rows, a->k, k_rows, st));
   else
     DSA_TRY(run_scores_bf16(a->d, a->H, p, a->q, q_rows, a->k, k_rows, st));
-  return launch_topk(topk_params(scores, static_cast<long long>(a->batch) * a->T, a->L, a->T,
+  return launch_topk(ws, topk_params(scores, static_cast<long long>(a->batch) * a->T, a->L, a->T,
                                  a->q_offset, 1, a->L, topk, out_idx, out_score, nullptr, 0, 1),
                      st);
 }
@@ -446,7 +452,7 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   ps.ldo = a->L;
   DSA_TRY(run_scores_bf16(a->d, h, ps, q_sel, BT * h, a->k, static_cast<long long>(a->batch) * a->L, st));
   if (kprime == 0) {
-    return launch_topk(topk_params(routed, BT, a->L, a->T, a->q_offset, 1, a->L, topk, out_idx,
+    return launch_topk(ws, topk_params(routed, BT, a->L, a->T, a->q_offset, 1, a->L, topk, out_idx,
                                    out_score, nullptr, 0, 1),
                        st);
   }
@@ -454,7 +460,7 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   int32_t* cand_ws = c.take<int32_t>(static_cast<size_t>(BT) * kprime);
   float* compact = c.take<float>(static_cast<size_t>(BT) * kprime);
   int32_t* cand = out_cand ? out_cand : cand_ws;
-  DSA_TRY(launch_topk(topk_params(routed, BT, a->L, a->T, a->q_offset, 1, a->L, kprime, cand,
+  DSA_TRY(launch_topk(ws, topk_params(routed, BT, a->L, a->T, a->q_offset, 1, a->L, kprime, cand,
                                   nullptr, nullptr, 0, 1),
                       st));
   ScoreParams pg = base_params(a, err);
@@ -466,7 +472,7 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   pg.blk = 1;
   pg.n_compact = kprime;
   DSA_TRY(run_gather(a->d, a->H, pg, a->q, BT * a->H, st));
-  return launch_topk(topk_params(compact, BT, kprime, a->T, a->q_offset, 0, kprime, topk, out_idx,
+  return launch_topk(ws, topk_params(compact, BT, kprime, a->T, a->q_offset, 0, kprime, topk, out_idx,
                                  out_score, cand, kprime, 1),
                      st);
 }
@@ -517,7 +523,7 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   pb.ldo = M;
   DSA_TRY(run_scores_bf16(a->d, a->H, pb, a->q, BT * a->H, kbar, a->batch * M, st));
   // 3. top-m blocks
-  DSA_TRY(launch_topk(topk_params(bscore, BT, M, a->T, a->q_offset, block, static_cast<int>(M), m,
+  DSA_TRY(launch_topk(ws, topk_params(bscore, BT, M, a->T, a->q_offset, block, static_cast<int>(M), m,
                                   blocks, nullptr, nullptr, 0, 1),
                       st));
   // 4. token scores inside the kept blocks (compact rows of m * block)
@@ -531,7 +537,7 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   pg.n_compact = ncomp;
   DSA_TRY(run_gather(a->d, a->H, pg, a->q, BT * a->H, st));
   // 5. top-k tokens
-  return launch_topk(topk_params(compact, BT, ncomp, a->T, a->q_offset, 0, ncomp, topk, out_idx,
+  return launch_topk(ws, topk_params(compact, BT, ncomp, a->T, a->q_offset, 0, ncomp, topk, out_idx,
                                  out_score, blocks, m, block),
                      st);
 }

@@ -34,6 +34,10 @@
 
 namespace dsa {
 
+#ifndef DSA_NACC_MAX
+#define DSA_NACC_MAX 8
+#endif
+
 enum class ScoreMode : int { kTma = 0, kGather = 1, kRouter = 2 };
 
 struct ScoreParams {
@@ -72,16 +76,24 @@ struct ScoreCfg {
                 "bad tile shape");
   static_assert(!GATHER || (QPT == 1 && ELEM == 2 && ROW_BYTES == 256),
                 "gather mode: one bf16 query per group, d = 128");
-  // Each producer warp owns the stages s with s % NPROD == its index, so every
-  // stage is refilled by one warp in order and a parity wait is never more
-  // than one phase behind.
-  static_assert(NSTAGE % (MODE_ == ScoreMode::kGather ? 4 : 1) == 0, "stages per producer warp");
+  // Gathers: the producer warps take tiles round robin. Stage s is refilled
+  // for tile i only after the MMAs of tile i - NSTAGE are done, and the MMA
+  // thread consumes tiles in order, so with NSTAGE >= NPROD a warp's wait on
+  // a stage is never more than one phase behind and the arrivals of two
+  // tiles never meet on one phase.
+  static constexpr int NPROD = GATHER ? 4 : 1;          // producer warps
+  static_assert(NSTAGE >= NPROD, "stages per producer warp");
   static constexpr int Q_BYTES = QROWS * ROW_BYTES;
   static constexpr int K_BYTES = KROWS * ROW_BYTES;
   static constexpr int NKSTEP = ROW_BYTES / 32;         // one MMA consumes 32 bytes of K
-  static constexpr int TMEM_COLS = (2 * MMA_N <= 32) ? 32 : (2 * MMA_N <= 64) ? 64
-                                 : (2 * MMA_N <= 128) ? 128 : (2 * MMA_N <= 256) ? 256 : 512;
-  static constexpr int NPROD = GATHER ? 4 : 1;          // producer warps
+  // TMEM accumulators: as many MMA_N-column buffers as fit in the 512
+  // columns (at most DSA_NACC_MAX). Narrow tiles (one query per group) carry
+  // little MMA work each, so with two buffers the MMA -> epilogue -> MMA
+  // round trip would set the pace; more buffers let the MMAs run ahead.
+  static constexpr int NACC = (512 / MMA_N < DSA_NACC_MAX) ? 512 / MMA_N : DSA_NACC_MAX;
+  static_assert(NACC >= 2 && (NACC & (NACC - 1)) == 0, "accumulator buffers");
+  static constexpr int TMEM_COLS = (NACC * MMA_N <= 32) ? 32 : (NACC * MMA_N <= 64) ? 64
+                                 : (NACC * MMA_N <= 128) ? 128 : (NACC * MMA_N <= 256) ? 256 : 512;
   static constexpr int MMA_WARP = NPROD;
   static constexpr int EPI_WARP0 = NPROD + 1;
   // Epilogue warps: EPIW = 4 * NSETS; each set of 4 warps covers the 128
@@ -97,16 +109,15 @@ struct ScoreCfg {
   // shared memory layout (offsets from a 1024-aligned base)
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_K = Q_BYTES;
-  // FP8: the per-key dequant scales of each stage's 128 keys ride with the tile
-  static constexpr int KSC_BYTES = (ELEM == 1 && !ROUTER && !GATHER) ? KROWS * 4 : 0;
-  static constexpr int SMEM_KSC = SMEM_K + NSTAGE * K_BYTES;
-  static constexpr int SMEM_BAR = SMEM_KSC + NSTAGE * KSC_BYTES;
-  static constexpr int NBAR = 2 * NSTAGE + 7;
+  // FP8: the epilogue applies per-key dequant scales (loaded from global
+  // memory by the thread that owns the key, ahead of the tile's MMAs)
+  static constexpr bool KEY_SCALES = ELEM == 1 && !ROUTER && !GATHER;
+  static constexpr int SMEM_BAR = SMEM_K + NSTAGE * K_BYTES;
+  static constexpr int NBAR = 2 * NSTAGE + 3 + 2 * NACC;
   static constexpr int SMEM_USED = SMEM_BAR + NBAR * 8 + 16;
   // Pad to more than half an SM so two CTAs never share an SM's TMEM.
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024 < 120 * 1024) ? 120 * 1024 : SMEM_USED + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-  static_assert(!KSC_BYTES || SPLIT_TILES, "key scales are read by one 4-warp set per tile");
 };
 
 // Iterates this CTA's (group, tile) pairs. Every thread runs its own copy;
@@ -250,8 +261,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t qfull = smem_u32(&bars[2 * C::NSTAGE]);
   const uint32_t qempty = smem_u32(&bars[2 * C::NSTAGE + 1]);
   auto tfull = [&](int b) { return smem_u32(&bars[2 * C::NSTAGE + 2 + b]); };
-  auto tempty = [&](int b) { return smem_u32(&bars[2 * C::NSTAGE + 4 + b]); };
-  const uint32_t mdone = smem_u32(&bars[2 * C::NSTAGE + 6]);
+  auto tempty = [&](int b) { return smem_u32(&bars[2 * C::NSTAGE + 2 + C::NACC + b]); };
+  const uint32_t mdone = smem_u32(&bars[2 * C::NSTAGE + 2 + 2 * C::NACC]);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -261,11 +272,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(full(i), (C::GATHER && !p.blk_tma) ? 32 : 1);
       // FP8: a stage is free once its MMAs are done and the epilogue warps of
       // its tile have read the stage's key scales
-      mbar_init(empty(i), C::KSC_BYTES ? 1 + 4 : 1);
+      mbar_init(empty(i), 1);
     }
     mbar_init(qfull, 1);
     mbar_init(qempty, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::NACC; ++b) {
       mbar_init(tfull(b), 1);
       mbar_init(tempty(b), C::TEMPTY_ARRIVALS);
     }
@@ -344,27 +355,25 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!mbar_wait(empty(stage), ph ^ 1u, p.err)) { ok = false; }
           else {
             const int krow0 = b * p.Lk + s.j * C::KROWS;
-            // scales of the tile's keys that exist (Lk % 4 == 0: 16-byte multiples)
-            const uint32_t ksc_bytes =
-                C::KSC_BYTES ? static_cast<uint32_t>(min(C::KROWS, p.Lk - s.j * C::KROWS)) * 4u : 0u;
-            mbar_arrive_expect_tx(full(stage), C::K_BYTES + ksc_bytes);
+            mbar_arrive_expect_tx(full(stage), C::K_BYTES);
 #pragma unroll
             for (int kb = 0; kb < C::KBLK; ++kb)
               tma_load_2d(s_k + stage * C::K_BYTES + kb * C::KROWS * 128, &tm_k, full(stage),
                           kb * (128 / C::ELEM), krow0);
-            if (C::KSC_BYTES)
-              bulk_load(s_base + C::SMEM_KSC + stage * C::KSC_BYTES, p.k_scale + krow0, ksc_bytes,
-                        full(stage));
           }
         }
       } else {
         // Gather 128 key rows (one per compact position) with 16-byte cp.async:
         // a half-warp copies one 256-byte row, chunk c of row r lands at its
         // 128-byte-swizzle slot (c ^ (r & 7)) so the tensor core sees the same
-        // layout a TMA load would have written.
+        // layout a TMA load would have written. Rows without a visible token
+        // are zero-filled by the same instruction (nothing is read).
         // The tile's 128 token ids are resolved first (lane l owns rows l,
         // l+32, l+64, l+96: four independent loads), then handed to the
         // copying lanes with shuffles, so no copy waits on a dependent load.
+        // Completion is asynchronous: every lane arrives on the stage's full
+        // barrier (32 arrivals) once its copies have landed, and the warp
+        // goes on to its next tile, so several tiles are in flight at once.
         const long long r = static_cast<long long>(b) * p.T + tg;
         const long long q_pos = p.q_offset + tg;
         long long toks[4];
@@ -373,33 +382,40 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!mbar_wait(empty(stage), ph ^ 1u, p.err)) ok = false;
         if (ok) {
           const int ch = lane & 15;
-          const uint32_t tile = s_k + stage * C::K_BYTES;
-#pragma unroll 8
-          for (int i = 0; i < C::KROWS / 2; ++i) {
-            const int row = 2 * i + (lane >> 4);
-            // row r lives in lane (r & 31) of toks[r >> 5]; rows 2i and 2i+1 share r >> 5
-            const long long tok = __shfl_sync(0xffffffffu, toks[(2 * i) >> 5], row & 31);
-            const int kb = ch >> 3;
-            const uint32_t dst = tile + kb * C::KROWS * 128 + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-            if (tok >= 0) {
-              const __nv_bfloat16* src = p.kg + (static_cast<long long>(b) * p.L_tok + tok) * C::D + ch * 8;
-              cp_async_16(dst, src);
-            } else {
-              asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+          const uint32_t tile = s_k + stage * C::K_BYTES + (ch >> 3) * C::KROWS * 128;
+          // per lane: the global address of its four rows and which of them exist
+          const __nv_bfloat16* kseq = p.kg + static_cast<long long>(b) * p.L_tok * C::D;
+          unsigned long long ga[4];
+          uint32_t vm[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            vm[u] = __ballot_sync(0xffffffffu, toks[u] >= 0);
+            ga[u] = reinterpret_cast<unsigned long long>(kseq + (toks[u] >= 0 ? toks[u] : 0) * C::D);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int rl = 2 * i + (lane >> 4);  // row 32u + rl lives in lane rl
+              const int row = 32 * u + rl;
+              const unsigned long long a = __shfl_sync(0xffffffffu, ga[u], rl);
+              const uint32_t dst = tile + row * 128 + (((ch & 7) ^ (rl & 7)) << 4);
+              cp_async_16_zfill(dst, reinterpret_cast<const void*>(a + ch * 16),
+                                ((vm[u] >> rl) & 1u) ? 16u : 0u);
             }
           }
-          cp_async_commit_wait_all();
-          fence_proxy_async_smem();
-          mbar_arrive(full(stage));
+          cp_async_mbar_arrive_noinc(full(stage));
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
     }
+    // cp.async gathers still in flight land before the CTA can release its
+    // shared memory (on the normal path the MMA warp has waited for them all)
+    if (C::GATHER && !p.blk_tma) cp_async_wait_all();
     if (!ok && lane == 0) {
       // Error path: wait (bounded) for the TMA loads that may still be in
-      // flight before the CTA releases its shared memory. cp.async gathers
-      // were already waited for before their arrive.
+      // flight before the CTA releases its shared memory.
       if (pw == 0 && gq > 0) mbar_drain(qfull, (gq - 1) & 1u);
       if (!C::GATHER || p.blk_tma) {
         const uint32_t lo = it > C::NSTAGE ? it - C::NSTAGE : 0;
@@ -415,10 +431,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (s.first && !mbar_wait(qfull, gq & 1u, p.err)) { ok = false; break; }
         const int stage = static_cast<int>(it % C::NSTAGE);
         const uint32_t ph = (it / C::NSTAGE) & 1u;
-        const int buf = static_cast<int>(it & 1u);
-        const uint32_t tph = (it >> 1) & 1u;
+        const int buf = static_cast<int>(it % C::NACC);
+        const uint32_t tph = (it / C::NACC) & 1u;
         if (!mbar_wait(tempty(buf), tph ^ 1u, p.err)) { ok = false; break; }
         if (!mbar_wait(full(stage), ph, p.err)) { ok = false; break; }
+        // cp.async gathers wrote the stage through the generic proxy: order
+        // those writes before the tensor core's (async proxy) reads
+        if (C::GATHER) fence_proxy_async_smem();
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::MMA_N);
         const uint32_t k_tile = s_k + stage * C::K_BYTES;
@@ -456,10 +475,25 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (; !s.done; s.next(p), ++it) {
       const int b = s.b;
       const int tg = s.tg;
-      const int buf = static_cast<int>(it & 1u);
-      const bool mine = C::SPLIT_TILES ? (buf == set) : true;
+      const int buf = static_cast<int>(it % C::NACC);
+      // split tiles: the two sets take alternate tiles (buffer b: set b & 1)
+      const bool mine = C::SPLIT_TILES ? (static_cast<int>(it & 1u) == set) : true;
       if (mine) {
-        if (!mbar_wait(tfull(buf), (it >> 1) & 1u, p.err)) break;
+        // gather mode: this row's token (and visibility), loaded before the
+        // wait so that its latency hides behind the tile's MMAs
+        long long gtok = -1;
+        if constexpr (C::GATHER) {
+          const int gkey = s.j * C::KROWS + row;
+          if (gkey < p.n_compact)
+            gtok = gathered_token(p, static_cast<long long>(b) * p.T + tg, gkey, p.q_offset + tg);
+        }
+        // FP8: this row's key dequant scale, likewise
+        float ks = 1.f;
+        if constexpr (C::KEY_SCALES) {
+          const int skey = s.j * C::KROWS + row;
+          if (skey < p.Lk) ks = __ldg(p.k_scale + static_cast<long long>(b) * p.Lk + skey);
+        }
+        if (!mbar_wait(tfull(buf), (it / C::NACC) & 1u, p.err)) break;
         tc_fence_after();
         const uint32_t taddr = lane_addr + static_cast<uint32_t>(buf * C::MMA_N);
         if constexpr (C::ROUTER) {
@@ -498,13 +532,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #endif
           const int q0 = C::SPLIT_TILES ? 0 : set * QH;          // first query (in group)
           const int key = s.j * C::KROWS + row;                  // key row / compact position
-          float ks = 1.f;                                        // FP8 key dequant scale
-          if constexpr (C::KSC_BYTES != 0) {
-            const int stage = static_cast<int>(it % C::NSTAGE);
-            ks = reinterpret_cast<const float*>(smem + C::SMEM_KSC + stage * C::KSC_BYTES)[row];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty(stage));
-          }
           const long long rbase = static_cast<long long>(b) * p.T + tg * C::QPT + q0;
           // head weights of this thread's columns are contiguous in w when every
           // query of the half-group exists
@@ -615,10 +642,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           if (C::GATHER) {
             const long long r = static_cast<long long>(b) * p.T + tg;
-            if (key < p.n_compact) {
-              const long long tok = gathered_token(p, r, key, p.q_offset + tg);
-              p.out[r * p.ldo + key] = tok >= 0 ? accq[0] : -INFINITY;
-            }
+            if (key < p.n_compact) p.out[r * p.ldo + key] = gtok >= 0 ? accq[0] : -INFINITY;
           } else if (key < p.Lk) {
             // query q0+ql sees this key iff key * pstride <= q_offset + t0 + ql
             const int t0 = tg * C::QPT + q0;

@@ -49,6 +49,7 @@ struct TopkParams {
   float* out_score;      // [rows, k] or nullptr
   const int* cand;       // optional map: position j -> cand[r * n_slots + j / blk] * blk + j % blk
   int n_slots, blk;
+  unsigned* err;         // device status word (bounded waits)
 };
 
 constexpr int TK_THREADS = 1024;     // one row per CTA, one CTA per SM
@@ -65,7 +66,7 @@ constexpr int TK_BITMAP_WORDS = 4096;
 // longer rows take the fallback path (their selection bitmap would not fit)
 constexpr long long TK_MAX_BITMAP_ROW = 32LL * TK_BITMAP_WORDS;
 constexpr int TK_SMEM_WORDS =
-    TK_BINS + 128 + TK_SAMPLE_MAX + 2 * TK_CAND_CAP + TK_BITMAP_WORDS + TK_SMEM_ROW;
+    TK_BINS + 128 + TK_SAMPLE_MAX + 2 * TK_CAND_CAP + TK_BITMAP_WORDS + TK_SMEM_ROW + 4;  // + barrier
 constexpr int TK_SMEM_BYTES = TK_SMEM_WORDS * 4;
 constexpr int TK_UNROLL = 8;         // float4 loads in flight per thread when staging a row
 
@@ -174,10 +175,12 @@ __device__ __forceinline__ bool present(float x) { return x > -INFINITY; }  // f
 // many keys equal to tau rank within the top `need`.
 template <class Src>
 __device__ void exact_select(const uint32_t* cbuf, const Src& src, int n, uint32_t need,
-                             uint32_t* hist, uint32_t* ws, uint32_t* vars) {
-  uint32_t prefix = 0;
+                             uint32_t* hist, uint32_t* ws, uint32_t* vars, int d0 = 0,
+                             uint32_t prefix0 = 0) {
+  // d0 > 0: every key shares its top bits with prefix0 (digits before d0 are known)
+  uint32_t prefix = prefix0;
 #pragma unroll 1
-  for (int d = 0; d < 3; ++d) {
+  for (int d = d0; d < 3; ++d) {
     const int sh = d == 0 ? 21 : (d == 1 ? 10 : 0);
     const uint32_t width = d == 2 ? 10u : 11u;
     const uint32_t hi_sh = sh + width;
@@ -215,9 +218,14 @@ __device__ __forceinline__ int value_bin(float x, float lo, float scale) {
 
 // One row of the selection (see the file comment). STAGED: the row fits in
 // shared memory and starts on a 16-byte boundary.
+// The staged scores of the next row may already be on their way (prefetched
+// by the previous row with a bulk copy on `sbar`); the row prefetches the
+// CTA's next row (nxt, n_nxt) as soon as its own staged scores are no longer
+// read. Returns whether it did.
 template <bool STAGED>
-__device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem, long long r, int n,
-                                         const float* row) {
+__device__ __forceinline__ bool topk_row(const TopkParams& p, uint32_t* tk_smem, long long r, int n,
+                                         const float* row, uint32_t sbar, uint32_t& sphase,
+                                         bool prefetched, const float* nxt, int n_nxt) {
   uint32_t* hist = tk_smem;                      // TK_BINS
   uint32_t* ws = hist + TK_BINS;                 // 64
   uint32_t* vars = ws + 64;                      // 64
@@ -252,30 +260,48 @@ __device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem,
   uint32_t keff = 0;
   bool done = false;      // row written by the bitmap path
 
+  bool issued_next = false;
+  // Prefetch the next row into the stage (thread 0; the caller's __syncthreads
+  // or this row's have retired every read of the stage).
+  auto prefetch_next = [&]() {
+    if constexpr (STAGED) {
+      if (nxt != nullptr) {
+        if (tid == 0) {
+          fence_proxy_async_smem();
+          const uint32_t bytes = static_cast<uint32_t>(n_nxt >> 2) * 16u;
+          if (bytes) {
+            mbar_arrive_expect_tx(sbar, bytes);
+            bulk_load(s_stage, nxt, bytes, sbar);
+          } else {
+            mbar_arrive(sbar);
+          }
+        }
+        issued_next = true;
+      }
+    }
+  };
+
   // ---- 1. stage (or sample only)
   if constexpr (STAGED) {
     const int n4 = n >> 2;
-    for (int base = 0; base < n4; base += TK_THREADS * TK_UNROLL) {
-      float4 x[TK_UNROLL];
-#pragma unroll
-      for (int u = 0; u < TK_UNROLL; ++u) {
-        const int i = base + u * TK_THREADS + tid;
-        x[u] = i < n4 ? __ldcg(reinterpret_cast<const float4*>(row) + i)
-                      : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-      }
-#pragma unroll
-      for (int u = 0; u < TK_UNROLL; ++u) {
-        const int i = base + u * TK_THREADS + tid;
-        if (i < n4) {
-          sts_f32x4(s_stage + 16u * static_cast<uint32_t>(i), x[u]);
-          if (((4 * i) & (S - 1)) == 0) fsamp[(4 * i) / S] = x[u].x;
-        }
+    if (!prefetched && tid == 0) {
+      fence_proxy_async_smem();  // earlier generic accesses of the stage before the copy
+      const uint32_t bytes = static_cast<uint32_t>(n4) * 16u;
+      if (bytes) {
+        mbar_arrive_expect_tx(sbar, bytes);
+        bulk_load(s_stage, row, bytes, sbar);
+      } else {
+        mbar_arrive(sbar);
       }
     }
-    for (int i = 4 * n4 + tid; i < n; i += TK_THREADS) {
-      const float x = __ldcg(row + i);
-      sts_f32(s_stage + 4u * static_cast<uint32_t>(i), x);
-      if ((i & (S - 1)) == 0) fsamp[i / S] = x;
+    for (int i = 4 * n4 + tid; i < n; i += TK_THREADS) sts_f32(s_stage + 4u * static_cast<uint32_t>(i), __ldcg(row + i));
+    // on a timeout (error recorded) the copy is still drained, bounded, so
+    // that no copy is left in flight when the CTA moves on or exits
+    if (!mbar_wait(sbar, sphase, p.err)) mbar_drain(sbar, sphase);
+    sphase ^= 1u;
+    __syncthreads();
+    if (fast) {
+      for (int m = tid; m < ns; m += TK_THREADS) fsamp[m] = src.get(m * S);
     }
   } else if (fast) {
 #pragma unroll 8
@@ -413,8 +439,18 @@ __device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem,
     const bool band_ok = keff < nvalid && cmax <= LIST && above_all < keff && keff <= above_all + nc;
     __syncthreads();
     if (band_ok) {
-      // ---- 4. exact select among the candidates
-      exact_select(lkey, src, TK_WARPS * LIST, keff - above_all, hist, ws, vars);
+      // the staged scores are not read past this point: start the next row's copy
+      prefetch_next();
+      // ---- 4. exact select among the candidates. Every candidate lies in
+      // [t_lo, t_hi]: digits on which both ends agree are skipped.
+      int d0 = 0;
+      uint32_t pre0 = 0;
+      if (t_lo > -INFINITY && t_hi < INFINITY) {
+        const uint32_t kl = score_key(t_lo), kh = score_key(t_hi);
+        if ((kl >> 10) == (kh >> 10)) { d0 = 2; pre0 = kl >> 10; }
+        else if ((kl >> 21) == (kh >> 21)) { d0 = 1; pre0 = kl >> 21; }
+      }
+      exact_select(lkey, src, TK_WARPS * LIST, keff - above_all, hist, ws, vars, d0, pre0);
       const uint32_t tau = vars[0];
       const uint32_t teq = vars[1];
       // eq counts per warp list -> prefix (lists are in position order)
@@ -473,7 +509,7 @@ __device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem,
           }
           if (out < static_cast<uint32_t>(k)) {  // holds by construction; guards the row
             oi[out] = idx;
-            if (os) { const float x = src.get(i); os[out] = x == 0.f ? 0.f : x; }
+            if (os) { const float x = __ldcg(row + i); os[out] = x == 0.f ? 0.f : x; }
           }
           ++out;
         }
@@ -607,25 +643,55 @@ __device__ __forceinline__ void topk_row(const TopkParams& p, uint32_t* tk_smem,
     oi[j] = -1;
     if (os) os[j] = -INFINITY;
   }
+  if (!issued_next) {
+    __syncthreads();  // every read of the stage is done
+    prefetch_next();
+  }
+  return issued_next;
+}
+
+__device__ __forceinline__ int row_length(const TopkParams& p, long long r) {
+  const int t = static_cast<int>(r % p.T);
+  long long nl = p.Lrow;
+  if (p.pstride > 0) {
+    nl = (p.q_offset + t) / p.pstride + 1;
+    if (nl > p.Lrow) nl = p.Lrow;
+    if (nl < 0) nl = 0;
+  }
+  return static_cast<int>(nl);
+}
+
+__device__ __forceinline__ bool row_staged(const float* row, int n) {
+  return n <= TK_SMEM_ROW && (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
 }
 
 __global__ void __launch_bounds__(TK_THREADS, TK_CTAS_PER_SM) topk_rows_kernel(const TopkParams p) {
   extern __shared__ uint32_t tk_smem[];
+  const uint32_t sbar = smem_u32(tk_smem + TK_SMEM_WORDS - 2);  // stage copy barrier (8-byte aligned)
+  if (threadIdx.x == 0) {
+    mbar_init(sbar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  uint32_t sphase = 0;
+  bool prefetched = false;
   for (long long r = blockIdx.x; r < p.rows; r += gridDim.x) {
-    const int t = static_cast<int>(r % p.T);
-    long long nl = p.Lrow;
-    if (p.pstride > 0) {
-      nl = (p.q_offset + t) / p.pstride + 1;
-      if (nl > p.Lrow) nl = p.Lrow;
-      if (nl < 0) nl = 0;
-    }
-    const int n = static_cast<int>(nl);
+    const int n = row_length(p, r);
     const float* row = p.scores + r * p.ld;
-    const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15u) == 0);
-    if (n <= TK_SMEM_ROW && vec) topk_row<true>(p, tk_smem, r, n, row);
-    else topk_row<false>(p, tk_smem, r, n, row);
+    const long long rn = r + gridDim.x;
+    const float* nrow = rn < p.rows ? p.scores + rn * p.ld : nullptr;
+    const int nn = nrow ? row_length(p, rn) : 0;
+    const float* nxt = (nrow && row_staged(nrow, nn)) ? nrow : nullptr;
+    if (row_staged(row, n)) {
+      prefetched = topk_row<true>(p, tk_smem, r, n, row, sbar, sphase, prefetched, nxt, nn);
+    } else {
+      topk_row<false>(p, tk_smem, r, n, row, sbar, sphase, false, nullptr, 0);
+      prefetched = false;
+    }
     __syncthreads();
   }
+  // a prefetch is only issued for a row this CTA processes next: nothing is
+  // left in flight here
 }
 
 }  // namespace dsa
