@@ -55,6 +55,7 @@ struct TopkParams {
 constexpr int TK_THREADS = 1024;     // one row per CTA, one CTA per SM
 constexpr int TK_CTAS_PER_SM = 1;
 constexpr int TK_WARPS = TK_THREADS / 32;
+static_assert(TK_WARPS == 32, "per-warp totals are reduced with one warp's shuffles");
 constexpr int TK_BINS = 2048;
 constexpr int TK_SMEM_ROW = 32768;   // rows up to this length are staged in shared memory
 constexpr int TK_LIST = 128;         // band candidates per warp segment (staged rows)
@@ -165,6 +166,20 @@ struct RowSrc {
     if constexpr (STAGED) return lds_f32(sbase + 4u * static_cast<uint32_t>(i));
     else return __ldcg(g + i);
   }
+  // entries i .. i+3 (i a multiple of 4), -inf from `end` on; one vector
+  // load when all four exist and the row start allows it (vec)
+  __device__ __forceinline__ float4 get4(int i, int end, bool vec) const {
+    if (i + 3 < end && (STAGED || vec)) {
+      if constexpr (STAGED) return lds_f32x4(sbase + 4u * static_cast<uint32_t>(i));
+      else return __ldcg(reinterpret_cast<const float4*>(g + i));
+    }
+    float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    if (i < end) v.x = get(i);
+    if (i + 1 < end) v.y = get(i + 1);
+    if (i + 2 < end) v.z = get(i + 2);
+    if (i + 3 < end) v.w = get(i + 3);
+    return v;
+  }
 };
 
 __device__ __forceinline__ bool present(float x) { return x > -INFINITY; }  // false for -inf, NaN
@@ -173,12 +188,16 @@ __device__ __forceinline__ bool present(float x) { return x > -INFINITY; }  // f
 // n keys) or of positions [0, n) of a row; keys equal to 0 (absent) are
 // ignored. Leaves vars[0] = tau, the need-th largest key, and vars[1] = how
 // many keys equal to tau rank within the top `need`.
+// lists != nullptr: cbuf holds one list per warp (stride `n`), warp w's first
+// lists[w] entries are its keys, and each warp scans its own list.
 template <class Src>
 __device__ void exact_select(const uint32_t* cbuf, const Src& src, int n, uint32_t need,
                              uint32_t* hist, uint32_t* ws, uint32_t* vars, int d0 = 0,
-                             uint32_t prefix0 = 0) {
+                             uint32_t prefix0 = 0, const uint32_t* lists = nullptr) {
   // d0 > 0: every key shares its top bits with prefix0 (digits before d0 are known)
   uint32_t prefix = prefix0;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int lcount = lists ? static_cast<int>(min(lists[wid], static_cast<uint32_t>(n))) : 0;
 #pragma unroll 1
   for (int d = d0; d < 3; ++d) {
     const int sh = d == 0 ? 21 : (d == 1 ? 10 : 0);
@@ -186,11 +205,19 @@ __device__ void exact_select(const uint32_t* cbuf, const Src& src, int n, uint32
     const uint32_t hi_sh = sh + width;
     for (int i = threadIdx.x; i < TK_BINS; i += TK_THREADS) hist[i] = 0;
     __syncthreads();
+    if (lists) {
+      for (int i = lane; i < lcount; i += 32) {
+        const uint32_t key = cbuf[wid * n + i];
+        if (key != 0u && (hi_sh >= 32 || (key >> hi_sh) == prefix))
+          atomicAdd(&hist[(key >> sh) & ((1u << width) - 1u)], 1u);
+      }
+    } else {
 #pragma unroll 4
-    for (int i = threadIdx.x; i < n; i += TK_THREADS) {
-      const uint32_t key = cbuf ? cbuf[i] : score_key(src.get(i));
-      if (key != 0u && (hi_sh >= 32 || (key >> hi_sh) == prefix))
-        atomicAdd(&hist[(key >> sh) & ((1u << width) - 1u)], 1u);
+      for (int i = threadIdx.x; i < n; i += TK_THREADS) {
+        const uint32_t key = cbuf ? cbuf[i] : score_key(src.get(i));
+        if (key != 0u && (hi_sh >= 32 || (key >> hi_sh) == prefix))
+          atomicAdd(&hist[(key >> sh) & ((1u << width) - 1u)], 1u);
+      }
     }
     __syncthreads();
     if (d < 2) radix_pick<2048 / TK_THREADS>(hist, need, ws, vars);
@@ -387,56 +414,85 @@ __device__ __forceinline__ bool topk_row(const TopkParams& p, uint32_t* tk_smem,
                                                    : lo + (static_cast<float>(b_lo) - 0.5f) / scale;
     __syncthreads();
 
-    // ---- 3. band pass: bitmap words of "> t_hi", per-warp candidate lists.
-    // Above / present counts are per lane and reduced once after the pass.
-    uint32_t c_above = 0, c_band = 0, c_present = 0;
+    // ---- 3. band pass: bitmap words of "> t_hi" (bmap) and of the band
+    // [t_lo, t_hi] (bbm, in the sample's space). A lane takes 4 consecutive
+    // entries; a word (32 entries) is the OR of the nibbles of 8 lanes.
+    // Present entries are not counted: with t_lo = -inf every present entry
+    // is above or in the band, otherwise the band test below needs no count.
+    const float t_lo_p = t_lo > -INFINITY ? t_lo : -3.402823466e+38f;  // x >= t_lo_p: present
+    const bool vec = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
+    uint32_t* bbm = samp;
     uint32_t* my_key = lkey + wid * LIST;
     uint32_t* my_pos = lpos + wid * LIST;
+    uint32_t c_above = 0;
     for (int base = s0; base < s1; base += 256) {
-      // the loads of two 128-entry chunks are issued before any of their uses
-      float xv[8];
+      float4 xv[2];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = base + 32 * j + lane;
-        xv[j] = i < s1 ? src.get(i) : -INFINITY;
-      }
+      for (int j = 0; j < 2; ++j) xv[j] = src.get4(base + 128 * j + 4 * lane, s1, vec);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = base + 32 * j + lane;
-        const float x = xv[j];
-        const bool up = x > t_hi;
-        const bool band = x >= t_lo && x <= t_hi && present(x);
-        c_above += up;
-        c_present += present(x);
-        const uint32_t ma = __ballot_sync(0xffffffffu, up);
-        if (lane == 0 && base + 32 * j < s1) bmap[(base + 32 * j) >> 5] = ma;
-        const uint32_t mb = __ballot_sync(0xffffffffu, band);
-        if (mb) {
-          if (band) {
-            const uint32_t slot = c_band + __popc(mb & lt_mask);
-            if (slot < LIST) { my_key[slot] = score_key(x); my_pos[slot] = static_cast<uint32_t>(i); }
-          }
-          c_band += __popc(mb);
+      for (int j = 0; j < 2; ++j) {
+        const int i4 = base + 128 * j + 4 * lane;
+        const float4 x = xv[j];
+        const uint32_t nib = static_cast<uint32_t>(x.x > t_hi) | (static_cast<uint32_t>(x.y > t_hi) << 1) |
+                             (static_cast<uint32_t>(x.z > t_hi) << 2) | (static_cast<uint32_t>(x.w > t_hi) << 3);
+        const uint32_t bnib =
+            (static_cast<uint32_t>(x.x >= t_lo_p) | (static_cast<uint32_t>(x.y >= t_lo_p) << 1) |
+             (static_cast<uint32_t>(x.z >= t_lo_p) << 2) | (static_cast<uint32_t>(x.w >= t_lo_p) << 3)) &
+            ~nib;
+        c_above += __popc(nib);
+        uint32_t word = nib << (4 * (lane & 7));
+        uint32_t bword = bnib << (4 * (lane & 7));
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+          word |= __shfl_xor_sync(0xffffffffu, word, o);
+          bword |= __shfl_xor_sync(0xffffffffu, bword, o);
         }
+        if ((lane & 7) == 0 && i4 < s1) { bmap[i4 >> 5] = word; bbm[i4 >> 5] = bword; }
       }
     }
+    __syncwarp();
+    // this warp's band entries -> its list, in position order
+    const int w0 = s0 >> 5;                              // this warp's words
+    const int w1 = s1 > s0 ? (s1 + 31) >> 5 : w0;      // (none for an empty segment)
+    uint32_t c_band = 0;
+    for (int wb = w0; wb < w1; wb += 32) {
+      const int wd = wb + lane;
+      uint32_t bits = wd < w1 ? bbm[wd] : 0u;
+      const uint32_t cnt = __popc(bits);
+      uint32_t inc = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      uint32_t slot = c_band + inc - cnt;
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        if (slot < LIST) {
+          const int i = wd * 32 + b;
+          my_key[slot] = score_key(src.get(i));
+          my_pos[slot] = static_cast<uint32_t>(i);
+        }
+        ++slot;
+      }
+      c_band += __shfl_sync(0xffffffffu, inc, 31);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c_above += __shfl_xor_sync(0xffffffffu, c_above, o);
+    uint32_t* lcnt = vars + 32;                          // per-warp list lengths
+    if (lane == 0) { ws[wid] = c_above; lcnt[wid] = c_band; }
+    __syncthreads();
+    uint32_t above_all = ws[lane], nc = lcnt[lane], cmax = lcnt[lane];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      c_above += __shfl_xor_sync(0xffffffffu, c_above, o);
-      c_present += __shfl_xor_sync(0xffffffffu, c_present, o);
+      above_all += __shfl_xor_sync(0xffffffffu, above_all, o);
+      nc += __shfl_xor_sync(0xffffffffu, nc, o);
+      cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
     }
-    for (int sl = static_cast<int>(c_band) + lane; sl < LIST; sl += 32) my_key[sl] = 0u;  // empty slots
-    if (lane == 0) { ws[wid] = c_above; ws[32 + wid] = c_present; samp[wid] = c_band; }
-    __syncthreads();
-    uint32_t above_all = 0, nvalid = 0, nc = 0, cmax = 0;
-    for (int w = 0; w < TK_WARPS; ++w) {
-      above_all += ws[w];
-      nvalid += ws[32 + w];
-      nc += samp[w];
-      cmax = max(cmax, samp[w]);
-    }
-    keff = min(static_cast<uint32_t>(k), nvalid);
-    const bool band_ok = keff < nvalid && cmax <= LIST && above_all < keff && keff <= above_all + nc;
+    // with t_lo = -inf the present entries are exactly above + band
+    keff = t_lo > -INFINITY ? static_cast<uint32_t>(k) : min(static_cast<uint32_t>(k), above_all + nc);
+    const bool band_ok = cmax <= LIST && above_all < keff && keff <= above_all + nc;
     __syncthreads();
     if (band_ok) {
       // the staged scores are not read past this point: start the next row's copy
@@ -450,19 +506,28 @@ __device__ __forceinline__ bool topk_row(const TopkParams& p, uint32_t* tk_smem,
         if ((kl >> 10) == (kh >> 10)) { d0 = 2; pre0 = kl >> 10; }
         else if ((kl >> 21) == (kh >> 21)) { d0 = 1; pre0 = kl >> 21; }
       }
-      exact_select(lkey, src, TK_WARPS * LIST, keff - above_all, hist, ws, vars, d0, pre0);
+      exact_select(lkey, src, LIST, keff - above_all, hist, ws, vars, d0, pre0, lcnt);
       const uint32_t tau = vars[0];
       const uint32_t teq = vars[1];
       // eq counts per warp list -> prefix (lists are in position order)
-      const uint32_t cb = samp[wid];
+      const uint32_t cb = lcnt[wid];
       uint32_t ceq = 0;
       for (int sl = lane; sl < static_cast<int>(cb); sl += 32) ceq += my_key[sl] == tau;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ceq += __shfl_xor_sync(0xffffffffu, ceq, o);
       if (lane == 0) ws[wid] = ceq;
       __syncthreads();
-      uint32_t eq_before = 0;
-      for (int w = 0; w < wid; ++w) eq_before += ws[w];
+      uint32_t eq_before;
+      {
+        const uint32_t e = ws[lane];                       // warps before this one
+        uint32_t inc = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += y;
+        }
+        eq_before = __shfl_sync(0xffffffffu, inc - e, wid);
+      }
       for (int base = 0; base < static_cast<int>(cb); base += 32) {
         const int sl = base + lane;
         const uint32_t key = sl < static_cast<int>(cb) ? my_key[sl] : 0u;
@@ -477,8 +542,6 @@ __device__ __forceinline__ bool topk_row(const TopkParams& p, uint32_t* tk_smem,
       }
       __syncthreads();
       // ---- 5. emit the bitmap in position order
-      const int w0 = s0 >> 5;                              // this warp's words
-      const int w1 = s1 > s0 ? (s1 + 31) >> 5 : w0;      // (none for an empty segment)
       const int per = (w1 - w0 + 31) / 32;                 // words per lane (contiguous)
       const int l0 = min(w1, w0 + lane * per), l1 = min(w1, l0 + per);
       uint32_t cnt = 0;
@@ -491,8 +554,17 @@ __device__ __forceinline__ bool topk_row(const TopkParams& p, uint32_t* tk_smem,
       }
       if (lane == 31) ws[32 + wid] = inc;
       __syncthreads();
-      uint32_t wbase = 0;
-      for (int w = 0; w < wid; ++w) wbase += ws[32 + w];
+      uint32_t wbase;
+      {
+        const uint32_t e = ws[32 + lane];
+        uint32_t winc = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, winc, o);
+          if (lane >= o) winc += y;
+        }
+        wbase = __shfl_sync(0xffffffffu, winc - e, wid);
+      }
       uint32_t out = wbase + inc - cnt;
       int32_t* oi = p.out_idx + r * p.k;
       float* os = p.out_score ? p.out_score + r * p.k : nullptr;
