@@ -425,12 +425,14 @@ __device__ __forceinline__ bool topk_row(const TopkParams& p, uint32_t* tk_smem,
     uint32_t* my_key = lkey + wid * LIST;
     uint32_t* my_pos = lpos + wid * LIST;
     uint32_t c_above = 0;
-    for (int base = s0; base < s1; base += 256) {
-      float4 xv[2];
+    // rows read from global memory keep more loads in flight
+    constexpr int UB = STAGED ? 2 : 4;
+    for (int base = s0; base < s1; base += 128 * UB) {
+      float4 xv[UB];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) xv[j] = src.get4(base + 128 * j + 4 * lane, s1, vec);
+      for (int j = 0; j < UB; ++j) xv[j] = src.get4(base + 128 * j + 4 * lane, s1, vec);
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      for (int j = 0; j < UB; ++j) {
         const int i4 = base + 128 * j + 4 * lane;
         const float4 x = xv[j];
         const uint32_t nib = static_cast<uint32_t>(x.x > t_hi) | (static_cast<uint32_t>(x.y > t_hi) << 1) |
@@ -568,22 +570,43 @@ __device__ __forceinline__ bool topk_row(const TopkParams& p, uint32_t* tk_smem,
       uint32_t out = wbase + inc - cnt;
       int32_t* oi = p.out_idx + r * p.k;
       float* os = p.out_score ? p.out_score + r * p.k : nullptr;
+      // positions are collected in shared memory (the candidate-list space,
+      // no longer read) and written out below with coalesced stores
+      uint32_t* obuf = ckey;
+      const bool via_smem = k <= 2 * TK_CAND_CAP;
       for (int wd = l0; wd < l1; ++wd) {
         uint32_t bits = bmap[wd];
         while (bits) {
           const int b = __ffs(bits) - 1;
           bits &= bits - 1u;
           const int i = wd * 32 + b;
+          if (out < static_cast<uint32_t>(k)) {  // holds by construction; guards the row
+            if (via_smem) {
+              obuf[out] = static_cast<uint32_t>(i);
+            } else {
+              int idx = i;
+              if (p.cand) {
+                const int slot = i / p.blk;
+                idx = __ldg(p.cand + r * p.n_slots + slot) * p.blk + (i - slot * p.blk);
+              }
+              oi[out] = idx;
+              if (os) { const float x = __ldcg(row + i); os[out] = x == 0.f ? 0.f : x; }
+            }
+          }
+          ++out;
+        }
+      }
+      if (via_smem) {
+        __syncthreads();
+        for (int j = tid; j < static_cast<int>(keff); j += TK_THREADS) {
+          const int i = static_cast<int>(obuf[j]);
           int idx = i;
           if (p.cand) {
             const int slot = i / p.blk;
             idx = __ldg(p.cand + r * p.n_slots + slot) * p.blk + (i - slot * p.blk);
           }
-          if (out < static_cast<uint32_t>(k)) {  // holds by construction; guards the row
-            oi[out] = idx;
-            if (os) { const float x = __ldcg(row + i); os[out] = x == 0.f ? 0.f : x; }
-          }
-          ++out;
+          oi[j] = idx;
+          if (os) { const float x = __ldcg(row + i); os[j] = x == 0.f ? 0.f : x; }
         }
       }
       done = true;
