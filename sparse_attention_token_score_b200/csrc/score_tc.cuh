@@ -112,7 +112,11 @@ struct ScoreCfg {
   // FP8: the epilogue applies per-key dequant scales (loaded from global
   // memory by the thread that owns the key, ahead of the tile's MMAs)
   static constexpr bool KEY_SCALES = ELEM == 1 && !ROUTER && !GATHER;
-  static constexpr int SMEM_BAR = SMEM_K + NSTAGE * K_BYTES;
+  // per epilogue warp: the head weights (x query scales) of its columns for
+  // the current query group, refilled when the group changes
+  static constexpr int NCOL_THREAD = ROUTER ? 0 : (SPLIT_TILES ? QROWS : QROWS / NSETS);
+  static constexpr int SMEM_COEF = SMEM_K + NSTAGE * K_BYTES;
+  static constexpr int SMEM_BAR = SMEM_COEF + EPIW * NCOL_THREAD * 4;
   static constexpr int NBAR = 2 * NSTAGE + 3 + 2 * NACC;
   static constexpr int SMEM_USED = SMEM_BAR + NBAR * 8 + 16;
   // Pad to more than half an SM so two CTAs never share an SM's TMEM.
@@ -471,6 +475,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int row = quarter * 32 + lane;       // accumulator row = TMEM lane
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     float racc = 0.f;                          // router partial sum
+    int coef_g = -1;                           // query group of the staged head weights
     uint32_t it = 0;
     for (; !s.done; s.next(p), ++it) {
       const int b = s.b;
@@ -535,9 +540,23 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const long long rbase = static_cast<long long>(b) * p.T + tg * C::QPT + q0;
           // head weights of this thread's columns are contiguous in w when every
           // query of the half-group exists
-          const bool full_group = tg * C::QPT + q0 + QH <= p.T;
-          const float* wrow = p.w + rbase * C::H;
-          const float* srow = (C::ELEM == 1) ? p.q_scale + rbase * C::H : nullptr;
+          // this warp's head weights for the group (queries past T reuse the
+          // last query's weights; their outputs are never stored)
+          static_assert(NC == C::NCOL_THREAD, "coefficient slot");
+          float* cw = reinterpret_cast<float*>(smem + C::SMEM_COEF) + e * NC;
+          if (s.g != coef_g) {
+            for (int c = lane; c < NC; c += 32) {
+              const int ql = c / C::H;
+              const int h = c % C::H;
+              const int tq = tg * C::QPT + q0 + ql;
+              const long long ci = (rbase + ql - (tq < p.T ? 0 : tq - p.T + 1)) * C::H + h;
+              float cv = __ldg(p.w + ci);
+              if (C::ELEM == 1) cv *= __ldg(p.q_scale + ci);
+              cw[c] = cv;
+            }
+            __syncwarp();
+            coef_g = s.g;
+          }
           float acc[QH][NP];
 #pragma unroll
           for (int i = 0; i < QH; ++i)
@@ -577,27 +596,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               const int cc = (ph * PH + c) * 32;
               const uint32_t (&v)[32] = vb[ph & 1][c];
               float coef[32];
-              if (full_group) {
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                  float4 c4 = __ldg(reinterpret_cast<const float4*>(wrow + cc + i));
-                  if (C::ELEM == 1) {
-                    const float4 s4 = __ldg(reinterpret_cast<const float4*>(srow + cc + i));
-                    c4.x *= s4.x; c4.y *= s4.y; c4.z *= s4.z; c4.w *= s4.w;
-                  }
-                  coef[i] = c4.x; coef[i + 1] = c4.y; coef[i + 2] = c4.z; coef[i + 3] = c4.w;
-                }
-              } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                  const int ql = (cc + i) / C::H;
-                  const int h = (cc + i) % C::H;
-                  const int tq = tg * C::QPT + q0 + ql;
-                  const long long ci = (rbase + ql - (tq < p.T ? 0 : tq - p.T + 1)) * C::H + h;
-                  float c = __ldg(p.w + ci);
-                  if (C::ELEM == 1) c *= __ldg(p.q_scale + ci);
-                  coef[i] = c;
-                }
+              for (int i = 0; i < 32; i += 4) {
+                const float4 c4 = *reinterpret_cast<const float4*>(cw + cc + i);
+                coef[i] = c4.x; coef[i + 1] = c4.y; coef[i + 2] = c4.z; coef[i + 3] = c4.w;
               }
 #if defined(DSA_NO_FFMA2)
 #pragma unroll
