@@ -165,20 +165,36 @@ dsa_status run_gather(int D, int H, ScoreParams p, const void* q, long long q_ro
 
 // ws: the call's workspace; its first word is the device status the
 // kernel's bounded waits report to.
+template <class C>
+dsa_status launch_topk_cfg(const TopkParams& tp, cudaStream_t st) {
+  static int ctas[kMaxDev] = {0};
+  const int dev = current_device();
+  if (ctas[dev] == 0) {
+    if (cudaFuncSetAttribute(topk_rows_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES) !=
+        cudaSuccess)
+      return DSA_ERR_CUDA;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, topk_rows_kernel<C>, C::NT, C::BYTES) !=
+            cudaSuccess ||
+        occ < 1)
+      return DSA_ERR_CUDA;
+    ctas[dev] = occ;
+  }
+  long long grid = static_cast<long long>(num_sms()) * ctas[dev];
+  if (tp.rows < grid) grid = tp.rows;
+  topk_rows_kernel<C><<<static_cast<int>(grid), C::NT, C::BYTES, st>>>(tp);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ws: the call's workspace (its first word is the device status word).
+// Rows up to 32768 scores use the short-row layout (more CTAs per SM); longer
+// rows use 256-thread CTAs when there are enough rows to fill the GPU, else
+// one 512-thread CTA per row.
 dsa_status launch_topk(void* ws, TopkParams tp, cudaStream_t st) {
   tp.err = static_cast<unsigned*>(ws);
-  static bool attr[kMaxDev] = {false};
-  const int dev = current_device();
-  if (!attr[dev]) {
-    if (cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             TK_SMEM_BYTES) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr[dev] = true;
-  }
-  long long grid = static_cast<long long>(num_sms()) * TK_CTAS_PER_SM;
-  if (tp.rows < grid) grid = tp.rows;
-  topk_rows_kernel<<<static_cast<int>(grid), TK_THREADS, TK_SMEM_BYTES, st>>>(tp);
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  if (tp.Lrow <= TkShort::MAX_ROW) return launch_topk_cfg<TkShort>(tp, st);
+  if (tp.rows >= static_cast<long long>(num_sms()) * TkLong::MIN_CTAS) return launch_topk_cfg<TkLong>(tp, st);
+  return launch_topk_cfg<TkWide>(tp, st);
 }
 
 bool h_supported_bf16(int H) { return H == 8 || H == 16 || H == 32 || H == 64; }

@@ -49,8 +49,12 @@ def _check(scores, idx, sc, expect, what):
     assert np.all(np.isneginf(sc[pad])), what
 
 
+# (20000, 5000) and (40000, 13000): more selected than the shared-memory output
+# staging holds (direct writes); (140000, 1000): longer than the band path's
+# bitmap (fallback only)
 @pytest.mark.parametrize("n,k", [(33, 5), (1000, 100), (32768, 2048), (32769, 2048), (40000, 3000),
-                                 (131072, 8192), (131072, 2048), (4096, 4096), (5000, 6000)])
+                                 (131072, 8192), (131072, 2048), (4096, 4096), (5000, 6000),
+                                 (20000, 5000), (40000, 13000), (140000, 1000)])
 def test_random_rows(n, k):
     rng = np.random.default_rng(n + k)
     s = (rng.standard_normal((6, n)) * 0.05).astype(np.float32)
@@ -105,3 +109,14 @@ def test_index_maps():
     s1 = rng.standard_normal((rows, 700)).astype(np.float32)
     idx, sc = _run(s1, rows, 0, 0, 700, 64, cand=cand1, n_slots=700, blk=1)
     _check(s1, idx, sc, _expect(s1, rows, 0, 0, 700, 64, cand=cand1, blk=1), "token map")
+
+
+def test_many_long_rows():
+    # enough rows longer than 32768 to fill the GPU with 256-thread CTAs
+    rng = np.random.default_rng(11)
+    rows, n, k = 320, 33000, 2048
+    s = (rng.standard_normal((rows, n)) * 0.05).astype(np.float32)
+    s[::7, : n // 3] = -np.inf  # some rows with absent entries
+    idx, sc = _run(s, rows, 0, 0, n, k)
+    exp = _expect(s, rows, 0, 0, n, k)
+    _check(s, idx, sc, exp, "many long rows")
