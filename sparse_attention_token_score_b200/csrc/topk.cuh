@@ -366,24 +366,42 @@ __device__ bool topk_row_band(const TopkParams& p, uint32_t* sm, long long r, in
   __syncthreads();
   if (!band_ok) return false;
 
-  // ---- 3. band entries -> candidate list, in position order
+  // ---- 3. band entries -> candidate list, in position order. A lane
+  // takes a contiguous run of the warp's words; the scores of its entries are
+  // re-read from L2 eight loads at a time.
   {
-    uint32_t slot0 = band_before;
-    for (int wb = w0; wb < w1; wb += 32) {
-      const int wd = wb + lane;
-      uint32_t bits = wd < w1 ? bbm[wd] : 0u;
-      const uint32_t cnt = __popc(bits);
-      const uint32_t inc = warp_incl_scan(cnt);
-      uint32_t slot = slot0 + inc - cnt;
-      while (bits) {
-        const int b = __ffs(bits) - 1;
-        bits &= bits - 1u;
-        const int i = wd * 32 + b;
-        lkey[slot] = score_key(__ldcg(row + i));
-        lpos[slot] = static_cast<uint32_t>(i);
-        ++slot;
+    const int per = (w1 - w0 + 31) / 32;
+    const int l0 = min(w1, w0 + lane * per), l1 = min(w1, l0 + per);
+    uint32_t cnt = 0;
+    for (int wd = l0; wd < l1; ++wd) cnt += __popc(bbm[wd]);
+    uint32_t slot = band_before + warp_incl_scan(cnt) - cnt;
+    int wd = l0;
+    uint32_t bits = wd < l1 ? bbm[wd] : 0u;
+    while (true) {
+      int pos[8];
+      int m = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        while (!bits && wd + 1 < l1) bits = bbm[++wd];
+        pos[u] = -1;
+        if (bits) {
+          pos[u] = wd * 32 + __ffs(bits) - 1;
+          bits &= bits - 1u;
+          ++m;
+        }
       }
-      slot0 += __shfl_sync(0xffffffffu, inc, 31);
+      if (m == 0) break;
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = pos[u] >= 0 ? __ldcg(row + pos[u]) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (pos[u] >= 0) {
+          lkey[slot] = score_key(v[u]);
+          lpos[slot] = static_cast<uint32_t>(pos[u]);
+          ++slot;
+        }
+      }
     }
   }
   __syncthreads();
