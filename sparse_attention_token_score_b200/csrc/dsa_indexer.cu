@@ -187,9 +187,9 @@ dsa_status launch_topk_cfg(const TopkParams& tp, cudaStream_t st) {
 }
 
 // ws: the call's workspace (its first word is the device status word).
-// Rows up to 32768 scores use the short-row layout (more CTAs per SM); longer
-// rows use 256-thread CTAs when there are enough rows to fill the GPU, else
-// one 512-thread CTA per row.
+// Rows up to 32768 scores use the short-row layout (4 CTAs of 256 threads per
+// SM); longer rows use 2 CTAs of 512 threads per SM when there are enough rows
+// to fill the GPU, else one 512-thread CTA (with more loads in flight) per row.
 dsa_status launch_topk(void* ws, TopkParams tp, cudaStream_t st) {
   tp.err = static_cast<unsigned*>(ws);
   if (tp.Lrow <= TkShort::MAX_ROW) return launch_topk_cfg<TkShort>(tp, st);

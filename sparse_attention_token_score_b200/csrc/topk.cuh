@@ -11,9 +11,9 @@
 // where integer order is needed; elsewhere scores are compared as floats
 // (which already treat -0 and +0 as equal).
 //
-// Work split: a CTA of 256 threads owns one row at a time and several CTAs
-// share an SM, so the barriers and latencies of one row overlap the work of
-// others. Rows are read from global memory (the sampling read brings a row
+// Work split: a CTA (256 or 512 threads) owns one row at a time and several
+// CTAs share an SM, so the barriers and latencies of one row overlap the work
+// of others. Rows are read from global memory (the sampling read brings a row
 // into L2, the band pass reads it from there). Per row:
 //   1. every S-th score is sampled (S a power of two, at most 4096 samples);
 //      a 2048-bin value histogram of the sample (bins evenly spaced between
@@ -83,7 +83,7 @@ struct TkCfg {
   static_assert(MINC_ * (BYTES + 1024) <= 228 * 1024, "shared memory for MIN_CTAS CTAs per SM");
 };
 using TkShort = TkCfg<1024, 2048, 4, 256, 4>;  // rows up to 32768: 44.5 KB, 4 CTAs per SM
-using TkLong = TkCfg<4096, 6144, 8, 256, 2>;   // rows up to 131072: 88.5 KB, 2 CTAs per SM
+using TkLong = TkCfg<4096, 6144, 4, 512, 2>;   // rows up to 131072: 88.5 KB, 2 CTAs per SM
 using TkWide = TkCfg<4096, 6144, 8, 512, 1>;   // as TkLong, one wider CTA per row for launches with few rows
 
 __device__ __forceinline__ uint32_t score_key(float x) {
