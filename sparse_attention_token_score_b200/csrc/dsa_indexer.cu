@@ -152,12 +152,19 @@ dsa_status run_router(int D, int H, const ScoreParams& p, const void* q, long lo
 // Gathered re-scoring (MISA-dagger candidates, HISA surviving blocks).
 // When blk is a multiple of 128, every 128-row tile is one contiguous key
 // run and is fetched with TMA; otherwise rows are gathered with cp.async.
+#ifndef DSA_GATHER_NS
+#define DSA_GATHER_NS 5
+#endif
+#ifndef DSA_GATHER_NQ
+#define DSA_GATHER_NQ 2
+#endif
 dsa_status run_gather(int D, int H, ScoreParams p, const void* q, long long q_rows,
                       cudaStream_t st) {
   p.blk_tma = (p.blk % 128 == 0) ? 1 : 0;
   const long long k_rows = static_cast<long long>(p.batch) * p.L_tok;
   if (D == 128 && H == 64)
-    return launch_score<ScoreCfg<2, 128, 64, 1, ScoreMode::kGather, 6>>(p, q, q_rows, p.kg, k_rows, st);
+    return launch_score<ScoreCfg<2, 128, 64, 1, ScoreMode::kGather, DSA_GATHER_NS, 8, DSA_GATHER_NQ>>(
+        p, q, q_rows, p.kg, k_rows, st);
   if (D == 128 && H == 32)
     return launch_score<ScoreCfg<2, 128, 32, 1, ScoreMode::kGather, 6>>(p, q, q_rows, p.kg, k_rows, st);
   return DSA_ERR_UNSUPPORTED;

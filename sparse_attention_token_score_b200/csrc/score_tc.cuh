@@ -38,6 +38,7 @@ namespace dsa {
 #define DSA_NACC_MAX 8
 #endif
 
+
 enum class ScoreMode : int { kTma = 0, kGather = 1, kRouter = 2 };
 
 struct ScoreParams {
@@ -59,7 +60,7 @@ struct ScoreParams {
   unsigned* err;            // device error word
 };
 
-template <int ELEM_, int D_, int H_, int QPT_, ScoreMode MODE_, int NSTAGE_, int EPIW_ = 8>
+template <int ELEM_, int D_, int H_, int QPT_, ScoreMode MODE_, int NSTAGE_, int EPIW_ = 8, int NQBUF_ = 1>
 struct ScoreCfg {
   static constexpr int ELEM = ELEM_;  // bytes per element: 2 = bf16, 1 = e4m3
   static constexpr int D = D_, H = H_, QPT = QPT_, NSTAGE = NSTAGE_;
@@ -106,9 +107,13 @@ struct ScoreCfg {
   static constexpr int NTHREADS = (EPI_WARP0 + EPIW) * 32;
   static constexpr int TEMPTY_ARRIVALS = SPLIT_TILES ? 4 : EPIW;
   static constexpr uint32_t IDESC = umma_idesc(ELEM == 2 ? 1u : 0u, 128, MMA_N);
-  // shared memory layout (offsets from a 1024-aligned base)
+  // shared memory layout (offsets from a 1024-aligned base). NQBUF query-tile
+  // buffers: with two, the next group's tile loads while the current group's
+  // keys still stream (pays off where groups are short, e.g. token gathers).
+  static constexpr int NQBUF = NQBUF_;
+  static_assert(NQBUF == 1 || NQBUF == 2, "query buffers");
   static constexpr int SMEM_Q = 0;
-  static constexpr int SMEM_K = Q_BYTES;
+  static constexpr int SMEM_K = NQBUF * Q_BYTES;
   // FP8: the epilogue applies per-key dequant scales (loaded from global
   // memory by the thread that owns the key, ahead of the tile's MMAs)
   static constexpr bool KEY_SCALES = ELEM == 1 && !ROUTER && !GATHER;
@@ -117,7 +122,7 @@ struct ScoreCfg {
   static constexpr int NCOL_THREAD = ROUTER ? 0 : (SPLIT_TILES ? QROWS : QROWS / NSETS);
   static constexpr int SMEM_COEF = SMEM_K + NSTAGE * K_BYTES;
   static constexpr int SMEM_BAR = SMEM_COEF + EPIW * NCOL_THREAD * 4;
-  static constexpr int NBAR = 2 * NSTAGE + 3 + 2 * NACC;
+  static constexpr int NBAR = 2 * NSTAGE + 2 * NQBUF + 2 * NACC + 1;
   static constexpr int SMEM_USED = SMEM_BAR + NBAR * 8 + 16;
   // Pad to more than half an SM so two CTAs never share an SM's TMEM.
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024 < 120 * 1024) ? 120 * 1024 : SMEM_USED + 1024;
@@ -262,11 +267,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   auto full = [&](int i) { return smem_u32(&bars[i]); };
   auto empty = [&](int i) { return smem_u32(&bars[C::NSTAGE + i]); };
-  const uint32_t qfull = smem_u32(&bars[2 * C::NSTAGE]);
-  const uint32_t qempty = smem_u32(&bars[2 * C::NSTAGE + 1]);
-  auto tfull = [&](int b) { return smem_u32(&bars[2 * C::NSTAGE + 2 + b]); };
-  auto tempty = [&](int b) { return smem_u32(&bars[2 * C::NSTAGE + 2 + C::NACC + b]); };
-  const uint32_t mdone = smem_u32(&bars[2 * C::NSTAGE + 2 + 2 * C::NACC]);
+  auto qfull = [&](int i) { return smem_u32(&bars[2 * C::NSTAGE + i]); };
+  auto qempty = [&](int i) { return smem_u32(&bars[2 * C::NSTAGE + C::NQBUF + i]); };
+  constexpr int TB = 2 * C::NSTAGE + 2 * C::NQBUF;
+  auto tfull = [&](int b) { return smem_u32(&bars[TB + b]); };
+  auto tempty = [&](int b) { return smem_u32(&bars[TB + C::NACC + b]); };
+  const uint32_t mdone = smem_u32(&bars[TB + 2 * C::NACC]);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -274,12 +280,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NSTAGE; ++i) {
       mbar_init(full(i), (C::GATHER && !p.blk_tma) ? 32 : 1);
-      // FP8: a stage is free once its MMAs are done and the epilogue warps of
-      // its tile have read the stage's key scales
-      mbar_init(empty(i), 1);
+      mbar_init(empty(i), 1);  // a stage is free once its MMAs are done
     }
-    mbar_init(qfull, 1);
-    mbar_init(qempty, 1);
+    for (int i = 0; i < C::NQBUF; ++i) {
+      mbar_init(qfull(i), 1);
+      mbar_init(qempty(i), 1);
+    }
     for (int b = 0; b < C::NACC; ++b) {
       mbar_init(tfull(b), 1);
       mbar_init(tempty(b), C::TEMPTY_ARRIVALS);
@@ -317,13 +323,15 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (s.first) {
         // The query tile is always loaded by warp 0, group by group in order.
         if (pw == 0 && lane == 0) {
-          if (!mbar_wait(qempty, (gq & 1u) ^ 1u, p.err)) { ok = false; }
+          const int qb = static_cast<int>(gq % C::NQBUF);
+          if (!mbar_wait(qempty(qb), ((gq / C::NQBUF) & 1u) ^ 1u, p.err)) { ok = false; }
           else {
-            mbar_arrive_expect_tx(qfull, C::Q_BYTES);
+            mbar_arrive_expect_tx(qfull(qb), C::Q_BYTES);
             const int row0 = (b * p.T + tg * C::QPT) * C::H;
 #pragma unroll
             for (int kb = 0; kb < C::KBLK; ++kb)
-              tma_load_2d(s_q + kb * C::QROWS * 128, &tm_q, qfull, kb * (128 / C::ELEM), row0);
+              tma_load_2d(s_q + qb * C::Q_BYTES + kb * C::QROWS * 128, &tm_q, qfull(qb),
+                          kb * (128 / C::ELEM), row0);
           }
         }
         ++gq;
@@ -420,7 +428,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (!ok && lane == 0) {
       // Error path: wait (bounded) for the TMA loads that may still be in
       // flight before the CTA releases its shared memory.
-      if (pw == 0 && gq > 0) mbar_drain(qfull, (gq - 1) & 1u);
+      if (pw == 0)
+        for (uint32_t g = gq > C::NQBUF ? gq - C::NQBUF : 0; g < gq; ++g)
+          mbar_drain(qfull(static_cast<int>(g % C::NQBUF)), (g / C::NQBUF) & 1u);
       if (!C::GATHER || p.blk_tma) {
         const uint32_t lo = it > C::NSTAGE ? it - C::NSTAGE : 0;
         for (uint32_t i = lo; i < it; ++i) mbar_drain(full(i % C::NSTAGE), (i / C::NSTAGE) & 1u);
@@ -432,7 +442,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       uint32_t it = 0, gq = 0;
       bool ok = true;
       for (; !s.done; s.next(p), ++it) {
-        if (s.first && !mbar_wait(qfull, gq & 1u, p.err)) { ok = false; break; }
+        const int qb = static_cast<int>(gq % C::NQBUF);
+        if (s.first && !mbar_wait(qfull(qb), (gq / C::NQBUF) & 1u, p.err)) { ok = false; break; }
         const int stage = static_cast<int>(it % C::NSTAGE);
         const uint32_t ph = (it / C::NSTAGE) & 1u;
         const int buf = static_cast<int>(it % C::NACC);
@@ -450,7 +461,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const int kb = (ks * 32) / 128;
           const int inner = (ks * 32) % 128;
           const uint64_t kdesc = umma_desc_sw128(k_tile + kb * C::KROWS * 128 + inner);
-          const uint64_t qdesc = umma_desc_sw128(s_q + kb * C::QROWS * 128 + inner);
+          const uint64_t qdesc = umma_desc_sw128(s_q + qb * C::Q_BYTES + kb * C::QROWS * 128 + inner);
           const uint64_t adesc = C::ROUTER ? qdesc : kdesc;
           const uint64_t bdesc = C::ROUTER ? kdesc : qdesc;
           if (C::ELEM == 2) mma_bf16(d_tmem, adesc, bdesc, C::IDESC, ks > 0 ? 1u : 0u);
@@ -458,7 +469,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         tc_commit(empty(stage));
         tc_commit(tfull(buf));
-        if (s.last) { tc_commit(qempty); ++gq; }
+        if (s.last) { tc_commit(qempty(qb)); ++gq; }
       }
       if (!ok) {
         // Error path: let every MMA already issued finish before TMEM is freed.
