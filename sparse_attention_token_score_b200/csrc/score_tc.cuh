@@ -10,12 +10,16 @@
 //
 // One persistent CTA per SM, warp-specialised:
 //   producer warp(s) -> shared-memory ring of key tiles (TMA, or cp.async
-//                       gathers of arbitrary key rows), plus the stationary
-//                       query tile of the current query group (TMA)
-//   MMA warp         -> one thread issues tcgen05.mma into a double-buffered
-//                       TMEM accumulator
-//   8 epilogue warps -> tcgen05.ld, ReLU, head-weighted sum, causal mask,
-//                       fp32 store. The [T, H, L] head logits never leave TMEM.
+//                       gathers of arbitrary key rows by four warps with
+//                       asynchronous completion), plus the stationary query
+//                       tile of the current query group (TMA; one or two
+//                       buffers)
+//   MMA warp         -> one thread issues tcgen05.mma into a ring of TMEM
+//                       accumulators (as many as fit in 512 columns, <= 8)
+//   8 epilogue warps -> tcgen05.ld, ReLU, head-weighted sum (head weights of
+//                       the query group staged in shared memory), causal
+//                       mask, fp32 store. The [T, H, L] head logits never
+//                       leave TMEM.
 //
 // Orientation (score modes): keys on the MMA M dimension (128 TMEM lanes, one
 // key per epilogue thread), QPT queries x H heads on N, so each thread reduces
