@@ -197,7 +197,7 @@ class Runner:
 # one ncu capture of the kernel named, valid only while its sources hash to
 # the value recorded with it (None otherwise). Full-size captures unless the
 # profile summary says it was scaled from a smaller case.
-_SC, _TK = "f4459abce1de", "b65c604b1af0"   # score_tc / topk_rows sources of the captures
+_SC, _TK = "483be90f01b3", "b877d4d6299f"   # score_tc / topk_rows sources of the captures
 TRAFFIC = {
     ("dsa", "score_tc<bf16>"): (86.33e6 + 448.97e6, _SC),
     ("dsa", "topk_rows"): (504.22e6 + 28.66e6, _TK),
@@ -216,12 +216,17 @@ KERNEL_SOURCES = {
 
 
 def source_hash(kernel_name):
+    """Hash of the kernel's source lines, full-line comments and blank lines
+    excluded (a comment edit does not invalidate a capture)."""
     import hashlib
     fam = "topk_rows" if kernel_name.startswith("topk_rows") else "score_tc"
     h = hashlib.sha1()
     for f in KERNEL_SOURCES[fam]:
-        with open(os.path.join(ROOT, "sparse_attention_token_score_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "sparse_attention_token_score_b200", "csrc", f)) as fh:
+            for line in fh:
+                t = line.strip()
+                if t and not t.startswith("//"):
+                    h.update(t.encode() + b"\n")
     return h.hexdigest()[:12]
 
 
