@@ -120,3 +120,13 @@ def test_many_long_rows():
     idx, sc = _run(s, rows, 0, 0, n, k)
     exp = _expect(s, rows, 0, 0, n, k)
     _check(s, idx, sc, exp, "many long rows")
+
+
+def test_many_long_rows_mass_ties():
+    # the long-row layout's fallback path: few distinct values, enough rows
+    # longer than 32768 to fill the GPU
+    rng = np.random.default_rng(12)
+    rows, n, k = 300, 36000, 1000
+    s = rng.integers(-3, 4, size=(rows, n)).astype(np.float32) * np.float32(0.5)
+    idx, sc = _run(s, rows, 0, 0, n, k)
+    _check(s, idx, sc, _expect(s, rows, 0, 0, n, k), "long rows, mass ties")
