@@ -32,6 +32,10 @@
  *     16-byte aligned.
  *   - Calls that share a workspace must not overlap in time (use one stream).
  *
+ *   - Calls may come from several host threads (each with its own
+ *     workspace); the current CUDA device is the one used. Device indices
+ *     of 64 and above return DSA_ERR_UNSUPPORTED.
+ *
  * Supported shapes: d in {64, 128}; bf16 H in {8, 16, 32, 64};
  * FP8 e4m3 (decode): d = 128, H in {32, 64}. Other shapes return
  * DSA_ERR_UNSUPPORTED.

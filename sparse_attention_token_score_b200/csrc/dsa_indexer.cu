@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <climits>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -65,33 +66,40 @@ bool make_tmap(CUtensorMap* m, const void* base, bool fp8, int D, long long rows
   return r == CUDA_SUCCESS;
 }
 
+// Per-device caches below are filled on first use; concurrent first calls
+// from several host threads may both fill an entry (idempotent), hence the
+// relaxed atomics.
 int current_device() {
   int dev = 0;
-  cudaGetDevice(&dev);
-  return dev < 0 || dev >= kMaxDev ? 0 : dev;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return -1;
+  return dev;
 }
 
 int num_sms() {
-  static int cache[kMaxDev] = {0};
+  static std::atomic<int> cache[kMaxDev];
   const int dev = current_device();
-  if (cache[dev] == 0) {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 1;
+  int n = dev >= 0 ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (n == 0) {
+    int d = 0;
+    cudaGetDevice(&d);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
+    if (n < 1) n = 1;
+    if (dev >= 0) cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 template <class C>
 dsa_status launch_score(const ScoreParams& p, const void* q, long long q_rows, const void* k,
                         long long k_rows, cudaStream_t st) {
-  static bool attr[kMaxDev] = {false};
+  static std::atomic<bool> attr[kMaxDev];
   const int dev = current_device();
-  if (!attr[dev]) {
+  if (dev < 0) return DSA_ERR_UNSUPPORTED;
+  if (!attr[dev].load(std::memory_order_relaxed)) {
     if (cudaFuncSetAttribute(score_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return DSA_ERR_CUDA;
-    attr[dev] = true;
+    attr[dev].store(true, std::memory_order_relaxed);
   }
   CUtensorMap tq, tk;
   if (!make_tmap(&tq, q, C::ELEM == 1, C::D, q_rows, C::QROWS)) return DSA_ERR_CUDA;
@@ -174,20 +182,21 @@ dsa_status run_gather(int D, int H, ScoreParams p, const void* q, long long q_ro
 // kernel's bounded waits report to.
 template <class C>
 dsa_status launch_topk_cfg(const TopkParams& tp, cudaStream_t st) {
-  static int ctas[kMaxDev] = {0};
+  static std::atomic<int> ctas[kMaxDev];
   const int dev = current_device();
-  if (ctas[dev] == 0) {
+  if (dev < 0) return DSA_ERR_UNSUPPORTED;
+  int occ = ctas[dev].load(std::memory_order_relaxed);
+  if (occ == 0) {
     if (cudaFuncSetAttribute(topk_rows_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES) !=
         cudaSuccess)
       return DSA_ERR_CUDA;
-    int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, topk_rows_kernel<C>, C::NT, C::BYTES) !=
             cudaSuccess ||
         occ < 1)
       return DSA_ERR_CUDA;
-    ctas[dev] = occ;
+    ctas[dev].store(occ, std::memory_order_relaxed);
   }
-  long long grid = static_cast<long long>(num_sms()) * ctas[dev];
+  long long grid = static_cast<long long>(num_sms()) * occ;
   if (tp.rows < grid) grid = tp.rows;
   topk_rows_kernel<C><<<static_cast<int>(grid), C::NT, C::BYTES, st>>>(tp);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
