@@ -93,6 +93,13 @@ DSA_EXPORT const char* dsa_status_string(dsa_status s);
  * last call that used this workspace, DSA_ERR_CUDA on a CUDA error, else OK. */
 DSA_EXPORT dsa_status dsa_device_status(void* workspace, void* stream);
 
+/* Self-test of the failure path (no counterpart on the pages): launches one
+ * warp whose bounded wait on a barrier that nothing completes gives up after
+ * the wait limit (2 s), records the timeout in the workspace's status word and
+ * returns; dsa_device_status then reports DSA_ERR_TIMEOUT and the context
+ * stays usable. Workspace: the 256-byte header only. */
+DSA_EXPORT dsa_status dsa_selftest_wait_timeout(void* workspace, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------ dense indexer
  * indexer_score_topk: for every query of every sequence, score all visible
  * keys with all H heads and keep the top `topk`.

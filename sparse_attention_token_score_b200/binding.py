@@ -42,6 +42,7 @@ _P = ctypes.c_void_p
 _SIGS = {
     "dsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dsa_device_status": (ctypes.c_int, [_P, _P]),
+    "dsa_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "indexer_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int]),
     "indexer_score_topk": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "indexer_score_topk_noalloc": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P]),
@@ -214,6 +215,11 @@ def hisa_block_filter_topk(args: IndexerArgs, block: int, m: int, topk: int, out
 
 def dsa_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(lib().dsa_device_status(_ptr(workspace), _stream_ptr(stream)))
+
+
+def dsa_selftest_wait_timeout(workspace: torch.Tensor, stream=None):
+    _check("dsa_selftest_wait_timeout",
+           lib().dsa_selftest_wait_timeout(_ptr(workspace), workspace.numel(), _stream_ptr(stream)))
 
 
 # ------------------------------------------------------------------ convenience

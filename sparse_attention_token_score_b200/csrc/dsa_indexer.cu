@@ -322,6 +322,14 @@ dsa_status dsa_device_status(void* workspace, void* stream) {
   return word ? DSA_ERR_TIMEOUT : DSA_OK;
 }
 
+dsa_status dsa_selftest_wait_timeout(void* workspace, size_t ws_bytes, void* stream) {
+  DSA_TRY(check_ws(workspace, ws_bytes, kHdr));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DSA_TRY(clear_status(workspace, st));
+  wait_timeout_kernel<<<1, 32, 0, st>>>(static_cast<unsigned*>(workspace));
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
 size_t indexer_workspace_size(const dsa_indexer_args* a, int topk) {
   (void)topk;
   if (!a || a->batch < 1 || a->T < 1 || a->L < 1) return 0;

@@ -83,4 +83,17 @@ __global__ void select_heads_kernel(const float* __restrict__ part, long long ro
   }
 }
 
+// Failure-path self-test: one warp waits on a barrier that nothing completes;
+// the bounded wait gives up after its limit and records the timeout in *err.
+__global__ void wait_timeout_kernel(unsigned* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, err);
+  __syncwarp();
+}
+
 }  // namespace dsa

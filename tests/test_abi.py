@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 13
+    assert len(names) == 14
     assert set(names) == set(B._SIGS)
     for n in names:
         assert getattr(lib, n) is not None
