@@ -18,6 +18,11 @@ widens them exactly to fp64 and follows the pages' steps in order:
 * HISA ("HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse
   Attention" review, section 3): score pooled block keys, keep the top-m
   blocks, score the tokens of the surviving blocks, keep the top-k.
+* DoSA certified pruning ("DoSA: Dots Sparse Attention" review, section 3):
+  a seed set scored with all heads bounds the k-th score from below, a
+  screened subset of heads bounds every other key's score from above, keys
+  whose bound is below the seeds' threshold are pruned, the survivors are
+  scored with all heads; the selection equals the dense one.
 
 Readings where the pages are silent (each is listed in the design notes):
 * Ties in any selection go to the lower index; a selection over fewer
@@ -30,6 +35,11 @@ Readings where the pages are silent (each is listed in the design notes):
   renormalisation.
 * FP8 inputs are dequantised exactly (scale * decoded byte) and scored in the
   unfactored form.
+* DoSA: the page names its bounds but gives no formulas; the upper bound
+  here keeps the screened heads' exact terms, bounds an unscreened head with
+  a positive weight by Cauchy-Schwarz and drops (bounds by 0) an unscreened
+  head with a non-positive weight; the seeds are the keys with the largest
+  screened partial scores.
 """
 from __future__ import annotations
 
@@ -343,3 +353,67 @@ def hisa(inp, block: int, m: int, topk: int, queries: Optional[Sequence[int]] = 
     out["blocks"] = np.array(out["blocks"], dtype=np.int64).reshape(len(queries), m)
     out["idx"] = np.array(out["idx"], dtype=np.int64).reshape(len(queries), topk)
     return out
+
+
+# ------------------------------------------------------------ DoSA (certified pruning)
+def dosa_upper_bound(q, k, w, t: int, keys: np.ndarray, screen: Sequence[int]):
+    """Upper bound on I[t,s] for each key s in ``keys`` from a subset of
+    heads ("DoSA: Dots Sparse Attention" review, section 3: screening dot
+    products and bound evaluation; the pages name the bounds but give no
+    formulas, this is the plainest sound choice):
+      - a screened head contributes its exact term w_h ReLU(q_h.k_s);
+      - an unscreened head with w_h > 0 contributes at most
+        w_h ||q_h|| ||k_s|| (Cauchy-Schwarz bounds ReLU(q_h.k_s));
+      - an unscreened head with w_h <= 0 contributes at most 0.
+    A relative slack of 1e-12 covers fp64 rounding. Returns (bound, screened
+    part of the score)."""
+    T, H, _ = q.shape
+    screen = np.unique(np.asarray(screen, dtype=np.int64))
+    hmask = np.zeros((T, H), dtype=np.uint8)
+    hmask[t, screen] = 1
+    keys = np.asarray(keys, dtype=np.int64)
+    part, pcond = score_pairs(q, k, w, np.full(keys.shape, t, dtype=np.int64), keys, hmask)
+    rest = np.setdiff1d(np.arange(H), screen)
+    pos = rest[w[t, rest] > 0]
+    a = float(np.sum(w[t, pos] * np.linalg.norm(q[t, pos], axis=1))) if pos.size else 0.0
+    kn = np.linalg.norm(np.asarray(k, dtype=np.float64)[keys], axis=1)
+    slack = 1e-12 * (pcond + a * kn) + 1e-300
+    return part + a * kn + slack, part
+
+
+def dosa_topk(inp, topk: int, screen: Sequence[int], n_seed: int,
+              queries: Optional[Sequence[int]] = None, b: int = 0):
+    """Certified exact top-k (DoSA review, section 3), per query:
+      1. the n_seed visible keys with the largest screened part of the score
+         (ties -> lower index) are scored with all heads; the topk-th best of
+         them, tau, is a lower bound on the row's k-th best score (-inf when
+         the seeds are fewer than topk);
+      2. every other visible key whose upper bound (dosa_upper_bound) is below
+         tau cannot be selected and is pruned;
+      3. the surviving keys are scored with all heads;
+      4. top-k (score descending, index ascending) over seeds and survivors.
+    The result equals dense_topk (lossless). Returns dict with 'idx'
+    [nq, topk], per query 'tau', 'survivors' (keys scored in step 3) and
+    'visible'."""
+    q, k, w = dequant(inp, b)
+    if queries is None:
+        queries = range(q.shape[0])
+    res = {"idx": [], "tau": [], "survivors": [], "visible": [], "queries": list(queries)}
+    for t in queries:
+        keys = np.arange(int(visible_count(inp.q_offset + t, k.shape[0])), dtype=np.int64)
+        bound, part = dosa_upper_bound(q, k, w, t, keys, screen)
+        order = np.lexsort((keys, -part))
+        seeds = np.sort(keys[order[:n_seed]])
+        _, s_seed, _ = dense_scores_row(q, k, w, t, inp.q_offset + t, keys=seeds)
+        tau = kth_score(s_seed, topk) if seeds.size >= topk else -np.inf
+        rest = np.setdiff1d(keys, seeds)
+        keep = rest[~(bound[rest] < tau)]
+        _, s_keep, _ = dense_scores_row(q, k, w, t, inp.q_offset + t, keys=keep)
+        cand = np.concatenate([seeds, keep])
+        res["idx"].append(select_topk(np.concatenate([s_seed, s_keep]), topk, index=cand))
+        res["tau"].append(tau)
+        res["survivors"].append(int(keep.size))
+        res["visible"].append(int(keys.size))
+    res["idx"] = np.array(res["idx"], dtype=np.int64).reshape(len(res["queries"]), topk)
+    return res
+

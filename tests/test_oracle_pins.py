@@ -335,3 +335,71 @@ def test_generator_deterministic_and_needles():
     qv = wl.bf16_bits_to_f32(a.q[0, a.meta["needle_src"][0]])
     assert np.array_equal(a.k[0, pos], wl.f32_to_bf16_bits(np.float32(0.5) * qv.mean(axis=1, dtype=np.float32)))
     assert wl.visible_pairs(16, 256, 200) == sum(min(201 + t, 256) for t in range(16))
+
+
+# ------------------------------------------------------------ DoSA certified pruning
+def _dosa_inp(seed, H=8, d=32, T=6, L=300, w_sign=0):
+    inp = wl.prefill_inputs(T=T, L=L, H=H, d=d, q_offset=L - T, seed=seed)
+    if w_sign < 0:
+        inp.w = -np.abs(inp.w)  # all heads negative: scores <= 0, mass ties at 0
+    return inp
+
+
+@pytest.mark.parametrize("screen", [[], [0], [1, 5], [0, 2, 4, 6], list(range(8))])
+def test_dosa_bound_is_sound(screen):
+    inp = _dosa_inp(41)
+    q, k, w = oracle.dequant(inp)
+    for t in range(inp.T):
+        p = inp.q_offset + t
+        keys = np.arange(p + 1)
+        bound, _ = oracle.dosa_upper_bound(q, k, w, t, keys, screen)
+        # exact scores by brute force (numpy, fp64), not through the oracle's core
+        x = np.einsum("hd,sd->hs", q[t], k[keys])
+        exact = (w[t][:, None] * np.maximum(x, 0.0)).sum(0)
+        assert np.all(bound >= exact)
+
+
+def test_dosa_bound_is_tight_with_every_head_screened():
+    inp = _dosa_inp(42)
+    q, k, w = oracle.dequant(inp)
+    keys = np.arange(inp.q_offset + 1)
+    bound, part = oracle.dosa_upper_bound(q, k, w, 0, keys, range(8))
+    x = np.einsum("hd,sd->hs", q[0], k[keys])
+    exact = (w[0][:, None] * np.maximum(x, 0.0)).sum(0)
+    assert np.allclose(bound, exact, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed,screen,n_seed,w_sign", [
+    (43, [0, 1], 64, 0), (44, [3], 32, 0), (45, [], 64, 0),       # no screened head: bounds from norms only
+    (46, [0, 1, 2, 3], 8, 0),                                      # fewer seeds than k: tau = -inf, no pruning
+    (47, [2, 6], 64, -1),                                          # all-negative weights: ties at 0
+])
+def test_dosa_equals_dense(seed, screen, n_seed, w_sign):
+    inp = _dosa_inp(seed, w_sign=w_sign)
+    if seed == 44:
+        inp.k[0, 100:110] = inp.k[0, 50]  # duplicate keys: exact ties across positions
+    topk = 16
+    dense = oracle.dense_topk(inp, topk)
+    dosa = oracle.dosa_topk(inp, topk, screen, n_seed)
+    assert np.array_equal(dense["idx"], dosa["idx"])
+    for i, t in enumerate(dense["queries"]):
+        kth = oracle.kth_score(dense["scores"][i], topk)
+        assert dosa["tau"][i] <= kth            # the seeds' k-th score bounds the row's from below
+    if n_seed < topk:
+        assert dosa["survivors"] == [v - min(n_seed, v) for v in dosa["visible"]]
+
+
+def test_dosa_planted_mistake_is_caught(monkeypatch):
+    # a bound that forgets the unscreened positive-weight heads is unsound;
+    # the selection then loses winners and no longer equals the dense one
+    real = oracle.dosa_upper_bound
+
+    def forgetful(q, k, w, t, keys, screen):
+        bound, part = real(q, k, w, t, keys, screen)
+        return part, part
+
+    monkeypatch.setattr(oracle, "dosa_upper_bound", forgetful)
+    inp = _dosa_inp(48, H=8, T=8, L=400)
+    dense = oracle.dense_topk(inp, 16)
+    dosa = oracle.dosa_topk(inp, 16, [0], 32)
+    assert not np.array_equal(dense["idx"], dosa["idx"])
