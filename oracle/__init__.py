@@ -36,10 +36,12 @@ Readings where the pages are silent (each is listed in the design notes):
 * FP8 inputs are dequantised exactly (scale * decoded byte) and scored in the
   unfactored form.
 * DoSA: the page names its bounds but gives no formulas; the upper bound
-  here keeps the screened heads' exact terms, bounds an unscreened head with
-  a positive weight by Cauchy-Schwarz and drops (bounds by 0) an unscreened
-  head with a non-positive weight; the seeds are the keys with the largest
-  screened partial scores.
+  here keeps the screened heads' exact terms, bounds the unscreened
+  positive-weight heads jointly through ReLU(x) = (x + |x|) / 2 (one
+  aggregated dot product plus Cauchy-Schwarz on |x|) and subtracts ReLU of
+  one aggregated dot product for the unscreened negative-weight heads
+  (subadditivity of ReLU); the seeds are the keys with the largest screened
+  partial scores.
 """
 from __future__ import annotations
 
@@ -359,12 +361,16 @@ def hisa(inp, block: int, m: int, topk: int, queries: Optional[Sequence[int]] = 
 def dosa_upper_bound(q, k, w, t: int, keys: np.ndarray, screen: Sequence[int]):
     """Upper bound on I[t,s] for each key s in ``keys`` from a subset of
     heads ("DoSA: Dots Sparse Attention" review, section 3: screening dot
-    products and bound evaluation; the pages name the bounds but give no
-    formulas, this is the plainest sound choice):
-      - a screened head contributes its exact term w_h ReLU(q_h.k_s);
-      - an unscreened head with w_h > 0 contributes at most
-        w_h ||q_h|| ||k_s|| (Cauchy-Schwarz bounds ReLU(q_h.k_s));
-      - an unscreened head with w_h <= 0 contributes at most 0.
+    products and bound evaluation; the page names a seed-set threshold,
+    nonnegative head projection, joint residual bounds and an aggregate of the
+    omitted negative heads, without formulas). With x_h = q_h.k_s:
+      - screened heads contribute their exact terms w_h ReLU(x_h);
+      - unscreened heads with w_h > 0 (set P): ReLU(x) = (x + |x|) / 2 gives
+        sum_P w_h ReLU(x_h) <= (k_s.v_P + A_P ||k_s||) / 2 with the aggregate
+        v_P = sum_P w_h q_h and A_P = sum_P w_h ||q_h|| (|x_h| <= ||q_h|| ||k_s||);
+      - unscreened heads with w_h < 0 (set N): ReLU is subadditive, so
+        sum_N |w_h| ReLU(x_h) >= ReLU(k_s.v_N) with v_N = sum_N |w_h| q_h, and
+        their (negative) contribution is at most -ReLU(k_s.v_N).
     A relative slack of 1e-12 covers fp64 rounding. Returns (bound, screened
     part of the score)."""
     T, H, _ = q.shape
@@ -374,11 +380,19 @@ def dosa_upper_bound(q, k, w, t: int, keys: np.ndarray, screen: Sequence[int]):
     keys = np.asarray(keys, dtype=np.int64)
     part, pcond = score_pairs(q, k, w, np.full(keys.shape, t, dtype=np.int64), keys, hmask)
     rest = np.setdiff1d(np.arange(H), screen)
-    pos = rest[w[t, rest] > 0]
-    a = float(np.sum(w[t, pos] * np.linalg.norm(q[t, pos], axis=1))) if pos.size else 0.0
-    kn = np.linalg.norm(np.asarray(k, dtype=np.float64)[keys], axis=1)
-    slack = 1e-12 * (pcond + a * kn) + 1e-300
-    return part + a * kn + slack, part
+    wt = np.asarray(w[t], dtype=np.float64)
+    qt = np.asarray(q[t], dtype=np.float64)
+    kk = np.asarray(k, dtype=np.float64)[keys]
+    pos, neg = rest[wt[rest] > 0], rest[wt[rest] < 0]
+    v_p = (wt[pos, None] * qt[pos]).sum(0)
+    a_p = float(np.sum(wt[pos] * np.linalg.norm(qt[pos], axis=1))) if pos.size else 0.0
+    v_n = (-wt[neg, None] * qt[neg]).sum(0)
+    kn = np.linalg.norm(kk, axis=1)
+    lin_p = kk @ v_p
+    up = 0.5 * (lin_p + a_p * kn)
+    down = np.maximum(kk @ v_n, 0.0)
+    slack = 1e-12 * (pcond + a_p * kn + np.abs(lin_p) + down) + 1e-300
+    return part + up - down + slack, part
 
 
 def dosa_topk(inp, topk: int, screen: Sequence[int], n_seed: int,
