@@ -94,3 +94,42 @@ def test_variant_argument_checks(lib):
     assert lib.hisa_block_filter_topk(ctypes.byref(h8), 128, 2, 16, out, None, None, ws, big, None) == -2
     assert lib.indexer_topk_rows(None, 4, 256, 4, 0, 1, 256, 16, None, 0, 1, out, None, ws, big, None) == -1
     assert lib.dsa_meanpool_keys(None, 1, 256, 128, 64, ws, None) == -1
+
+
+def test_stage_entry_point_checks(lib):
+    a = _args()
+    out = ctypes.c_void_p(0x40000)
+    ws = ctypes.c_void_p(0x50000)
+    big = 1 << 40
+    # indexer_scores: row pitch below L, missing output, missing workspace
+    assert lib.indexer_scores(ctypes.byref(a), out, 255, ws, big, None) == -1
+    assert lib.indexer_scores(ctypes.byref(a), None, 256, ws, big, None) == -1
+    assert lib.indexer_scores(ctypes.byref(a), out, 256, None, big, None) == -3
+    # indexer_score_gathered: missing candidates, empty slots, pitch below the
+    # compact row, head counts / dims / dtype the gather does not support
+    cand = ctypes.c_void_p(0x60000)
+    assert lib.indexer_score_gathered(ctypes.byref(a), None, 8, 1, out, 8, ws, big, None) == -1
+    assert lib.indexer_score_gathered(ctypes.byref(a), cand, 0, 1, out, 8, ws, big, None) == -1
+    assert lib.indexer_score_gathered(ctypes.byref(a), cand, 8, 128, out, 1000, ws, big, None) == -1
+    assert lib.indexer_score_gathered(ctypes.byref(_args(H=16)), cand, 8, 1, out, 8, ws, big, None) == -2
+    assert lib.indexer_score_gathered(ctypes.byref(_args(d=64)), cand, 8, 1, out, 8, ws, big, None) == -2
+    f = _args(qk_dtype=B.DSA_FP8_E4M3, q_scale=0x60000, k_scale=0x70000)
+    assert lib.indexer_score_gathered(ctypes.byref(f), cand, 8, 1, out, 8, ws, big, None) == -2
+    # indexer_topk_rows: pitch below the row, index map shorter than the row,
+    # k out of range, negative position stride
+    sc = ctypes.c_void_p(0x80000)
+    assert lib.indexer_topk_rows(sc, 4, 100, 4, 0, 0, 256, 16, None, 0, 1, out, None, ws, big, None) == -1
+    assert lib.indexer_topk_rows(sc, 4, 256, 4, 0, 0, 256, 16, cand, 3, 64, out, None, ws, big, None) == -1
+    assert lib.indexer_topk_rows(sc, 4, 256, 4, 0, 0, 256, (1 << 24) + 1, None, 0, 1, out, None, ws, big,
+                                 None) == -1
+    assert lib.indexer_topk_rows(sc, 4, 256, 4, 0, -1, 256, 16, None, 0, 1, out, None, ws, big, None) == -1
+
+
+def test_selftest_and_noalloc_checks(lib):
+    assert lib.dsa_selftest_wait_timeout(None, 256, None) == -3
+    assert lib.dsa_selftest_wait_timeout(ctypes.c_void_p(0x50010), 256, None) == -1
+    assert lib.dsa_selftest_wait_timeout(ctypes.c_void_p(0x50000), 100, None) == -3
+    # the static scratch holds the scores of at most 16 M pairs: larger problems
+    # are refused before any CUDA call
+    a = _args(T=4, L=5_000_000, q_offset=4_999_996)
+    assert lib.indexer_score_topk_noalloc(ctypes.byref(a), 16, ctypes.c_void_p(0x40000), None, None) == -3
