@@ -52,3 +52,21 @@ def test_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     f.write_text(f.read_text() + "\nstatic int changed_code = 1;\n")  # code does
     assert bench.traffic_for(*key) is None
     assert bench.traffic_for("dsa", "no such kernel") is None
+
+
+def test_reference_arm_json_line():
+    # the oracle arm needs no GPU: one JSON line with the contract's keys
+    import json
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, check=True).stdout
+    line = json.loads(out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["warmup"] == 3
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    assert line["config"]["workload"].startswith("tiny_prefill")
