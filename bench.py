@@ -3,28 +3,32 @@
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-One step = one pass of the indexer hot path over one batch of resident inputs:
-for the default workload (the DeepSeek-V3.2-shaped prefill chunk: T=4096
-queries at the end of a 32768-token prefix, H_I=64, d=128, top-k=2048) that is
-tcgen05 scoring of every visible (query, key) pair followed by the per-query
-radix top-k, both through the C-ABI entry point indexer_score_topk.
-Other workloads: tiny, decode (FP8), misa (MISA-dagger), hisa.
+One step = one pass of the indexer hot path over one batch of resident inputs.
+The headline line is the DeepSeek-V3.2-shaped prefill chunk (T=4096 queries at
+the end of a 32768-token prefix, H_I=64, d=128, top-k=2048): tcgen05 scoring of
+every visible (query, key) pair followed by the per-query radix top-k, both
+through the C-ABI entry point indexer_score_topk. By default the same run also
+measures the other four workloads (tiny prefill, FP8 decode, MISA-dagger,
+HISA) and reports each under "workloads" with the same fields; --workload
+NAME measures one workload alone as the headline.
 
 The metric is scored query-key pairs per second (visible pairs of the dense
 problem, so routed / filtered variants show their speed-up in the same unit).
-Timing: W warm-up steps, then K steps, each preceded by a 256 MiB L2 flush
-and timed with CUDA events on the launching stream; a barrier + synchronize
-bracket the timed region; the max over ranks is reported. With N > 1 every
-rank runs an independent replica on its own GPU (the path has no exchange
-step), so the aggregate is weak scaling.
+Timing: W warm-up steps, then K steps (sub-records: at least 60 ms of steps),
+each preceded by a 256 MiB L2 flush and timed with CUDA events on the
+launching stream; a barrier + synchronize bracket the timed region; the max
+over ranks is reported. With N > 1 every rank runs an independent replica on
+its own GPU (the path has no exchange step), so the aggregate is weak scaling.
 
-Extra keys: roofline of the dominant kernel (every kernel of the step timed
-alone on the inputs the step gives it; the slowest is the roofline's, all are
-listed under "kernels"),
-cpu_baseline (the fp64 oracle on a bounded sample, host cores), e2e (host
-buffers: every step copies its inputs in and its indices out inside the timed
-region, double-buffered so copies overlap the previous step's call), clocks
-sampled during the timed region, gpu_launches.
+Extra keys: roofline of the dominant kernel (after the timed region, the
+same number of steps runs again with the library's launch profiler on: every
+launch bracketed by CUDA events on its stream; all kernels are listed under
+"kernels" with their time per step, and the slowest one with known
+algorithmic work is the roofline's), cpu_baseline (the fp64 oracle on a
+bounded sample, host cores), e2e (host buffers: every step copies its inputs
+in and its indices out inside the timed region, double-buffered so copies
+overlap the previous step's call), clocks sampled by NVML every 5 ms during
+the timed region, gpu_launches (counted by the profiler).
 """
 from __future__ import annotations
 
@@ -32,9 +36,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -70,14 +72,22 @@ def workload_desc(name, queries=None, batch=None):
     batch = c.get("batch", 1)
     off = c.get("q_offset", c["L"] - 1)
     pairs = wl.visible_pairs(c["T"], c["L"], off, batch)
+    if name == "indexcache":  # pairs of the dense problem of every layer
+        pairs *= len(c["pattern"])
     tag = {"tiny": "tiny_prefill", "dsa": "dsa_chunk", "decode": "decode_fp8",
-           "misa": "misa_dagger", "hisa": "hisa"}[name]
+           "misa": "misa_dagger", "hisa": "hisa", "dsa_fp8": "dsa_chunk_fp8",
+           "indexcache": "indexcache_dsa_chunk"}[name]
     label = f"{tag}_B{batch}_T{c['T']}_L{c['L']}_H{c['H']}_d{c['d']}_k{c['topk']}"
     if name == "misa":
         label += f"_blk{c['block']}_h{c['h']}_kp{c['kprime']}"
     if name == "hisa":
         label += f"_blk{c['block']}_m{c['m']}"
+    if name == "indexcache":
+        label += f"_layers{c['pattern']}"
     return c, batch, off, pairs, label
+
+
+DENSE = ("tiny", "dsa", "decode", "dsa_fp8", "indexcache")  # workloads whose F layer is indexer_score_topk
 
 
 class Runner:
@@ -95,22 +105,27 @@ class Runner:
         self.topk = c["topk"]
         self.idx = torch.empty((self.batch, c["T"], self.topk), dtype=torch.int32, device="cuda")
         a = self.ix.args
-        if name in ("tiny", "dsa", "decode"):
+        if name in DENSE:
             self.ws = B.alloc_workspace(B.indexer_workspace_size(a, self.topk))
-            self.launches = 2
+            if name == "indexcache":
+                pat = c["pattern"]
+                assert pat.count("F") == 1, "the bench's IndexCache slice has one F layer"
+                self.shared = B.IndexerArgs(batch=self.batch, T=c["T"])  # S layers: shape only
         elif name == "misa":
             self.ws = B.alloc_workspace(B.misa_workspace_size(a, c["block"], c["h"], self.topk, c["kprime"]))
-            self.launches = 7  # meanpool, router, select_heads, routed score, top-k', gather score, top-k
         else:
             self.ws = B.alloc_workspace(B.hisa_workspace_size(a, c["block"], c["m"], self.topk))
-            self.launches = 5  # meanpool, block score, top-m, gather score, top-k
         self.dtype = "e4m3" if inp.dtype != "bf16" else "bf16"
 
     def step(self, args=None, out=None):
         B, c = self.B, self.c
         a = self.ix.args if args is None else args
         o = self.idx if out is None else out
-        if self.name in ("tiny", "dsa", "decode"):
+        if self.name == "indexcache":
+            # S layers share the F layer's index buffer (the page's index cache)
+            layers = [a if r == "F" else self.shared for r in c["pattern"]]
+            B.indexcache_score_topk(layers, c["pattern"], self.topk, [o] * len(layers), None, self.ws)
+        elif self.name in DENSE:
             B.indexer_score_topk(a, self.topk, o, None, self.ws)
         elif self.name == "misa":
             B.misa_route_score_topk(a, c["block"], c["h"], self.topk, c["kprime"], o, None, None,
@@ -118,79 +133,54 @@ class Runner:
         else:
             B.hisa_block_filter_topk(a, c["block"], c["m"], self.topk, o, None, None, self.ws)
 
-    # ---- the step's kernels, each launched alone through the C-ABI on the
-    # inputs the step gives it (roofline and per-kernel shares)
-    def kernels(self):
-        """List of (name, callable, algorithmic units per launch, bound), in
-        the step's order. Units: FLOPs for tensor-bound kernels (2 * d per
-        head per scored pair), bytes for HBM-bound ones."""
-        B, torch, c = self.B, self.torch, self.c
+    # ---- algorithmic units of the step's kernels (per step), by the name the
+    # library's launch profiler files them under
+    def kernel_units(self, name):
+        """(units per step, bound) of a profiled kernel, or (None, None) when
+        its work depends on data the host does not see (list lengths, sample
+        sizes). Units: FLOPs (2 * d per head per scored pair) for the tensor
+        core kernels, bytes for the HBM-bound ones."""
+        c, inp = self.c, self.inp
         T, L, H, d, k = c["T"], c["L"], c["H"], c["d"], self.topk
         rows = self.batch * T
-        ws = B.alloc_workspace(256)
-        keep = [ws]
-        out = []
-        if self.name in ("tiny", "dsa", "decode"):
-            sc = torch.empty((self.batch, T, L), dtype=torch.float32, device="cuda")
-            idx = torch.empty((self.batch, T, k), dtype=torch.int32, device="cuda")
-            keep += [sc, idx]
-            f_score = lambda: B.indexer_scores(self.ix.args, sc, L, ws)
-            f_score()
-            if self.name == "decode":
-                # one FP8 key row + its fp32 scale per visible pair
-                out.append(("score_tc<fp8>", f_score, self.pairs * (d + 4), "hbm"))
-            else:
-                out.append(("score_tc<bf16>", f_score, self.pairs * 2.0 * d * H, "tensor"))
-            # every visible score read once, k indices written per row
-            out.append(("topk_rows", lambda: B.indexer_topk_rows(sc, rows, L, T, self.inp.q_offset, 1, L, k,
-                                                                 None, 0, 1, idx, None, ws),
-                        self.pairs * 4 + rows * k * 4, "hbm"))
-        elif self.name == "misa":
-            h, kp = c["h"], c["kprime"]
-            q, kk, w, _, _ = self.dev
-            # the routed pass scores with h heads per query: the same kernel on a
-            # query tensor of h heads (head choice does not change its cost)
-            qh, wh = q[:, :, :h].contiguous(), w[:, :, :h].contiguous()
-            ah = B.make_args(qh, kk, wh, self.inp.q_offset)
-            routed = torch.empty((self.batch, T, L), dtype=torch.float32, device="cuda")
-            cand = torch.empty((self.batch, T, kp), dtype=torch.int32, device="cuda")
-            comp = torch.empty((self.batch, T, kp), dtype=torch.float32, device="cuda")
-            idx = torch.empty((self.batch, T, k), dtype=torch.int32, device="cuda")
-            keep += [qh, wh, ah, routed, cand, comp, idx]
-            B.misa_route_score_topk(self.ix.args, c["block"], h, k, kp, idx, None, None, cand, self.ws)
-            f_routed = lambda: B.indexer_scores(ah, routed, L, ws)
-            f_routed()
-            out.append(("score_tc<bf16,h=%d> (routed)" % h, f_routed, self.pairs * 2.0 * d * h, "tensor"))
-            out.append(("topk_rows (k'=%d over routed rows)" % kp,
-                        lambda: B.indexer_topk_rows(routed, rows, L, T, self.inp.q_offset, 1, L, kp, None,
-                                                    0, 1, cand, None, ws),
-                        self.pairs * 4 + rows * kp * 4, "hbm"))
-            f_gather = lambda: B.indexer_score_gathered(self.ix.args, cand, kp, 1, comp, kp, ws)
-            f_gather()
-            out.append(("score_tc<bf16> gathered (MISA-dagger re-score)", f_gather,
-                        rows * kp * 2.0 * d * H, "tensor"))
-            out.append(("topk_rows (k=%d over k' candidates)" % k,
-                        lambda: B.indexer_topk_rows(comp, rows, kp, T, self.inp.q_offset, 0, kp, k, cand,
-                                                    kp, 1, idx, None, ws),
-                        rows * kp * 4 + rows * k * 8, "hbm"))
-        else:
-            m, blk = c["m"], c["block"]
-            nc = m * blk
-            blocks = torch.empty((self.batch, T, m), dtype=torch.int32, device="cuda")
-            comp = torch.empty((self.batch, T, nc), dtype=torch.float32, device="cuda")
-            idx = torch.empty((self.batch, T, k), dtype=torch.int32, device="cuda")
-            keep += [blocks, comp, idx]
-            B.hisa_block_filter_topk(self.ix.args, blk, m, k, idx, None, blocks, self.ws)
-            f_gather = lambda: B.indexer_score_gathered(self.ix.args, blocks, m, blk, comp, nc, ws)
-            f_gather()
-            out.append(("score_tc<bf16> gathered (HISA kept blocks)", f_gather,
-                        rows * nc * 2.0 * d * H, "tensor"))
-            out.append(("topk_rows (k=%d over m*block tokens)" % k,
-                        lambda: B.indexer_topk_rows(comp, rows, nc, T, self.inp.q_offset, 0, nc, k, blocks,
-                                                    m, blk, idx, None, ws),
-                        rows * nc * 4 + rows * k * 8, "hbm"))
-        self._keep = keep
-        return out
+        pos = inp.q_offset + np.arange(T, dtype=np.int64)
+        label = name.split(": ")[-1]
+        stage = name.split(": ")[0] if ": " in name else ""
+        if "sample pass" in stage or "candidate lists)" in label:
+            return None, None
+        if self.name in DENSE:
+            pairs = self.pairs // len(c.get("pattern", "F"))  # the F layer's pairs (indexcache)
+            if label.startswith("score_tc"):
+                if self.name == "decode":
+                    return pairs * (d + 4), "hbm"          # one FP8 key row + its scale per pair
+                return pairs * 2.0 * d * H, ("tensor_fp8" if self.name == "dsa_fp8" else "tensor")
+            if label == "topk_rows":
+                return pairs * 4 + rows * k * 4, "hbm"    # every visible score read, k ids written
+        if self.name == "misa":
+            blk, h, kp = c["block"], c["h"], c["kprime"]
+            M = -(-L // blk)
+            vis_blocks = int(self.batch * np.minimum(pos // blk + 1, M).sum())
+            if stage == "router":
+                return vis_blocks * 2.0 * d * H, "tensor"
+            if stage == "routed" and label.startswith("score_tc"):
+                return self.pairs * 2.0 * d * h, "tensor"
+            if stage == "routed" and label == "topk_rows":
+                return self.pairs * 4 + rows * kp * 4, "hbm"
+            if stage == "re-score" and label.startswith("score_tc"):
+                return rows * kp * 2.0 * d * H, "tensor"
+            if stage == "re-score" and label == "topk_rows":
+                return rows * kp * 4 + rows * k * 8, "hbm"
+        if self.name == "hisa":
+            blk, m = c["block"], c["m"]
+            M = -(-L // blk)
+            vis_blocks = int(self.batch * np.minimum(pos // blk + 1, M).sum())
+            if stage == "blocks" and label.startswith("score_tc"):
+                return vis_blocks * 2.0 * d * H, "tensor"
+            if stage == "tokens" and label.startswith("score_"):
+                return rows * m * blk * 2.0 * d * H, "tensor"
+            if stage == "tokens" and label == "topk_rows":
+                return rows * m * blk * 4 + rows * k * 8, "hbm"
+        return None, None
 
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
@@ -328,39 +318,85 @@ def run_e2e(r, inp, steps, torch, barrier):
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons sampled while the GPU works: NVML polled
+    from a thread every 5 ms (nvidia-smi at 200 ms where NVML is missing).
+    Only samples taken between mark_start() and mark_stop() are reported, so
+    the record covers exactly the timed region."""
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
 
-    def __init__(self, gpu_index):
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+    def __init__(self, device_index):
+        import threading
+        self.samples = []          # (monotonic s, sm MHz, max MHz, reason bits)
+        self.t0 = self.t1 = None
+        self.stop_flag = threading.Event()
+        self.nvml = None
         try:
-            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                       "-i", str(gpu_index), "-lms", "200"], stdout=self.f,
-                                      stderr=subprocess.DEVNULL)
-        except OSError:
-            self.p = None
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.nvml = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.nvml = None
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _reasons(self):
+        p = self.nvml
+        f = getattr(p, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(p, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return int(f(self.h))
+
+    def _run(self):
+        if self.nvml is None:
+            return
+        p = self.nvml
+        while not self.stop_flag.is_set():
+            try:
+                sm = float(p.nvmlDeviceGetClockInfo(self.h, p.NVML_CLOCK_SM))
+                self.samples.append((time.monotonic(), sm, self.max_mhz, self._reasons()))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_stop(self):
+        self.t1 = time.monotonic()
 
     def stop(self):
-        if self.p is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
-        self.p.terminate()
-        self.p.wait(timeout=10)
-        self.f.flush()
-        self.f.seek(0)
-        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.count(",") >= 8]
-        os.unlink(self.f.name)
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v and "Not" not in v})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        if self.nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["NVML unavailable"], "samples": 0}
+        return self.summarize(self.samples, self.t0, self.t1, self.max_mhz)
+
+    @classmethod
+    def summarize(cls, samples, t0, t1, max_mhz):
+        """Median SM clock and the throttle reasons seen in samples with
+        t0 <= time <= t1; the samples just before t0 and just after t1 are kept
+        too, so a region shorter than the polling interval still has a record."""
+        if t0 is None:
+            return {"sm_mhz": None, "sm_max_mhz": max_mhz, "reasons": [], "samples": 0}
+        t1 = t1 if t1 is not None else float("inf")
+        inside = [r for r in samples if t0 <= r[0] <= t1]
+        before = [r for r in samples if r[0] < t0][-1:]
+        after = [r for r in samples if r[0] > t1][:1]
+        rows = before + inside + after
+        sm = [r[1] for r in rows]
+        reasons = sorted({n for r in rows for n, bit in cls.REASONS.items() if r[3] & bit})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max_mhz,
+                "reasons": reasons, "samples": len(rows), "samples_inside": len(inside),
+                "source": "NVML, every 5 ms"}
 
 
 # ------------------------------------------------------------------ oracle (CPU) timing
-def oracle_sample(name, inp, budget_s=10.0, max_q=4096):
+def oracle_sample(name, inp, budget_s=10.0, max_q=4096, with_pairs=False):
     """Time the fp64 oracle, as it stands, on a bounded sample of this workload's
     queries (the same computation as one GPU step, restricted to the sample)."""
     import oracle
@@ -380,8 +416,10 @@ def oracle_sample(name, inp, budget_s=10.0, max_q=4096):
         return time.perf_counter() - t0
 
     def pairs(qs, b=0):
+        # IndexCache: the oracle runs the F layer; its S layers reuse the indices
+        # (as on the GPU), and the dense pairs of every layer count
         off = inp.q_offset
-        return int(sum(min(off + int(t) + 1, inp.L) for t in qs))
+        return int(sum(min(off + int(t) + 1, inp.L) for t in qs)) * len(c.get("pattern", "F"))
 
     if name == "decode":
         # one unit = one sequence's query; add sequences until budget_s is spent
@@ -389,7 +427,8 @@ def oracle_sample(name, inp, budget_s=10.0, max_q=4096):
         while t < budget_s and nb < inp.batch:
             t += run([0], b=nb)
             nb += 1
-        return nb * inp.L / t / 1e9, f"{nb} of {inp.batch} sequences (all {inp.L} keys each)", nb, t
+        res = (nb * inp.L / t / 1e9, f"{nb} of {inp.batch} sequences (all {inp.L} keys each)", nb, t)
+        return res + (nb * inp.L,) if with_pairs else res
     # grow the sample until one run takes at least budget_s (or covers every query)
     n = 8
     while True:
@@ -399,31 +438,48 @@ def oracle_sample(name, inp, budget_s=10.0, max_q=4096):
         if t >= budget_s or n >= min(T, max_q):
             break
         n = int(n * min(8.0, max(2.0, 1.2 * budget_s / max(t, 1e-3))))
-    return pairs(qs) / t / 1e9, f"{len(qs)} of {T} queries (uniform sample)", len(qs), t
+    res = (pairs(qs) / t / 1e9, f"{len(qs)} of {T} queries (uniform sample)", len(qs), t)
+    return res + (pairs(qs),) if with_pairs else res
+
+
+def workload_config(r_c, batch, label, q_offset, pairs, world):
+    """The `config` object of a JSON line (the same for both arms)."""
+    return {"workload": label, "batch": batch, "T": r_c["T"], "L": r_c["L"], "H": r_c["H"],
+            "d": r_c["d"], "topk": r_c["topk"], "q_offset": q_offset, "pairs_per_step": pairs,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "256 MiB buffer written before every timed step"}
 
 
 def run_reference(args):
-    """The oracle arm: fp64 CPU oracle on host cores, bounded sample per step."""
+    """The oracle arm: the fp64 CPU oracle, as it stands, on the host cores; each
+    step is a bounded query sample of the headline workload, timed as it runs
+    (ms_per_step is that sample's time, value its pairs / time)."""
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
     import oracle
     from sparse_attention_token_score_b200 import workloads as wl
-    c, batch, off, pairs, label = workload_desc(args.workload)
-    inp = wl.make_inputs(args.workload, seed=0)
+    name = "dsa" if args.workload == "all" else args.workload
+    c, batch, off, pairs, label = workload_desc(name)
+    inp = wl.make_inputs(name, seed=0)
     per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
-    vals, samples = [], None
+    vals, secs, npairs, samples = [], [], [], None
     for i in range(args.warmup + args.steps):
-        v, samples, _, _ = oracle_sample(args.workload, inp, budget_s=per_step / 2)
+        v, samples, _, t, p = oracle_sample(name, inp, budget_s=per_step / 2, with_pairs=True)
         if i >= args.warmup:
             vals.append(v)
-    value = float(np.mean(vals))
+            secs.append(t)
+            npairs.append(p)
+    value = float(sum(npairs) / sum(secs) / 1e9)
     cores = oracle.num_threads()
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": pairs / (value * 1e9) * 1e3, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(secs)), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": label, "pairs_per_step": pairs, "parallelism": "host cores"},
+            "config": workload_config(c, batch, label, off, pairs, world),
+            "sample": {"what": samples, "pairs_per_timed_step": int(np.mean(npairs)),
+                       "note": "each step times the oracle on this query sample of the workload"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": samples},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -451,22 +507,128 @@ def make_inputs(name, seed, queries=0, batch=0):
 
 
 # ------------------------------------------------------------------ main
+SUB_WORKLOADS = ("tiny", "decode", "misa", "hisa", "dsa_fp8", "indexcache")
+MIN_TIMED_MS = 60.0  # sub-records run enough steps that the clock sampler sees the GPU busy
+
+
+def measure_workload(name, args, torch, world, rank, local, flush, barrier, rmax, steps,
+                     cpu_budget_s, min_timed_ms=0.0):
+    """Everything one JSON record says about a workload, measured in this
+    process: timed steps, each kernel alone (roofline), end to end through
+    host buffers, clocks during the timed region, and the oracle's CPU rate."""
+    inp = make_inputs(name, rank, args.queries, args.batch)
+    r = Runner(name, inp, torch, args.queries, args.batch)
+    for _ in range(args.warmup):
+        r.step()
+    torch.cuda.synchronize()
+    if min_timed_ms > 0:  # lengthen short workloads' timed regions (same count on every rank)
+        probe = statistics.median(time_steps(r.step, 3, torch, flush))
+        steps = max(steps, int(np.ceil(min_timed_ms / max(probe, 1e-3))))
+        if world > 1:
+            steps = int(rmax(steps))
+
+    # ---- timed region
+    sampler = ClockSampler(local) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark_start()
+    times = time_steps(r.step, steps, torch, flush)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark_stop()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms, pairs_per_s = aggregate_ranks(float(sum(times)), r.pairs, steps, world, rmax)
+    assert r.ix.device_status() == 0, "device wait timed out"
+
+    # ---- every launch of the step, timed by the library's launch profiler
+    # (CUDA events on the launching stream) over `steps` more steps with the
+    # same L2 flush; the kernel with the largest time per step is the roofline's
+    peaks, peak_src = load_peaks()
+    from sparse_attention_token_score_b200 import binding as B
+    B.dsa_profile_begin()
+    for _ in range(steps):
+        l2_flush(flush)
+        r.step()
+    recs = B.dsa_profile_end()
+    per_name = {}
+    for nm, ms in recs:
+        e = per_name.setdefault(nm, [0.0, 0])
+        e[0] += ms
+        e[1] += 1
+    per_kernel = []
+    for nm, (ms_tot, n) in per_name.items():
+        kms = ms_tot / steps
+        units, bound = r.kernel_units(nm)
+        rec_k = {"kernel": nm, "ms": kms, "launches_per_step": n / steps, "bound": bound,
+                 "algorithmic_units_per_step": units, "traffic": traffic_for(name, nm)}
+        if units is not None:
+            if bound == "tensor":
+                rec_k.update(achieved=units / (kms / 1e3) / 1e12, peak=peaks["bf16_tflops"], unit="TFLOP/s")
+            elif bound == "tensor_fp8":  # measured bf16 burst x the nominal dense fp8 : bf16 ratio (2)
+                rec_k.update(achieved=units / (kms / 1e3) / 1e12, peak=2.0 * peaks["bf16_tflops"], unit="TFLOP/s")
+            else:
+                rec_k.update(achieved=units / (kms / 1e3) / 1e9, peak=peaks["hbm_gbs"], unit="GB/s")
+            rec_k["frac"] = rec_k["achieved"] / rec_k["peak"]
+        per_kernel.append(rec_k)
+    kernel_sum = sum(e["ms"] for e in per_kernel)
+    for e in per_kernel:
+        e["share_of_step"] = e["ms"] / kernel_sum
+    launches_per_step = len(recs) / steps
+    dom = max((e for e in per_kernel if "frac" in e), key=lambda e: e["ms"])
+    psrc = {"tensor": "bf16 burst", "tensor_fp8": "bf16 burst x 2, the nominal fp8:bf16 dense ratio",
+            "hbm": "HBM copy"}[dom["bound"]]
+    roof = {"bound": "tensor" if dom["bound"].startswith("tensor") else dom["bound"],
+            "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],
+            "frac": dom["frac"], "traffic": dom["traffic"], "kernel": dom["kernel"], "kernel_ms": dom["ms"],
+            "algorithmic_units_per_launch": dom["algorithmic_units_per_step"] / dom["launches_per_step"],
+            "largest_kernel": max(per_kernel, key=lambda e: e["ms"])["kernel"],
+            "peak_source": f"{peak_src} ({psrc})"}
+
+    # ---- end to end: host buffers, H2D + call + D2H in every step
+    e_total, h2d, d2h = run_e2e(r, inp, steps, torch, barrier)
+    e_ms, e_pairs_per_s = aggregate_ranks(e_total, r.pairs, steps, world, rmax)
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        v, sample, _, secs = oracle_sample(name, inp, budget_s=cpu_budget_s)
+        cpu = {"value": v, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": sample, "seconds": round(secs, 2)}
+    c = r.c
+    rec = {
+        "value": pairs_per_s / 1e9, "unit": UNIT, "steps": steps, "ms_per_step": total_ms / steps,
+        "dtype": r.dtype,
+        "config": workload_config(c, r.batch, r.label, inp.q_offset, r.pairs, world),
+        "queries_per_s": world * r.batch * c["T"] * steps / (total_ms / 1e3),
+        "roofline": roof, "kernels": per_kernel, "cpu_baseline": cpu,
+        "e2e": {"value": e_pairs_per_s / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e_ms / steps, "pipeline": "2 buffer sets, copy-in / call / copy-out streams"},
+        "gpu_launches": int(round(launches_per_step * steps)), "clocks": clocks,
+        "step_ms": {"min": min(times), "median": statistics.median(times), "max": max(times)},
+    }
+    del r, inp
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="dsa", choices=["tiny", "dsa", "decode", "misa", "hisa"])
+    ap.add_argument("--workload", default="all", choices=["all", "tiny", "dsa", "decode", "misa", "hisa", "dsa_fp8", "indexcache"],
+                    help="all (default): the dsa chunk is the headline line, the other four "
+                         "workloads are measured in the same run under 'workloads'")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--queries", type=int, default=0,
                     help="profiling: use only the last N queries of the chunk")
     ap.add_argument("--batch", type=int, default=0,
                     help="profiling: use only the first N sequences (decode)")
-    ap.add_argument("--kernel-only", action="store_true",
-                    help="profiling: launch only one kernel of the step (W + K times)")
-    ap.add_argument("--kernel", type=int, default=0,
-                    help="with --kernel-only: index into the step's kernel list (0 = first)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -475,7 +637,6 @@ def main():
 
     import torch
     import torch.distributed as dist
-    from sparse_attention_token_score_b200 import workloads as wl
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -492,92 +653,30 @@ def main():
         if world > 1:
             dist.barrier()
 
-    inp = make_inputs(args.workload, rank, args.queries, args.batch)
-    r = Runner(args.workload, inp, torch, args.queries, args.batch)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    if args.kernel_only:
-        kname, fn, _, _ = r.kernels()[args.kernel]
-        kt = time_steps(fn, args.warmup + args.steps, torch, flush)[args.warmup:]
-        print(json.dumps({"kernel": kname, "workload": r.label, "kernel_ms": kt}), flush=True)
-        return 0
-    for _ in range(args.warmup):
-        r.step()
-    torch.cuda.synchronize()
-
-    # ---- timed region
-    sampler = ClockSampler(local) if rank == 0 else None
-    barrier()
-    torch.cuda.synchronize()
-    times = time_steps(r.step, args.steps, torch, flush)
-    torch.cuda.synchronize()
-    barrier()
-    clocks = sampler.stop() if sampler else None
+    head = "dsa" if args.workload == "all" else args.workload
     rmax = dist_max(dist, "cuda") if world > 1 else None
-    total_ms, pairs_per_s = aggregate_ranks(float(sum(times)), r.pairs, args.steps, world, rmax)
-    ms_per_step = total_ms / args.steps
-    value = pairs_per_s / 1e9
-    assert r.ix.device_status() == 0, "device wait timed out"
 
-    # ---- each kernel alone; the one with the largest time is the roofline's
-    peaks, peak_src = load_peaks()
-    per_kernel = []
-    for kname, fn, units, bound in r.kernels():
-        for _ in range(3):
-            fn()
-        kms = statistics.mean(time_steps(fn, args.steps, torch, flush))
-        if bound == "tensor":
-            achieved, peak, unit = units / (kms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-        else:
-            achieved, peak, unit = units / (kms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
-        per_kernel.append({"kernel": kname, "bound": bound, "ms": kms, "achieved": achieved, "peak": peak,
-                           "unit": unit, "frac": achieved / peak, "algorithmic_units_per_launch": units,
-                           "traffic": traffic_for(args.workload, kname)})
-    dom = max(per_kernel, key=lambda e: e["ms"])
-    kernel_sum = sum(e["ms"] for e in per_kernel)
-    for e in per_kernel:
-        e["share_of_listed"] = e["ms"] / kernel_sum
-    roof = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],
-            "frac": dom["frac"], "traffic": dom["traffic"], "kernel": dom["kernel"], "kernel_ms": dom["ms"],
-            "algorithmic_units_per_launch": dom["algorithmic_units_per_launch"],
-            "peak_source": f"{peak_src} ({'bf16 burst' if dom['bound'] == 'tensor' else 'HBM copy'})"}
-
-    # ---- end to end: host buffers, H2D + call + D2H in every step
-    e_total, h2d, d2h = run_e2e(r, inp, args.steps, torch, barrier)
-    e_ms, e_pairs_per_s = aggregate_ranks(e_total, r.pairs, args.steps, world, rmax)
-    e2e_value = e_pairs_per_s / 1e9
-
-    # ---- CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        v, sample, _, secs = oracle_sample(args.workload, inp)
-        cpu = {"value": v, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-               "sample": sample, "seconds": round(secs, 2)}
-
+    rec = measure_workload(head, args, torch, world, rank, local, flush, barrier, rmax, args.steps, 10.0)
+    subs = {}
+    if args.workload == "all":
+        for name in SUB_WORKLOADS:
+            subs[name] = measure_workload(name, args, torch, world, rank, local, flush, barrier, rmax,
+                                          args.steps, 5.0, min_timed_ms=MIN_TIMED_MS)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    c = r.c
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": r.dtype, "data": "synthetic",
-        "config": {"workload": r.label, "batch": r.batch, "T": c["T"], "L": c["L"], "H": c["H"],
-                   "d": c["d"], "topk": c["topk"], "q_offset": inp.q_offset,
-                   "pairs_per_step": r.pairs, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "256 MiB buffer written before every timed step"},
-        "queries_per_s": world * r.batch * c["T"] * args.steps / (total_ms / 1e3),
-        "roofline": roof,
-        "kernels": per_kernel,
-        "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e_ms / args.steps,
-                "pipeline": "2 buffer sets, copy-in / call / copy-out streams"},
-        "gpu_launches": r.launches * args.steps,
-        "clocks": clocks,
-        "step_ms": {"min": min(times), "median": statistics.median(times), "max": max(times)},
+        "metric": METRIC, "value": rec["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": rec["dtype"], "data": "synthetic",
+        "config": rec["config"], "queries_per_s": rec["queries_per_s"], "roofline": rec["roofline"],
+        "kernels": rec["kernels"], "cpu_baseline": rec["cpu_baseline"], "e2e": rec["e2e"],
+        "gpu_launches": rec["gpu_launches"], "clocks": rec["clocks"], "step_ms": rec["step_ms"],
     }
+    if subs:
+        line["workloads"] = subs
     print(json.dumps(line), flush=True)
     return 0
 

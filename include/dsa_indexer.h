@@ -37,7 +37,7 @@
  *     of 64 and above return DSA_ERR_UNSUPPORTED.
  *
  * Supported shapes: d in {64, 128}; bf16 H in {8, 16, 32, 64};
- * FP8 e4m3 (decode): d = 128, H in {32, 64}. Other shapes return
+ * FP8 e4m3 (decode and prefill): d = 128, H in {32, 64}. Other shapes return
  * DSA_ERR_UNSUPPORTED.
  */
 #ifndef DSA_INDEXER_H
@@ -113,25 +113,35 @@ DSA_EXPORT dsa_status indexer_score_topk(const dsa_indexer_args* a, int topk, in
                               float* out_score, void* workspace, size_t ws_bytes, void* stream);
 
 /* indexer_score_topk_noalloc: the same dense score + top-k as
- * indexer_score_topk, for callers that cannot allocate device memory: code
- * running inside a stream capture whose graph must not contain allocations,
- * plugins handed a fixed memory arena by a host runtime that owns every
- * device allocation, and callers with no allocator at all (no torch, no
- * cudaMalloc permission). It takes no workspace: its scores scratch is a
- * 64 MiB array in the library's own device memory (reserved on every GPU
- * that loads the library, until the process exits), so it accepts problems
- * with 256 + 4 * batch * T * L <= 64 MiB (e.g. 64 decode sequences of
- * 131072 keys) and returns DSA_ERR_WORKSPACE for larger ones.
- * It allocates nothing and calls no allocating routine. The first call on a
- * device looks the scratch's device address up (cudaGetSymbolAddress, with
- * that device current) and caches it; make that first call before any stream
- * capture. Every call on a device shares the one scratch array: calls that
- * may overlap on the GPU (different streams, no ordering between them) race
- * and must not be issued. The status word at the start of the scratch is
- * cleared by each call. No method page has a counterpart of this entry
- * point; it is plumbing. */
+ * indexer_score_topk, for callers that cannot allocate device memory: a
+ * plugin handed a fixed memory arena by a host runtime that owns every device
+ * allocation, a latency-critical loop where cudaMalloc (which may synchronise
+ * the device) is not allowed, or a caller with no allocator at all (no torch,
+ * no permission to grow its device footprint). It takes no workspace: its
+ * scores scratch is a 64 MiB array in the library's own device memory
+ * (reserved on every GPU that loads the library, until the process exits), so
+ * it accepts problems with 256 + 4 * batch * T * L <= 64 MiB (e.g. 64 decode
+ * sequences of 131072 keys) and returns DSA_ERR_WORKSPACE for larger ones.
+ * It allocates nothing and calls no allocating routine. Every call looks the
+ * scratch's device address up (cudaGetSymbolAddress, on the current device);
+ * the first call on a device also loads the library's module there, and the
+ * first call of each shape class (head dim, head count, dtype, row length
+ * class) sets that kernel's shared-memory attribute on the host, so make one
+ * call of every shape before a phase that must not do either.
+ * Every call on a device shares the one scratch array, which keeps the last
+ * call's scores: calls that may overlap on the GPU (different streams, no
+ * ordering between them) race and must not be issued. The status word at the
+ * start of the scratch is cleared by each call; dsa_noalloc_status reads it.
+ * No method page has a counterpart of this entry point; it is plumbing. */
 DSA_EXPORT dsa_status indexer_score_topk_noalloc(const dsa_indexer_args* a, int topk,
                                                  int32_t* out_idx, float* out_score, void* stream);
+
+/* Synchronise `stream`, then report and clear the status word of the static
+ * scratch that indexer_score_topk_noalloc uses on the current device:
+ * DSA_ERR_TIMEOUT if a bounded device wait gave up inside such a call since
+ * the last read, DSA_ERR_CUDA on a CUDA error, else DSA_OK (the analogue of
+ * dsa_device_status for the call that has no workspace). */
+DSA_EXPORT dsa_status dsa_noalloc_status(void* stream);
 
 /* Stage 1 alone: write the scores I[t,s] of all visible keys into
  * out_scores[(b*T + t) * ld + s] (ld >= L). Entries with s > q_offset + t are
@@ -205,6 +215,58 @@ DSA_EXPORT size_t hisa_workspace_size(const dsa_indexer_args* a, int block, int 
 DSA_EXPORT dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, int topk,
                                   int32_t* out_idx, float* out_score, int32_t* out_blocks,
                                   void* workspace, size_t ws_bytes, void* stream);
+
+/* HISA token refinement alone (HISA review, section 3 and Figure 1), block
+ * major: the kept blocks [batch*T, m] (block ids, -1 = empty slot) are
+ * inverted into per-block lists of the queries that kept them, and each kept
+ * 128-token key tile is loaded once and scored against all of those queries:
+ *     out[r * ld + slot * blk + i] = I[t, blocks[r, slot] * blk + i]   (r = b*T + t)
+ * and -inf where that token is past L or not visible (> q_offset + t), or the
+ * slot is empty. The same values as indexer_score_gathered with these blocks
+ * (which fetches every kept block once per query). hisa_block_filter_topk
+ * uses this path when blk is a multiple of 128.
+ * bf16 only; d = 128, H in {32, 64}, blk a multiple of 128. Workspace:
+ * hisa_refine_workspace_size bytes (the 256-byte header plus the lists). */
+DSA_EXPORT size_t hisa_refine_workspace_size(const dsa_indexer_args* a, int m, int blk);
+DSA_EXPORT dsa_status hisa_refine_scores(const dsa_indexer_args* a, const int32_t* blocks, int m, int blk,
+                                         float* out, long long ld, void* workspace, size_t ws_bytes,
+                                         void* stream);
+
+/* Launch profiling (plumbing; no counterpart on the pages). Between
+ * dsa_profile_begin and dsa_profile_end every kernel the library launches, on
+ * any stream, is bracketed by two CUDA events recorded on that stream and
+ * filed under a name: the stage of the chain ("sample pass", "routed",
+ * "re-score", "blocks", "tokens", "router"), a colon, and the kernel's label.
+ * dsa_profile_end stops recording, waits for the recorded events, and writes
+ * the launches in launch order: NUL-separated names into `names` (capacity
+ * names_bytes) and each launch's time in milliseconds into ms; it returns
+ * how many it wrote (at most max_entries), or -1 if an event could not be
+ * read. Profiling adds two event records per launch; time steps without it. */
+DSA_EXPORT dsa_status dsa_profile_begin(void);
+DSA_EXPORT int dsa_profile_end(char* names, size_t names_bytes, float* ms, int max_entries);
+
+/* ------------------------------------------------------------ IndexCache
+ * indexcache_score_topk ("IndexCache: Accelerating Sparse Attention via
+ * Cross-Layer Index Reuse", section 2): n_layers indexer layers, each marked
+ * in `pattern` (n_layers characters) as 'F' (full: runs its own dense indexer,
+ * as indexer_score_topk, and its top-k becomes the cached index set) or 'S'
+ * (shared: skips the indexer and takes the indices of the nearest preceding F
+ * layer). pattern[0] must be 'F'.
+ *   layers    [n_layers] problems; an S layer's entry only needs batch and T,
+ *             equal to its F layer's (q, k, w are not read)
+ *   out_idx   [n_layers] pointers to [batch, T, topk] int32; an S layer whose
+ *             pointer equals its F layer's shares that buffer (no copy),
+ *             otherwise the indices are copied on the stream
+ *   out_score NULL, or [n_layers] pointers (entries may be NULL) to fp32
+ *             [batch, T, topk]; an S layer's scores are its F layer's
+ * Workspace: the largest indexer_workspace_size of the F layers, reused by
+ * each F layer in turn. Every argument is validated before the first launch. */
+DSA_EXPORT size_t indexcache_workspace_size(const dsa_indexer_args* layers, int n_layers,
+                                            const char* pattern, int topk);
+DSA_EXPORT dsa_status indexcache_score_topk(const dsa_indexer_args* layers, int n_layers,
+                                            const char* pattern, int topk, int32_t* const* out_idx,
+                                            float* const* out_score, void* workspace, size_t ws_bytes,
+                                            void* stream);
 
 #ifdef __cplusplus
 }

@@ -18,6 +18,10 @@ widens them exactly to fp64 and follows the pages' steps in order:
 * HISA ("HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse
   Attention" review, section 3): score pooled block keys, keep the top-m
   blocks, score the tokens of the surviving blocks, keep the top-k.
+* IndexCache ("IndexCache: Accelerating Sparse Attention via Cross-Layer
+  Index Reuse", section 2): layers marked F run their own indexer and cache
+  its top-k; layers marked S skip the indexer and reuse the cache of the
+  nearest preceding F layer.
 * DoSA certified pruning ("DoSA: Dots Sparse Attention" review, section 3):
   a seed set scored with all heads bounds the k-th score from below, a
   screened subset of heads bounds every other key's score from above, keys
@@ -357,6 +361,22 @@ def hisa(inp, block: int, m: int, topk: int, queries: Optional[Sequence[int]] = 
     return out
 
 
+# ------------------------------------------------------------ IndexCache
+def indexcache(layer_inputs, pattern: str, topk: int):
+    """Per-layer top-k indices [batch, T, topk] of an F/S layer pattern: an F
+    layer runs the dense indexer on its own inputs (dense_topk, every sequence)
+    and becomes the cache; an S layer returns the cache of the nearest F layer
+    before it. pattern[0] must be 'F'."""
+    if len(pattern) != len(layer_inputs) or not pattern or pattern[0] != "F" or set(pattern) - {"F", "S"}:
+        raise ValueError("pattern: one 'F' or 'S' per layer, starting with 'F'")
+    out, cache = [], None
+    for inp, role in zip(layer_inputs, pattern):
+        if role == "F":
+            cache = np.stack([dense_topk(inp, topk, b=b)["idx"] for b in range(inp.batch)])
+        out.append(cache)
+    return out
+
+
 # ------------------------------------------------------------ DoSA (certified pruning)
 def dosa_upper_bound(q, k, w, t: int, keys: np.ndarray, screen: Sequence[int]):
     """Upper bound on I[t,s] for each key s in ``keys`` from a subset of
@@ -431,3 +451,89 @@ def dosa_topk(inp, topk: int, screen: Sequence[int], n_seed: int,
     res["idx"] = np.array(res["idx"], dtype=np.int64).reshape(len(res["queries"]), topk)
     return res
 
+
+
+def dosa_screen_heads(q_t: np.ndarray, w_t: np.ndarray, n_screen: int) -> np.ndarray:
+    """The screened heads of one query: the n_screen heads with the largest
+    |w_h| * ||q_h|| (the heads that can move the score most; ties -> lower h),
+    ascending."""
+    g = np.abs(np.asarray(w_t, dtype=np.float64)) * np.linalg.norm(np.asarray(q_t, dtype=np.float64), axis=1)
+    sel = select_topk(g, n_screen)
+    return sel[sel >= 0]
+
+
+def sample_threshold(sample_scores: np.ndarray, k: int, V: int) -> float:
+    """A threshold the k-th best of V scores is very likely to reach, from the
+    scores of every S-th key (ns of them): the r_lo-th best sample with r_lo =
+    ceil(ns p + 4 sqrt(ns p (1 - p)) + 4), p = k / V; -inf when V <= k or the
+    sample is too small. Any value is safe for the exact selection that uses
+    it (the count of scores reaching it is checked); it only decides how much
+    work is skipped."""
+    ns = int(np.size(sample_scores))
+    if V <= k:
+        return -np.inf
+    p = k / V
+    r_lo = int(np.ceil(ns * p + 4.0 * np.sqrt(ns * p * (1.0 - p)) + 4.0))
+    if r_lo > ns:
+        return -np.inf
+    return float(np.sort(np.asarray(sample_scores, dtype=np.float64))[::-1][r_lo - 1])
+
+
+def dosa_tile_topk(inp, topk: int, n_screen: int, S: int, qpt: int, tile: int = 128, b: int = 0,
+                   groups: Optional[Sequence[int]] = None):
+    """DoSA certified pruning at tile granularity ("DoSA: Dots Sparse
+    Attention" review, section 3: screening dot products, bound evaluation,
+    pruning and candidate compaction, full-head dot products of the survivors,
+    original-score reduction with sparse writeback, exact selection), for the
+    queries of sequence b grouped qpt at a time (the queries that share a
+    tensor-core tile) and keys in tiles of `tile`:
+      1. per query, a threshold thr from the full scores of every S-th visible
+         key (sample_threshold);
+      2. per query and key, the upper bound of dosa_upper_bound with the
+         query's n_screen screened heads (dosa_screen_heads);
+      3. a key tile stays live for a group when some query of the group has a
+         visible key in it whose bound reaches that query's thr; other tiles
+         are pruned (every key in them scores below thr for every query);
+      4. each query scores the visible keys of its group's live tiles; if at
+         least min(k, V) of those scores reach thr (the certificate: the k-th
+         best of the row then reaches thr, so no pruned key can be a winner),
+         the top-k comes from them, else from the whole row (fallback);
+      5. top-k (score descending, index ascending).
+    The result equals dense_topk. Returns dict with 'idx' [nq, topk] (queries
+    of the groups, in order), 'queries', 'thr', 'live' [n_groups, n_tiles]
+    (1 live, 0 pruned), 'fallback' per query and 'groups'."""
+    q, k, w = dequant(inp, b)
+    T, H, _ = q.shape
+    L = k.shape[0]
+    n_groups = -(-T // qpt)
+    n_tiles = -(-L // tile)
+    groups = range(n_groups) if groups is None else groups
+    out = {"idx": [], "queries": [], "thr": [], "fallback": [], "groups": list(groups),
+           "live": np.zeros((len(groups), n_tiles), dtype=np.uint8)}
+    for gi, g in enumerate(groups):
+        qs = list(range(g * qpt, min(T, (g + 1) * qpt)))
+        rows = []
+        for t in qs:
+            p = inp.q_offset + t
+            V = int(visible_count(p, L))
+            _, samp, _ = dense_scores_row(q, k, w, t, p, keys=np.arange(0, V, S, dtype=np.int64))
+            thr = sample_threshold(samp, topk, V)
+            keys = np.arange(V, dtype=np.int64)
+            bound, _ = dosa_upper_bound(q, k, w, t, keys, dosa_screen_heads(q[t], w[t], n_screen))
+            live_keys = keys[bound >= thr]
+            out["live"][gi, np.unique(live_keys // tile)] = 1
+            rows.append((t, p, V, thr))
+        for t, p, V, thr in rows:
+            keys = np.arange(V, dtype=np.int64)
+            cand = keys[out["live"][gi, keys // tile] == 1]
+            _, s, _ = dense_scores_row(q, k, w, t, p, keys=cand)
+            fb = int(np.sum(s >= thr)) < min(topk, V)
+            if fb:
+                _, s, _ = dense_scores_row(q, k, w, t, p)
+                cand = keys
+            out["idx"].append(select_topk(s, topk, index=cand))
+            out["queries"].append(t)
+            out["thr"].append(thr)
+            out["fallback"].append(fb)
+    out["idx"] = np.array(out["idx"], dtype=np.int64).reshape(len(out["queries"]), topk)
+    return out

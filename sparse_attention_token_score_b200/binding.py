@@ -46,6 +46,7 @@ _SIGS = {
     "indexer_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int]),
     "indexer_score_topk": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "indexer_score_topk_noalloc": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P]),
+    "dsa_noalloc_status": (ctypes.c_int, [_P]),
     "indexer_scores": (ctypes.c_int, [_P, _P, ctypes.c_longlong, _P, ctypes.c_size_t, _P]),
     "indexer_score_gathered": (ctypes.c_int, [_P, _P, ctypes.c_int, ctypes.c_int, _P,
                                               ctypes.c_longlong, _P, ctypes.c_size_t, _P]),
@@ -59,6 +60,14 @@ _SIGS = {
                                               ctypes.c_int]),
     "misa_route_score_topk": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "hisa_refine_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int, ctypes.c_int]),
+    "hisa_refine_scores": (ctypes.c_int, [_P, _P, ctypes.c_int, ctypes.c_int, _P, ctypes.c_longlong, _P,
+                                          ctypes.c_size_t, _P]),
+    "dsa_profile_begin": (ctypes.c_int, []),
+    "dsa_profile_end": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_size_t, _P, ctypes.c_int]),
+    "indexcache_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int, ctypes.c_char_p, ctypes.c_int]),
+    "indexcache_score_topk": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_char_p, ctypes.c_int, _P, _P, _P,
+                                             ctypes.c_size_t, _P]),
     "hisa_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "hisa_block_filter_topk": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P,
                                               _P, _P, _P, ctypes.c_size_t, _P]),
@@ -156,6 +165,11 @@ def indexer_score_topk_noalloc(args: IndexerArgs, topk: int, out_idx: torch.Tens
                                             _ptr(out_score), _stream_ptr(stream)))
 
 
+def dsa_noalloc_status(stream=None) -> int:
+    """Status word of the static scratch of indexer_score_topk_noalloc (0 = ok)."""
+    return int(lib().dsa_noalloc_status(_stream_ptr(stream)))
+
+
 def indexer_scores(args: IndexerArgs, out_scores: torch.Tensor, ld: int, workspace: torch.Tensor,
                    stream=None):
     _check("indexer_scores",
@@ -211,6 +225,63 @@ def hisa_block_filter_topk(args: IndexerArgs, block: int, m: int, topk: int, out
            lib().hisa_block_filter_topk(ctypes.byref(args), block, m, topk, _ptr(out_idx),
                                         _ptr(out_score), _ptr(out_blocks), _ptr(workspace),
                                         workspace.numel(), _stream_ptr(stream)))
+
+
+def hisa_refine_workspace_size(args: IndexerArgs, m: int, blk: int) -> int:
+    return int(lib().hisa_refine_workspace_size(ctypes.byref(args), m, blk))
+
+
+def hisa_refine_scores(args: IndexerArgs, blocks: torch.Tensor, m: int, blk: int, out: torch.Tensor, ld: int,
+                       workspace: torch.Tensor, stream=None):
+    _check("hisa_refine_scores",
+           lib().hisa_refine_scores(ctypes.byref(args), _ptr(blocks), m, blk, _ptr(out), ld, _ptr(workspace),
+                                    workspace.numel(), _stream_ptr(stream)))
+
+
+def dsa_profile_begin():
+    _check("dsa_profile_begin", lib().dsa_profile_begin())
+
+
+def dsa_profile_end(max_entries: int = 4096):
+    """Launches recorded since dsa_profile_begin: list of (name, ms)."""
+    names = ctypes.create_string_buffer(max_entries * 96)
+    ms = (ctypes.c_float * max_entries)()
+    n = lib().dsa_profile_end(names, len(names), ctypes.cast(ms, ctypes.c_void_p), max_entries)
+    if n < 0:
+        raise DsaError("dsa_profile_end", -4)
+    out, raw = [], names.raw
+    pos = 0
+    for i in range(n):
+        end = raw.index(b"\0", pos)
+        out.append((raw[pos:end].decode(), float(ms[i])))
+        pos = end + 1
+    return out
+
+
+def _args_array(layers):
+    arr = (IndexerArgs * len(layers))()
+    for i, a in enumerate(layers):
+        arr[i] = a
+    return arr
+
+
+def indexcache_workspace_size(layers, pattern: str, topk: int) -> int:
+    return int(lib().indexcache_workspace_size(_args_array(layers), len(layers), pattern.encode(), topk))
+
+
+def indexcache_score_topk(layers, pattern: str, topk: int, out_idx, out_score, workspace: torch.Tensor,
+                          stream=None):
+    """layers: list of IndexerArgs (an S layer's entry needs only batch and T);
+    out_idx: list of [batch, T, topk] int32 tensors (an S layer may pass its F
+    layer's tensor to share it); out_score: None or a list (entries may be None)."""
+    n = len(layers)
+    pi = (ctypes.c_void_p * n)(*[t.data_ptr() for t in out_idx])
+    ps = None
+    if out_score is not None:
+        ps = (ctypes.c_void_p * n)(*[t.data_ptr() if t is not None else None for t in out_score])
+    _check("indexcache_score_topk",
+           lib().indexcache_score_topk(_args_array(layers), n, pattern.encode(), topk, pi, ps,
+                                       _ptr(workspace), workspace.numel(), _stream_ptr(stream)))
 
 
 def dsa_device_status(workspace: torch.Tensor, stream=None) -> int:

@@ -5,12 +5,18 @@
 
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <climits>
+#include <cmath>
+#include <cstring>
 #include <atomic>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "common.cuh"
 #include "misc.cuh"
+#include "score_inv.cuh"
 #include "score_tc.cuh"
 #include "topk.cuh"
 
@@ -22,6 +28,7 @@ constexpr size_t kHdr = 256;
 constexpr int kMaxDev = 64;
 
 size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+long long blocks_of(long long L, int block) { return (L + block - 1) / block; }
 
 struct Carve {
   char* base;
@@ -51,12 +58,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 2-D map over a row-major [rows, D] tensor, 128-byte swizzle, box of one
 // 128-byte column block x box_rows rows. Out-of-range rows read as zero.
-bool make_tmap(CUtensorMap* m, const void* base, bool fp8, int D, long long rows, int box_rows) {
+// `stride` is the distance between rows in elements (D for a dense tensor;
+// S * D views every S-th row).
+bool make_tmap(CUtensorMap* m, const void* base, bool fp8, int D, long long rows, int box_rows,
+               long long stride = 0) {
   auto fn = encode_fn();
   if (!fn) return false;
   const int elem = fp8 ? 1 : 2;
   cuuint64_t gdim[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
-  cuuint64_t gstr[1] = {static_cast<cuuint64_t>(D) * elem};
+  cuuint64_t gstr[1] = {static_cast<cuuint64_t>(stride > 0 ? stride : D) * elem};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t es[2] = {1, 1};
   const CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
@@ -89,9 +99,51 @@ int num_sms() {
   return n;
 }
 
+// ------------------------------------------------------------ launch profiling (dsa_profile_*)
+// While enabled, every kernel launch of the library is bracketed by a pair of
+// CUDA events recorded on the launching stream and filed under a name: the
+// current stage of the chain (if any) and the kernel's label.
+namespace prof {
+std::atomic<bool> on{false};
+std::mutex mu;
+struct Rec {
+  std::string name;
+  cudaEvent_t a, b;
+};
+std::vector<Rec> recs;
+thread_local std::string stage;  // nested stages joined by '/'
+
+struct Stage {  // names the launches made while it lives ("routed", "sample pass", ...)
+  size_t prev;
+  explicit Stage(const char* s) : prev(stage.size()) {
+    if (!stage.empty()) stage += '/';
+    stage += s;
+  }
+  ~Stage() { stage.resize(prev); }
+};
+
+struct Launch {  // construct right before a launch, destroy right after it
+  cudaStream_t st;
+  cudaEvent_t a = nullptr, b = nullptr;
+  std::string name;
+  Launch(cudaStream_t s, const char* label) : st(s) {
+    if (!on.load(std::memory_order_relaxed)) return;
+    name = stage.empty() ? std::string(label) : stage + ": " + label;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) { a = b = nullptr; return; }
+    cudaEventRecord(a, st);
+  }
+  ~Launch() {
+    if (!a) return;
+    cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> lock(mu);
+    recs.push_back({name, a, b});
+  }
+};
+}  // namespace prof
+
 template <class C>
 dsa_status launch_score(const ScoreParams& p, const void* q, long long q_rows, const void* k,
-                        long long k_rows, cudaStream_t st) {
+                        long long k_rows, cudaStream_t st, long long k_stride = 0) {
   static std::atomic<bool> attr[kMaxDev];
   const int dev = current_device();
   if (dev < 0) return DSA_ERR_UNSUPPORTED;
@@ -104,43 +156,55 @@ dsa_status launch_score(const ScoreParams& p, const void* q, long long q_rows, c
   CUtensorMap tq, tk;
   if (!make_tmap(&tq, q, C::ELEM == 1, C::D, q_rows, C::QROWS)) return DSA_ERR_CUDA;
   if (C::GATHER && !p.blk_tma) tk = tq;  // token gathers copy rows with cp.async (no key map)
-  else if (!make_tmap(&tk, k, C::ELEM == 1, C::D, k_rows, C::KROWS)) return DSA_ERR_CUDA;
+  else if (!make_tmap(&tk, k, C::ELEM == 1, C::D, k_rows, C::KROWS, k_stride)) return DSA_ERR_CUDA;
   int grid = num_sms();
   if (C::ROUTER) {
     const long long G = static_cast<long long>(p.batch) * ((p.T + C::QPT - 1) / C::QPT);
     if (G < grid) grid = static_cast<int>(G);
   }
+  prof::Launch pl(st, C::ROUTER ? "score_tc router" : C::GATHER ? "score_tc gathered"
+                     : C::CMP ? (C::ELEM == 1 ? "score_tc fp8 + candidate lists" : "score_tc + candidate lists")
+                     : (C::ELEM == 1 ? "score_tc fp8" : "score_tc"));
   score_tc_kernel<C><<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(tq, tk, p);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 // Dense / routed / block scoring, bf16: N = 256 columns = (256 / H) queries x H heads.
+// cmp: the epilogue also appends scores >= the row threshold to candidate
+// lists (p.cthr ... p.ccap); k_stride: key rows every k_stride elements.
 dsa_status run_scores_bf16(int D, int H, const ScoreParams& p, const void* q, long long q_rows,
-                           const void* k, long long k_rows, cudaStream_t st) {
+                           const void* k, long long k_rows, cudaStream_t st, bool cmp = false,
+                           long long k_stride = 0) {
 #ifndef DSA_EPIW
 #define DSA_EPIW 8
 #endif
-#define DSA_CASE(DD, HH)                                                                          \
-  if (D == DD && H == HH)                                                                         \
-    return launch_score<                                                                          \
-        ScoreCfg<2, DD, HH, 256 / HH, ScoreMode::kTma, (DD == 128 ? 4 : 8), DSA_EPIW>>(          \
-        p, q, q_rows, k, k_rows, st);
+#define DSA_CASE(DD, HH)                                                                            \
+  if (D == DD && H == HH)                                                                           \
+    return cmp ? launch_score<ScoreCfg<2, DD, HH, 256 / HH, ScoreMode::kTma, (DD == 128 ? 4 : 8),   \
+                                       DSA_EPIW, 1, true>>(p, q, q_rows, k, k_rows, st, k_stride)   \
+               : launch_score<ScoreCfg<2, DD, HH, 256 / HH, ScoreMode::kTma, (DD == 128 ? 4 : 8),   \
+                                       DSA_EPIW>>(p, q, q_rows, k, k_rows, st, k_stride);
   DSA_CASE(64, 8) DSA_CASE(64, 16) DSA_CASE(64, 32) DSA_CASE(64, 64)
   DSA_CASE(128, 8) DSA_CASE(128, 16) DSA_CASE(128, 32) DSA_CASE(128, 64)
 #undef DSA_CASE
   return DSA_ERR_UNSUPPORTED;
 }
 
-// FP8 decode scoring: one query per group, N = H.
+// FP8 scoring (kind::f8f6f4). Decode (one query per sequence): one query per
+// group, N = H. Prefill (T > 1): 256 / H queries per group, N = 256, as the
+// bf16 path.
 #ifndef DSA_FP8_NSTAGE
 #define DSA_FP8_NSTAGE 8
 #endif
 dsa_status run_scores_fp8(int D, int H, const ScoreParams& p, const void* q, long long q_rows,
                           const void* k, long long k_rows, cudaStream_t st) {
+  const bool prefill = p.T > 1;
   if (D == 128 && H == 64)
-    return launch_score<ScoreCfg<1, 128, 64, 1, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
+    return prefill ? launch_score<ScoreCfg<1, 128, 64, 4, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st)
+                   : launch_score<ScoreCfg<1, 128, 64, 1, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
   if (D == 128 && H == 32)
-    return launch_score<ScoreCfg<1, 128, 32, 1, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
+    return prefill ? launch_score<ScoreCfg<1, 128, 32, 8, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st)
+                   : launch_score<ScoreCfg<1, 128, 32, 1, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
   return DSA_ERR_UNSUPPORTED;
 }
 
@@ -198,6 +262,7 @@ dsa_status launch_topk_cfg(const TopkParams& tp, cudaStream_t st) {
   }
   long long grid = static_cast<long long>(num_sms()) * occ;
   if (tp.rows < grid) grid = tp.rows;
+  prof::Launch pl(st, tp.cres ? "topk_rows (candidate lists)" : "topk_rows");
   topk_rows_kernel<C><<<static_cast<int>(grid), C::NT, C::BYTES, st>>>(tp);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
@@ -211,6 +276,110 @@ dsa_status launch_topk(void* ws, TopkParams tp, cudaStream_t st) {
   if (tp.Lrow <= TkShort::MAX_ROW) return launch_topk_cfg<TkShort>(tp, st);
   if (tp.rows >= static_cast<long long>(num_sms()) * TkLong::MIN_CTAS) return launch_topk_cfg<TkLong>(tp, st);
   return launch_topk_cfg<TkWide>(tp, st);
+}
+
+// ------------------------------------------------------------ block-major HISA refinement
+// Workspace of the inverted kept-block lists (after the caller's own parts):
+// counts, cursors, list starts, item starts, the item total and the list.
+struct InvWs {
+  int* cnt;
+  int* cursor;
+  int* qoff;
+  int* ioff;
+  long long* total;
+  int2* list;
+};
+
+size_t inv_ws_bytes(long long rows, int m, long long nb) {
+  return 4 * al256(static_cast<size_t>(nb + 1) * sizeof(int)) + al256(sizeof(long long)) +
+         al256(static_cast<size_t>(rows) * m * sizeof(int2));
+}
+
+InvWs inv_carve(Carve& c, long long rows, int m, long long nb) {
+  InvWs w;
+  w.cnt = c.take<int>(nb + 1);
+  w.cursor = c.take<int>(nb + 1);
+  w.qoff = c.take<int>(nb + 1);
+  w.ioff = c.take<int>(nb + 1);
+  w.total = c.take<long long>(1);
+  w.list = c.take<int2>(static_cast<size_t>(rows) * m);
+  return w;
+}
+
+// The block-major kernel takes kept blocks whose size is a multiple of 128
+// (whole key tiles), bf16, d = 128, H in {32, 64}.
+bool inv_supported(const dsa_indexer_args* a, int blk) {
+  return blk % 128 == 0 && a->qk_dtype == DSA_BF16 && a->d == 128 && (a->H == 32 || a->H == 64);
+}
+
+template <class C>
+dsa_status launch_inv(const InvParams& p, const void* q, long long q_rows, const void* k, long long k_rows,
+                      const long long* total, cudaStream_t st) {
+  static std::atomic<bool> attr[kMaxDev];
+  const int dev = current_device();
+  if (dev < 0) return DSA_ERR_UNSUPPORTED;
+  if (!attr[dev].load(std::memory_order_relaxed)) {
+    if (cudaFuncSetAttribute(score_inv_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    attr[dev].store(true, std::memory_order_relaxed);
+  }
+  CUtensorMap tq, tk;
+  if (!make_tmap(&tq, q, false, C::D, q_rows, C::H)) return DSA_ERR_CUDA;     // one query per box
+  if (!make_tmap(&tk, k, false, C::D, k_rows, C::KROWS)) return DSA_ERR_CUDA;
+  prof::Launch pl(st, "score_inv (block-major)");
+  score_inv_kernel<C><<<num_sms(), C::NTHREADS, C::SMEM_BYTES, st>>>(tq, tk, p, total);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+#ifndef DSA_INV_NSTAGE
+#define DSA_INV_NSTAGE 4
+#endif
+// Invert the kept blocks [rows, m] and score every kept (query, block) pair:
+// out[r * ldo + slot * blk + i] = I[t, blocks[r, slot] * blk + i], -inf where
+// that token is not visible, past L, or the slot is empty.
+dsa_status run_refine_inverted(const dsa_indexer_args* a, const int32_t* blocks, int m, int blk, float* out,
+                               long long ldo, const InvWs& w, unsigned* err, cudaStream_t st) {
+  const long long rows = static_cast<long long>(a->batch) * a->T;
+  const long long M = blocks_of(a->L, blk);
+  const long long nb = a->batch * M;
+  if (cudaMemsetAsync(w.cnt, 0, static_cast<size_t>(nb) * sizeof(int), st) != cudaSuccess) return DSA_ERR_CUDA;
+  const long long n = rows * m;
+  const int grid = static_cast<int>(std::min<long long>((n + 255) / 256, 8LL * num_sms()));
+  {
+    prof::Launch pl(st, "invert_count");
+    invert_count_kernel<<<grid, 256, 0, st>>>(blocks, rows, m, a->T, static_cast<int>(M), blk, w.cnt, out, ldo);
+  }
+  {
+    prof::Launch pl(st, "invert_scan");
+    invert_scan_kernel<1024><<<1, 1024, 0, st>>>(w.cnt, static_cast<int>(nb), blk / 128, 128 / a->H, w.qoff,
+                                               w.ioff, w.cursor, w.total);
+  }
+  {
+    prof::Launch pl(st, "invert_fill");
+    invert_fill_kernel<<<grid, 256, 0, st>>>(blocks, rows, m, a->T, static_cast<int>(M), w.qoff, w.cursor, w.list);
+  }
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  InvParams p{};
+  p.batch = a->batch;
+  p.T = a->T;
+  p.L = a->L;
+  p.M = static_cast<int>(M);
+  p.blk = blk;
+  p.m = m;
+  p.q_offset = a->q_offset;
+  p.w = a->w;
+  p.out = out;
+  p.ldo = ldo;
+  p.cnt = w.cnt;
+  p.qoff = w.qoff;
+  p.ioff = w.ioff;
+  p.list = w.list;
+  p.err = err;
+  const long long q_rows = rows * a->H;
+  const long long k_rows = static_cast<long long>(a->batch) * a->L;
+  if (a->H == 32) return launch_inv<InvCfg<32, DSA_INV_NSTAGE>>(p, a->q, q_rows, a->k, k_rows, w.total, st);
+  return launch_inv<InvCfg<64, DSA_INV_NSTAGE>>(p, a->q, q_rows, a->k, k_rows, w.total, st);
 }
 
 bool h_supported_bf16(int H) { return H == 8 || H == 16 || H == 32 || H == 64; }
@@ -290,11 +459,151 @@ TopkParams topk_params(const float* scores, long long rows, long long ld, int T,
     if (s_ != DSA_OK) return s_;    \
   } while (0)
 
+// ------------------------------------------------------------ fused score -> candidate lists -> top-k
+// LiteTopK's idea ("DoSA: Dots Sparse Attention" review: scoring fused with
+// filtering to cut memory traffic), kept exact: a first pass scores every S-th
+// key; from that sample each row gets a threshold its k-th score is very
+// likely to reach; the full pass then appends every visible score >= the
+// threshold to the row's candidate list, and the top-k selects from the lists.
+// A row whose list holds fewer than k (or more than its capacity) is selected
+// from its full scores, which the full pass still writes.
+struct FusedPlan {
+  bool on;
+  int S;       // sample stride (keys)
+  int ns_max;  // samples per full row (L / S)
+  int cap;     // candidate list capacity per row
+  int qpt;     // queries per group of the score kernel (256 / heads)
+  int ntiles;  // key tiles per full row
+};
+
+FusedPlan fused_plan(int L, int topk, bool bf16, int heads) {
+  FusedPlan f{false, 0, 0, 0, 0, 0};
+  if (!bf16 || L < 4096 || static_cast<long long>(topk) * 8 > L || heads < 1 || 256 % heads != 0) return f;
+  int S = 16;
+  while (L / S > 4096) S <<= 1;  // 2048 .. 4096 samples per full row
+  if (L % S != 0) return f;
+  f.on = true;
+  f.S = S;
+  f.ns_max = L / S;
+  // twice the expected list length at the longest rows (k plus the
+  // threshold's margin: 4 standard deviations + 4 samples, each sample
+  // standing for S keys), plus the unused tails of the reserved chunks (two
+  // chunks per warp, four warps per query, a few CTAs per query group)
+  const double c = 2.0 * (topk + 4.0 * std::sqrt(static_cast<double>(topk) * S) + 4.0 * S) + 32.0 * CCHUNK;
+  f.cap = static_cast<int>((static_cast<long long>(std::ceil(c)) + 255) / 256 * 256);
+  f.qpt = 256 / heads;
+  f.ntiles = (L + 127) / 128;
+  return f;
+}
+
+long long fused_groups(long long batch, int T, const FusedPlan& f) { return batch * ((T + f.qpt - 1) / f.qpt); }
+
+size_t fused_ws_bytes(long long batch, int T, const FusedPlan& f) {
+  if (!f.on) return 0;
+  const size_t rows = static_cast<size_t>(batch) * T;
+  return al256(rows * f.ns_max * sizeof(float)) + 3 * al256(rows * 4) + 2 * al256(rows * f.cap * 4) +
+         al256(static_cast<size_t>(fused_groups(batch, T, f)) * f.ntiles);
+}
+
+struct FusedWs {
+  float* samp;
+  float* thr;
+  int* cres;
+  int* creal;
+  float* cval;
+  int* cidx;
+  uint8_t* fb;  // [groups, ntiles] tiles the fallback pass computes
+};
+
+FusedWs fused_carve(Carve& c, long long batch, int T, const FusedPlan& f) {
+  const long long rows = batch * T;
+  FusedWs w;
+  w.samp = c.take<float>(static_cast<size_t>(rows) * f.ns_max);
+  w.thr = c.take<float>(rows);
+  w.cres = c.take<int>(rows);
+  w.creal = c.take<int>(rows);
+  c.take<int>(rows);  // spare (keeps the two counters apart)
+  w.cval = c.take<float>(static_cast<size_t>(rows) * f.cap);
+  w.cidx = c.take<int>(static_cast<size_t>(rows) * f.cap);
+  w.fb = c.take<uint8_t>(static_cast<size_t>(fused_groups(batch, T, f)) * f.ntiles);
+  return w;
+}
+
+// Scores of every visible key with the Hh heads of q ([rows * Hh, D] bf16;
+// weights in base.w) and the top-k of every row through candidate lists;
+// scores [rows, L] receives full scores only for rows whose list fails the
+// check (and the winners' scores). base: batch, T, q_offset, w, err set.
+dsa_status fused_score_topk(int D, int Hh, const ScoreParams& base, const void* q, const void* k, int L,
+                            int topk, int32_t* out_idx, float* out_score, float* scores, const FusedPlan& f,
+                            const FusedWs& w, void* ws, cudaStream_t st) {
+  const long long rows = static_cast<long long>(base.batch) * base.T;
+  const long long groups = fused_groups(base.batch, base.T, f);
+  if (cudaMemsetAsync(w.cres, 0, 2 * al256(static_cast<size_t>(rows) * 4), st) != cudaSuccess ||
+      cudaMemsetAsync(w.fb, 0, static_cast<size_t>(groups) * f.ntiles, st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  // 1. sample pass: keys 0, S, 2S, ... (a strided view of the key rows)
+  {
+    prof::Stage sample_stage("sample pass");
+    ScoreParams ps = base;
+    ps.Lk = f.ns_max;
+    ps.pstride = f.S;
+    ps.out = w.samp;
+    ps.ldo = f.ns_max;
+    DSA_TRY(run_scores_bf16(D, Hh, ps, q, rows * Hh, k, static_cast<long long>(base.batch) * f.ns_max, st, false,
+                            static_cast<long long>(f.S) * D));
+  }
+  // 2. thresholds
+  const int tgrid = static_cast<int>(std::min<long long>(rows, 8LL * num_sms()));
+  {
+    prof::Launch pl(st, "thresholds");
+    topk_threshold_kernel<256><<<tgrid, 256, 0, st>>>(w.samp, rows, f.ns_max, base.T, base.q_offset, f.S, f.ns_max,
+                                                       L, topk, w.thr);
+  }
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  // 3. candidate lists (no full scores)
+  ScoreParams pm = base;
+  pm.Lk = L;
+  pm.pstride = 1;
+  pm.out = nullptr;
+  pm.cthr = w.thr;
+  pm.cval = w.cval;
+  pm.cidx = w.cidx;
+  pm.cres = w.cres;
+  pm.creal = w.creal;
+  pm.ccap = f.cap;
+  DSA_TRY(run_scores_bf16(D, Hh, pm, q, rows * Hh, k, static_cast<long long>(base.batch) * L, st, true));
+  // 4. rows whose list is short (or overflowed): full scores of their groups
+  {
+    prof::Launch pl(st, "list check");
+    fused_check_kernel<<<static_cast<int>((rows + 255) / 256), 256, 0, st>>>(
+        w.cres, w.creal, rows, base.T, base.q_offset, L, topk, f.cap, f.qpt, f.ntiles, w.fb);
+  }
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  {
+    prof::Stage fb_stage("fallback");
+    ScoreParams pf = base;
+    pf.Lk = L;
+    pf.pstride = 1;
+    pf.out = scores;
+    pf.ldo = L;
+    pf.tile_live = w.fb;
+    pf.live_ld = f.ntiles;
+    DSA_TRY(run_scores_bf16(D, Hh, pf, q, rows * Hh, k, static_cast<long long>(base.batch) * L, st));
+  }
+  // 5. top-k from the lists (from the full scores where a list failed)
+  TopkParams tp = topk_params(scores, rows, L, base.T, base.q_offset, 1, L, topk, out_idx, out_score, nullptr, 0, 1);
+  tp.cval = w.cval;
+  tp.cidx = w.cidx;
+  tp.cres = w.cres;
+  tp.creal = w.creal;
+  tp.ccap = f.cap;
+  return launch_topk(ws, tp, st);
+}
+
 dsa_status clear_status(void* ws, cudaStream_t st) {
   return cudaMemsetAsync(ws, 0, 4, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
-long long blocks_of(long long L, int block) { return (L + block - 1) / block; }
 
 }  // namespace
 
@@ -331,9 +640,10 @@ dsa_status dsa_selftest_wait_timeout(void* workspace, size_t ws_bytes, void* str
 }
 
 size_t indexer_workspace_size(const dsa_indexer_args* a, int topk) {
-  (void)topk;
   if (!a || a->batch < 1 || a->T < 1 || a->L < 1) return 0;
-  return kHdr + al256(static_cast<size_t>(a->batch) * a->T * a->L * sizeof(float));
+  const size_t rows = static_cast<size_t>(a->batch) * a->T;
+  return kHdr + al256(rows * a->L * sizeof(float)) +
+         fused_ws_bytes(a->batch, a->T, fused_plan(a->L, topk, a->qk_dtype == DSA_BF16, a->H));
 }
 
 dsa_status indexer_scores(const dsa_indexer_args* a, float* out, long long ld, void* ws,
@@ -392,27 +702,40 @@ dsa_status indexer_topk_rows(const float* scores, long long rows, long long ld, 
                      st);
 }
 
-dsa_status indexer_score_topk(const dsa_indexer_args* a, int topk, int32_t* out_idx,
-                              float* out_score, void* ws, size_t ws_bytes, void* stream) {
+// The dense score + top-k; `fused` picks the candidate-list chain where it
+// applies (fused_plan), otherwise full scores then the row top-k.
+static dsa_status dense_score_topk(const dsa_indexer_args* a, int topk, int32_t* out_idx, float* out_score,
+                                   void* ws, size_t ws_bytes, void* stream, bool fused) {
   DSA_TRY(validate(a, false));
   if (!out_idx || topk < 1 || topk > (1 << 24)) return DSA_ERR_ARG;
-  DSA_TRY(check_ws(ws, ws_bytes, indexer_workspace_size(a, topk)));
+  const size_t rows = static_cast<size_t>(a->batch) * a->T;
+  const FusedPlan f = fused ? fused_plan(a->L, topk, a->qk_dtype == DSA_BF16, a->H) : FusedPlan{};
+  DSA_TRY(check_ws(ws, ws_bytes, kHdr + al256(rows * a->L * sizeof(float)) + fused_ws_bytes(a->batch, a->T, f)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DSA_TRY(clear_status(ws, st));
   Carve c{static_cast<char*>(ws), kHdr};
-  float* scores = c.take<float>(static_cast<size_t>(a->batch) * a->T * a->L);
+  float* scores = c.take<float>(rows * a->L);
   ScoreParams p = base_params(a, static_cast<unsigned*>(ws));
-  p.out = scores;
-  p.ldo = a->L;
   const long long q_rows = static_cast<long long>(a->batch) * a->T * a->H;
   const long long k_rows = static_cast<long long>(a->batch) * a->L;
+  if (f.on) {
+    const FusedWs w = fused_carve(c, a->batch, a->T, f);
+    return fused_score_topk(a->d, a->H, p, a->q, a->k, a->L, topk, out_idx, out_score, scores, f, w, ws, st);
+  }
+  p.out = scores;
+  p.ldo = a->L;
   if (a->qk_dtype == DSA_FP8_E4M3)
     DSA_TRY(run_scores_fp8(a->d, a->H, p, a->q, q_rows, a->k, k_rows, st));
   else
     DSA_TRY(run_scores_bf16(a->d, a->H, p, a->q, q_rows, a->k, k_rows, st));
-  return launch_topk(ws, topk_params(scores, static_cast<long long>(a->batch) * a->T, a->L, a->T,
-                                 a->q_offset, 1, a->L, topk, out_idx, out_score, nullptr, 0, 1),
+  return launch_topk(ws, topk_params(scores, static_cast<long long>(rows), a->L, a->T, a->q_offset, 1, a->L, topk,
+                                 out_idx, out_score, nullptr, 0, 1),
                      st);
+}
+
+dsa_status indexer_score_topk(const dsa_indexer_args* a, int topk, int32_t* out_idx, float* out_score, void* ws,
+                              size_t ws_bytes, void* stream) {
+  return dense_score_topk(a, topk, out_idx, out_score, ws, ws_bytes, stream, true);
 }
 
 dsa_status dsa_meanpool_keys(const void* k, int batch, int L, int d, int block, void* kbar,
@@ -421,6 +744,7 @@ dsa_status dsa_meanpool_keys(const void* k, int batch, int L, int d, int block, 
   const long long M = blocks_of(L, block);
   if (static_cast<long long>(batch) * M > INT_MAX) return DSA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  prof::Launch pl(st, "meanpool");
   meanpool_kernel<<<static_cast<int>(batch * M), d < 128 ? d : 128, 0, st>>>(
       static_cast<const __nv_bfloat16*>(k), L, d, block, static_cast<int>(M),
       static_cast<__nv_bfloat16*>(kbar));
@@ -440,6 +764,7 @@ size_t misa_workspace_size(const dsa_indexer_args* a, int block, int h, int topk
   n += al256(BT * h * sizeof(float));             // their weights
   n += al256(BT * h * sizeof(int32_t));           // kept heads
   n += al256(BT * a->L * sizeof(float));          // routed scores
+  n += fused_ws_bytes(a->batch, a->T, fused_plan(a->L, kprime > 0 ? kprime : topk, true, h));
   if (kprime > 0) {
     n += al256(BT * kprime * sizeof(int32_t));    // candidates
     n += al256(BT * kprime * sizeof(float));      // full-H candidate scores
@@ -472,37 +797,54 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   int32_t* heads_ws = c.take<int32_t>(static_cast<size_t>(BT) * h);
   float* routed = c.take<float>(static_cast<size_t>(BT) * a->L);
   int32_t* heads = out_heads ? out_heads : heads_ws;
+  const FusedPlan fp = fused_plan(a->L, kprime > 0 ? kprime : topk, true, h);
+  const FusedWs fw = fp.on ? fused_carve(c, a->batch, a->T, fp) : FusedWs{};
 
   // 1. pooled keys
   DSA_TRY(dsa_meanpool_keys(a->k, a->batch, a->L, a->d, block, kbar, stream));
   // 2. router affinities (partial ReLU sums over visible pooled keys)
+  prof::Stage route_stage("router");
   ScoreParams pr = base_params(a, err);
   pr.Lk = static_cast<int>(M);
   pr.pstride = block;
   pr.out = part;
   DSA_TRY(run_router(a->d, a->H, pr, a->q, BT * a->H, kbar, a->batch * M, st));
   // 3. top-h heads per query; gather their query rows and weights
-  select_heads_kernel<<<static_cast<int>((BT + 7) / 8), 256, 0, st>>>(
-      part, BT, a->H, h, a->w, static_cast<const __nv_bfloat16*>(a->q), a->d, heads, q_sel, w_sel);
+  {
+    prof::Launch pl(st, "select_heads");
+    select_heads_kernel<<<static_cast<int>((BT + 7) / 8), 256, 0, st>>>(
+        part, BT, a->H, h, a->w, static_cast<const __nv_bfloat16*>(a->q), a->d, heads, q_sel, w_sel);
+  }
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  // 4. routed token scores with the kept heads only
+  // 4. routed token scores with the kept heads only, and their top-k (or
+  // top-k' candidates), through candidate lists where that applies
+  prof::Stage routed_stage("routed");
   ScoreParams ps = base_params(a, err);
   ps.w = w_sel;
   ps.out = routed;
   ps.ldo = a->L;
-  DSA_TRY(run_scores_bf16(a->d, h, ps, q_sel, BT * h, a->k, static_cast<long long>(a->batch) * a->L, st));
-  if (kprime == 0) {
-    return launch_topk(ws, topk_params(routed, BT, a->L, a->T, a->q_offset, 1, a->L, topk, out_idx,
-                                   out_score, nullptr, 0, 1),
-                       st);
+  const long long k_rows = static_cast<long long>(a->batch) * a->L;
+  int32_t* cand = nullptr;
+  float* compact = nullptr;
+  if (kprime > 0) {
+    int32_t* cand_ws = c.take<int32_t>(static_cast<size_t>(BT) * kprime);
+    compact = c.take<float>(static_cast<size_t>(BT) * kprime);
+    cand = out_cand ? out_cand : cand_ws;
   }
-  // 5. MISA-dagger: top-k' candidates, full-H re-score, top-k
-  int32_t* cand_ws = c.take<int32_t>(static_cast<size_t>(BT) * kprime);
-  float* compact = c.take<float>(static_cast<size_t>(BT) * kprime);
-  int32_t* cand = out_cand ? out_cand : cand_ws;
-  DSA_TRY(launch_topk(ws, topk_params(routed, BT, a->L, a->T, a->q_offset, 1, a->L, kprime, cand,
-                                  nullptr, nullptr, 0, 1),
-                      st));
+  const int ksel = kprime > 0 ? kprime : topk;
+  int32_t* sel = kprime > 0 ? cand : out_idx;
+  float* sel_score = kprime > 0 ? nullptr : out_score;
+  if (fp.on) {
+    DSA_TRY(fused_score_topk(a->d, h, ps, q_sel, a->k, a->L, ksel, sel, sel_score, routed, fp, fw, ws, st));
+  } else {
+    DSA_TRY(run_scores_bf16(a->d, h, ps, q_sel, BT * h, a->k, k_rows, st));
+    DSA_TRY(launch_topk(ws, topk_params(routed, BT, a->L, a->T, a->q_offset, 1, a->L, ksel, sel, sel_score,
+                                    nullptr, 0, 1),
+                        st));
+  }
+  if (kprime == 0) return DSA_OK;
+  // 5. MISA-dagger: full-H re-score of the k' candidates, top-k
+  prof::Stage rescore_stage("re-score");
   ScoreParams pg = base_params(a, err);
   pg.out = compact;
   pg.ldo = kprime;
@@ -527,7 +869,30 @@ size_t hisa_workspace_size(const dsa_indexer_args* a, int block, int m, int topk
   n += al256(BT * M * sizeof(float));                         // block scores
   n += al256(BT * m * sizeof(int32_t));                       // kept blocks
   n += al256(BT * static_cast<size_t>(m) * block * sizeof(float));  // token scores of kept blocks
+  if (inv_supported(a, block)) n += inv_ws_bytes(static_cast<long long>(BT), m, a->batch * static_cast<long long>(M));
   return n;
+}
+
+size_t hisa_refine_workspace_size(const dsa_indexer_args* a, int m, int blk) {
+  if (!a || a->batch < 1 || a->T < 1 || a->L < 1 || m < 1 || blk < 1) return 0;
+  return kHdr + inv_ws_bytes(static_cast<long long>(a->batch) * a->T, m, a->batch * blocks_of(a->L, blk));
+}
+
+dsa_status hisa_refine_scores(const dsa_indexer_args* a, const int32_t* blocks, int m, int blk, float* out,
+                              long long ld, void* ws, size_t ws_bytes, void* stream) {
+  DSA_TRY(validate(a, true));
+  if (!blocks || !out || m < 1 || blk < 1 || !aligned(blocks, 4) || !aligned(out, 4)) return DSA_ERR_ARG;
+  if (static_cast<long long>(m) * blk > INT_MAX / 2) return DSA_ERR_UNSUPPORTED;
+  if (ld < static_cast<long long>(m) * blk) return DSA_ERR_ARG;
+  if (!inv_supported(a, blk)) return DSA_ERR_UNSUPPORTED;
+  if (a->batch * blocks_of(a->L, blk) > INT_MAX / 2) return DSA_ERR_UNSUPPORTED;
+  DSA_TRY(check_ws(ws, ws_bytes, hisa_refine_workspace_size(a, m, blk)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DSA_TRY(clear_status(ws, st));
+  Carve c{static_cast<char*>(ws), kHdr};
+  const long long rows = static_cast<long long>(a->batch) * a->T;
+  const InvWs w = inv_carve(c, rows, m, a->batch * blocks_of(a->L, blk));
+  return run_refine_inverted(a, blocks, m, blk, out, ld, w, static_cast<unsigned*>(ws), st);
 }
 
 dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, int topk,
@@ -556,6 +921,7 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   // 1. pooled keys
   DSA_TRY(dsa_meanpool_keys(a->k, a->batch, a->L, a->d, block, kbar, stream));
   // 2. block scores on the pooled keys (block m visible iff m * block <= p_t)
+  prof::Stage block_stage("blocks");
   ScoreParams pb = base_params(a, err);
   pb.Lk = static_cast<int>(M);
   pb.pstride = block;
@@ -566,7 +932,17 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   DSA_TRY(launch_topk(ws, topk_params(bscore, BT, M, a->T, a->q_offset, block, static_cast<int>(M), m,
                                   blocks, nullptr, nullptr, 0, 1),
                       st));
-  // 4. token scores inside the kept blocks (compact rows of m * block)
+  prof::Stage token_stage("tokens");
+  // 4. token scores inside the kept blocks (compact rows of m * block):
+  // block-major over the inverted kept-block lists when blocks are whole key
+  // tiles, else one query per tile with gathered rows
+  if (inv_supported(a, block)) {
+    const InvWs w = inv_carve(c, BT, m, a->batch * M);
+    DSA_TRY(run_refine_inverted(a, blocks, m, block, compact, ncomp, w, err, st));
+    return launch_topk(ws, topk_params(compact, BT, ncomp, a->T, a->q_offset, 0, ncomp, topk, out_idx,
+                                   out_score, blocks, m, block),
+                       st);
+  }
   ScoreParams pg = base_params(a, err);
   pg.out = compact;
   pg.ldo = ncomp;
@@ -582,6 +958,109 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
                      st);
 }
 
+// ------------------------------------------------------------ launch profiling
+dsa_status dsa_profile_begin(void) {
+  std::lock_guard<std::mutex> lock(prof::mu);
+  for (auto& r : prof::recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  prof::recs.clear();
+  prof::on.store(true);
+  return DSA_OK;
+}
+
+int dsa_profile_end(char* names, size_t names_bytes, float* ms, int max_entries) {
+  prof::on.store(false);
+  std::lock_guard<std::mutex> lock(prof::mu);
+  int n = 0;
+  size_t used = 0;
+  bool failed = false;
+  for (auto& r : prof::recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) failed = true;
+    if (n < max_entries && ms && names && used + r.name.size() + 1 <= names_bytes) {
+      ms[n] = t;
+      std::memcpy(names + used, r.name.c_str(), r.name.size() + 1);
+      used += r.name.size() + 1;
+      ++n;
+    }
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  prof::recs.clear();
+  return failed ? -1 : n;
+}
+
+// ------------------------------------------------------------ IndexCache
+// Layers marked 'F' run their own indexer; layers marked 'S' reuse the top-k
+// indices of the nearest preceding 'F' layer ("IndexCache: Accelerating Sparse
+// Attention via Cross-Layer Index Reuse", section 2). Every F layer is
+// validated before the first launch; S layers only need batch and T (their
+// output shape), which must match their F layer's.
+static dsa_status indexcache_check(const dsa_indexer_args* layers, int n_layers, const char* pattern,
+                                   int topk, int32_t* const* out_idx, float* const* out_score) {
+  if (!layers || !pattern || !out_idx || n_layers < 1 || topk < 1 || topk > (1 << 24)) return DSA_ERR_ARG;
+  if (pattern[0] != 'F') return DSA_ERR_ARG;
+  int f = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    if (!out_idx[l]) return DSA_ERR_ARG;
+    if (pattern[l] == 'F') {
+      DSA_TRY(validate(&layers[l], false));
+      f = l;
+    } else if (pattern[l] == 'S') {
+      if (layers[l].batch != layers[f].batch || layers[l].T != layers[f].T) return DSA_ERR_ARG;
+      if (out_score && out_score[l] && !out_score[f]) return DSA_ERR_ARG;  // no scores to reuse
+    } else {
+      return DSA_ERR_ARG;  // includes a pattern shorter than n_layers
+    }
+  }
+  return DSA_OK;
+}
+
+size_t indexcache_workspace_size(const dsa_indexer_args* layers, int n_layers, const char* pattern,
+                                 int topk) {
+  if (!layers || !pattern || n_layers < 1) return 0;
+  size_t n = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    if (pattern[l] != 'F' && pattern[l] != 'S') return 0;
+    if (pattern[l] == 'F') {
+      const size_t m = indexer_workspace_size(&layers[l], topk);
+      if (m == 0) return 0;
+      if (m > n) n = m;
+    }
+  }
+  return n;
+}
+
+dsa_status indexcache_score_topk(const dsa_indexer_args* layers, int n_layers, const char* pattern,
+                                 int topk, int32_t* const* out_idx, float* const* out_score, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  DSA_TRY(indexcache_check(layers, n_layers, pattern, topk, out_idx, out_score));
+  DSA_TRY(check_ws(ws, ws_bytes, indexcache_workspace_size(layers, n_layers, pattern, topk)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int f = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    float* os = out_score ? out_score[l] : nullptr;
+    if (pattern[l] == 'F') {
+      f = l;
+      DSA_TRY(indexer_score_topk(&layers[l], topk, out_idx[l], os, ws, ws_bytes, stream));
+      continue;
+    }
+    // S: the cached indices of layer f (no copy when the caller aliases the buffers)
+    const size_t n = static_cast<size_t>(layers[l].batch) * layers[l].T * topk;
+    if (out_idx[l] != out_idx[f] &&
+        cudaMemcpyAsync(out_idx[l], out_idx[f], n * sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    const float* fs = out_score ? out_score[f] : nullptr;
+    if (os && os != fs) {
+      if (cudaMemcpyAsync(os, fs, n * sizeof(float), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    }
+  }
+  return DSA_OK;
+}
+
 }  // extern "C"
 
 // ------------------------------------------------------------------ no-allocation variant
@@ -589,28 +1068,23 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
 // scores scratch lives in a file-scope __device__ array that every device
 // loading this library reserves until exit. Host code must not pass
 // `g_noalloc_scratch` itself to a kernel: on the host that name is only a
-// stand-in for the device symbol. The device address is looked up once per
-// device with cudaGetSymbolAddress (the first call on a device, with that
-// device current) and cached.
+// stand-in for the device symbol. Its device address is looked up with
+// cudaGetSymbolAddress on every call, with the caller's device current, so a
+// new primary context (after cudaDeviceReset, say), where the module may sit
+// at another address, never sees a stale pointer. The lookup is a host-side
+// table read once the module is loaded; the first call on a device loads it.
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDev] = {nullptr};
-
 dsa_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDev) return DSA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+  *out = p;
   return DSA_OK;
 }
 
@@ -621,10 +1095,21 @@ extern "C" dsa_status indexer_score_topk_noalloc(const dsa_indexer_args* a, int 
                                                  void* stream) {
   DSA_TRY(validate(a, false));
   if (!out_idx || topk < 1 || topk > (1 << 24)) return DSA_ERR_ARG;
-  if (indexer_workspace_size(a, topk) > kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
+  if (kHdr + al256(static_cast<size_t>(a->batch) * a->T * a->L * sizeof(float)) > kNoAllocScratchBytes)
+    return DSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   DSA_TRY(noalloc_scratch(&scratch));
-  // Same launches as indexer_score_topk; its status word (first 4 bytes of
-  // the scratch) is cleared on the stream before the kernels run.
-  return indexer_score_topk(a, topk, out_idx, out_score, scratch, kNoAllocScratchBytes, stream);
+  // Full scores then the row top-k (the selection indexer_score_topk makes,
+  // without its candidate lists); the status word (first 4 bytes of the
+  // scratch) is cleared on the stream before the kernels run.
+  return dense_score_topk(a, topk, out_idx, out_score, scratch, kNoAllocScratchBytes, stream, false);
+}
+
+// The status word of the static scratch: a bounded wait that gave up inside an
+// indexer_score_topk_noalloc call on this device is reported here, as
+// dsa_device_status reports it for a caller workspace.
+extern "C" dsa_status dsa_noalloc_status(void* stream) {
+  void* scratch = nullptr;
+  DSA_TRY(noalloc_scratch(&scratch));
+  return dsa_device_status(scratch, stream);
 }

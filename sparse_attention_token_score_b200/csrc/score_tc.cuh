@@ -62,15 +62,41 @@ struct ScoreParams {
   int n_slots, blk, n_compact;  // compact position c -> cand[c / blk] * blk + c % blk
   int blk_tma;              // gather mode, blk % 128 == 0: a tile is one contiguous key run (TMA)
   unsigned* err;            // device error word
+  // Optional compaction (score mode, ScoreCfg CMP): every visible score >=
+  // cthr[row] is appended, with its key, to the row's candidate list
+  // (cval / cidx [rows, ccap]). Each epilogue warp reserves slots CCHUNK at a
+  // time (cres[row] counts reserved slots, requested one chunk ahead) and
+  // fills the unused rest of its chunks with sentinels (-inf, -1) when it
+  // leaves the group; creal[row] counts the real entries. Slots past ccap are
+  // not written (cres then exceeds ccap). out may be null: no full scores.
+  const float* cthr;
+  float* cval;
+  int* cidx;
+  int* cres;
+  int* creal;
+  int ccap;
+  // Optional tile mask (score mode): tile j of query group g (g counted over
+  // all sequences) is computed only if tile_live[g * live_ld + j] != 0; for
+  // the others nothing is loaded or multiplied and, with dead_fill, the
+  // visible entries of the full scores are set to -inf.
+  const uint8_t* tile_live;
+  long long live_ld;
+  int dead_fill;
 };
 
-template <int ELEM_, int D_, int H_, int QPT_, ScoreMode MODE_, int NSTAGE_, int EPIW_ = 8, int NQBUF_ = 1>
+constexpr int CCHUNK = 64;  // candidate slots reserved per warp and query at a time
+
+template <int ELEM_, int D_, int H_, int QPT_, ScoreMode MODE_, int NSTAGE_, int EPIW_ = 8, int NQBUF_ = 1,
+          bool CMP_ = false>
 struct ScoreCfg {
   static constexpr int ELEM = ELEM_;  // bytes per element: 2 = bf16, 1 = e4m3
   static constexpr int D = D_, H = H_, QPT = QPT_, NSTAGE = NSTAGE_;
   static constexpr ScoreMode MODE = MODE_;
   static constexpr bool ROUTER = MODE_ == ScoreMode::kRouter;
   static constexpr bool GATHER = MODE_ == ScoreMode::kGather;
+  // candidate compaction in the epilogue (ScoreParams::ccnt and friends)
+  static constexpr bool CMP = CMP_;
+  static_assert(!CMP || (MODE_ == ScoreMode::kTma && QPT_ > 1), "compaction: score mode, several queries per group");
   static constexpr int ROW_BYTES = D * ELEM;
   static_assert(ROW_BYTES == 128 || ROW_BYTES == 256, "rows must be 1 or 2 swizzle atoms wide");
   static constexpr int KBLK = ROW_BYTES / 128;          // 128-byte column blocks per row
@@ -257,6 +283,13 @@ __device__ __forceinline__ long long gathered_token(const ScoreParams& p, long l
   return tok;
 }
 
+// Whether the current (group, tile) is computed (ScoreParams::tile_live).
+template <class C, class S>
+__device__ __forceinline__ bool tile_live(const ScoreParams& p, const S& s) {
+  if (C::ROUTER || C::GATHER || p.tile_live == nullptr) return true;
+  return __ldg(p.tile_live + static_cast<long long>(s.g) * p.live_ld + s.j) != 0;
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -318,9 +351,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int pw = warp;
     uint32_t it = 0, gq = 0;
     bool ok = true;
-    for (; !s.done; s.next(p), ++it) {
+    for (; !s.done; s.next(p)) {
       const int b = s.b;
       const int tg = s.tg;
+      const bool live = tile_live<C>(p, s);
       // gathers: tiles round-robin over the producer warps (each owns its
       // stages); contiguous block tiles (TMA): warp 0 loads every tile
       const bool mine = C::GATHER ? (p.blk_tma ? pw == 0 : static_cast<int>(it % C::NPROD) == pw) : true;
@@ -342,7 +376,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      if (!mine) continue;
+      if (!live) continue;  // a pruned tile: no keys (the query tile bookkeeping above still runs)
+      if (!mine) { ++it; continue; }
       const int stage = static_cast<int>(it % C::NSTAGE);
       const uint32_t ph = (it / C::NSTAGE) & 1u;
       if (C::GATHER && p.blk_tma) {
@@ -425,6 +460,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
+      ++it;
     }
     // cp.async gathers still in flight land before the CTA can release its
     // shared memory (on the normal path the MMA warp has waited for them all)
@@ -445,9 +481,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (lane == 0) {
       uint32_t it = 0, gq = 0;
       bool ok = true;
-      for (; !s.done; s.next(p), ++it) {
+      for (; !s.done; s.next(p)) {
         const int qb = static_cast<int>(gq % C::NQBUF);
         if (s.first && !mbar_wait(qfull(qb), (gq / C::NQBUF) & 1u, p.err)) { ok = false; break; }
+        if (!tile_live<C>(p, s)) {
+          if (s.last) { tc_commit(qempty(qb)); ++gq; }
+          continue;
+        }
         const int stage = static_cast<int>(it % C::NSTAGE);
         const uint32_t ph = (it / C::NSTAGE) & 1u;
         const int buf = static_cast<int>(it % C::NACC);
@@ -474,6 +514,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_commit(empty(stage));
         tc_commit(tfull(buf));
         if (s.last) { tc_commit(qempty(qb)); ++gq; }
+        ++it;
       }
       if (!ok) {
         // Error path: let every MMA already issued finish before TMEM is freed.
@@ -492,9 +533,41 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float racc = 0.f;                          // router partial sum
     int coef_g = -1;                           // query group of the staged head weights
     uint32_t it = 0;
-    for (; !s.done; s.next(p), ++it) {
+    // candidate lists (CMP): lane ql keeps the reservation state of this
+    // warp's query ql: current chunk (base, used), whether the next chunk has
+    // been requested (and where it starts), and the real entries written
+    constexpr int QHC = (C::ROUTER || C::GATHER || C::SPLIT_TILES) ? 1 : C::QPT / C::NSETS;
+    int cbase = -1, cused = CCHUNK, chas = 0, cnext = 0, creal = 0;
+    for (; !s.done; s.next(p)) {
       const int b = s.b;
       const int tg = s.tg;
+      const bool live = tile_live<C>(p, s);
+      const int q0s = C::SPLIT_TILES ? 0 : set * QHC;            // this set's first query (in group)
+      const long long rbase_s = static_cast<long long>(b) * p.T + tg * C::QPT + q0s;
+      if constexpr (C::CMP) {
+        // a new group (or this CTA's first tile): request the first chunk of
+        // every query now, so it has landed by the first kept score
+        if (s.first && lane < QHC && tg * C::QPT + q0s + lane < p.T) {
+          cbase = -1;
+          cused = CCHUNK;
+          chas = 1;
+          creal = 0;
+          cnext = atomicAdd(p.cres + rbase_s + lane, CCHUNK);
+        }
+      }
+      if (!live) {
+        if (!C::ROUTER && !C::GATHER && p.dead_fill && p.out != nullptr && (!C::SPLIT_TILES || set == 0)) {
+          // pruned tile: its visible entries read as -inf
+          const int key = s.j * C::KROWS + row;
+          const int t0 = tg * C::QPT + q0s;
+          const long long e = static_cast<long long>(key) * p.pstride - (p.q_offset + t0);
+          if (key < p.Lk) {
+#pragma unroll
+            for (int ql = 0; ql < QHC; ++ql)
+              if (t0 + ql < p.T && e <= ql) p.out[(rbase_s + ql) * p.ldo + key] = -INFINITY;
+          }
+        }
+      } else {
       const int buf = static_cast<int>(it % C::NACC);
       // split tiles: the two sets take alternate tiles (buffer b: set b & 1)
       const bool mine = C::SPLIT_TILES ? (static_cast<int>(it & 1u) == set) : true;
@@ -512,6 +585,17 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if constexpr (C::KEY_SCALES) {
           const int skey = s.j * C::KROWS + row;
           if (skey < p.Lk) ks = __ldg(p.k_scale + static_cast<long long>(b) * p.Lk + skey);
+        }
+        // candidate thresholds of this thread's queries (compaction only)
+        constexpr int QHT = QHC;
+        float cthr[QHT];
+#pragma unroll
+        for (int ql = 0; ql < QHT; ++ql) cthr[ql] = INFINITY;
+        if constexpr (C::CMP) {
+          const int tq0 = tg * C::QPT + (C::SPLIT_TILES ? 0 : set * QHT);
+#pragma unroll
+          for (int ql = 0; ql < QHT; ++ql)
+            if (tq0 + ql < p.T) cthr[ql] = __ldg(p.cthr + static_cast<long long>(b) * p.T + tq0 + ql);
         }
         if (!mbar_wait(tfull(buf), (it / C::NACC) & 1u, p.err)) break;
         tc_fence_after();
@@ -542,6 +626,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (lane == 0) mbar_arrive(tempty(buf));
         } else {
           constexpr int QH = C::SPLIT_TILES ? 1 : C::QPT / C::NSETS;   // queries per thread
+          static_assert(QH == QHT, "threshold slots");
           constexpr int NC = QH * C::H;                          // columns per thread
           constexpr int NCH = NC / 32;                           // 32-column chunks
           // independent partial sums per query (breaks the FMA dependency chain)
@@ -660,16 +745,95 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (C::GATHER) {
             const long long r = static_cast<long long>(b) * p.T + tg;
             if (key < p.n_compact) p.out[r * p.ldo + key] = gtok >= 0 ? accq[0] : -INFINITY;
-          } else if (key < p.Lk) {
+          } else {
             // query q0+ql sees this key iff key * pstride <= q_offset + t0 + ql
             const int t0 = tg * C::QPT + q0;
             const long long e = static_cast<long long>(key) * p.pstride - (p.q_offset + t0);
-            float* orow = p.out + rbase * p.ldo + key;
+            if (key < p.Lk && (!C::CMP || p.out != nullptr)) {
+              float* orow = p.out + rbase * p.ldo + key;
 #pragma unroll
-            for (int ql = 0; ql < QH; ++ql) {
-              if (t0 + ql < p.T && e <= ql) orow[ql * p.ldo] = ks * accq[ql];
+              for (int ql = 0; ql < QH; ++ql) {
+                if (t0 + ql < p.T && e <= ql) orow[ql * p.ldo] = ks * accq[ql];
+              }
+            }
+            if constexpr (C::CMP) {
+              // candidate lists: the warp's kept scores of query ql fill
+              // consecutive slots of its current chunk (lane ql holds the
+              // chunk state, uniform across the warp after the shuffles); a
+              // full chunk continues in the requested next one, and the chunk
+              // after that is requested once half of the current one is used,
+              // so the atomic's latency hides behind later tiles
+              const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+              for (int ql = 0; ql < QH; ++ql) {
+                const float sc = ks * accq[ql];
+                const bool keep = key < p.Lk && t0 + ql < p.T && e <= ql && sc >= cthr[ql];
+                const uint32_t msk = __ballot_sync(0xffffffffu, keep);
+                if (msk == 0u) continue;
+                const int n = __popc(msk);
+                const int pre = __popc(msk & lt);
+                const int used = __shfl_sync(0xffffffffu, cused, ql);
+                const int base = __shfl_sync(0xffffffffu, cbase, ql);
+                int slot;
+                if (used + n <= CCHUNK) {
+                  slot = base + used + pre;
+                  if (lane == ql) cused = used + n;
+                } else {
+                  int nxt;
+                  if (__shfl_sync(0xffffffffu, chas, ql)) {
+                    nxt = __shfl_sync(0xffffffffu, cnext, ql);
+                  } else {
+                    int v = 0;
+                    if (lane == ql) v = atomicAdd(p.cres + rbase + ql, CCHUNK);
+                    nxt = __shfl_sync(0xffffffffu, v, ql);
+                  }
+                  const int room = CCHUNK - used;
+                  slot = pre < room ? base + used + pre : nxt + (pre - room);
+                  if (lane == ql) { cbase = nxt; cused = n - room; chas = 0; }
+                }
+                if (keep && slot < p.ccap) {
+                  const long long o = (rbase + ql) * p.ccap + slot;
+                  p.cval[o] = sc;
+                  p.cidx[o] = key;
+                }
+                if (lane == ql) {
+                  creal += n;
+                  if (!chas && cused >= CCHUNK / 2) {
+                    cnext = atomicAdd(p.cres + rbase + ql, CCHUNK);
+                    chas = 1;
+                  }
+                }
+              }
             }
           }
+        }
+      }
+      ++it;
+      }  // live tile
+      if constexpr (C::CMP) {
+        if (s.last) {
+          // leaving the group: sentinels over the unused slots of this warp's
+          // chunks, then the real entries are counted
+#pragma unroll 1
+          for (int ql = 0; ql < QHC; ++ql) {
+            if (tg * C::QPT + q0s + ql >= p.T) break;
+            const long long orow = (rbase_s + ql) * p.ccap;
+            const int base = __shfl_sync(0xffffffffu, cbase, ql);
+            const int used = __shfl_sync(0xffffffffu, cused, ql);
+            const int has = __shfl_sync(0xffffffffu, chas, ql);
+            const int nxt = __shfl_sync(0xffffffffu, cnext, ql);
+            if (base >= 0)
+              for (int i = used + lane; i < CCHUNK; i += 32)
+                if (base + i < p.ccap) { p.cval[orow + base + i] = -INFINITY; p.cidx[orow + base + i] = -1; }
+            if (has)
+              for (int i = lane; i < CCHUNK; i += 32)
+                if (nxt + i < p.ccap) { p.cval[orow + nxt + i] = -INFINITY; p.cidx[orow + nxt + i] = -1; }
+            if (lane == ql && creal > 0) atomicAdd(p.creal + rbase_s + ql, creal);
+          }
+          cbase = -1;
+          cused = CCHUNK;
+          chas = 0;
+          creal = 0;
         }
       }
       if (C::ROUTER && s.last) {

@@ -54,6 +54,17 @@ struct TopkParams {
   const int* cand;       // optional map: position j -> cand[r * n_slots + j / blk] * blk + j % blk
   int n_slots, blk;
   unsigned* err;         // device status word (unused: the kernel has no waits)
+  // Optional candidate lists written by the score pass (every visible score
+  // >= a per-row threshold): row r's entries (value, position) fill slots
+  // [0, cres[r]) of cval / cidx[r * ccap + i], unused slots hold (-inf, -1);
+  // creal[r] counts the real ones. When a row holds at least min(k, n) real
+  // entries and cres[r] <= ccap, its top-k lies among them and the row's full
+  // scores are not read.
+  const float* cval;
+  const int* cidx;
+  const int* cres;
+  const int* creal;
+  int ccap;
 };
 
 constexpr int TK_BINS = 2048;        // histogram bins (11-bit digits, value bins)
@@ -215,6 +226,51 @@ __device__ __forceinline__ int map_index(const TopkParams& p, long long r, int i
   if (!p.cand) return i;
   const int slot = i / p.blk;
   return __ldg(p.cand + r * p.n_slots + slot) * p.blk + (i - slot * p.blk);
+}
+
+// Write the positions set in the bitmap words [l0, l1) of each thread (the
+// ranges ordered by thread) in ascending order: per-thread popcounts, a
+// prefix over the CTA, then the positions (staged in shared memory when they
+// fit, for coalesced stores) mapped through the index map; scores re-read
+// from the row. keff positions in all.
+template <class C>
+__device__ void emit_bitmap(const TopkParams& p, uint32_t* sm, long long r, int l0, int l1, uint32_t keff,
+                            const float* row) {
+  uint32_t* ws = sm + C::W_WS;
+  const uint32_t* bmap = sm + C::W_BMAP;
+  uint32_t* obuf = sm + C::W_KEY;  // key + position space (no longer read)
+  uint32_t cnt = 0;
+  for (int wd = l0; wd < l1; ++wd) cnt += __popc(bmap[wd]);
+  uint32_t tot;
+  uint32_t out = block_excl_scan<C::NT>(cnt, ws, tot);  // threads in order = positions in order
+  int32_t* oi = p.out_idx + r * p.k;
+  float* os = p.out_score ? p.out_score + r * p.k : nullptr;
+  const bool via_smem = keff <= static_cast<uint32_t>(C::OUT_CAP);
+  for (int wd = l0; wd < l1; ++wd) {
+    uint32_t bits = bmap[wd];
+    while (bits) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      const int i = wd * 32 + b;
+      if (out < keff) {  // holds by construction; guards the row
+        if (via_smem) {
+          obuf[out] = static_cast<uint32_t>(i);
+        } else {
+          oi[out] = map_index(p, r, i);
+          if (os) { const float x = __ldcg(row + i); os[out] = x == 0.f ? 0.f : x; }
+        }
+      }
+      ++out;
+    }
+  }
+  if (via_smem) {
+    __syncthreads();
+    for (int j = threadIdx.x; j < static_cast<int>(keff); j += C::NT) {
+      const int i = static_cast<int>(obuf[j]);
+      oi[j] = map_index(p, r, i);
+      if (os) { const float x = __ldcg(row + i); os[j] = x == 0.f ? 0.f : x; }
+    }
+  }
 }
 
 // ---------------------------------------------------------------- band path
@@ -444,40 +500,72 @@ __device__ bool topk_row_band(const TopkParams& p, uint32_t* sm, long long r, in
   // ---- 5. emit the bitmap in position order
   const int per = (w1 - w0 + 31) / 32;  // words per lane (contiguous)
   const int l0 = min(w1, w0 + lane * per), l1 = min(w1, l0 + per);
-  uint32_t cnt = 0;
-  for (int wd = l0; wd < l1; ++wd) cnt += __popc(bmap[wd]);
-  uint32_t tot;
-  uint32_t out = block_excl_scan<TK_NT>(cnt, ws, tot);  // lanes in order, warps in order = positions in order
-  int32_t* oi = p.out_idx + r * p.k;
-  float* os = p.out_score ? p.out_score + r * p.k : nullptr;
-  uint32_t* obuf = lkey;  // key + position space (no longer read)
-  const bool via_smem = keff <= static_cast<uint32_t>(C::OUT_CAP);
-  for (int wd = l0; wd < l1; ++wd) {
-    uint32_t bits = bmap[wd];
-    while (bits) {
-      const int b = __ffs(bits) - 1;
-      bits &= bits - 1u;
-      const int i = wd * 32 + b;
-      if (out < keff) {  // holds by construction; guards the row
-        if (via_smem) {
-          obuf[out] = static_cast<uint32_t>(i);
-        } else {
-          oi[out] = map_index(p, r, i);
-          if (os) { const float x = __ldcg(row + i); os[out] = x == 0.f ? 0.f : x; }
-        }
-      }
-      ++out;
-    }
-  }
-  if (via_smem) {
-    __syncthreads();
-    for (int j = tid; j < static_cast<int>(keff); j += TK_NT) {
-      const int i = static_cast<int>(obuf[j]);
-      oi[j] = map_index(p, r, i);
-      if (os) { const float x = __ldcg(row + i); os[j] = x == 0.f ? 0.f : x; }
-    }
-  }
+  emit_bitmap<C>(p, sm, r, l0, l1, keff, row);
   keff_out = keff;
+  return true;
+}
+
+// ---------------------------------------------------------------- candidate-list path
+// The score pass appended every visible score >= the row's threshold to the
+// row's candidate list, in no particular order. With at least min(k, n) of
+// them (and none lost past the capacity) the row's k-th score is >= the
+// threshold, so its top-k lies in the list: exact select of rank k over the
+// candidates' score keys (unused slots hold -inf, key 0, and never count); if
+// more scores equal the k-th than are taken, a second select over the
+// inverted positions of those takes the lowest positions; the winners go into
+// a position bitmap, emitted in order. Returns false (nothing written) when
+// the row must use its full scores.
+template <class C>
+__device__ bool topk_row_compact(const TopkParams& p, uint32_t* sm, long long r, int n, const float* row,
+                                 uint32_t& keff_out) {
+  constexpr int TK_NT = C::NT;
+  const int nc = __ldg(p.cres + r);
+  const int keff_i = min(p.k, n);
+  if (__ldg(p.creal + r) < keff_i || nc > p.ccap || n > C::MAX_ROW || n < 1) return false;
+  uint32_t* hist = sm + C::W_HIST;
+  uint32_t* ws = sm + C::W_WS;
+  uint32_t* vars = sm + C::W_VARS;
+  uint32_t* bmap = sm + C::W_BMAP;
+  const int tid = threadIdx.x;
+  const float* cv = p.cval + r * p.ccap;
+  const int* ci = p.cidx + r * p.ccap;
+  const uint32_t k = static_cast<uint32_t>(keff_i);
+  exact_select<TK_NT>([&](int i) { return score_key(__ldcg(cv + i)); }, nc, k, hist, ws, vars);
+  const uint32_t tau = vars[0];
+  const uint32_t teq = vars[1];
+  uint32_t neq = 0;
+  for (int i = tid; i < nc; i += TK_NT) neq += score_key(__ldcg(cv + i)) == tau;
+  uint32_t tot;
+  block_excl_scan<TK_NT>(neq, ws, tot);
+  const bool all_eq = tot == teq;
+  uint32_t tau2 = 0;
+  if (!all_eq) {
+    exact_select<TK_NT>(
+        [&](int i) { return score_key(__ldcg(cv + i)) == tau ? ~static_cast<uint32_t>(__ldcg(ci + i)) : 0u; },
+        nc, teq, hist, ws, vars);
+    tau2 = vars[0];
+  }
+  const int w1 = (n + 31) >> 5;
+  for (int wd = tid; wd < w1; wd += TK_NT) bmap[wd] = 0u;
+  __syncthreads();
+  // The winners' scores go into the row's own buffer (library scratch that
+  // the compacting score pass leaves unwritten), where the emit reads them.
+  float* srow = const_cast<float*>(row);
+  for (int i = tid; i < nc; i += TK_NT) {
+    const float v = __ldcg(cv + i);
+    const uint32_t key = score_key(v);
+    const uint32_t pos = static_cast<uint32_t>(__ldcg(ci + i));
+    const bool take = key > tau || (key == tau && (all_eq || ~pos >= tau2));
+    if (take) {
+      atomicOr(&bmap[pos >> 5], 1u << (pos & 31u));
+      if (p.out_score) srow[pos] = v;
+    }
+  }
+  __syncthreads();
+  const int per = (w1 + TK_NT - 1) / TK_NT;
+  const int l0 = min(w1, tid * per), l1 = min(w1, l0 + per);
+  emit_bitmap<C>(p, sm, r, l0, l1, k, row);
+  keff_out = k;
   return true;
 }
 
@@ -628,7 +716,8 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) topk_rows_kernel(const Top
     const float* row = p.scores + r * p.ld;
     uint32_t keff = 0;
     bool done = false;
-    if (n > p.k && n <= C::MAX_ROW) done = topk_row_band<C>(p, tk_smem, r, n, row, keff);
+    if (p.cres != nullptr) done = topk_row_compact<C>(p, tk_smem, r, n, row, keff);
+    if (!done && n > p.k && n <= C::MAX_ROW) done = topk_row_band<C>(p, tk_smem, r, n, row, keff);
     if (!done) topk_row_fallback<C>(p, tk_smem, r, n, row, keff);
     int32_t* oi = p.out_idx + r * p.k;
     float* os = p.out_score ? p.out_score + r * p.k : nullptr;
@@ -636,6 +725,59 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) topk_rows_kernel(const Top
       oi[j] = -1;
       if (os) os[j] = -INFINITY;
     }
+    __syncthreads();
+  }
+}
+
+// Rows whose candidate list cannot certify their top-k (fewer real entries
+// than min(k, visible), or entries lost past the capacity) mark every key
+// tile of their query group (qpt queries) for the fallback score pass.
+__global__ void fused_check_kernel(const int* __restrict__ cres, const int* __restrict__ creal, long long rows,
+                                   int T, long long q_offset, int L, int k, int cap, int qpt, int ntiles,
+                                   uint8_t* __restrict__ fb) {
+  const long long r = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (r >= rows) return;
+  const int t = static_cast<int>(r % T);
+  const long long V = min(q_offset + t + 1, static_cast<long long>(L));
+  const int need = static_cast<int>(min(static_cast<long long>(k), V));
+  if (cres[r] <= cap && creal[r] >= need) return;
+  const long long g = (r / T) * ((T + qpt - 1) / qpt) + t / qpt;
+  for (int j = 0; j < ntiles; ++j) fb[g * ntiles + j] = 1;
+}
+
+// ---------------------------------------------------------------- candidate thresholds
+// Per row, from the scores of every S-th key (samp[r * lds + i] is the score
+// of key i * S; the row has ns = min(p_t / S + 1, ns_max) of them): a
+// threshold the row's k-th score is very likely to reach, the r_lo-th largest
+// sample with r_lo = the sample rank expected for the k-th score + 4 standard
+// deviations (binomial) + 4. -inf keeps every visible score (rows with no
+// more than k visible keys, or too few samples). A wrong guess only costs
+// time: rows whose lists come out short are selected from their full scores.
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_threshold_kernel(const float* __restrict__ samp, long long rows,
+                                                            long long lds, int T, long long q_offset, int S,
+                                                            int ns_max, int L, int k, float* __restrict__ thr) {
+  __shared__ uint32_t hist[TK_BINS];
+  __shared__ uint32_t ws[64];
+  __shared__ uint32_t vars[64];
+  for (long long r = blockIdx.x; r < rows; r += gridDim.x) {
+    const long long pos = q_offset + r % T;
+    const long long V = min(pos + 1, static_cast<long long>(L));
+    const int ns = static_cast<int>(min(pos / S + 1, static_cast<long long>(ns_max)));
+    float t = -INFINITY;
+    if (V > k) {
+      const float pr = static_cast<float>(k) / static_cast<float>(V);
+      const float mean = pr * ns;
+      const float sd = sqrtf(static_cast<float>(ns) * pr * (1.f - pr));
+      const int r_lo = static_cast<int>(ceilf(mean + 4.f * sd + 4.f));
+      if (r_lo <= ns) {
+        const float* row = samp + r * lds;
+        exact_select<NT>([&](int i) { return score_key(__ldcg(row + i)); }, ns, static_cast<uint32_t>(r_lo), hist,
+                         ws, vars);
+        t = key_score(vars[0]);
+      }
+    }
+    if (threadIdx.x == 0) thr[r] = t;
     __syncthreads();
   }
 }

@@ -20,6 +20,11 @@ Distributions follow the five workloads the indexer is measured on:
              heads, top-k=2048, MISA-dagger k'=8192
 * ``hisa``   T=1024 at the end of a 262144 prefix, H_I=32 (GLM-5 head count),
              block 128, top-128 blocks, top-k=2048, recency ramp on key dim 0
+* ``indexcache`` four layers of ``dsa`` chunks with the IndexCache pattern
+             FSSS: one layer runs the indexer, three reuse its indices (only
+             the F layer has inputs: S layers compute no indexer projections)
+* ``dsa_fp8`` the ``dsa`` chunk quantised to FP8 e4m3 the way the decode cache
+             is (per-token key scale, per-(query, head) query scale)
 
 Random streams: one numpy PCG64 stream per tensor, spawned from
 ``SeedSequence(seed)``; the decode K cache uses one child stream per sequence so
@@ -27,6 +32,8 @@ the values do not depend on how generation is chunked.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 from typing import Optional
 
@@ -180,19 +187,39 @@ def decode_inputs(batch: int, L: int, H: int, d: int, seed: int = 0,
     centres = rc.standard_normal((n_centres, d), dtype=np.float32)
     k8 = np.empty((batch, L, d), dtype=np.uint8)
     ks = np.empty((batch, L), dtype=np.float32)
-    n_clustered = 0
-    for b in range(batch):
+
+    def one_sequence(b):
         kb = kst[b].standard_normal((L, d), dtype=np.float32)
         pick = kst[b].random(L) < cluster_frac
         which = kst[b].integers(0, n_centres, size=L)
         kb[pick] = centres[which[pick]]
-        n_clustered += int(pick.sum())
         k8[b], ks[b] = quantize_rows_e4m3(kb)
+        return int(pick.sum())
+
+    # every sequence draws from its own stream, so the values do not depend
+    # on the order the threads run in
+    with ThreadPoolExecutor(max_workers=max(1, min(16, os.cpu_count() or 1, batch))) as ex:
+        n_clustered = sum(ex.map(one_sequence, range(batch)))
     q32 = rq.standard_normal((batch, 1, H, d), dtype=np.float32) * np.float32(1.0 / np.sqrt(d))
     q8, qs = quantize_rows_e4m3(q32)
     w = (rw.standard_normal((batch, 1, H), dtype=np.float32) * np.float32(w_std)).astype(np.float32)
     return IndexerInputs(q=q8, k=k8, w=w, q_offset=L - 1, dtype="fp8_e4m3",
                          q_scale=qs, k_scale=ks, meta={"clustered_tokens": n_clustered})
+
+
+def fp8_prefill_inputs(T: int, L: int, H: int, d: int, q_offset: Optional[int] = None,
+                       seed: int = 0, batch: int = 1, w_std: Optional[float] = None,
+                       needles: int = 0) -> IndexerInputs:
+    """FP8 prefill chunk: the bf16 chunk of ``prefill_inputs`` (same streams,
+    needles included), widened to fp32 and quantised the way the decode cache
+    is: keys per token, queries per (query, head) row, e4m3 with scale
+    absmax/448."""
+    base = prefill_inputs(T, L, H, d, q_offset=q_offset, seed=seed, batch=batch, w_std=w_std,
+                          needles=needles)
+    q8, qs = quantize_rows_e4m3(bf16_bits_to_f32(base.q))
+    k8, ks = quantize_rows_e4m3(bf16_bits_to_f32(base.k))
+    return IndexerInputs(q=q8, k=k8, w=base.w, q_offset=base.q_offset, dtype="fp8_e4m3",
+                         q_scale=qs, k_scale=ks, meta=base.meta)
 
 
 # ----------------------------------------------------------------- workloads
@@ -201,6 +228,10 @@ CONFIGS = {
     "dsa": dict(kind="dense", T=4096, L=32768, H=64, d=128, q_offset=28672, topk=2048,
                 needles=64, w_std=0.125),
     "decode": dict(kind="decode", batch=64, T=1, L=131072, H=64, d=128, topk=2048),
+    "indexcache": dict(kind="indexcache", pattern="FSSS", T=4096, L=32768, H=64, d=128, q_offset=28672,
+                       topk=2048, needles=64, w_std=0.125),
+    "dsa_fp8": dict(kind="dense_fp8", T=4096, L=32768, H=64, d=128, q_offset=28672, topk=2048,
+                    needles=64, w_std=0.125),
     "misa": dict(kind="misa", T=2048, L=131072, H=64, d=128, q_offset=129024, topk=2048,
                  block=64, h=8, kprime=8192, w_std=0.125),
     "hisa": dict(kind="hisa", T=1024, L=262144, H=32, d=128, q_offset=261120, topk=2048,
@@ -213,6 +244,12 @@ def make_inputs(name: str, seed: int = 0) -> IndexerInputs:
     c = CONFIGS[name]
     if c["kind"] == "decode":
         return decode_inputs(c["batch"], c["L"], c["H"], c["d"], seed=seed)
+    if c["kind"] == "indexcache":  # the inputs of the (single) F layer
+        return prefill_inputs(c["T"], c["L"], c["H"], c["d"], q_offset=c["q_offset"], seed=seed,
+                              w_std=c.get("w_std"), needles=c.get("needles", 0))
+    if c["kind"] == "dense_fp8":
+        return fp8_prefill_inputs(c["T"], c["L"], c["H"], c["d"], q_offset=c["q_offset"], seed=seed,
+                                  w_std=c.get("w_std"), needles=c.get("needles", 0))
     return prefill_inputs(c["T"], c["L"], c["H"], c["d"], q_offset=c["q_offset"], seed=seed,
                           w_std=c.get("w_std"), needles=c.get("needles", 0),
                           recency=c.get("recency", 0.0))

@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 14
+    assert len(names) == 21
     assert set(names) == set(B._SIGS)
     for n in names:
         assert getattr(lib, n) is not None
@@ -133,3 +133,45 @@ def test_selftest_and_noalloc_checks(lib):
     # are refused before any CUDA call
     a = _args(T=4, L=5_000_000, q_offset=4_999_996)
     assert lib.indexer_score_topk_noalloc(ctypes.byref(a), 16, ctypes.c_void_p(0x40000), None, None) == -3
+
+
+def test_indexcache_checks(lib):
+    F = _args()
+    S = B.IndexerArgs(batch=1, T=4, L=0, H=0, d=0, q_offset=0, qk_dtype=0)  # only batch, T read
+    arr = (B.IndexerArgs * 3)(F, S, F)
+    P = ctypes.c_void_p
+    outs = (P * 3)(0x40000, 0x40000, 0x41000)
+    ws, big = ctypes.c_void_p(0x50000), 1 << 30
+    one = lib.indexer_workspace_size(ctypes.byref(F), 16)
+    assert lib.indexcache_workspace_size(arr, 3, b"FSF", 16) == one
+    assert lib.indexcache_workspace_size(arr, 3, b"FXF", 16) == 0
+    # rejected before any launch: bad pattern, first layer shared, mismatched
+    # S shape, missing output, unsupported F layer, small workspace
+    assert lib.indexcache_score_topk(arr, 3, b"SFF", 16, outs, None, ws, big, None) == -1
+    assert lib.indexcache_score_topk(arr, 3, b"FXF", 16, outs, None, ws, big, None) == -1
+    assert lib.indexcache_score_topk(arr, 3, b"FS", 16, outs, None, ws, big, None) == -1
+    bad_s = (B.IndexerArgs * 3)(F, B.IndexerArgs(batch=1, T=5), F)
+    assert lib.indexcache_score_topk(bad_s, 3, b"FSF", 16, outs, None, ws, big, None) == -1
+    assert lib.indexcache_score_topk(arr, 3, b"FSF", 16, (P * 3)(0x40000, None, 0x41000), None, ws, big,
+                                     None) == -1
+    bad_f = (B.IndexerArgs * 3)(F, S, _args(H=48))
+    assert lib.indexcache_score_topk(bad_f, 3, b"FSF", 16, outs, None, ws, big, None) == -2
+    assert lib.indexcache_score_topk(arr, 3, b"FSF", 16, outs, None, ws, one - 1, None) == -3
+    # scores requested for an S layer whose F layer has none
+    assert lib.indexcache_score_topk(arr, 3, b"FSF", 16, outs, (P * 3)(None, 0x60000, None), ws, big,
+                                     None) == -1
+
+
+def test_hisa_refine_checks(lib):
+    a = _args(L=1000, q_offset=996)
+    blocks, out, ws, big = ctypes.c_void_p(0x40000), ctypes.c_void_p(0x60000), ctypes.c_void_p(0x50000), 1 << 30
+    need = lib.hisa_refine_workspace_size(ctypes.byref(a), 4, 128)
+    assert need > 256
+    assert lib.hisa_refine_scores(ctypes.byref(a), None, 4, 128, out, 512, ws, big, None) == -1
+    assert lib.hisa_refine_scores(ctypes.byref(a), blocks, 4, 128, out, 511, ws, big, None) == -1  # ld < m*blk
+    assert lib.hisa_refine_scores(ctypes.byref(a), blocks, 4, 96, out, 512, ws, big, None) == -2  # blk % 128
+    assert lib.hisa_refine_scores(ctypes.byref(_args(H=16, L=1000, q_offset=996)), blocks, 4, 128, out, 512,
+                                  ws, big, None) == -2
+    assert lib.hisa_refine_scores(ctypes.byref(a), blocks, 4, 128, out, 512, ws, need - 1, None) == -3
+    # the HISA workspace grows by the inverted lists when blocks are whole key tiles
+    assert lib.hisa_workspace_size(ctypes.byref(a), 128, 4, 16) > lib.hisa_workspace_size(ctypes.byref(a), 96, 4, 16)

@@ -9,15 +9,16 @@ import bench
 from sparse_attention_token_score_b200 import workloads as wl
 
 
-@pytest.mark.parametrize("name", ["tiny", "dsa", "decode", "misa", "hisa"])
+@pytest.mark.parametrize("name", ["tiny", "dsa", "decode", "misa", "hisa", "dsa_fp8", "indexcache"])
 def test_pairs_are_the_dense_visible_pairs(name):
     c, batch, off, pairs, label = bench.workload_desc(name)
     T = c["T"]
     # query t at position off + t sees off + t + 1 keys (never more than L)
-    expect = batch * sum(min(c["L"], off + t + 1) for t in range(T))
+    expect = batch * sum(min(c["L"], off + t + 1) for t in range(T)) * len(c.get("pattern", "F"))
     assert pairs == expect
     assert label.startswith({"tiny": "tiny_prefill", "dsa": "dsa_chunk", "decode": "decode_fp8",
-                              "misa": "misa_dagger", "hisa": "hisa"}[name])
+                              "misa": "misa_dagger", "hisa": "hisa", "dsa_fp8": "dsa_chunk_fp8",
+                              "indexcache": "indexcache_dsa_chunk"}[name])
 
 
 def test_dsa_chunk_size():
@@ -45,6 +46,8 @@ def test_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     shutil.copytree(src, dst)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     key = ("dsa", "score_tc<bf16>")
+    # a capture recorded against the current source stays valid ...
+    monkeypatch.setitem(bench.TRAFFIC, key, (123.0e6, bench.source_hash(key[1])))
     assert bench.traffic_for(*key) == bench.TRAFFIC[key][0]
     f = dst / "score_tc.cuh"
     f.write_text("// a comment line\n" + f.read_text())         # comments do not count
@@ -70,3 +73,21 @@ def test_reference_arm_json_line():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     assert line["config"]["workload"].startswith("tiny_prefill")
+    # same config object as the GPU arm's line, and a step time that is the
+    # sampled step's own (not an extrapolation to the full workload)
+    c, batch, off, pairs, label = bench.workload_desc("tiny")
+    assert line["config"] == bench.workload_config(c, batch, label, off, pairs, 1)
+    assert line["ms_per_step"] * line["steps"] / 1e3 < 600
+    assert line["sample"]["pairs_per_timed_step"] <= pairs
+
+
+def test_clock_summary_keeps_the_timed_window():
+    S = bench.ClockSampler
+    rows = [(0.00, 1900.0, 1965.0, 0), (0.01, 1950.0, 1965.0, 0x4), (0.02, 1960.0, 1965.0, 0),
+            (0.03, 1000.0, 1965.0, 0x40), (0.10, 1100.0, 1965.0, 0x8)]
+    st = S.summarize(rows, 0.005, 0.025, 1965.0)
+    # the sample before the window, the two inside and the first one after
+    assert st["samples"] == 4 and st["samples_inside"] == 2
+    assert st["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert st["sm_mhz"] == 1925.0
+    assert S.summarize(rows, None, None, 1965.0)["samples"] == 0

@@ -403,3 +403,107 @@ def test_dosa_planted_mistake_is_caught(monkeypatch):
     dense = oracle.dense_topk(inp, 16)
     dosa = oracle.dosa_topk(inp, 16, [0], 32)
     assert not np.array_equal(dense["idx"], dosa["idx"])
+
+
+def test_indexcache_layers_follow_the_pattern():
+    # F layers are the dense indexer on their own inputs; an S layer is the
+    # nearest preceding F layer's result, whatever its own inputs are
+    layers = [wl.prefill_inputs(6, 300, 8, 64, q_offset=294, seed=100 + i, batch=2) for i in range(5)]
+    got = oracle.indexcache(layers, "FSFSS", 20)
+    dense = [np.stack([oracle.dense_topk(x, 20, b=b)["idx"] for b in range(2)]) for x in layers]
+    for i, j in enumerate([0, 0, 2, 2, 2]):
+        assert np.array_equal(got[i], dense[j])
+    assert not np.array_equal(dense[0], dense[1])  # the layers differ, so reuse is visible
+    all_f = oracle.indexcache(layers, "FFFFF", 20)
+    assert all(np.array_equal(a, b) for a, b in zip(all_f, dense))
+    for bad in ("SFFFF", "FFF", "FXFFF"):
+        with pytest.raises(ValueError):
+            oracle.indexcache(layers, bad, 20)
+
+
+# ------------------------------------------------------------ DoSA at tile granularity
+def test_sample_threshold_closed_form():
+    # V = 1000 keys, k = 50: p = 0.05; 100 samples -> r_lo = ceil(5 + 4 sqrt(4.75) + 4) = 18
+    samp = np.arange(100, dtype=np.float64)[::-1] * 0.5          # 49.5, 49.0, ...
+    assert oracle.sample_threshold(samp, 50, 1000) == 49.5 - 17 * 0.5
+    assert oracle.sample_threshold(samp, 1000, 1000) == -np.inf  # V <= k keeps every key
+    assert oracle.sample_threshold(samp[:6], 50, 1000) == -np.inf  # r_lo = 7 beyond the sample
+
+
+def test_dosa_screen_heads_rank_by_weighted_norm():
+    q = np.zeros((4, 2))
+    q[:, 0] = [1.0, 2.0, 1.0, 4.0]
+    w = np.array([-3.0, 1.0, 2.0, 0.25])     # |w| ||q||: 3, 2, 2, 1
+    assert oracle.dosa_screen_heads(q, w, 2).tolist() == [0, 1]   # tie 2 = 2 -> lower head
+    assert oracle.dosa_screen_heads(q, w, 4).tolist() == [0, 1, 2, 3]
+
+
+def _low_norm_population(seed, T=8, L=4096, H=8, d=32, live_every=4):
+    """Keys of most 128-key tiles shrunk 100x (a low-norm population no query
+    can rank high); every live_every-th tile keeps its norm. Non-negative head
+    weights, so every query's best scores are clearly positive."""
+    inp = wl.prefill_inputs(T=T, L=L, H=H, d=d, q_offset=L - T, seed=seed)
+    inp.w = np.abs(inp.w)
+    kf = wl.bf16_bits_to_f32(inp.k)
+    tile = np.arange(L) // 128
+    kf[0, tile % live_every != 0] *= np.float32(0.01)
+    inp.k = wl.f32_to_bf16_bits(kf)
+    return inp
+
+
+@pytest.mark.parametrize("seed,n_screen,S,qpt,w_sign", [
+    (51, 3, 16, 4, 0), (52, 0, 8, 2, 0), (53, 8, 16, 4, 0),   # no screened head / every head screened
+    (54, 2, 16, 8, -1),                                         # all-negative weights: ties at 0
+])
+def test_dosa_tile_equals_dense(seed, n_screen, S, qpt, w_sign):
+    inp = _dosa_inp(seed, w_sign=w_sign, T=12, L=700)
+    if seed == 52:
+        inp.k[0, 300:320] = inp.k[0, 40]  # duplicate keys: exact ties across positions
+    dense = oracle.dense_topk(inp, 16)
+    got = oracle.dosa_tile_topk(inp, 16, n_screen, S, qpt)
+    assert got["queries"] == list(range(12))
+    assert np.array_equal(dense["idx"], got["idx"])
+
+
+def test_dosa_tile_prunes_a_low_norm_population():
+    inp = _low_norm_population(55)
+    dense = oracle.dense_topk(inp, 16)
+    got = oracle.dosa_tile_topk(inp, 16, 3, 16, 4)
+    assert np.array_equal(dense["idx"], got["idx"])
+    assert got["live"].mean() <= 0.5          # at least half of the tiles pruned
+    assert not any(got["fallback"])
+    # the live tiles hold every winner
+    for i, t in enumerate(got["queries"]):
+        assert np.all(got["live"][t // 4, dense["idx"][i] // 128] == 1)
+
+
+def test_dosa_tile_short_certificate_falls_back():
+    # the sampled keys (every 16th) are the strongest: thresholds come out so
+    # high that fewer than k scores reach them; the rows fall back to all keys
+    inp = _dosa_inp(56, T=8, L=900)
+    q, _, _ = oracle.dequant(inp)
+    kf = wl.bf16_bits_to_f32(inp.k)
+    inp.w = np.abs(inp.w)
+    kf[0, ::16] = 3.0 * q.mean(axis=(0, 1)) / np.linalg.norm(q.mean(axis=(0, 1)))
+    inp.k = wl.f32_to_bf16_bits(kf)
+    dense = oracle.dense_topk(inp, 100)
+    got = oracle.dosa_tile_topk(inp, 100, 3, 16, 4)
+    assert any(got["fallback"])
+    assert np.array_equal(dense["idx"], got["idx"])
+
+
+def test_dosa_tile_planted_mistake_is_caught(monkeypatch):
+    # a bound without the unscreened positive heads prunes tiles that hold
+    # winners; the certificate still rescues rows whose count comes out short,
+    # so the mistake must show as a different selection somewhere
+    real = oracle.dosa_upper_bound
+
+    def forgetful(q, k, w, t, keys, screen):
+        bound, part = real(q, k, w, t, keys, screen)
+        return part, part
+
+    monkeypatch.setattr(oracle, "dosa_upper_bound", forgetful)
+    inp = _dosa_inp(57, T=16, L=1500)
+    dense = oracle.dense_topk(inp, 16)
+    got = oracle.dosa_tile_topk(inp, 16, 1, 16, 4)
+    assert not np.array_equal(dense["idx"], got["idx"])

@@ -1,11 +1,13 @@
 """indexer_score_topk_noalloc: the dense score + top-k for callers that cannot
-allocate device memory (inside a stream capture that must stay free of
-allocations, in a plugin whose host runtime owns every device allocation, or
-with no allocator at all). It uses the library's own static scratch instead of
-a caller workspace. These checks compare it, through the C ABI, with the
-workspace entry point on the same inputs, twice in a row (the second call
-reuses scratch that still holds the first call's scores), and check that a
-problem too large for the scratch is refused before any launch.
+allocate device memory (a plugin whose host runtime owns every device
+allocation, a loop where cudaMalloc and its possible device synchronisation
+are not allowed, or code with no allocator at all). It uses the library's own
+static scratch instead of a caller workspace. These checks compare it, through
+the C ABI, with the workspace entry point on the same inputs, twice in a row
+(the second call reuses scratch that still holds the first call's scores),
+check after each call that the scratch's status word (dsa_noalloc_status)
+reads "ok", and check that a problem too large for the scratch is refused
+before any launch.
 
 This file is collected last so that a run stopping at the first failure has
 already run every other test."""
@@ -36,7 +38,9 @@ def _compare(inp, topk, rtol):
                                             ctypes.c_void_p(sc.data_ptr()),
                                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0, B.STATUS.get(st, st)
-    torch.cuda.synchronize()
+    # a bounded device wait that gave up inside the call would show here
+    st = B.lib().dsa_noalloc_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0, B.STATUS.get(st, st)
     ref_idx, ref_sc, idx, sc = (t.cpu().numpy() for t in (ref_idx, ref_sc, idx, sc))
     assert np.array_equal(idx, ref_idx)
     pad = ref_idx < 0
