@@ -76,7 +76,8 @@ def workload_desc(name, queries=None, batch=None):
         pairs *= len(c["pattern"])
     tag = {"tiny": "tiny_prefill", "dsa": "dsa_chunk", "decode": "decode_fp8",
            "misa": "misa_dagger", "hisa": "hisa", "dsa_fp8": "dsa_chunk_fp8",
-           "indexcache": "indexcache_dsa_chunk"}[name]
+           "indexcache": "indexcache_dsa_chunk", "dosa": "dosa_dsa_chunk",
+           "dosa_lownorm": "dosa_lownorm_dsa_chunk", "dsa_lists": "dsa_chunk_lists"}[name]
     label = f"{tag}_B{batch}_T{c['T']}_L{c['L']}_H{c['H']}_d{c['d']}_k{c['topk']}"
     if name == "misa":
         label += f"_blk{c['block']}_h{c['h']}_kp{c['kprime']}"
@@ -84,10 +85,14 @@ def workload_desc(name, queries=None, batch=None):
         label += f"_blk{c['block']}_m{c['m']}"
     if name == "indexcache":
         label += f"_layers{c['pattern']}"
+    if name in ("dosa", "dosa_lownorm"):
+        label += f"_screen{c['n_screen']}"
     return c, batch, off, pairs, label
 
 
 DENSE = ("tiny", "dsa", "decode", "dsa_fp8", "indexcache")  # workloads whose F layer is indexer_score_topk
+DOSA = ("dosa", "dosa_lownorm")                              # dosa_score_topk
+LISTS = ("dsa_lists",)                                       # indexer_score_topk_lists
 
 
 class Runner:
@@ -111,6 +116,14 @@ class Runner:
                 pat = c["pattern"]
                 assert pat.count("F") == 1, "the bench's IndexCache slice has one F layer"
                 self.shared = B.IndexerArgs(batch=self.batch, T=c["T"])  # S layers: shape only
+        elif name in LISTS:
+            self.ws = B.alloc_workspace(B.indexer_lists_workspace_size(a, self.topk))
+        elif name in DOSA:
+            self.ws = B.alloc_workspace(B.dosa_workspace_size(a, self.topk, c["n_screen"]))
+            qpt = 256 // c["H"]
+            self.live = torch.empty((self.batch, -(-c["T"] // qpt), -(-c["L"] // 128)), dtype=torch.uint8,
+                                    device="cuda")
+            self.live_pairs = None
         elif name == "misa":
             self.ws = B.alloc_workspace(B.misa_workspace_size(a, c["block"], c["h"], self.topk, c["kprime"]))
         else:
@@ -127,6 +140,10 @@ class Runner:
             B.indexcache_score_topk(layers, c["pattern"], self.topk, [o] * len(layers), None, self.ws)
         elif self.name in DENSE:
             B.indexer_score_topk(a, self.topk, o, None, self.ws)
+        elif self.name in LISTS:
+            B.indexer_score_topk_lists(a, self.topk, o, None, self.ws)
+        elif self.name in DOSA:
+            B.dosa_score_topk(a, self.topk, c["n_screen"], o, None, self.live, self.ws)
         elif self.name == "misa":
             B.misa_route_score_topk(a, c["block"], c["h"], self.topk, c["kprime"], o, None, None,
                                     None, self.ws)
@@ -146,13 +163,17 @@ class Runner:
         pos = inp.q_offset + np.arange(T, dtype=np.int64)
         label = name.split(": ")[-1]
         stage = name.split(": ")[0] if ": " in name else ""
-        if "sample pass" in stage or "candidate lists)" in label:
+        if "sample pass" in stage or "fallback" in stage or "candidate lists)" in label:
             return None, None
-        if self.name in DENSE:
+        if self.name in DENSE + DOSA + LISTS:
             pairs = self.pairs // len(c.get("pattern", "F"))  # the F layer's pairs (indexcache)
+            if stage == "bounds" and label.startswith("score_tc"):
+                return pairs * 2.0 * d * 8, "tensor"          # 8 augmented heads per pair
             if label.startswith("score_tc"):
                 if self.name == "decode":
                     return pairs * (d + 4), "hbm"          # one FP8 key row + its scale per pair
+                if self.name in DOSA:                      # the live tiles' pairs only
+                    return self.live_pairs * 2.0 * d * H if self.live_pairs is not None else None, "tensor"
                 return pairs * 2.0 * d * H, ("tensor_fp8" if self.name == "dsa_fp8" else "tensor")
             if label == "topk_rows":
                 return pairs * 4 + rows * k * 4, "hbm"    # every visible score read, k ids written
@@ -160,7 +181,7 @@ class Runner:
             blk, h, kp = c["block"], c["h"], c["kprime"]
             M = -(-L // blk)
             vis_blocks = int(self.batch * np.minimum(pos // blk + 1, M).sum())
-            if stage == "router":
+            if stage == "router" and label.startswith("score_tc"):
                 return vis_blocks * 2.0 * d * H, "tensor"
             if stage == "routed" and label.startswith("score_tc"):
                 return self.pairs * 2.0 * d * h, "tensor"
@@ -181,6 +202,26 @@ class Runner:
             if stage == "tokens" and label == "topk_rows":
                 return rows * m * blk * 4 + rows * k * 8, "hbm"
         return None, None
+
+    def dosa_live(self):
+        """Fraction of the visible (query group, key tile) pairs the bound kept,
+        and the visible pairs of the kept tiles (from the last step's mask)."""
+        c = self.c
+        live = self.live.cpu().numpy()[0]
+        qpt, T, L = 256 // c["H"], c["T"], c["L"]
+        kept = total = 0
+        pairs = 0
+        for g in range(live.shape[0]):
+            t0, t1 = g * qpt, min(T, (g + 1) * qpt)
+            pos = self.inp.q_offset + np.arange(t0, t1)
+            nt = -(-min(pos[-1] + 1, L) // 128)
+            kept += int(live[g, :nt].sum())
+            total += nt
+            for j in np.flatnonzero(live[g, :nt]):
+                lo, hi = 128 * j, min(128 * (j + 1), L)
+                pairs += int(np.clip(pos + 1 - lo, 0, hi - lo).sum())
+        self.live_pairs = pairs
+        return kept / total, pairs
 
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
@@ -507,7 +548,7 @@ def make_inputs(name, seed, queries=0, batch=0):
 
 
 # ------------------------------------------------------------------ main
-SUB_WORKLOADS = ("tiny", "decode", "misa", "hisa", "dsa_fp8", "indexcache")
+SUB_WORKLOADS = ("tiny", "decode", "misa", "hisa", "dsa_fp8", "indexcache", "dsa_lists", "dosa", "dosa_lownorm")
 MIN_TIMED_MS = 60.0  # sub-records run enough steps that the clock sampler sees the GPU busy
 
 
@@ -542,6 +583,12 @@ def measure_workload(name, args, torch, world, rank, local, flush, barrier, rmax
     total_ms, pairs_per_s = aggregate_ranks(float(sum(times)), r.pairs, steps, world, rmax)
     assert r.ix.device_status() == 0, "device wait timed out"
 
+    dosa = None
+    if name in DOSA:
+        frac_live, live_pairs = r.dosa_live()
+        dosa = {"live_tile_fraction": frac_live, "pruned_tile_fraction": 1.0 - frac_live,
+                "refined_pairs_per_step": live_pairs,
+                "pruned_pair_fraction": 1.0 - live_pairs / (r.pairs / len(r.c.get("pattern", "F")))}
     # ---- every launch of the step, timed by the library's launch profiler
     # (CUDA events on the launching stream) over `steps` more steps with the
     # same L2 flush; the kernel with the largest time per step is the roofline's
@@ -609,6 +656,8 @@ def measure_workload(name, args, torch, world, rank, local, flush, barrier, rmax
         "gpu_launches": int(round(launches_per_step * steps)), "clocks": clocks,
         "step_ms": {"min": min(times), "median": statistics.median(times), "max": max(times)},
     }
+    if dosa is not None:
+        rec["dosa"] = dosa
     del r, inp
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
@@ -620,7 +669,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="all", choices=["all", "tiny", "dsa", "decode", "misa", "hisa", "dsa_fp8", "indexcache"],
+    ap.add_argument("--workload", default="all", choices=["all", "tiny", "dsa", "decode", "misa", "hisa", "dsa_fp8", "indexcache", "dosa",
+                             "dosa_lownorm", "dsa_lists"],
                     help="all (default): the dsa chunk is the headline line, the other four "
                          "workloads are measured in the same run under 'workloads'")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

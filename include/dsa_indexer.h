@@ -143,6 +143,29 @@ DSA_EXPORT dsa_status indexer_score_topk_noalloc(const dsa_indexer_args* a, int 
  * dsa_device_status for the call that has no workspace). */
 DSA_EXPORT dsa_status dsa_noalloc_status(void* stream);
 
+/* indexer_score_topk_lists: the same selection as indexer_score_topk with the
+ * scoring fused with a filter (the LiteTopK idea named in the "DoSA: Dots
+ * Sparse Attention" review: scoring and filtering fused to cut memory
+ * traffic), kept exact:
+ *   1. every S-th visible key (S = 16, or larger so a row has at most 4096)
+ *      is scored; from that sample each query gets a threshold its k-th
+ *      score very likely reaches (the sample rank expected for the k-th score
+ *      + 4 binomial standard deviations + 4);
+ *   2. the score pass keeps no full scores: every visible score >= the
+ *      query's threshold goes, with its key, to the query's candidate list;
+ *   3. a query whose list holds at least min(k, visible) entries has its
+ *      top-k in the list (its k-th score reaches the threshold); the other
+ *      queries' groups (256 / H queries) are re-scored in full;
+ *   4. top-k from the lists (or the full scores), score descending, index
+ *      ascending.
+ * Output and ordering as indexer_score_topk, bit for bit. bf16; rows of at
+ * least 4096 keys, L a multiple of S, topk <= L / 8, else
+ * DSA_ERR_UNSUPPORTED. Workspace: indexer_lists_workspace_size bytes (0
+ * when unsupported). */
+DSA_EXPORT size_t indexer_lists_workspace_size(const dsa_indexer_args* a, int topk);
+DSA_EXPORT dsa_status indexer_score_topk_lists(const dsa_indexer_args* a, int topk, int32_t* out_idx,
+                                               float* out_score, void* workspace, size_t ws_bytes, void* stream);
+
 /* Stage 1 alone: write the scores I[t,s] of all visible keys into
  * out_scores[(b*T + t) * ld + s] (ld >= L). Entries with s > q_offset + t are
  * left untouched. Workspace: the 256-byte header only. */
@@ -231,6 +254,37 @@ DSA_EXPORT size_t hisa_refine_workspace_size(const dsa_indexer_args* a, int m, i
 DSA_EXPORT dsa_status hisa_refine_scores(const dsa_indexer_args* a, const int32_t* blocks, int m, int blk,
                                          float* out, long long ld, void* workspace, size_t ws_bytes,
                                          void* stream);
+
+/* ------------------------------------------------------------ DoSA
+ * dosa_score_topk ("DoSA: Dots Sparse Attention" review, section 3): the
+ * dense selection of indexer_score_topk, computed with certified pruning.
+ *   1. every 16th (or 32nd...) visible key is scored with all heads; from that
+ *      sample each query gets a threshold thr its k-th score very likely
+ *      reaches;
+ *   2. screening: per query the n_screen heads with the largest
+ *      |w_h| * ||q_h|| are kept exactly; the other positive-weight heads are
+ *      bounded through ReLU(x) = (x + |x|) / 2 and Cauchy-Schwarz, the other
+ *      negative-weight heads subtract ReLU(k . sum |w_h| q_h); the bound is
+ *      evaluated on the tensor cores over n_screen + 3 augmented heads;
+ *   3. a 128-key tile stays live for a group of 256 / H queries when some
+ *      visible key of it has bound >= thr for some query of the group; the
+ *      other tiles are not scored;
+ *   4. live tiles are scored with all H heads, scores >= thr are kept per
+ *      query; a query with at least min(k, visible) of them has its top-k
+ *      among them (its k-th score reaches thr, and every pruned key scores
+ *      below thr); other queries have their whole group re-scored;
+ *   5. top-k (score descending, index ascending).
+ * The selection (and out_score) equals indexer_score_topk's exactly.
+ *   out_live NULL or [batch, ceil(T / (256 / H)), ceil(L / 128)] bytes: 1 for
+ *            the tiles step 3 kept, 0 for the pruned ones
+ * bf16; d in {64, 128}; H in {16, 32, 64}; 0 <= n_screen < H, n_screen <= 13;
+ * rows long enough for sampled thresholds (L >= 4096, L a multiple of the
+ * sample stride, topk <= L / 8), else DSA_ERR_UNSUPPORTED. Workspace:
+ * dosa_workspace_size bytes (0 when unsupported). */
+DSA_EXPORT size_t dosa_workspace_size(const dsa_indexer_args* a, int topk, int n_screen);
+DSA_EXPORT dsa_status dosa_score_topk(const dsa_indexer_args* a, int topk, int n_screen, int32_t* out_idx,
+                                      float* out_score, uint8_t* out_live, void* workspace, size_t ws_bytes,
+                                      void* stream);
 
 /* Launch profiling (plumbing; no counterpart on the pages). Between
  * dsa_profile_begin and dsa_profile_end every kernel the library launches, on

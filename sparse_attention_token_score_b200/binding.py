@@ -47,6 +47,8 @@ _SIGS = {
     "indexer_score_topk": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "indexer_score_topk_noalloc": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P]),
     "dsa_noalloc_status": (ctypes.c_int, [_P]),
+    "indexer_lists_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int]),
+    "indexer_score_topk_lists": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "indexer_scores": (ctypes.c_int, [_P, _P, ctypes.c_longlong, _P, ctypes.c_size_t, _P]),
     "indexer_score_gathered": (ctypes.c_int, [_P, _P, ctypes.c_int, ctypes.c_int, _P,
                                               ctypes.c_longlong, _P, ctypes.c_size_t, _P]),
@@ -63,6 +65,8 @@ _SIGS = {
     "hisa_refine_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int, ctypes.c_int]),
     "hisa_refine_scores": (ctypes.c_int, [_P, _P, ctypes.c_int, ctypes.c_int, _P, ctypes.c_longlong, _P,
                                           ctypes.c_size_t, _P]),
+    "dosa_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int, ctypes.c_int]),
+    "dosa_score_topk": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "dsa_profile_begin": (ctypes.c_int, []),
     "dsa_profile_end": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_size_t, _P, ctypes.c_int]),
     "indexcache_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int, ctypes.c_char_p, ctypes.c_int]),
@@ -165,6 +169,17 @@ def indexer_score_topk_noalloc(args: IndexerArgs, topk: int, out_idx: torch.Tens
                                             _ptr(out_score), _stream_ptr(stream)))
 
 
+def indexer_lists_workspace_size(args: IndexerArgs, topk: int) -> int:
+    return int(lib().indexer_lists_workspace_size(ctypes.byref(args), topk))
+
+
+def indexer_score_topk_lists(args: IndexerArgs, topk: int, out_idx: torch.Tensor,
+                             out_score: Optional[torch.Tensor], workspace: torch.Tensor, stream=None):
+    _check("indexer_score_topk_lists",
+           lib().indexer_score_topk_lists(ctypes.byref(args), topk, _ptr(out_idx), _ptr(out_score),
+                                          _ptr(workspace), workspace.numel(), _stream_ptr(stream)))
+
+
 def dsa_noalloc_status(stream=None) -> int:
     """Status word of the static scratch of indexer_score_topk_noalloc (0 = ok)."""
     return int(lib().dsa_noalloc_status(_stream_ptr(stream)))
@@ -236,6 +251,18 @@ def hisa_refine_scores(args: IndexerArgs, blocks: torch.Tensor, m: int, blk: int
     _check("hisa_refine_scores",
            lib().hisa_refine_scores(ctypes.byref(args), _ptr(blocks), m, blk, _ptr(out), ld, _ptr(workspace),
                                     workspace.numel(), _stream_ptr(stream)))
+
+
+def dosa_workspace_size(args: IndexerArgs, topk: int, n_screen: int) -> int:
+    return int(lib().dosa_workspace_size(ctypes.byref(args), topk, n_screen))
+
+
+def dosa_score_topk(args: IndexerArgs, topk: int, n_screen: int, out_idx: torch.Tensor,
+                    out_score: Optional[torch.Tensor], out_live: Optional[torch.Tensor], workspace: torch.Tensor,
+                    stream=None):
+    _check("dosa_score_topk",
+           lib().dosa_score_topk(ctypes.byref(args), topk, n_screen, _ptr(out_idx), _ptr(out_score), _ptr(out_live),
+                                 _ptr(workspace), workspace.numel(), _stream_ptr(stream)))
 
 
 def dsa_profile_begin():

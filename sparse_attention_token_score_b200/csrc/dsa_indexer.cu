@@ -15,6 +15,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "dosa.cuh"
 #include "misc.cuh"
 #include "score_inv.cuh"
 #include "score_tc.cuh"
@@ -115,7 +116,10 @@ thread_local std::string stage;  // nested stages joined by '/'
 
 struct Stage {  // names the launches made while it lives ("routed", "sample pass", ...)
   size_t prev;
-  explicit Stage(const char* s) : prev(stage.size()) {
+  explicit Stage(const char* s) : prev(stage.size()) { set(s); }
+  // replaces this stage's name (the steps of one chain, one after another)
+  void set(const char* s) {
+    stage.resize(prev);
     if (!stage.empty()) stage += '/';
     stage += s;
   }
@@ -163,30 +167,47 @@ dsa_status launch_score(const ScoreParams& p, const void* q, long long q_rows, c
     if (G < grid) grid = static_cast<int>(G);
   }
   prof::Launch pl(st, C::ROUTER ? "score_tc router" : C::GATHER ? "score_tc gathered"
-                     : C::CMP ? (C::ELEM == 1 ? "score_tc fp8 + candidate lists" : "score_tc + candidate lists")
+                     : C::CMP ? "score_tc + candidate lists" : C::BND ? "score_tc bounds"
                      : (C::ELEM == 1 ? "score_tc fp8" : "score_tc"));
   score_tc_kernel<C><<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(tq, tk, p);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 // Dense / routed / block scoring, bf16: N = 256 columns = (256 / H) queries x H heads.
-// cmp: the epilogue also appends scores >= the row threshold to candidate
-// lists (p.cthr ... p.ccap); k_stride: key rows every k_stride elements.
+// epi: kEpiStore (full scores), kEpiCand (candidate lists: p.cthr ...
+// p.ccap), kEpiBound (DoSA live tiles: p.knorm ... p.live_gpb; H = 8 or 16
+// augmented heads); k_stride: key rows every k_stride elements; p.pairs set:
+// only the listed (group, tile) pairs (work-list instantiations).
 dsa_status run_scores_bf16(int D, int H, const ScoreParams& p, const void* q, long long q_rows,
-                           const void* k, long long k_rows, cudaStream_t st, bool cmp = false,
+                           const void* k, long long k_rows, cudaStream_t st, int epi = kEpiStore,
                            long long k_stride = 0) {
 #ifndef DSA_EPIW
 #define DSA_EPIW 8
 #endif
-#define DSA_CASE(DD, HH)                                                                            \
-  if (D == DD && H == HH)                                                                           \
-    return cmp ? launch_score<ScoreCfg<2, DD, HH, 256 / HH, ScoreMode::kTma, (DD == 128 ? 4 : 8),   \
-                                       DSA_EPIW, 1, true>>(p, q, q_rows, k, k_rows, st, k_stride)   \
-               : launch_score<ScoreCfg<2, DD, HH, 256 / HH, ScoreMode::kTma, (DD == 128 ? 4 : 8),   \
-                                       DSA_EPIW>>(p, q, q_rows, k, k_rows, st, k_stride);
+  const bool list = p.pairs != nullptr;
+#define DSA_CFG(DD, HH, EE, LL) \
+  ScoreCfg<2, DD, HH, 256 / HH, ScoreMode::kTma, (DD == 128 ? 4 : 8), DSA_EPIW, 1, EE, LL>
+#define DSA_LAUNCH(DD, HH, EE, LL) return launch_score<DSA_CFG(DD, HH, EE, LL)>(p, q, q_rows, k, k_rows, st, k_stride);
+#define DSA_CASE(DD, HH)                                            \
+  if (D == DD && H == HH) {                                         \
+    if (epi == kEpiCand) {                                          \
+      if (list && HH >= 16) { DSA_LAUNCH(DD, HH, kEpiCand, true) }  \
+      if (!list) { DSA_LAUNCH(DD, HH, kEpiCand, false) }            \
+      return DSA_ERR_UNSUPPORTED;                                   \
+    }                                                               \
+    if (list) { DSA_LAUNCH(DD, HH, kEpiStore, true) }               \
+    DSA_LAUNCH(DD, HH, kEpiStore, false)                            \
+  }
+#define DSA_CASE_B(DD, HH) \
+  if (D == DD && H == HH && epi == kEpiBound && !list) { DSA_LAUNCH(DD, HH, kEpiBound, false) }
+  DSA_CASE_B(64, 8) DSA_CASE_B(64, 16) DSA_CASE_B(128, 8) DSA_CASE_B(128, 16)
+  if (epi == kEpiBound) return DSA_ERR_UNSUPPORTED;
   DSA_CASE(64, 8) DSA_CASE(64, 16) DSA_CASE(64, 32) DSA_CASE(64, 64)
   DSA_CASE(128, 8) DSA_CASE(128, 16) DSA_CASE(128, 32) DSA_CASE(128, 64)
 #undef DSA_CASE
+#undef DSA_CASE_B
+#undef DSA_LAUNCH
+#undef DSA_CFG
   return DSA_ERR_UNSUPPORTED;
 }
 
@@ -271,6 +292,9 @@ dsa_status launch_topk_cfg(const TopkParams& tp, cudaStream_t st) {
 // Rows up to 32768 scores use the short-row layout (4 CTAs of 256 threads per
 // SM); longer rows use 2 CTAs of 512 threads per SM when there are enough rows
 // to fill the GPU, else one 512-thread CTA (with more loads in flight) per row.
+// (One CTA per SM for long rows, so fewer rows in flight stay in L2 between
+// the sampling read and the band pass, measured slower: 0.72 vs 0.59 ms on
+// the MISA-dagger k' selection.)
 dsa_status launch_topk(void* ws, TopkParams tp, cudaStream_t st) {
   tp.err = static_cast<unsigned*>(ws);
   if (tp.Lrow <= TkShort::MAX_ROW) return launch_topk_cfg<TkShort>(tp, st);
@@ -288,21 +312,35 @@ struct InvWs {
   int* ioff;
   long long* total;
   int2* list;
+  int* it_tile;
+  int4* it_row;
+  int4* it_slot;
 };
 
-size_t inv_ws_bytes(long long rows, int m, long long nb) {
-  return 4 * al256(static_cast<size_t>(nb + 1) * sizeof(int)) + al256(sizeof(long long)) +
-         al256(static_cast<size_t>(rows) * m * sizeof(int2));
+// Items: at most tiles-per-block x (kept pairs / queries per item + blocks).
+long long inv_max_items(long long rows, int m, long long nb, int blk, int H) {
+  return static_cast<long long>(blk / 128) * (rows * m / (128 / H) + nb + 1);
 }
 
-InvWs inv_carve(Carve& c, long long rows, int m, long long nb) {
+size_t inv_ws_bytes(long long rows, int m, long long nb, int blk, int H) {
+  const size_t items = static_cast<size_t>(inv_max_items(rows, m, nb, blk, H));
+  return 4 * al256(static_cast<size_t>(nb + 1) * sizeof(int)) + al256(sizeof(long long)) +
+         al256(static_cast<size_t>(rows) * m * sizeof(int2)) + al256(items * sizeof(int)) +
+         2 * al256(items * sizeof(int4));
+}
+
+InvWs inv_carve(Carve& c, long long rows, int m, long long nb, int blk, int H) {
   InvWs w;
+  const size_t items = static_cast<size_t>(inv_max_items(rows, m, nb, blk, H));
   w.cnt = c.take<int>(nb + 1);
   w.cursor = c.take<int>(nb + 1);
   w.qoff = c.take<int>(nb + 1);
   w.ioff = c.take<int>(nb + 1);
   w.total = c.take<long long>(1);
   w.list = c.take<int2>(static_cast<size_t>(rows) * m);
+  w.it_tile = c.take<int>(items);
+  w.it_row = c.take<int4>(items);
+  w.it_slot = c.take<int4>(items);
   return w;
 }
 
@@ -359,6 +397,12 @@ dsa_status run_refine_inverted(const dsa_indexer_args* a, const int32_t* blocks,
     prof::Launch pl(st, "invert_fill");
     invert_fill_kernel<<<grid, 256, 0, st>>>(blocks, rows, m, a->T, static_cast<int>(M), w.qoff, w.cursor, w.list);
   }
+  {
+    prof::Launch pl(st, "invert_items");
+    invert_items_kernel<<<static_cast<int>((nb + 7) / 8), 256, 0, st>>>(w.cnt, w.qoff, w.ioff, w.list,
+                                                                       static_cast<int>(nb), blk / 128, 128 / a->H,
+                                                                       w.it_tile, w.it_row, w.it_slot);
+  }
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   InvParams p{};
   p.batch = a->batch;
@@ -371,10 +415,9 @@ dsa_status run_refine_inverted(const dsa_indexer_args* a, const int32_t* blocks,
   p.w = a->w;
   p.out = out;
   p.ldo = ldo;
-  p.cnt = w.cnt;
-  p.qoff = w.qoff;
-  p.ioff = w.ioff;
-  p.list = w.list;
+  p.it_tile = w.it_tile;
+  p.it_row = w.it_row;
+  p.it_slot = w.it_slot;
   p.err = err;
   const long long q_rows = rows * a->H;
   const long long k_rows = static_cast<long long>(a->batch) * a->L;
@@ -497,12 +540,32 @@ FusedPlan fused_plan(int L, int topk, bool bf16, int heads) {
 }
 
 long long fused_groups(long long batch, int T, const FusedPlan& f) { return batch * ((T + f.qpt - 1) / f.qpt); }
+// Pair lists of the score kernel's work-list mode: flags [groups, ntiles],
+// the list and its length.
+size_t pairs_ws_bytes(long long groups, int ntiles) {
+  return al256(static_cast<size_t>(groups) * ntiles) + al256(static_cast<size_t>(groups) * ntiles * sizeof(int2)) +
+         al256(sizeof(int));
+}
 
 size_t fused_ws_bytes(long long batch, int T, const FusedPlan& f) {
   if (!f.on) return 0;
   const size_t rows = static_cast<size_t>(batch) * T;
   return al256(rows * f.ns_max * sizeof(float)) + 3 * al256(rows * 4) + 2 * al256(rows * f.cap * 4) +
-         al256(static_cast<size_t>(fused_groups(batch, T, f)) * f.ntiles);
+         pairs_ws_bytes(fused_groups(batch, T, f), f.ntiles);
+}
+
+struct PairWs {
+  uint8_t* flags;  // [groups, ntiles]
+  int2* list;      // [groups * ntiles]
+  int* n;
+};
+
+PairWs pairs_carve(Carve& c, long long groups, int ntiles) {
+  PairWs w;
+  w.flags = c.take<uint8_t>(static_cast<size_t>(groups) * ntiles);
+  w.list = c.take<int2>(static_cast<size_t>(groups) * ntiles);
+  w.n = c.take<int>(1);
+  return w;
 }
 
 struct FusedWs {
@@ -512,7 +575,7 @@ struct FusedWs {
   int* creal;
   float* cval;
   int* cidx;
-  uint8_t* fb;  // [groups, ntiles] tiles the fallback pass computes
+  PairWs fb;  // the fallback pass's tiles
 };
 
 FusedWs fused_carve(Carve& c, long long batch, int T, const FusedPlan& f) {
@@ -525,22 +588,52 @@ FusedWs fused_carve(Carve& c, long long batch, int T, const FusedPlan& f) {
   c.take<int>(rows);  // spare (keeps the two counters apart)
   w.cval = c.take<float>(static_cast<size_t>(rows) * f.cap);
   w.cidx = c.take<int>(static_cast<size_t>(rows) * f.cap);
-  w.fb = c.take<uint8_t>(static_cast<size_t>(fused_groups(batch, T, f)) * f.ntiles);
+  w.fb = pairs_carve(c, fused_groups(batch, T, f), f.ntiles);
   return w;
+}
+
+// Clear a pair workspace (stream-ordered).
+dsa_status pairs_clear(const PairWs& w, long long groups, int ntiles, cudaStream_t st) {
+  if (cudaMemsetAsync(w.flags, 0, static_cast<size_t>(groups) * ntiles, st) != cudaSuccess ||
+      cudaMemsetAsync(w.n, 0, sizeof(int), st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+// flags -> work list (pairs_build_kernel).
+dsa_status pairs_build(const PairWs& w, long long groups, int ntiles, int T, int qpt, long long q_offset, int L,
+                       cudaStream_t st) {
+  prof::Launch pl(st, "work list");
+  const int gpb = (T + qpt - 1) / qpt;
+  pairs_build_kernel<<<static_cast<int>((groups + 7) / 8), 256, 0, st>>>(w.flags, ntiles, static_cast<int>(groups), gpb,
+                                                                         T, qpt, q_offset, L, w.list, w.n);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 // Scores of every visible key with the Hh heads of q ([rows * Hh, D] bf16;
 // weights in base.w) and the top-k of every row through candidate lists;
 // scores [rows, L] receives full scores only for rows whose list fails the
 // check (and the winners' scores). base: batch, T, q_offset, w, err set.
+// DoSA pruning between the thresholds and the candidate pass: the bound pass
+// marks the key tiles each query group must score (live), the candidate pass
+// skips the others.
+struct Prune {
+  const void* q_aug;  // [rows, ha, D] bf16 augmented heads
+  const float* w_aug; // [rows, ha]
+  const float* cb;    // [rows] norm coefficient c_t
+  const float* kn;    // [batch * L] key norms
+  int ha;             // augmented heads (8 or 16)
+  PairWs live;        // tiles the bound pass keeps
+};
+
 dsa_status fused_score_topk(int D, int Hh, const ScoreParams& base, const void* q, const void* k, int L,
                             int topk, int32_t* out_idx, float* out_score, float* scores, const FusedPlan& f,
-                            const FusedWs& w, void* ws, cudaStream_t st) {
+                            const FusedWs& w, void* ws, cudaStream_t st, const Prune* prune = nullptr) {
   const long long rows = static_cast<long long>(base.batch) * base.T;
   const long long groups = fused_groups(base.batch, base.T, f);
-  if (cudaMemsetAsync(w.cres, 0, 2 * al256(static_cast<size_t>(rows) * 4), st) != cudaSuccess ||
-      cudaMemsetAsync(w.fb, 0, static_cast<size_t>(groups) * f.ntiles, st) != cudaSuccess)
-    return DSA_ERR_CUDA;
+  if (cudaMemsetAsync(w.cres, 0, 2 * al256(static_cast<size_t>(rows) * 4), st) != cudaSuccess) return DSA_ERR_CUDA;
+  DSA_TRY(pairs_clear(w.fb, groups, f.ntiles, st));
+  if (prune) DSA_TRY(pairs_clear(prune->live, groups, f.ntiles, st));
   // 1. sample pass: keys 0, S, 2S, ... (a strided view of the key rows)
   {
     prof::Stage sample_stage("sample pass");
@@ -549,7 +642,7 @@ dsa_status fused_score_topk(int D, int Hh, const ScoreParams& base, const void* 
     ps.pstride = f.S;
     ps.out = w.samp;
     ps.ldo = f.ns_max;
-    DSA_TRY(run_scores_bf16(D, Hh, ps, q, rows * Hh, k, static_cast<long long>(base.batch) * f.ns_max, st, false,
+    DSA_TRY(run_scores_bf16(D, Hh, ps, q, rows * Hh, k, static_cast<long long>(base.batch) * f.ns_max, st, kEpiStore,
                             static_cast<long long>(f.S) * D));
   }
   // 2. thresholds
@@ -560,8 +653,31 @@ dsa_status fused_score_topk(int D, int Hh, const ScoreParams& base, const void* 
                                                        L, topk, w.thr);
   }
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  // 2b. DoSA: bounds over the augmented heads -> live key tiles
+  if (prune) {
+    prof::Stage bound_stage("bounds");
+    ScoreParams pb = base;
+    pb.Lk = L;
+    pb.pstride = 1;
+    pb.out = nullptr;
+    pb.w = prune->w_aug;
+    pb.cthr = w.thr;
+    pb.cbound = prune->cb;
+    pb.knorm = prune->kn;
+    pb.live_out = prune->live.flags;
+    pb.live_ld = f.ntiles;
+    pb.live_qpt = f.qpt;
+    pb.live_gpb = (base.T + f.qpt - 1) / f.qpt;
+    DSA_TRY(run_scores_bf16(D, prune->ha, pb, prune->q_aug, rows * prune->ha, k, static_cast<long long>(base.batch) * L,
+                            st, kEpiBound));
+    DSA_TRY(pairs_build(prune->live, groups, f.ntiles, base.T, f.qpt, base.q_offset, L, st));
+  }
   // 3. candidate lists (no full scores)
   ScoreParams pm = base;
+  if (prune) {
+    pm.pairs = prune->live.list;
+    pm.pairs_n = prune->live.n;
+  }
   pm.Lk = L;
   pm.pstride = 1;
   pm.out = nullptr;
@@ -571,14 +687,15 @@ dsa_status fused_score_topk(int D, int Hh, const ScoreParams& base, const void* 
   pm.cres = w.cres;
   pm.creal = w.creal;
   pm.ccap = f.cap;
-  DSA_TRY(run_scores_bf16(D, Hh, pm, q, rows * Hh, k, static_cast<long long>(base.batch) * L, st, true));
+  DSA_TRY(run_scores_bf16(D, Hh, pm, q, rows * Hh, k, static_cast<long long>(base.batch) * L, st, kEpiCand));
   // 4. rows whose list is short (or overflowed): full scores of their groups
   {
     prof::Launch pl(st, "list check");
     fused_check_kernel<<<static_cast<int>((rows + 255) / 256), 256, 0, st>>>(
-        w.cres, w.creal, rows, base.T, base.q_offset, L, topk, f.cap, f.qpt, f.ntiles, w.fb);
+        w.cres, w.creal, rows, base.T, base.q_offset, L, topk, f.cap, f.qpt, f.ntiles, w.fb.flags);
   }
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  DSA_TRY(pairs_build(w.fb, groups, f.ntiles, base.T, f.qpt, base.q_offset, L, st));
   {
     prof::Stage fb_stage("fallback");
     ScoreParams pf = base;
@@ -586,8 +703,8 @@ dsa_status fused_score_topk(int D, int Hh, const ScoreParams& base, const void* 
     pf.pstride = 1;
     pf.out = scores;
     pf.ldo = L;
-    pf.tile_live = w.fb;
-    pf.live_ld = f.ntiles;
+    pf.pairs = w.fb.list;
+    pf.pairs_n = w.fb.n;
     DSA_TRY(run_scores_bf16(D, Hh, pf, q, rows * Hh, k, static_cast<long long>(base.batch) * L, st));
   }
   // 5. top-k from the lists (from the full scores where a list failed)
@@ -640,10 +757,9 @@ dsa_status dsa_selftest_wait_timeout(void* workspace, size_t ws_bytes, void* str
 }
 
 size_t indexer_workspace_size(const dsa_indexer_args* a, int topk) {
+  (void)topk;
   if (!a || a->batch < 1 || a->T < 1 || a->L < 1) return 0;
-  const size_t rows = static_cast<size_t>(a->batch) * a->T;
-  return kHdr + al256(rows * a->L * sizeof(float)) +
-         fused_ws_bytes(a->batch, a->T, fused_plan(a->L, topk, a->qk_dtype == DSA_BF16, a->H));
+  return kHdr + al256(static_cast<size_t>(a->batch) * a->T * a->L * sizeof(float));
 }
 
 dsa_status indexer_scores(const dsa_indexer_args* a, float* out, long long ld, void* ws,
@@ -702,28 +818,22 @@ dsa_status indexer_topk_rows(const float* scores, long long rows, long long ld, 
                      st);
 }
 
-// The dense score + top-k; `fused` picks the candidate-list chain where it
-// applies (fused_plan), otherwise full scores then the row top-k.
-static dsa_status dense_score_topk(const dsa_indexer_args* a, int topk, int32_t* out_idx, float* out_score,
-                                   void* ws, size_t ws_bytes, void* stream, bool fused) {
+// The dense score + top-k: full scores, then the row top-k.
+dsa_status indexer_score_topk(const dsa_indexer_args* a, int topk, int32_t* out_idx, float* out_score, void* ws,
+                              size_t ws_bytes, void* stream) {
   DSA_TRY(validate(a, false));
   if (!out_idx || topk < 1 || topk > (1 << 24)) return DSA_ERR_ARG;
-  const size_t rows = static_cast<size_t>(a->batch) * a->T;
-  const FusedPlan f = fused ? fused_plan(a->L, topk, a->qk_dtype == DSA_BF16, a->H) : FusedPlan{};
-  DSA_TRY(check_ws(ws, ws_bytes, kHdr + al256(rows * a->L * sizeof(float)) + fused_ws_bytes(a->batch, a->T, f)));
+  DSA_TRY(check_ws(ws, ws_bytes, indexer_workspace_size(a, topk)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DSA_TRY(clear_status(ws, st));
   Carve c{static_cast<char*>(ws), kHdr};
+  const size_t rows = static_cast<size_t>(a->batch) * a->T;
   float* scores = c.take<float>(rows * a->L);
   ScoreParams p = base_params(a, static_cast<unsigned*>(ws));
-  const long long q_rows = static_cast<long long>(a->batch) * a->T * a->H;
-  const long long k_rows = static_cast<long long>(a->batch) * a->L;
-  if (f.on) {
-    const FusedWs w = fused_carve(c, a->batch, a->T, f);
-    return fused_score_topk(a->d, a->H, p, a->q, a->k, a->L, topk, out_idx, out_score, scores, f, w, ws, st);
-  }
   p.out = scores;
   p.ldo = a->L;
+  const long long q_rows = static_cast<long long>(a->batch) * a->T * a->H;
+  const long long k_rows = static_cast<long long>(a->batch) * a->L;
   if (a->qk_dtype == DSA_FP8_E4M3)
     DSA_TRY(run_scores_fp8(a->d, a->H, p, a->q, q_rows, a->k, k_rows, st));
   else
@@ -733,9 +843,29 @@ static dsa_status dense_score_topk(const dsa_indexer_args* a, int topk, int32_t*
                      st);
 }
 
-dsa_status indexer_score_topk(const dsa_indexer_args* a, int topk, int32_t* out_idx, float* out_score, void* ws,
-                              size_t ws_bytes, void* stream) {
-  return dense_score_topk(a, topk, out_idx, out_score, ws, ws_bytes, stream, true);
+// The dense selection through candidate lists (fused_score_topk).
+size_t indexer_lists_workspace_size(const dsa_indexer_args* a, int topk) {
+  if (!a || a->batch < 1 || a->T < 1 || a->L < 1) return 0;
+  const FusedPlan f = fused_plan(a->L, topk, a->qk_dtype == DSA_BF16, a->H);
+  if (!f.on) return 0;
+  return kHdr + al256(static_cast<size_t>(a->batch) * a->T * a->L * sizeof(float)) +
+         fused_ws_bytes(a->batch, a->T, f);
+}
+
+dsa_status indexer_score_topk_lists(const dsa_indexer_args* a, int topk, int32_t* out_idx, float* out_score,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  DSA_TRY(validate(a, true));
+  if (!out_idx || topk < 1 || topk > (1 << 24)) return DSA_ERR_ARG;
+  const FusedPlan f = fused_plan(a->L, topk, true, a->H);
+  if (!f.on) return DSA_ERR_UNSUPPORTED;
+  DSA_TRY(check_ws(ws, ws_bytes, indexer_lists_workspace_size(a, topk)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DSA_TRY(clear_status(ws, st));
+  Carve c{static_cast<char*>(ws), kHdr};
+  float* scores = c.take<float>(static_cast<size_t>(a->batch) * a->T * a->L);
+  const FusedWs w = fused_carve(c, a->batch, a->T, f);
+  const ScoreParams p = base_params(a, static_cast<unsigned*>(ws));
+  return fused_score_topk(a->d, a->H, p, a->q, a->k, a->L, topk, out_idx, out_score, scores, f, w, ws, st);
 }
 
 dsa_status dsa_meanpool_keys(const void* k, int batch, int L, int d, int block, void* kbar,
@@ -764,7 +894,6 @@ size_t misa_workspace_size(const dsa_indexer_args* a, int block, int h, int topk
   n += al256(BT * h * sizeof(float));             // their weights
   n += al256(BT * h * sizeof(int32_t));           // kept heads
   n += al256(BT * a->L * sizeof(float));          // routed scores
-  n += fused_ws_bytes(a->batch, a->T, fused_plan(a->L, kprime > 0 ? kprime : topk, true, h));
   if (kprime > 0) {
     n += al256(BT * kprime * sizeof(int32_t));    // candidates
     n += al256(BT * kprime * sizeof(float));      // full-H candidate scores
@@ -797,13 +926,11 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   int32_t* heads_ws = c.take<int32_t>(static_cast<size_t>(BT) * h);
   float* routed = c.take<float>(static_cast<size_t>(BT) * a->L);
   int32_t* heads = out_heads ? out_heads : heads_ws;
-  const FusedPlan fp = fused_plan(a->L, kprime > 0 ? kprime : topk, true, h);
-  const FusedWs fw = fp.on ? fused_carve(c, a->batch, a->T, fp) : FusedWs{};
 
   // 1. pooled keys
   DSA_TRY(dsa_meanpool_keys(a->k, a->batch, a->L, a->d, block, kbar, stream));
   // 2. router affinities (partial ReLU sums over visible pooled keys)
-  prof::Stage route_stage("router");
+  prof::Stage misa_stage("router");
   ScoreParams pr = base_params(a, err);
   pr.Lk = static_cast<int>(M);
   pr.pstride = block;
@@ -818,7 +945,7 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   // 4. routed token scores with the kept heads only, and their top-k (or
   // top-k' candidates), through candidate lists where that applies
-  prof::Stage routed_stage("routed");
+  misa_stage.set("routed");
   ScoreParams ps = base_params(a, err);
   ps.w = w_sel;
   ps.out = routed;
@@ -834,17 +961,13 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   const int ksel = kprime > 0 ? kprime : topk;
   int32_t* sel = kprime > 0 ? cand : out_idx;
   float* sel_score = kprime > 0 ? nullptr : out_score;
-  if (fp.on) {
-    DSA_TRY(fused_score_topk(a->d, h, ps, q_sel, a->k, a->L, ksel, sel, sel_score, routed, fp, fw, ws, st));
-  } else {
-    DSA_TRY(run_scores_bf16(a->d, h, ps, q_sel, BT * h, a->k, k_rows, st));
-    DSA_TRY(launch_topk(ws, topk_params(routed, BT, a->L, a->T, a->q_offset, 1, a->L, ksel, sel, sel_score,
-                                    nullptr, 0, 1),
-                        st));
-  }
+  DSA_TRY(run_scores_bf16(a->d, h, ps, q_sel, BT * h, a->k, k_rows, st));
+  DSA_TRY(launch_topk(ws, topk_params(routed, BT, a->L, a->T, a->q_offset, 1, a->L, ksel, sel, sel_score, nullptr,
+                                  0, 1),
+                      st));
   if (kprime == 0) return DSA_OK;
   // 5. MISA-dagger: full-H re-score of the k' candidates, top-k
-  prof::Stage rescore_stage("re-score");
+  misa_stage.set("re-score");
   ScoreParams pg = base_params(a, err);
   pg.out = compact;
   pg.ldo = kprime;
@@ -869,13 +992,15 @@ size_t hisa_workspace_size(const dsa_indexer_args* a, int block, int m, int topk
   n += al256(BT * M * sizeof(float));                         // block scores
   n += al256(BT * m * sizeof(int32_t));                       // kept blocks
   n += al256(BT * static_cast<size_t>(m) * block * sizeof(float));  // token scores of kept blocks
-  if (inv_supported(a, block)) n += inv_ws_bytes(static_cast<long long>(BT), m, a->batch * static_cast<long long>(M));
+  if (inv_supported(a, block))
+    n += inv_ws_bytes(static_cast<long long>(BT), m, a->batch * static_cast<long long>(M), block, a->H);
   return n;
 }
 
 size_t hisa_refine_workspace_size(const dsa_indexer_args* a, int m, int blk) {
   if (!a || a->batch < 1 || a->T < 1 || a->L < 1 || m < 1 || blk < 1) return 0;
-  return kHdr + inv_ws_bytes(static_cast<long long>(a->batch) * a->T, m, a->batch * blocks_of(a->L, blk));
+  return kHdr + inv_ws_bytes(static_cast<long long>(a->batch) * a->T, m, a->batch * blocks_of(a->L, blk), blk,
+                             a->H > 0 ? a->H : 1);
 }
 
 dsa_status hisa_refine_scores(const dsa_indexer_args* a, const int32_t* blocks, int m, int blk, float* out,
@@ -891,7 +1016,7 @@ dsa_status hisa_refine_scores(const dsa_indexer_args* a, const int32_t* blocks, 
   DSA_TRY(clear_status(ws, st));
   Carve c{static_cast<char*>(ws), kHdr};
   const long long rows = static_cast<long long>(a->batch) * a->T;
-  const InvWs w = inv_carve(c, rows, m, a->batch * blocks_of(a->L, blk));
+  const InvWs w = inv_carve(c, rows, m, a->batch * blocks_of(a->L, blk), blk, a->H);
   return run_refine_inverted(a, blocks, m, blk, out, ld, w, static_cast<unsigned*>(ws), st);
 }
 
@@ -921,7 +1046,7 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   // 1. pooled keys
   DSA_TRY(dsa_meanpool_keys(a->k, a->batch, a->L, a->d, block, kbar, stream));
   // 2. block scores on the pooled keys (block m visible iff m * block <= p_t)
-  prof::Stage block_stage("blocks");
+  prof::Stage hisa_stage("blocks");
   ScoreParams pb = base_params(a, err);
   pb.Lk = static_cast<int>(M);
   pb.pstride = block;
@@ -932,12 +1057,12 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   DSA_TRY(launch_topk(ws, topk_params(bscore, BT, M, a->T, a->q_offset, block, static_cast<int>(M), m,
                                   blocks, nullptr, nullptr, 0, 1),
                       st));
-  prof::Stage token_stage("tokens");
+  hisa_stage.set("tokens");
   // 4. token scores inside the kept blocks (compact rows of m * block):
   // block-major over the inverted kept-block lists when blocks are whole key
   // tiles, else one query per tile with gathered rows
   if (inv_supported(a, block)) {
-    const InvWs w = inv_carve(c, BT, m, a->batch * M);
+    const InvWs w = inv_carve(c, BT, m, a->batch * M, block, a->H);
     DSA_TRY(run_refine_inverted(a, blocks, m, block, compact, ncomp, w, err, st));
     return launch_topk(ws, topk_params(compact, BT, ncomp, a->T, a->q_offset, 0, ncomp, topk, out_idx,
                                    out_score, blocks, m, block),
@@ -956,6 +1081,89 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   return launch_topk(ws, topk_params(compact, BT, ncomp, a->T, a->q_offset, 0, ncomp, topk, out_idx,
                                  out_score, blocks, m, block),
                      st);
+}
+
+// ------------------------------------------------------------ DoSA
+static int dosa_aug_heads(int n_screen) { return n_screen + 3 <= 8 ? 8 : 16; }
+
+static dsa_status dosa_check(const dsa_indexer_args* a, int topk, int n_screen, FusedPlan* f) {
+  DSA_TRY(validate(a, true));
+  if (topk < 1 || topk > (1 << 24) || n_screen < 0) return DSA_ERR_ARG;
+  if (n_screen + 3 > 16 || n_screen >= a->H || (a->H != 16 && a->H != 32 && a->H != 64)) return DSA_ERR_UNSUPPORTED;
+  *f = fused_plan(a->L, topk, true, a->H);
+  if (!f->on) return DSA_ERR_UNSUPPORTED;  // rows too short for sampled thresholds
+  return DSA_OK;
+}
+
+static size_t dosa_extra_bytes(const dsa_indexer_args* a, int n_screen, const FusedPlan& f) {
+  const size_t rows = static_cast<size_t>(a->batch) * a->T;
+  const int ha = dosa_aug_heads(n_screen);
+  return al256(rows * ha * a->d * 2) + al256(rows * ha * 4) + al256(rows * 4) +
+         al256(static_cast<size_t>(a->batch) * a->L * 4) + pairs_ws_bytes(fused_groups(a->batch, a->T, f), f.ntiles);
+}
+
+size_t dosa_workspace_size(const dsa_indexer_args* a, int topk, int n_screen) {
+  if (!a || a->batch < 1 || a->T < 1 || a->L < 1 || n_screen < 0) return 0;
+  FusedPlan f;
+  if (dosa_check(a, topk, n_screen, &f) == DSA_ERR_UNSUPPORTED || !f.on) return 0;
+  const size_t rows = static_cast<size_t>(a->batch) * a->T;
+  return kHdr + al256(rows * a->L * sizeof(float)) + fused_ws_bytes(a->batch, a->T, f) +
+         dosa_extra_bytes(a, n_screen, f);
+}
+
+dsa_status dosa_score_topk(const dsa_indexer_args* a, int topk, int n_screen, int32_t* out_idx, float* out_score,
+                           uint8_t* out_live, void* ws, size_t ws_bytes, void* stream) {
+  FusedPlan f;
+  DSA_TRY(dosa_check(a, topk, n_screen, &f));
+  if (!out_idx) return DSA_ERR_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes, dosa_workspace_size(a, topk, n_screen)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DSA_TRY(clear_status(ws, st));
+  const long long rows = static_cast<long long>(a->batch) * a->T;
+  const int ha = dosa_aug_heads(n_screen);
+  Carve c{static_cast<char*>(ws), kHdr};
+  float* scores = c.take<float>(static_cast<size_t>(rows) * a->L);
+  const FusedWs w = fused_carve(c, a->batch, a->T, f);
+  Prune pr;
+  __nv_bfloat16* q_aug = c.take<__nv_bfloat16>(static_cast<size_t>(rows) * ha * a->d);
+  float* w_aug = c.take<float>(static_cast<size_t>(rows) * ha);
+  float* cb = c.take<float>(rows);
+  float* kn = c.take<float>(static_cast<size_t>(a->batch) * a->L);
+  pr.live = pairs_carve(c, fused_groups(a->batch, a->T, f), f.ntiles);
+  pr.q_aug = q_aug;
+  pr.w_aug = w_aug;
+  pr.cb = cb;
+  pr.kn = kn;
+  pr.ha = ha;
+  const size_t live_bytes = static_cast<size_t>(fused_groups(a->batch, a->T, f)) * f.ntiles;
+  {
+    prof::Stage prep_stage("bounds");
+    {
+      prof::Launch pl(st, "dosa_prep");
+      const int grid = static_cast<int>((rows + 7) / 8);
+      if (a->d == 128)
+        dosa_prep_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a->q), a->w, rows, a->H,
+                                                    n_screen, ha, q_aug, w_aug, cb);
+      else
+        dosa_prep_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a->q), a->w, rows, a->H,
+                                                   n_screen, ha, q_aug, w_aug, cb);
+    }
+    {
+      prof::Launch pl(st, "key_norm");
+      const long long nk = static_cast<long long>(a->batch) * a->L;
+      const int grid = static_cast<int>(std::min<long long>((nk + 255) / 256, 8LL * num_sms()));
+      if (a->d == 128)
+        key_norm_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a->k), nk, kn);
+      else
+        key_norm_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a->k), nk, kn);
+    }
+    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  ScoreParams p = base_params(a, static_cast<unsigned*>(ws));
+  DSA_TRY(fused_score_topk(a->d, a->H, p, a->q, a->k, a->L, topk, out_idx, out_score, scores, f, w, ws, st, &pr));
+  if (out_live && cudaMemcpyAsync(out_live, pr.live.flags, live_bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
 }
 
 // ------------------------------------------------------------ launch profiling
@@ -1095,14 +1303,12 @@ extern "C" dsa_status indexer_score_topk_noalloc(const dsa_indexer_args* a, int 
                                                  void* stream) {
   DSA_TRY(validate(a, false));
   if (!out_idx || topk < 1 || topk > (1 << 24)) return DSA_ERR_ARG;
-  if (kHdr + al256(static_cast<size_t>(a->batch) * a->T * a->L * sizeof(float)) > kNoAllocScratchBytes)
-    return DSA_ERR_WORKSPACE;
+  if (indexer_workspace_size(a, topk) > kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   DSA_TRY(noalloc_scratch(&scratch));
-  // Full scores then the row top-k (the selection indexer_score_topk makes,
-  // without its candidate lists); the status word (first 4 bytes of the
-  // scratch) is cleared on the stream before the kernels run.
-  return dense_score_topk(a, topk, out_idx, out_score, scratch, kNoAllocScratchBytes, stream, false);
+  // Same launches as indexer_score_topk; its status word (first 4 bytes of
+  // the scratch) is cleared on the stream before the kernels run.
+  return indexer_score_topk(a, topk, out_idx, out_score, scratch, kNoAllocScratchBytes, stream);
 }
 
 // The status word of the static scratch: a bounded wait that gave up inside an

@@ -13,9 +13,9 @@
 // kept it; the queries (H * d * 2 bytes each) are what streams.
 //
 // Work items, in order: (block g, key tile u of the block, chunk c of QC of
-// its queries). Item counts per block are a prefix sum (ioff), so a CTA finds
-// its first item by binary search and walks on from there; all items cost
-// one MMA tile.
+// its queries), one record each (key tile, query rows, slots) built after the
+// inversion; a CTA takes a contiguous range of items and every role reads
+// their records 32 at a time; all items cost one MMA tile.
 //
 // One persistent CTA per SM, warp-specialised as the other score kernels:
 // one TMA producer warp (key tile into one of two stationary buffers, query
@@ -36,10 +36,9 @@ struct InvParams {
   const float* w;           // [batch*T, H]
   float* out;               // [batch*T, ldo] compact rows: position slot * blk + i
   long long ldo;
-  const int* cnt;           // [batch*M] queries that kept each block
-  const int* qoff;          // [batch*M + 1] start of each block's list
-  const int* ioff;          // [batch*M + 1] start of each block's items
-  const int2* list;         // [total kept] (row, slot), grouped by block
+  const int* it_tile;       // [items] key tile of item i: g * (blk / 128) + u (g = b * M + j)
+  const int4* it_row;       // [items] the item's query rows (-1 past its queries)
+  const int4* it_slot;      // [items] their slots in the compact rows
   unsigned* err;
 };
 
@@ -72,65 +71,83 @@ struct InvCfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-// Walks this CTA's items; every thread runs its own copy, all copies visit
-// the same sequence.
-template <class C>
-struct InvSched {
-  long long i, i1;     // current item, end of this CTA's range
-  int g;               // current block (global: b * M + j)
-  int loc;             // item index inside the block
-  int nq;              // queries of block g
-  int nch;             // chunks of block g
-  int u, ch;           // key tile inside the block, chunk
-  bool first, last, done;
+// A warp's walk over this CTA's items [i0, i1). Lane l holds the records of
+// items bbase + l (current batch) and bbase + 32 + l (next batch), loaded 32
+// at a time with coalesced loads, so per item only shuffles remain. All 32
+// lanes call cur() and advance() together.
+struct ItemWalk {
+  long long i, i0, i1, bbase;
+  int tile_c, tile_n;
+  int4 row_c, row_n, slot_c, slot_n;
+  int prev_tile;
+  // the current item (uniform over the warp after cur())
+  int tile;
+  int4 rows, slots;
+  bool first, last;
 
-  __device__ __forceinline__ void load_block(const InvParams& p) {
-    nq = __ldg(p.cnt + g);
-    nch = (nq + C::QC - 1) / C::QC;
+  __device__ __forceinline__ void load(const InvParams& p, long long base, int& t, int4& r, int4& sl,
+                                       bool with_slots) {
+    const long long idx = base + (threadIdx.x & 31);
+    t = -1;
+    r = make_int4(-1, -1, -1, -1);
+    sl = make_int4(0, 0, 0, 0);
+    if (idx < i1) {
+      t = __ldg(p.it_tile + idx);
+      r = __ldg(p.it_row + idx);
+      if (with_slots) sl = __ldg(p.it_slot + idx);
+    }
   }
-  __device__ __forceinline__ void set_pos(const InvParams& p) {
-    u = loc / nch;
-    ch = loc - u * nch;
-    // the key tile changes at the first chunk of every tile (and at this
-    // CTA's first item); it is released after its last chunk (or this CTA's
-    // last item)
-    last = (ch == nch - 1) || (i + 1 == i1);
-  }
-  __device__ __forceinline__ void init(const InvParams& p, long long total) {
+  __device__ __forceinline__ void init(const InvParams& p, long long total, bool with_slots) {
     const long long G = gridDim.x;
-    i = total * blockIdx.x / G;
+    i0 = i = total * blockIdx.x / G;
     i1 = total * (blockIdx.x + 1) / G;
-    done = i >= i1;
-    if (done) return;
-    // block with ioff[g] <= i < ioff[g + 1] (ioff is non-decreasing)
-    int lo = 0, hi = p.batch * p.M - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (__ldg(p.ioff + mid) <= i) lo = mid;
-      else hi = mid - 1;
-    }
-    g = lo;
-    loc = static_cast<int>(i - __ldg(p.ioff + g));
-    load_block(p);
-    set_pos(p);
-    first = true;
+    bbase = i0;
+    prev_tile = -1;
+    load(p, bbase, tile_c, row_c, slot_c, with_slots);
+    load(p, bbase + 32, tile_n, row_n, slot_n, with_slots);
   }
-  __device__ __forceinline__ void next(const InvParams& p) {
-    if (++i >= i1) { done = true; return; }
-    const int prev_u = u;
-    ++loc;
-    if (loc == (p.blk / 128) * nch) {
-      do { ++g; } while (__ldg(p.ioff + g + 1) == __ldg(p.ioff + g));
-      loc = 0;
-      load_block(p);
-      set_pos(p);
-      first = true;
-      return;
+  __device__ __forceinline__ void cur() {
+    const int l = static_cast<int>(i - bbase);
+    tile = __shfl_sync(0xffffffffu, tile_c, l);
+    rows.x = __shfl_sync(0xffffffffu, row_c.x, l);
+    rows.y = __shfl_sync(0xffffffffu, row_c.y, l);
+    rows.z = __shfl_sync(0xffffffffu, row_c.z, l);
+    rows.w = __shfl_sync(0xffffffffu, row_c.w, l);
+    slots.x = __shfl_sync(0xffffffffu, slot_c.x, l);
+    slots.y = __shfl_sync(0xffffffffu, slot_c.y, l);
+    slots.z = __shfl_sync(0xffffffffu, slot_c.z, l);
+    slots.w = __shfl_sync(0xffffffffu, slot_c.w, l);
+    const int nl = __shfl_sync(0xffffffffu, l + 1 < 32 ? tile_c : tile_n, (l + 1) & 31);
+    first = i == i0 || prev_tile != tile;
+    last = nl != tile;  // -1 past the range
+  }
+  // query rows of item i + ahead (1 <= ahead <= 32); -1s past the range
+  __device__ __forceinline__ int4 peek_rows(int ahead) const {
+    const int l2 = static_cast<int>(i - bbase) + ahead;
+    const bool in_c = l2 < 32;
+    int4 v;
+    v.x = __shfl_sync(0xffffffffu, in_c ? row_c.x : row_n.x, l2 & 31);
+    v.y = __shfl_sync(0xffffffffu, in_c ? row_c.y : row_n.y, l2 & 31);
+    v.z = __shfl_sync(0xffffffffu, in_c ? row_c.z : row_n.z, l2 & 31);
+    v.w = __shfl_sync(0xffffffffu, in_c ? row_c.w : row_n.w, l2 & 31);
+    if (i + ahead >= i1) v = make_int4(-1, -1, -1, -1);
+    return v;
+  }
+  __device__ __forceinline__ void advance(const InvParams& p, bool with_slots) {
+    prev_tile = tile;
+    if (++i - bbase == 32) {
+      bbase += 32;
+      tile_c = tile_n;
+      row_c = row_n;
+      slot_c = slot_n;
+      load(p, bbase + 32, tile_n, row_n, slot_n, with_slots);
     }
-    set_pos(p);
-    first = (u != prev_u);
   }
 };
+
+__device__ __forceinline__ int item_row(const int4& r, int i) {
+  return i == 0 ? r.x : i == 1 ? r.y : i == 2 ? r.z : r.w;
+}
 
 template <class C>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
@@ -185,79 +202,98 @@ score_inv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  InvSched<C> s;
-  s.init(p, *total_items);
+  const long long total = *total_items;
+  ItemWalk s;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    s.init(p, total, false);
     uint32_t it = 0, gk = 0;
     bool ok = true;
-    if (lane == 0) {
-      for (; !s.done; s.next(p), ++it) {
-        const int b = s.g / p.M;
-        const int j = s.g - b * p.M;
+    for (; s.i < s.i1; s.advance(p, false), ++it) {
+      s.cur();
+      if (lane == 0) {
         if (s.first) {
           const int kb_ = static_cast<int>(gk % C::NKBUF);
-          if (!mbar_wait(kempty(kb_), ((gk / C::NKBUF) & 1u) ^ 1u, p.err)) { ok = false; break; }
-          mbar_arrive_expect_tx(kfull(kb_), C::K_BYTES);
-          const int row0 = b * p.L + j * p.blk + s.u * 128;
+          if (!mbar_wait(kempty(kb_), ((gk / C::NKBUF) & 1u) ^ 1u, p.err)) {
+            ok = false;
+          } else {
+            const int U = p.blk / 128;
+            const int g = s.tile / U;
+            const int b = g / p.M;
+            const int row0 = b * p.L + (g - b * p.M) * p.blk + (s.tile - g * U) * 128;
+            mbar_arrive_expect_tx(kfull(kb_), C::K_BYTES);
 #pragma unroll
-          for (int cb = 0; cb < C::KBLK; ++cb)
-            tma_load_2d(s_k + kb_ * C::K_BYTES + cb * C::KROWS * 128, &tm_k, kfull(kb_), cb * 64, row0);
-          ++gk;
+            for (int cb = 0; cb < C::KBLK; ++cb)
+              tma_load_2d(s_k + kb_ * C::K_BYTES + cb * C::KROWS * 128, &tm_k, kfull(kb_), cb * 64, row0);
+            ++gk;
+          }
         }
         const int stage = static_cast<int>(it % C::NSTAGE);
-        if (!mbar_wait(empty(stage), ((it / C::NSTAGE) & 1u) ^ 1u, p.err)) { ok = false; break; }
-        const int q0 = __ldg(p.qoff + s.g) + s.ch * C::QC;
-        const int nq = min(C::QC, s.nq - s.ch * C::QC);
-        mbar_arrive_expect_tx(full(stage), static_cast<uint32_t>(nq * C::H * C::ROW_BYTES));
-        for (int i = 0; i < nq; ++i) {
-          const int r = __ldg(&p.list[q0 + i].x);
+        if (ok && !mbar_wait(empty(stage), ((it / C::NSTAGE) & 1u) ^ 1u, p.err)) ok = false;
+        if (ok) {
+          int nq = 0;
 #pragma unroll
-          for (int cb = 0; cb < C::KBLK; ++cb)
-            tma_load_2d(s_q + stage * C::Q_BYTES + cb * C::NROWS * 128 + i * C::H * 128, &tm_q, full(stage),
-                        cb * 64, r * C::H);
+          for (int i = 0; i < C::QC; ++i) nq += item_row(s.rows, i) >= 0;
+          mbar_arrive_expect_tx(full(stage), static_cast<uint32_t>(nq * C::H * C::ROW_BYTES));
+#pragma unroll
+          for (int i = 0; i < C::QC; ++i) {
+            const int r = item_row(s.rows, i);
+            if (r < 0) continue;
+#pragma unroll
+            for (int cb = 0; cb < C::KBLK; ++cb)
+              tma_load_2d(s_q + stage * C::Q_BYTES + cb * C::NROWS * 128 + i * C::H * 128, &tm_q, full(stage),
+                          cb * 64, r * C::H);
+          }
         }
       }
-      if (!ok) {
-        // error path: the loads already issued land before shared memory is released
-        for (uint32_t g2 = gk > C::NKBUF ? gk - C::NKBUF : 0; g2 < gk; ++g2)
-          mbar_drain(kfull(static_cast<int>(g2 % C::NKBUF)), (g2 / C::NKBUF) & 1u);
-        const uint32_t lo = it > C::NSTAGE ? it - C::NSTAGE : 0;
-        for (uint32_t i = lo; i < it; ++i) mbar_drain(full(i % C::NSTAGE), (i / C::NSTAGE) & 1u);
-      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+    }
+    if (!ok && lane == 0) {
+      // error path: the loads already issued land before shared memory is released
+      for (uint32_t g2 = gk > C::NKBUF ? gk - C::NKBUF : 0; g2 < gk; ++g2)
+        mbar_drain(kfull(static_cast<int>(g2 % C::NKBUF)), (g2 / C::NKBUF) & 1u);
+      const uint32_t lo = it > C::NSTAGE ? it - C::NSTAGE : 0;
+      for (uint32_t i = lo; i < it; ++i) mbar_drain(full(i % C::NSTAGE), (i / C::NSTAGE) & 1u);
     }
     __syncwarp();
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t it = 0, gk = 0;
-      bool ok = true;
-      for (; !s.done; s.next(p), ++it) {
+    s.init(p, total, false);
+    uint32_t it = 0, gk = 0;
+    bool ok = true;
+    for (; s.i < s.i1; s.advance(p, false), ++it) {
+      s.cur();
+      if (lane == 0) {
         const int kb_ = static_cast<int>(gk % C::NKBUF);
-        if (s.first && !mbar_wait(kfull(kb_), (gk / C::NKBUF) & 1u, p.err)) { ok = false; break; }
         const int stage = static_cast<int>(it % C::NSTAGE);
         const int buf = static_cast<int>(it % C::NACC);
-        if (!mbar_wait(tempty(buf), ((it / C::NACC) & 1u) ^ 1u, p.err)) { ok = false; break; }
-        if (!mbar_wait(full(stage), (it / C::NSTAGE) & 1u, p.err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::NROWS);
+        if (s.first && !mbar_wait(kfull(kb_), (gk / C::NKBUF) & 1u, p.err)) ok = false;
+        if (ok && !mbar_wait(tempty(buf), ((it / C::NACC) & 1u) ^ 1u, p.err)) ok = false;
+        if (ok && !mbar_wait(full(stage), (it / C::NSTAGE) & 1u, p.err)) ok = false;
+        if (ok) {
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::NROWS);
 #pragma unroll
-        for (int ks = 0; ks < C::NKSTEP; ++ks) {
-          const int cb = (ks * 32) / 128;
-          const int inner = (ks * 32) % 128;
-          const uint64_t adesc = umma_desc_sw128(s_k + kb_ * C::K_BYTES + cb * C::KROWS * 128 + inner);
-          const uint64_t bdesc = umma_desc_sw128(s_q + stage * C::Q_BYTES + cb * C::NROWS * 128 + inner);
-          mma_bf16(d_tmem, adesc, bdesc, C::IDESC, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < C::NKSTEP; ++ks) {
+            const int cb = (ks * 32) / 128;
+            const int inner = (ks * 32) % 128;
+            const uint64_t adesc = umma_desc_sw128(s_k + kb_ * C::K_BYTES + cb * C::KROWS * 128 + inner);
+            const uint64_t bdesc = umma_desc_sw128(s_q + stage * C::Q_BYTES + cb * C::NROWS * 128 + inner);
+            mma_bf16(d_tmem, adesc, bdesc, C::IDESC, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(empty(stage));
+          tc_commit(tfull(buf));
+          if (s.last) { tc_commit(kempty(kb_)); ++gk; }
         }
-        tc_commit(empty(stage));
-        tc_commit(tfull(buf));
-        if (s.last) { tc_commit(kempty(kb_)); ++gk; }
       }
-      if (!ok) {
-        tc_commit(mdone);
-        mbar_drain(mdone, 0);
-      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+    }
+    if (!ok && lane == 0) {
+      tc_commit(mdone);
+      mbar_drain(mdone, 0);
     }
     __syncwarp();
   } else {
@@ -268,30 +304,36 @@ score_inv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int row = quarter * 32 + lane;       // key of the tile = TMEM lane
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     float* cw = reinterpret_cast<float*>(smem + C::SMEM_COEF) + e * C::NROWS;
+    s.init(p, total, true);
+    // lane l stages coefficients 4l .. 4l+3 of an item (of its query 4l / H;
+    // columns of missing queries take the item's first query's, their sums
+    // are never stored); the loads for the set's next item are issued while
+    // the current item is processed
+    const int c0 = 4 * lane;
+    auto coef_load = [&](const int4& rows) {
+      int r = item_row(rows, c0 / C::H);
+      if (r < 0) r = rows.x;
+      if (r < 0) return make_float4(0.f, 0.f, 0.f, 0.f);  // no such item
+      return __ldg(reinterpret_cast<const float4*>(p.w + static_cast<long long>(r) * C::H + (c0 % C::H)));
+    };
+    float4 wnext = make_float4(0.f, 0.f, 0.f, 0.f);
+    {
+      s.cur();
+      wnext = coef_load(set == 0 ? s.rows : s.peek_rows(1));
+    }
     uint32_t it = 0;
-    for (; !s.done; s.next(p), ++it) {
+    for (; s.i < s.i1; s.advance(p, true), ++it) {
+      s.cur();
       if (static_cast<int>(it & 1u) != set) continue;
       const int buf = static_cast<int>(it % C::NACC);
-      const int b = s.g / p.M;
-      const int j = s.g - b * p.M;
-      const int q0 = __ldg(p.qoff + s.g) + s.ch * C::QC;
-      const int nq = min(C::QC, s.nq - s.ch * C::QC);
-      // this item's queries (row, slot) and their head weights, before the wait
-      int2 ent[C::QC];
-#pragma unroll
-      for (int i = 0; i < C::QC; ++i) ent[i] = i < nq ? __ldg(p.list + q0 + i) : make_int2(-1, 0);
-      {
-        // lane l stages coefficients 4l .. 4l+3 (of query 4l / H; columns of
-        // queries past nq take query 0's, their sums are never stored)
-        const int c0 = 4 * lane;
-        const int qi = c0 / C::H;
-        const int2 eq = __ldg(p.list + q0 + (qi < nq ? qi : 0));
-        const float4 wv = __ldg(reinterpret_cast<const float4*>(p.w + static_cast<long long>(eq.x) * C::H +
-                                                                (c0 % C::H)));
-        *reinterpret_cast<float4*>(cw + c0) = wv;
-        __syncwarp();
-      }
-      const int tok = j * p.blk + s.u * 128 + row;  // token of this lane's key in its sequence
+      const int U = p.blk / 128;
+      const int g = s.tile / U;
+      const int u = s.tile - g * U;
+      const int j = g - (g / p.M) * p.M;
+      *reinterpret_cast<float4*>(cw + c0) = wnext;
+      __syncwarp();
+      wnext = coef_load(s.peek_rows(2));
+      const int tok = j * p.blk + u * 128 + row;  // token of this lane's key in its sequence
       if (!mbar_wait(tfull(buf), (it / C::NACC) & 1u, p.err)) break;
       tc_fence_after();
       const uint32_t taddr = lane_addr + static_cast<uint32_t>(buf * C::NROWS);
@@ -327,15 +369,15 @@ score_inv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
 #pragma unroll
       for (int i = 0; i < C::QC; ++i) {
-        if (i >= nq) continue;
+        const int r = item_row(s.rows, i);
+        if (r < 0) continue;
         const float2 f0 = unpack2(acc2[i][0]);
         const float2 f1 = unpack2(acc2[i][1]);
         const float score = (f0.x + f0.y) + (f1.x + f1.y);
-        const int r = ent[i].x;
         const long long pos = p.q_offset + (r % p.T);
         const bool vis = tok < p.L && tok <= pos;
-        p.out[static_cast<long long>(r) * p.ldo + static_cast<long long>(ent[i].y) * p.blk + s.u * 128 + row] =
-            vis ? score : -INFINITY;
+        p.out[static_cast<long long>(r) * p.ldo + static_cast<long long>(item_row(s.slots, i)) * p.blk + u * 128 +
+              row] = vis ? score : -INFINITY;
       }
     }
   }
@@ -426,6 +468,38 @@ __global__ void invert_fill_kernel(const int* __restrict__ blocks, long long row
     const int g = static_cast<int>((r / T) * M + jb);
     const int at = atomicAdd(cursor + g, 1);
     list[qoff[g] + at] = make_int2(static_cast<int>(r), static_cast<int>(e - r * m));
+  }
+}
+
+// Item records: one warp per block g; item loc of the block is (key tile
+// u = loc / nch, chunk c = loc % nch) and holds queries c*QC .. c*QC+QC-1 of
+// the block's list.
+__global__ void invert_items_kernel(const int* __restrict__ cnt, const int* __restrict__ qoff,
+                                    const int* __restrict__ ioff, const int2* __restrict__ list, int nb, int U,
+                                    int qc, int* __restrict__ it_tile, int4* __restrict__ it_row,
+                                    int4* __restrict__ it_slot) {
+  const int lane = threadIdx.x & 31;
+  const int g = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (g >= nb) return;
+  const int nq = cnt[g];
+  const int nch = (nq + qc - 1) / qc;
+  const int base = ioff[g];
+  const int q0 = qoff[g];
+  for (int loc = lane; loc < U * nch; loc += 32) {
+    const int u = loc / nch;
+    const int c = loc - u * nch;
+    int rr[4] = {-1, -1, -1, -1}, ss[4] = {0, 0, 0, 0};
+    for (int i = 0; i < qc && i < 4; ++i) {
+      const int q = c * qc + i;
+      if (q < nq) {
+        const int2 e = list[q0 + q];
+        rr[i] = e.x;
+        ss[i] = e.y;
+      }
+    }
+    it_tile[base + loc] = g * U + u;
+    it_row[base + loc] = make_int4(rr[0], rr[1], rr[2], rr[3]);
+    it_slot[base + loc] = make_int4(ss[0], ss[1], ss[2], ss[3]);
   }
 }
 

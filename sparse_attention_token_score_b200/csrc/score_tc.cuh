@@ -75,28 +75,47 @@ struct ScoreParams {
   int* cres;
   int* creal;
   int ccap;
-  // Optional tile mask (score mode): tile j of query group g (g counted over
-  // all sequences) is computed only if tile_live[g * live_ld + j] != 0; for
-  // the others nothing is loaded or multiplied and, with dead_fill, the
-  // visible entries of the full scores are set to -inf.
-  const uint8_t* tile_live;
+  // Optional work list (score mode): only the (query group, key tile) pairs
+  // pairs[0 .. *pairs_n) are computed (groups counted over all sequences;
+  // each group's tiles contiguous and ascending), split evenly over the CTAs.
+  const int2* pairs;
+  const int* pairs_n;
+
+  // DoSA bound pass (ScoreCfg kEpiBound): the score computed is the bound's
+  // augmented-head part; adding cbound[row] * knorm[key] gives the bound, and
+  // a key tile becomes live for the refinement pass's query group
+  // (live_qpt queries per group, live_gpb groups per sequence) when a visible
+  // key of the tile has bound >= cthr[row]: live_out[group * live_ld + tile] = 1.
+  const float* knorm;
+  const float* cbound;
+  uint8_t* live_out;
   long long live_ld;
-  int dead_fill;
+  int live_qpt, live_gpb;
 };
 
 constexpr int CCHUNK = 64;  // candidate slots reserved per warp and query at a time
 
+// Epilogue variants of the score mode: full scores (kEpiStore), candidate
+// lists (kEpiCand), DoSA bounds -> live key tiles (kEpiBound).
+enum : int { kEpiStore = 0, kEpiCand = 1, kEpiBound = 2 };
+
 template <int ELEM_, int D_, int H_, int QPT_, ScoreMode MODE_, int NSTAGE_, int EPIW_ = 8, int NQBUF_ = 1,
-          bool CMP_ = false>
+          int EPI_ = kEpiStore, bool LIST_ = false>
 struct ScoreCfg {
   static constexpr int ELEM = ELEM_;  // bytes per element: 2 = bf16, 1 = e4m3
   static constexpr int D = D_, H = H_, QPT = QPT_, NSTAGE = NSTAGE_;
   static constexpr ScoreMode MODE = MODE_;
   static constexpr bool ROUTER = MODE_ == ScoreMode::kRouter;
   static constexpr bool GATHER = MODE_ == ScoreMode::kGather;
-  // candidate compaction in the epilogue (ScoreParams::ccnt and friends)
-  static constexpr bool CMP = CMP_;
-  static_assert(!CMP || (MODE_ == ScoreMode::kTma && QPT_ > 1), "compaction: score mode, several queries per group");
+  // candidate compaction in the epilogue (ScoreParams::cres and friends) or
+  // DoSA bounds (ScoreParams::knorm and friends)
+  static constexpr bool CMP = EPI_ == kEpiCand;
+  static constexpr bool BND = EPI_ == kEpiBound;
+  static_assert(EPI_ == kEpiStore || (MODE_ == ScoreMode::kTma && QPT_ > 1),
+                "epilogue variants: score mode, several queries per group");
+  // work-list mode (ScoreParams::pairs): only listed (group, tile) pairs
+  static constexpr bool LIST = LIST_;
+  static_assert(!LIST || MODE_ == ScoreMode::kTma, "work lists: score mode");
   static constexpr int ROW_BYTES = D * ELEM;
   static_assert(ROW_BYTES == 128 || ROW_BYTES == 256, "rows must be 1 or 2 swizzle atoms wide");
   static constexpr int KBLK = ROW_BYTES / 128;          // 128-byte column blocks per row
@@ -150,8 +169,11 @@ struct ScoreCfg {
   // per epilogue warp: the head weights (x query scales) of its columns for
   // the current query group, refilled when the group changes
   static constexpr int NCOL_THREAD = ROUTER ? 0 : (SPLIT_TILES ? QROWS : QROWS / NSETS);
+  // DoSA bounds: (threshold, norm coefficient) of each query of the warp's
+  // set, staged with the head weights
+  static constexpr int NBND_THREAD = (EPI_ == 2) ? 2 * (QPT_ / NSETS) : 0;
   static constexpr int SMEM_COEF = SMEM_K + NSTAGE * K_BYTES;
-  static constexpr int SMEM_BAR = SMEM_COEF + EPIW * NCOL_THREAD * 4;
+  static constexpr int SMEM_BAR = SMEM_COEF + EPIW * (NCOL_THREAD + NBND_THREAD) * 4;
   static constexpr int NBAR = 2 * NSTAGE + 2 * NQBUF + 2 * NACC + 1;
   static constexpr int SMEM_USED = SMEM_BAR + NBAR * 8 + 16;
   // Pad to more than half an SM so two CTAs never share an SM's TMEM.
@@ -185,12 +207,34 @@ struct TileSched {
     return ntile_tg(p, grp % gpb);
   }
 
+  // pair-list mode: position li of the list (left pairs to go, this included)
+  int li;
+
+  __device__ __forceinline__ void load_pair(const ScoreParams& p, bool at_start) {
+    const int2 e = __ldg(p.pairs + li);
+    g = e.x;
+    j = e.y;
+    b = g / gpb;
+    tg = g - b * gpb;
+    first = at_start || __ldg(&p.pairs[li - 1].x) != g;
+    last = left == 1 || __ldg(&p.pairs[li + 1].x) != g;
+  }
+
   // All 32 lanes of the warp call init together (warp-cooperative scans).
   __device__ __forceinline__ void init(const ScoreParams& p) {
     gpb = (p.T + C::QPT - 1) / C::QPT;
     G = p.batch * gpb;
     done = false;
     const int lane = threadIdx.x & 31;
+    if constexpr (C::LIST) {
+      const long long W = __ldg(p.pairs_n);
+      const long long i0 = W * blockIdx.x / gridDim.x;
+      left = W * (blockIdx.x + 1) / gridDim.x - i0;
+      li = static_cast<int>(i0);
+      if (left <= 0) { done = true; return; }
+      load_pair(p, true);
+      return;
+    }
     if (C::ROUTER) {
       left = 0;
       g = blockIdx.x;
@@ -239,6 +283,12 @@ struct TileSched {
   }
 
   __device__ __forceinline__ void next(const ScoreParams& p) {
+    if constexpr (C::LIST) {
+      if (--left == 0) { done = true; return; }
+      ++li;
+      load_pair(p, false);
+      return;
+    }
     if (C::ROUTER) {
       if (++j == nt) {
         g += gridDim.x;
@@ -283,11 +333,38 @@ __device__ __forceinline__ long long gathered_token(const ScoreParams& p, long l
   return tok;
 }
 
-// Whether the current (group, tile) is computed (ScoreParams::tile_live).
-template <class C, class S>
-__device__ __forceinline__ bool tile_live(const ScoreParams& p, const S& s) {
-  if (C::ROUTER || C::GATHER || p.tile_live == nullptr) return true;
-  return __ldg(p.tile_live + static_cast<long long>(s.g) * p.live_ld + s.j) != 0;
+// Work list for the score kernel's pair-list mode: the (group, tile) pairs
+// whose flag is set (flags[g * ld + j]), each group's tiles ascending and
+// contiguous, j below the group's visible tile count (queries of a group are
+// qpt consecutive ones; tiles of 128 keys). One warp per group; the group's
+// run is placed with one atomic, so groups come in no particular order.
+__global__ void pairs_build_kernel(const uint8_t* __restrict__ flags, long long ld, int groups, int gpb, int T,
+                                   int qpt, long long q_offset, int L, int2* __restrict__ pairs,
+                                   int* __restrict__ count) {
+  const int lane = threadIdx.x & 31;
+  const int g = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (g >= groups) return;
+  const int tg = g % gpb;
+  const long long t_last = min(T, (tg + 1) * qpt) - 1;
+  const long long nk = min(q_offset + t_last + 1, static_cast<long long>(L));
+  const int nt = static_cast<int>((nk + 127) / 128);
+  const uint8_t* f = flags + static_cast<long long>(g) * ld;
+  int cnt = 0;
+  for (int j0 = 0; j0 < nt; j0 += 32) {
+    const int j = j0 + lane;
+    cnt += __popc(__ballot_sync(0xffffffffu, j < nt && f[j] != 0));
+  }
+  if (cnt == 0) return;
+  int base = 0;
+  if (lane == 0) base = atomicAdd(count, cnt);
+  base = __shfl_sync(0xffffffffu, base, 0);
+  for (int j0 = 0; j0 < nt; j0 += 32) {
+    const int j = j0 + lane;
+    const bool on = j < nt && f[j] != 0;
+    const uint32_t m = __ballot_sync(0xffffffffu, on);
+    if (on) pairs[base + __popc(m & ((1u << lane) - 1u))] = make_int2(g, j);
+    base += __popc(m);
+  }
 }
 
 template <class C>
@@ -354,7 +431,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (; !s.done; s.next(p)) {
       const int b = s.b;
       const int tg = s.tg;
-      const bool live = tile_live<C>(p, s);
       // gathers: tiles round-robin over the producer warps (each owns its
       // stages); contiguous block tiles (TMA): warp 0 loads every tile
       const bool mine = C::GATHER ? (p.blk_tma ? pw == 0 : static_cast<int>(it % C::NPROD) == pw) : true;
@@ -376,7 +452,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      if (!live) continue;  // a pruned tile: no keys (the query tile bookkeeping above still runs)
       if (!mine) { ++it; continue; }
       const int stage = static_cast<int>(it % C::NSTAGE);
       const uint32_t ph = (it / C::NSTAGE) & 1u;
@@ -484,10 +559,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (; !s.done; s.next(p)) {
         const int qb = static_cast<int>(gq % C::NQBUF);
         if (s.first && !mbar_wait(qfull(qb), (gq / C::NQBUF) & 1u, p.err)) { ok = false; break; }
-        if (!tile_live<C>(p, s)) {
-          if (s.last) { tc_commit(qempty(qb)); ++gq; }
-          continue;
-        }
         const int stage = static_cast<int>(it % C::NSTAGE);
         const uint32_t ph = (it / C::NSTAGE) & 1u;
         const int buf = static_cast<int>(it % C::NACC);
@@ -541,7 +612,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (; !s.done; s.next(p)) {
       const int b = s.b;
       const int tg = s.tg;
-      const bool live = tile_live<C>(p, s);
       const int q0s = C::SPLIT_TILES ? 0 : set * QHC;            // this set's first query (in group)
       const long long rbase_s = static_cast<long long>(b) * p.T + tg * C::QPT + q0s;
       if constexpr (C::CMP) {
@@ -555,19 +625,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           cnext = atomicAdd(p.cres + rbase_s + lane, CCHUNK);
         }
       }
-      if (!live) {
-        if (!C::ROUTER && !C::GATHER && p.dead_fill && p.out != nullptr && (!C::SPLIT_TILES || set == 0)) {
-          // pruned tile: its visible entries read as -inf
-          const int key = s.j * C::KROWS + row;
-          const int t0 = tg * C::QPT + q0s;
-          const long long e = static_cast<long long>(key) * p.pstride - (p.q_offset + t0);
-          if (key < p.Lk) {
-#pragma unroll
-            for (int ql = 0; ql < QHC; ++ql)
-              if (t0 + ql < p.T && e <= ql) p.out[(rbase_s + ql) * p.ldo + key] = -INFINITY;
-          }
-        }
-      } else {
+      {
       const int buf = static_cast<int>(it % C::NACC);
       // split tiles: the two sets take alternate tiles (buffer b: set b & 1)
       const bool mine = C::SPLIT_TILES ? (static_cast<int>(it & 1u) == set) : true;
@@ -585,6 +643,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if constexpr (C::KEY_SCALES) {
           const int skey = s.j * C::KROWS + row;
           if (skey < p.Lk) ks = __ldg(p.k_scale + static_cast<long long>(b) * p.Lk + skey);
+        }
+        // DoSA: this row's key norm, likewise
+        float kn = 0.f;
+        if constexpr (C::BND) {
+          const int nkey = s.j * C::KROWS + row;
+          if (nkey < p.Lk) kn = __ldg(p.knorm + static_cast<long long>(b) * p.Lk + nkey);
         }
         // candidate thresholds of this thread's queries (compaction only)
         constexpr int QHT = QHC;
@@ -643,7 +707,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           // this warp's head weights for the group (queries past T reuse the
           // last query's weights; their outputs are never stored)
           static_assert(NC == C::NCOL_THREAD, "coefficient slot");
-          float* cw = reinterpret_cast<float*>(smem + C::SMEM_COEF) + e * NC;
+          float* cw = reinterpret_cast<float*>(smem + C::SMEM_COEF) + e * (NC + C::NBND_THREAD);
           if (s.g != coef_g) {
             for (int c = lane; c < NC; c += 32) {
               const int ql = c / C::H;
@@ -653,6 +717,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               float cv = __ldg(p.w + ci);
               if (C::ELEM == 1) cv *= __ldg(p.q_scale + ci);
               cw[c] = cv;
+            }
+            if constexpr (C::BND) {
+              for (int ql = lane; ql < QH; ql += 32) {
+                const bool in = tg * C::QPT + q0 + ql < p.T;
+                cw[NC + 2 * ql] = in ? __ldg(p.cthr + rbase + ql) : INFINITY;
+                cw[NC + 2 * ql + 1] = in ? __ldg(p.cbound + rbase + ql) : 0.f;
+              }
             }
             __syncwarp();
             coef_g = s.g;
@@ -749,7 +820,26 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // query q0+ql sees this key iff key * pstride <= q_offset + t0 + ql
             const int t0 = tg * C::QPT + q0;
             const long long e = static_cast<long long>(key) * p.pstride - (p.q_offset + t0);
-            if (key < p.Lk && (!C::CMP || p.out != nullptr)) {
+            if constexpr (C::BND) {
+              // DoSA: bound >= threshold for some visible key of the warp ->
+              // the tile is live for the query's refinement group
+#pragma unroll
+              uint32_t lmask = 0;  // bit ql: this key is live for query ql
+              for (int ql = 0; ql < QH; ++ql) {
+                const float2 tc = *reinterpret_cast<const float2*>(cw + NC + 2 * ql);  // (thr, c_t)
+                const bool live = key < p.Lk && e <= ql && fmaf(tc.y, kn, accq[ql]) >= tc.x;
+                lmask |= static_cast<uint32_t>(live) << ql;
+              }
+              // one flag per refinement group of live_qpt queries (t0 is a
+              // multiple of QH, which is a multiple of live_qpt or covers a
+              // part of one group)
+              const int qg = p.live_qpt < QH ? p.live_qpt : QH;
+              for (int g0 = 0; g0 < QH; g0 += qg) {
+                const uint32_t gm = qg >= 32 ? 0xffffffffu : ((1u << qg) - 1u) << g0;
+                if (__ballot_sync(0xffffffffu, (lmask & gm) != 0u) != 0u && lane == 0)
+                  p.live_out[(static_cast<long long>(b) * p.live_gpb + (t0 + g0) / p.live_qpt) * p.live_ld + s.j] = 1;
+              }
+            } else if (key < p.Lk && (!C::CMP || p.out != nullptr)) {
               float* orow = p.out + rbase * p.ldo + key;
 #pragma unroll
               for (int ql = 0; ql < QH; ++ql) {
@@ -809,7 +899,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       ++it;
-      }  // live tile
+      }
       if constexpr (C::CMP) {
         if (s.last) {
           // leaving the group: sentinels over the unused slots of this warp's

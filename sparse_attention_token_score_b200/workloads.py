@@ -23,6 +23,10 @@ Distributions follow the five workloads the indexer is measured on:
 * ``indexcache`` four layers of ``dsa`` chunks with the IndexCache pattern
              FSSS: one layer runs the indexer, three reuse its indices (only
              the F layer has inputs: S layers compute no indexer projections)
+* ``dsa_lists`` the ``dsa`` chunk through the candidate-list selection
+* ``dosa``   the ``dsa`` chunk through DoSA's certified pruning (5 screened heads)
+* ``dosa_lownorm`` the ``dsa`` shape with three of every four key tiles shrunk
+             100x and non-negative head weights: most tiles can be pruned
 * ``dsa_fp8`` the ``dsa`` chunk quantised to FP8 e4m3 the way the decode cache
              is (per-token key scale, per-(query, head) query scale)
 
@@ -222,6 +226,21 @@ def fp8_prefill_inputs(T: int, L: int, H: int, d: int, q_offset: Optional[int] =
                          q_scale=qs, k_scale=ks, meta=base.meta)
 
 
+def lownorm_inputs(T: int, L: int, H: int, d: int, q_offset: Optional[int] = None, seed: int = 0,
+                   w_std: Optional[float] = None, live_every: int = 4, shrink: float = 0.01) -> IndexerInputs:
+    """A prefill chunk where most keys cannot rank high for any query: the
+    keys of every 128-key tile except each live_every-th one are scaled by
+    ``shrink`` before rounding, and the head weights are non-negative (|w|),
+    so every query's best scores come from the full-norm tiles."""
+    base = prefill_inputs(T, L, H, d, q_offset=q_offset, seed=seed, w_std=w_std)
+    kf = bf16_bits_to_f32(base.k)
+    tile = np.arange(L) // 128
+    kf[:, tile % live_every != 0] *= np.float32(shrink)
+    base.k = f32_to_bf16_bits(kf)
+    base.w = np.abs(base.w)
+    return base
+
+
 # ----------------------------------------------------------------- workloads
 CONFIGS = {
     "tiny": dict(kind="dense", T=2048, L=2048, H=8, d=64, q_offset=0, topk=256),
@@ -230,6 +249,12 @@ CONFIGS = {
     "decode": dict(kind="decode", batch=64, T=1, L=131072, H=64, d=128, topk=2048),
     "indexcache": dict(kind="indexcache", pattern="FSSS", T=4096, L=32768, H=64, d=128, q_offset=28672,
                        topk=2048, needles=64, w_std=0.125),
+    "dsa_lists": dict(kind="dosa", T=4096, L=32768, H=64, d=128, q_offset=28672, topk=2048, needles=64,
+                      w_std=0.125),
+    "dosa": dict(kind="dosa", T=4096, L=32768, H=64, d=128, q_offset=28672, topk=2048, needles=64,
+                 w_std=0.125, n_screen=5),
+    "dosa_lownorm": dict(kind="dosa_lownorm", T=4096, L=32768, H=64, d=128, q_offset=28672, topk=2048,
+                         w_std=0.125, n_screen=5, live_every=4, shrink=0.01),
     "dsa_fp8": dict(kind="dense_fp8", T=4096, L=32768, H=64, d=128, q_offset=28672, topk=2048,
                     needles=64, w_std=0.125),
     "misa": dict(kind="misa", T=2048, L=131072, H=64, d=128, q_offset=129024, topk=2048,
@@ -244,7 +269,10 @@ def make_inputs(name: str, seed: int = 0) -> IndexerInputs:
     c = CONFIGS[name]
     if c["kind"] == "decode":
         return decode_inputs(c["batch"], c["L"], c["H"], c["d"], seed=seed)
-    if c["kind"] == "indexcache":  # the inputs of the (single) F layer
+    if c["kind"] == "dosa_lownorm":
+        return lownorm_inputs(c["T"], c["L"], c["H"], c["d"], q_offset=c["q_offset"], seed=seed,
+                              w_std=c["w_std"], live_every=c["live_every"], shrink=c["shrink"])
+    if c["kind"] in ("indexcache", "dosa"):  # the dsa chunk (indexcache: its single F layer)
         return prefill_inputs(c["T"], c["L"], c["H"], c["d"], q_offset=c["q_offset"], seed=seed,
                               w_std=c.get("w_std"), needles=c.get("needles", 0))
     if c["kind"] == "dense_fp8":

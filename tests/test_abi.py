@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 21
+    assert len(names) == 25
     assert set(names) == set(B._SIGS)
     for n in names:
         assert getattr(lib, n) is not None
@@ -175,3 +175,32 @@ def test_hisa_refine_checks(lib):
     assert lib.hisa_refine_scores(ctypes.byref(a), blocks, 4, 128, out, 512, ws, need - 1, None) == -3
     # the HISA workspace grows by the inverted lists when blocks are whole key tiles
     assert lib.hisa_workspace_size(ctypes.byref(a), 128, 4, 16) > lib.hisa_workspace_size(ctypes.byref(a), 96, 4, 16)
+
+
+def test_dosa_checks(lib):
+    a = _args(T=64, L=8192, q_offset=8128)
+    big, ws = 1 << 34, ctypes.c_void_p(0x50000)
+    out = ctypes.c_void_p(0x40000)
+    assert lib.dosa_workspace_size(ctypes.byref(a), 512, 5) > lib.indexer_workspace_size(ctypes.byref(a), 512)
+    assert lib.dosa_score_topk(ctypes.byref(a), 512, 5, None, None, None, ws, big, None) == -1
+    assert lib.dosa_score_topk(ctypes.byref(a), 512, 14, out, None, None, ws, big, None) == -2    # > 13 screened
+    assert lib.dosa_score_topk(ctypes.byref(_args(T=64, L=2048, q_offset=1984)), 128, 5, out, None, None, ws, big,
+                               None) == -2                                                       # rows too short
+    assert lib.dosa_score_topk(ctypes.byref(_args(H=8, T=64, L=8192, q_offset=8128)), 512, 5, out, None, None, ws,
+                               big, None) == -2                                                  # H = 8
+    assert lib.dosa_workspace_size(ctypes.byref(_args(T=64, L=2048, q_offset=1984)), 128, 5) == 0
+    need = lib.dosa_workspace_size(ctypes.byref(a), 512, 5)
+    assert lib.dosa_score_topk(ctypes.byref(a), 512, 5, out, None, None, ws, need - 1, None) == -3
+
+
+def test_lists_checks(lib):
+    a = _args(T=64, L=8192, q_offset=8128)
+    ws, big, out = ctypes.c_void_p(0x50000), 1 << 34, ctypes.c_void_p(0x40000)
+    need = lib.indexer_lists_workspace_size(ctypes.byref(a), 512)
+    assert need > lib.indexer_workspace_size(ctypes.byref(a), 512)
+    assert lib.indexer_lists_workspace_size(ctypes.byref(_args(T=4, L=2048, q_offset=2044)), 64) == 0
+    assert lib.indexer_score_topk_lists(ctypes.byref(_args(T=4, L=2048, q_offset=2044)), 64, out, None, ws, big,
+                                        None) == -2                     # rows too short for the sample
+    assert lib.indexer_score_topk_lists(ctypes.byref(a), 2048, out, None, ws, big, None) == -2   # k > L / 8
+    assert lib.indexer_score_topk_lists(ctypes.byref(a), 512, None, None, ws, big, None) == -1
+    assert lib.indexer_score_topk_lists(ctypes.byref(a), 512, out, None, ws, need - 1, None) == -3

@@ -179,8 +179,14 @@ def _unfused(ix, inp, topk):
 
 def _fused_equals_unfused(inp, topk):
     ix = _indexer(inp)
-    idx, val = ix.dense(topk, with_score=True)
-    assert ix.device_status() == 0
+    shape = (inp.batch, inp.T, topk)
+    idx = torch.full(shape, -7, dtype=torch.int32, device="cuda")
+    val = torch.full(shape, float("nan"), device="cuda")
+    ws = B.alloc_workspace(B.indexer_lists_workspace_size(ix.args, topk))
+    B.indexer_score_topk_lists(ix.args, topk, idx, val, ws)
+    assert B.dsa_device_status(ws) == 0
+    d_idx, d_val = ix.dense(topk, with_score=True)
+    assert torch.equal(idx, d_idx) and torch.equal(val, d_val)
     uidx, uval = _unfused(ix, inp, topk)
     assert torch.equal(idx, uidx), "candidate-list selection differs from the full-row selection"
     assert torch.equal(val, uval)
@@ -194,8 +200,9 @@ def _fused_equals_unfused(inp, topk):
 ])
 def test_fused_selection_equals_full_rows(shape):
     """The candidate-list chain (sample pass, thresholds, compacting score
-    pass, list top-k) selects exactly what the top-k of the full rows selects,
-    bit for bit, and matches the oracle within the near-tie rule."""
+    pass, list top-k, fallback for short lists) selects exactly what the top-k
+    of the full rows selects, bit for bit (and what indexer_score_topk
+    selects), and matches the oracle within the near-tie rule."""
     b, T, L, H, d, topk = shape
     inp = wl.prefill_inputs(T, L, H, d, q_offset=L - T, seed=80 + H, batch=b)
     idx, val = _fused_equals_unfused(inp, topk)
@@ -223,7 +230,7 @@ def _common_direction_inputs(T, L, seed):
 
 def test_fused_selection_short_lists_fall_back():
     # every 16th key (the sampled ones) is a strong, distinct key: thresholds
-    # come out high, the lists hold fewer than k, every row uses its full scores
+    # come out high, the lists hold fewer than k, every group is re-scored
     inp, u, rng = _common_direction_inputs(32, 8192, 90)
     strong = 3.0 * u[None, :] + 0.05 * rng.standard_normal((512, 128)).astype(np.float32)
     inp.k[0, ::16] = wl.f32_to_bf16_bits(strong)
@@ -250,6 +257,99 @@ def test_misa_fused_routed_selection():
     inp = wl.prefill_inputs(36, 16384, 64, 128, q_offset=16348, seed=92, w_std=0.125)
     _misa_check(inp, block=64, h=8, topk=256, kprime=1024, queries=range(0, 36, 5), what="misa fused")
     _misa_check(inp, block=64, h=8, topk=512, kprime=0, queries=range(0, 36, 7), what="misa fused plain")
+
+
+# ------------------------------------------------------------------ DoSA certified pruning
+def _dosa_run(inp, topk, n_screen):
+    ix = _indexer(inp)
+    a = ix.args
+    shape = (inp.batch, inp.T, topk)
+    idx = torch.full(shape, -7, dtype=torch.int32, device="cuda")
+    val = torch.full(shape, float("nan"), device="cuda")
+    qpt = 256 // inp.H
+    live = torch.full((inp.batch, -(-inp.T // qpt), -(-inp.L // 128)), 9, dtype=torch.uint8, device="cuda")
+    ws = B.alloc_workspace(B.dosa_workspace_size(a, topk, n_screen))
+    B.dosa_score_topk(a, topk, n_screen, idx, val, live, ws)
+    assert B.dsa_device_status(ws) == 0
+    uidx, uval = _unfused(ix, inp, topk)
+    assert torch.equal(idx, uidx), "DoSA selection differs from the full-row selection"
+    assert torch.equal(val, uval)
+    return idx.cpu().numpy(), live.cpu().numpy()
+
+
+def _visible_live_fraction(inp, live):
+    qpt = 256 // inp.H
+    fr = []
+    for g in range(live.shape[1]):
+        p_last = inp.q_offset + min(inp.T, (g + 1) * qpt) - 1
+        nt = -(-min(p_last + 1, inp.L) // 128)
+        fr.append(live[0, g, :nt].mean())
+    return float(np.mean(fr))
+
+
+@pytest.mark.parametrize("H,n_screen", [(64, 5), (32, 13), (16, 2)])
+def test_dosa_equals_dense_selection(H, n_screen):
+    """Random keys and signed head weights (the bound prunes little): the
+    pruned selection equals the full-row selection bit for bit."""
+    inp = wl.prefill_inputs(48, 8192, H, 128, q_offset=8192 - 48, seed=100 + H, batch=2)
+    idx, live = _dosa_run(inp, 300, n_screen)
+    assert set(np.unique(live)) <= {0, 1}
+    res = oracle.dense_topk(inp, 300, queries=[0, 47])
+    for i, t in enumerate(res["queries"]):
+        s_, c_ = res["scores"][i], res["cond"][i]
+        check_selection(idx[0, t], np.arange(s_.size), s_, c_, 300, what=f"dosa H={H} t={t}")
+
+
+def _low_norm_keys(inp, live_every=4, shrink=0.01):
+    kf = wl.bf16_bits_to_f32(inp.k)
+    tile = np.arange(inp.L) // 128
+    kf[:, tile % live_every != 0] *= np.float32(shrink)
+    inp.k = wl.f32_to_bf16_bits(kf)
+
+
+def test_dosa_prunes_a_low_norm_population():
+    """Three of every four key tiles hold low-norm keys no query can rank
+    high: the bound prunes them (more than half of the visible tiles), and the
+    selection still equals the full-row one. The oracle's tile-granular DoSA
+    prunes about as much on the same input."""
+    inp = wl.prefill_inputs(64, 8192, 64, 128, q_offset=8128, seed=110)
+    inp.w = np.abs(inp.w)
+    _low_norm_keys(inp)
+    idx, live = _dosa_run(inp, 256, 5)
+    frac = _visible_live_fraction(inp, live)
+    assert frac < 0.5, frac
+    ref = oracle.dosa_tile_topk(inp, 256, 5, 16, 4, groups=[0, 15])
+    for gi, g in enumerate(ref["groups"]):
+        # every tile the oracle needs is live on the GPU
+        assert np.all(live[0, g][ref["live"][gi] == 1] == 1)
+    dense = oracle.dense_topk(inp, 256, queries=ref["queries"])
+    assert np.array_equal(ref["idx"], dense["idx"])
+    for i, t in enumerate(dense["queries"]):
+        s_, c_ = dense["scores"][i], dense["cond"][i]
+        check_selection(idx[0, t], np.arange(s_.size), s_, c_, 256, what=f"dosa low-norm t={t}")
+
+
+def test_dosa_mass_ties_and_full_lists():
+    # 256 copies of one strong key at the sampled positions: the certified
+    # lists hold more keys tied at the k-th score than are taken (lowest
+    # positions win); then every key identical: every list overflows its
+    # capacity and every group is re-scored in full
+    inp, u, _ = _common_direction_inputs(24, 8192, 112)
+    inp.k[0, 0:4096:16] = wl.f32_to_bf16_bits(3.0 * u)[None, :]
+    idx, _ = _dosa_run(inp, 100, 5)
+    assert np.array_equal(idx[0, 0], np.arange(0, 1600, 16))
+    inp.k[0, :] = inp.k[0, 0]
+    idx, _ = _dosa_run(inp, 100, 5)
+    assert np.array_equal(idx[0, 5], np.arange(100))
+
+
+def test_dosa_short_certificates_fall_back():
+    # the sampled keys are the strongest: thresholds too high to certify,
+    # every group is re-scored in full; the selection is still exact
+    inp, u, rng = _common_direction_inputs(32, 8192, 111)
+    strong = 3.0 * u[None, :] + 0.05 * rng.standard_normal((512, 128)).astype(np.float32)
+    inp.k[0, ::16] = wl.f32_to_bf16_bits(strong)
+    _dosa_run(inp, 512, 5)
 
 
 # ------------------------------------------------------------------ FP8 prefill
