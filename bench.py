@@ -77,11 +77,12 @@ def workload_desc(name, queries=None, batch=None):
     tag = {"tiny": "tiny_prefill", "dsa": "dsa_chunk", "decode": "decode_fp8",
            "misa": "misa_dagger", "hisa": "hisa", "dsa_fp8": "dsa_chunk_fp8",
            "indexcache": "indexcache_dsa_chunk", "dosa": "dosa_dsa_chunk",
-           "dosa_lownorm": "dosa_lownorm_dsa_chunk", "dsa_lists": "dsa_chunk_lists"}[name]
+           "dosa_lownorm": "dosa_lownorm_dsa_chunk", "dsa_lists": "dsa_chunk_lists",
+           "hisa_decode": "hisa_decode_fp8"}[name]
     label = f"{tag}_B{batch}_T{c['T']}_L{c['L']}_H{c['H']}_d{c['d']}_k{c['topk']}"
     if name == "misa":
         label += f"_blk{c['block']}_h{c['h']}_kp{c['kprime']}"
-    if name == "hisa":
+    if name in ("hisa", "hisa_decode"):
         label += f"_blk{c['block']}_m{c['m']}"
     if name == "indexcache":
         label += f"_layers{c['pattern']}"
@@ -191,14 +192,15 @@ class Runner:
                 return rows * kp * 2.0 * d * H, "tensor"
             if stage == "re-score" and label == "topk_rows":
                 return rows * kp * 4 + rows * k * 8, "hbm"
-        if self.name == "hisa":
+        if self.name in ("hisa", "hisa_decode"):
+            fp8 = self.name == "hisa_decode"
             blk, m = c["block"], c["m"]
             M = -(-L // blk)
             vis_blocks = int(self.batch * np.minimum(pos // blk + 1, M).sum())
             if stage == "blocks" and label.startswith("score_tc"):
-                return vis_blocks * 2.0 * d * H, "tensor"
+                return vis_blocks * 2.0 * d * H, "tensor_fp8" if fp8 else "tensor"
             if stage == "tokens" and label.startswith("score_"):
-                return rows * m * blk * 2.0 * d * H, "tensor"
+                return rows * m * blk * 2.0 * d * H, "tensor_fp8" if fp8 else "tensor"
             if stage == "tokens" and label == "topk_rows":
                 return rows * m * blk * 4 + rows * k * 8, "hbm"
         return None, None
@@ -450,7 +452,7 @@ def oracle_sample(name, inp, budget_s=10.0, max_q=4096, with_pairs=False):
         t0 = time.perf_counter()
         if name == "misa":
             oracle.misa(inp, c["block"], c["h"], c["topk"], kprime=c["kprime"], queries=qs, b=b)
-        elif name == "hisa":
+        elif name in ("hisa", "hisa_decode"):
             oracle.hisa(inp, c["block"], c["m"], c["topk"], queries=qs, b=b)
         else:
             oracle.dense_topk(inp, c["topk"], queries=qs, b=b)
@@ -462,7 +464,7 @@ def oracle_sample(name, inp, budget_s=10.0, max_q=4096, with_pairs=False):
         off = inp.q_offset
         return int(sum(min(off + int(t) + 1, inp.L) for t in qs)) * len(c.get("pattern", "F"))
 
-    if name == "decode":
+    if name in ("decode", "hisa_decode"):
         # one unit = one sequence's query; add sequences until budget_s is spent
         t, nb = 0.0, 0
         while t < budget_s and nb < inp.batch:
@@ -548,7 +550,8 @@ def make_inputs(name, seed, queries=0, batch=0):
 
 
 # ------------------------------------------------------------------ main
-SUB_WORKLOADS = ("tiny", "decode", "misa", "hisa", "dsa_fp8", "indexcache", "dsa_lists", "dosa", "dosa_lownorm")
+SUB_WORKLOADS = ("tiny", "decode", "misa", "hisa", "hisa_decode", "dsa_fp8", "indexcache", "dsa_lists", "dosa",
+                 "dosa_lownorm")
 MIN_TIMED_MS = 60.0  # sub-records run enough steps that the clock sampler sees the GPU busy
 
 
@@ -670,7 +673,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="all", choices=["all", "tiny", "dsa", "decode", "misa", "hisa", "dsa_fp8", "indexcache", "dosa",
-                             "dosa_lownorm", "dsa_lists"],
+                             "dosa_lownorm", "dsa_lists", "hisa_decode"],
                     help="all (default): the dsa chunk is the headline line, the other four "
                          "workloads are measured in the same run under 'workloads'")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

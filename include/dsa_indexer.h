@@ -180,7 +180,9 @@ DSA_EXPORT dsa_status indexer_scores(const dsa_indexer_args* a, float* out_score
  * blk = 1: token candidates; blk = B: candidate blocks of B tokens (a block
  * size that is a multiple of 128 fetches whole blocks with TMA).
  *   cand [batch*T, n_slots] int32; out [batch*T, ld] fp32, ld >= n_slots * blk.
- * bf16 only; d = 128, H in {32, 64}. Workspace: the 256-byte header only. */
+ * d = 128, H in {32, 64}; bf16 or FP8 e4m3 (FP8: 128-byte key rows, each
+ * gathered key's score times its k_scale, the head weights times q_scale).
+ * Workspace: the 256-byte header only. */
 DSA_EXPORT dsa_status indexer_score_gathered(const dsa_indexer_args* a, const int32_t* cand,
                                              int n_slots, int blk, float* out, long long ld,
                                              void* workspace, size_t ws_bytes, void* stream);
@@ -216,8 +218,13 @@ DSA_EXPORT dsa_status dsa_meanpool_keys(const void* k, int batch, int L, int d, 
  *   out_score [batch, T, topk] fp32 (routed scores; full-H scores for MISA-dagger) or NULL
  *   out_heads [batch, T, h] int32 chosen heads (ascending) or NULL
  *   out_cand  [batch, T, kprime] int32 MISA-dagger candidates (ascending, -1 padded) or NULL
- * bf16 only; h in {8, 16, 32, 64}, h <= H; MISA-dagger needs d = 128 and
- * H in {32, 64}. */
+ * h in {8, 16, 32, 64}, h <= H; MISA-dagger needs d = 128 and H in {32, 64}.
+ * bf16, or FP8 e4m3 (d = 128, H in {32, 64}; a prefill chunk or the decode
+ * cache): the pooled keys are kept in the cache's format (per block the fp64
+ * mean of the dequantised keys, scale absmax/448, e4m3 codes of mean / scale,
+ * nearest even); the router weights each pooled key by its scale and each
+ * affinity by q_scale[t,h]; the routed pass reads the kept heads' e4m3 rows
+ * and scales; the MISA-dagger re-score gathers 128-byte e4m3 key rows. */
 DSA_EXPORT size_t misa_workspace_size(const dsa_indexer_args* a, int block, int h, int topk, int kprime);
 DSA_EXPORT dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, int topk,
                                  int kprime, int32_t* out_idx, float* out_score,
@@ -233,7 +240,13 @@ DSA_EXPORT dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block
  *   out_idx    [batch, T, topk] int32 token indices
  *   out_score  [batch, T, topk] fp32 token scores or NULL
  *   out_blocks [batch, T, m] int32 kept blocks (ascending, -1 padded) or NULL
- * bf16 only; token refinement needs d = 128 and H in {32, 64}. */
+ * d = 128 and H in {32, 64}. bf16 or FP8 e4m3 (a prefill chunk or the decode
+ * cache): with FP8 the pooled keys are kept in the cache's format (per block
+ * the fp64 mean of the dequantised keys, scale absmax/448, e4m3 codes of
+ * mean / scale, nearest even), the block scores and the token scores use FP8
+ * MMAs with the per-token / per-block and per-(query, head) scales, and block
+ * must be a multiple of 128. Blocks that are whole 128-key tiles are refined
+ * block major (hisa_refine_scores); others one query per tile (bf16). */
 DSA_EXPORT size_t hisa_workspace_size(const dsa_indexer_args* a, int block, int m, int topk);
 DSA_EXPORT dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, int topk,
                                   int32_t* out_idx, float* out_score, int32_t* out_blocks,
@@ -248,7 +261,8 @@ DSA_EXPORT dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int bloc
  * slot is empty. The same values as indexer_score_gathered with these blocks
  * (which fetches every kept block once per query). hisa_block_filter_topk
  * uses this path when blk is a multiple of 128.
- * bf16 only; d = 128, H in {32, 64}, blk a multiple of 128. Workspace:
+ * bf16 or FP8 e4m3 (scores k_scale[s] * sum_h (w * q_scale) ReLU(q8 . k8));
+ * d = 128, H in {32, 64}, blk a multiple of 128. Workspace:
  * hisa_refine_workspace_size bytes (the 256-byte header plus the lists). */
 DSA_EXPORT size_t hisa_refine_workspace_size(const dsa_indexer_args* a, int m, int blk);
 DSA_EXPORT dsa_status hisa_refine_scores(const dsa_indexer_args* a, const int32_t* blocks, int m, int blk,

@@ -17,7 +17,9 @@ widens them exactly to fp64 and follows the pages' steps in order:
   candidates, the full H_I-head indexer re-scores them, keep the top-k.
 * HISA ("HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse
   Attention" review, section 3): score pooled block keys, keep the top-m
-  blocks, score the tokens of the surviving blocks, keep the top-k.
+  blocks, score the tokens of the surviving blocks, keep the top-k. On an
+  FP8 key cache the pooled keys of MISA and HISA are kept in the cache's
+  format (e4m3 with a per-block scale).
 * IndexCache ("IndexCache: Accelerating Sparse Attention via Cross-Layer
   Index Reuse", section 2): layers marked F run their own indexer and cache
   its top-k; layers marked S skip the indexer and reuse the cache of the
@@ -122,6 +124,46 @@ E4M3_TABLE = np.array([_e4m3_value(c) for c in range(256)], dtype=np.float64)
 def decode_e4m3(codes: np.ndarray) -> np.ndarray:
     """FP8 e4m3 bytes -> fp64 (exact)."""
     return E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
+
+
+# e4m3 codes 0x00 .. 0x7E (non-negative finite values, increasing with the code)
+_E4M3_POS = E4M3_TABLE[:0x7F]
+
+
+def f64_to_e4m3(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to OCP FP8 E4M3 codes: nearest representable value,
+    ties to the even code (even mantissa), saturating at +-448; zero keeps its
+    sign. Brute force over the 127 non-negative finite codes."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), 448.0)
+    d = np.abs(a[..., None] - _E4M3_POS)                     # distance to every code
+    best = d.min(axis=-1, keepdims=True)
+    cand = d == best
+    # ties: two neighbours at the same distance; take the even code
+    code = np.where(cand.sum(-1) > 1, np.argmax(cand & (np.arange(0x7F) % 2 == 0), axis=-1),
+                    np.argmax(cand, axis=-1)).astype(np.uint8)
+    sign = np.signbit(x).astype(np.uint8) << 7
+    return code | sign
+
+
+def meanpool_e4m3(k_codes: np.ndarray, k_scale: np.ndarray, B: int):
+    """Pooled keys of an FP8 cache, stored in the cache's format: the fp64
+    mean of the block's dequantised keys, a scale absmax/448 (fp32 absmax
+    divided in fp32; 1 when the mean is zero), codes e4m3(mean / scale).
+    Returns (codes [M, d] uint8, scales [M] fp32)."""
+    k = decode_e4m3(k_codes) * np.asarray(k_scale, dtype=np.float64)[:, None]
+    L, d = k.shape
+    M = -(-L // B)
+    codes = np.empty((M, d), dtype=np.uint8)
+    scales = np.empty(M, dtype=np.float32)
+    for m in range(M):
+        blk = k[m * B:min((m + 1) * B, L)]
+        mean = blk.sum(axis=0) / blk.shape[0]
+        amax = np.float32(np.max(np.abs(mean)))
+        sc = np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+        scales[m] = sc
+        codes[m] = f64_to_e4m3(mean / np.float64(sc))
+    return codes, scales
 
 
 def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -278,18 +320,26 @@ def misa(inp, block: int, h: int, topk: int, kprime: int = 0,
          heads_given: Optional[np.ndarray] = None, cand_given: Optional[np.ndarray] = None):
     """MISA routed indexer (kprime == 0) or MISA-dagger (kprime > 0).
 
+    bf16 or FP8 inputs: with an FP8 cache every stage reads the dequantised
+    values (q = q_scale * e4m3(q), k = k_scale * e4m3(k)) and the pooled keys
+    stay in the cache's format (``meanpool_e4m3``), as in ``hisa``.
+
     heads_given [nq, h] / cand_given [nq, kprime]: run the later stages on these
     choices instead of the oracle's own (lets a test condition each stage on
     the GPU's previous discrete choice). Returns a dict with every stage."""
-    assert inp.dtype == "bf16"
     q, k, w = dequant(inp, b)
     T, H, d = q.shape
     L = k.shape[0]
     if queries is None:
         queries = np.arange(T)
     queries = np.asarray(queries, dtype=np.int64)
-    kbar_bits = meanpool_bf16(inp.k[b], block)
-    kbar = widen_bf16(kbar_bits)
+    if inp.dtype == "bf16":
+        kbar_bits = meanpool_bf16(inp.k[b], block)
+        kbar = widen_bf16(kbar_bits)
+    else:  # FP8 cache: pooled keys in the cache's format, as for HISA
+        codes, scales = meanpool_e4m3(inp.k[b], inp.k_scale[b], block)
+        kbar_bits = (codes, scales)
+        kbar = decode_e4m3(codes) * scales.astype(np.float64)[:, None]
     M = kbar.shape[0]
     p = inp.q_offset + queries
     a = router_affinity(q[queries], kbar, w[queries], visible_blocks(p, block, M))
@@ -327,15 +377,19 @@ def hisa(inp, block: int, m: int, topk: int, queries: Optional[Sequence[int]] = 
 
     blocks_given [nq, m]: run the token stage on these blocks instead of the
     oracle's own choice."""
-    assert inp.dtype == "bf16"
     q, k, w = dequant(inp, b)
     T, H, d = q.shape
     L = k.shape[0]
     if queries is None:
         queries = np.arange(T)
     queries = np.asarray(queries, dtype=np.int64)
-    kbar_bits = meanpool_bf16(inp.k[b], block)
-    kbar = widen_bf16(kbar_bits)
+    if inp.dtype == "bf16":
+        kbar_bits = meanpool_bf16(inp.k[b], block)
+        kbar = widen_bf16(kbar_bits)
+    else:  # FP8 cache: pooled keys in the cache's format (meanpool_e4m3)
+        codes, scales = meanpool_e4m3(inp.k[b], inp.k_scale[b], block)
+        kbar_bits = (codes, scales)
+        kbar = decode_e4m3(codes) * scales.astype(np.float64)[:, None]
     M = kbar.shape[0]
     p = inp.q_offset + queries
     nvb = visible_blocks(p, block, M)

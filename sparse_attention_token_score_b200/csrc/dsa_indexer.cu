@@ -220,6 +220,15 @@ dsa_status run_scores_bf16(int D, int H, const ScoreParams& p, const void* q, lo
 dsa_status run_scores_fp8(int D, int H, const ScoreParams& p, const void* q, long long q_rows,
                           const void* k, long long k_rows, cudaStream_t st) {
   const bool prefill = p.T > 1;
+  // 8 or 16 heads (MISA's routed pass): each of the two epilogue warp sets
+  // takes at least 32 columns, so a group has 64 / H queries even in decode,
+  // where only the first of them exists
+  if (D == 128 && H == 16)
+    return prefill ? launch_score<ScoreCfg<1, 128, 16, 16, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st)
+                   : launch_score<ScoreCfg<1, 128, 16, 4, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
+  if (D == 128 && H == 8)
+    return prefill ? launch_score<ScoreCfg<1, 128, 8, 32, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st)
+                   : launch_score<ScoreCfg<1, 128, 8, 8, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
   if (D == 128 && H == 64)
     return prefill ? launch_score<ScoreCfg<1, 128, 64, 4, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st)
                    : launch_score<ScoreCfg<1, 128, 64, 1, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
@@ -242,6 +251,18 @@ dsa_status run_router(int D, int H, const ScoreParams& p, const void* q, long lo
   return DSA_ERR_UNSUPPORTED;
 }
 
+// MISA router on an FP8 cache: e4m3 queries against e4m3 pooled keys,
+// p.k_scale = the pooled keys' scales (the router weights its columns by
+// them; the query scales are applied with |w| when the heads are chosen).
+dsa_status run_router_fp8(int D, int H, const ScoreParams& p, const void* q, long long q_rows,
+                          const void* kbar, long long k_rows, cudaStream_t st) {
+  if (D == 128 && H == 64)
+    return launch_score<ScoreCfg<1, 128, 64, 2, ScoreMode::kRouter, 4>>(p, q, q_rows, kbar, k_rows, st);
+  if (D == 128 && H == 32)
+    return launch_score<ScoreCfg<1, 128, 32, 4, ScoreMode::kRouter, 4>>(p, q, q_rows, kbar, k_rows, st);
+  return DSA_ERR_UNSUPPORTED;
+}
+
 // Gathered re-scoring (MISA-dagger candidates, HISA surviving blocks).
 // When blk is a multiple of 128, every 128-row tile is one contiguous key
 // run and is fetched with TMA; otherwise rows are gathered with cp.async.
@@ -251,10 +272,22 @@ dsa_status run_router(int D, int H, const ScoreParams& p, const void* q, long lo
 #ifndef DSA_GATHER_NQ
 #define DSA_GATHER_NQ 2
 #endif
+#ifndef DSA_GATHER8_NS
+#define DSA_GATHER8_NS 8
+#endif
 dsa_status run_gather(int D, int H, ScoreParams p, const void* q, long long q_rows,
-                      cudaStream_t st) {
+                      cudaStream_t st, bool fp8 = false) {
   p.blk_tma = (p.blk % 128 == 0) ? 1 : 0;
   const long long k_rows = static_cast<long long>(p.batch) * p.L_tok;
+  if (fp8) {  // e4m3 rows of 128 bytes, per-token key scales (p.k_scale)
+    if (D == 128 && H == 64)
+      return launch_score<ScoreCfg<1, 128, 64, 1, ScoreMode::kGather, DSA_GATHER8_NS, 8, DSA_GATHER_NQ>>(
+          p, q, q_rows, p.kg, k_rows, st);
+    if (D == 128 && H == 32)
+      return launch_score<ScoreCfg<1, 128, 32, 1, ScoreMode::kGather, DSA_GATHER8_NS, 8, DSA_GATHER_NQ>>(
+          p, q, q_rows, p.kg, k_rows, st);
+    return DSA_ERR_UNSUPPORTED;
+  }
   if (D == 128 && H == 64)
     return launch_score<ScoreCfg<2, 128, 64, 1, ScoreMode::kGather, DSA_GATHER_NS, 8, DSA_GATHER_NQ>>(
         p, q, q_rows, p.kg, k_rows, st);
@@ -347,7 +380,7 @@ InvWs inv_carve(Carve& c, long long rows, int m, long long nb, int blk, int H) {
 // The block-major kernel takes kept blocks whose size is a multiple of 128
 // (whole key tiles), bf16, d = 128, H in {32, 64}.
 bool inv_supported(const dsa_indexer_args* a, int blk) {
-  return blk % 128 == 0 && a->qk_dtype == DSA_BF16 && a->d == 128 && (a->H == 32 || a->H == 64);
+  return blk % 128 == 0 && a->d == 128 && (a->H == 32 || a->H == 64);
 }
 
 template <class C>
@@ -363,8 +396,8 @@ dsa_status launch_inv(const InvParams& p, const void* q, long long q_rows, const
     attr[dev].store(true, std::memory_order_relaxed);
   }
   CUtensorMap tq, tk;
-  if (!make_tmap(&tq, q, false, C::D, q_rows, C::H)) return DSA_ERR_CUDA;     // one query per box
-  if (!make_tmap(&tk, k, false, C::D, k_rows, C::KROWS)) return DSA_ERR_CUDA;
+  if (!make_tmap(&tq, q, C::ELEM == 1, C::D, q_rows, C::H)) return DSA_ERR_CUDA;     // one query per box
+  if (!make_tmap(&tk, k, C::ELEM == 1, C::D, k_rows, C::KROWS)) return DSA_ERR_CUDA;
   prof::Launch pl(st, "score_inv (block-major)");
   score_inv_kernel<C><<<num_sms(), C::NTHREADS, C::SMEM_BYTES, st>>>(tq, tk, p, total);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
@@ -413,6 +446,8 @@ dsa_status run_refine_inverted(const dsa_indexer_args* a, const int32_t* blocks,
   p.m = m;
   p.q_offset = a->q_offset;
   p.w = a->w;
+  p.q_scale = a->q_scale;
+  p.k_scale = a->k_scale;
   p.out = out;
   p.ldo = ldo;
   p.it_tile = w.it_tile;
@@ -421,8 +456,12 @@ dsa_status run_refine_inverted(const dsa_indexer_args* a, const int32_t* blocks,
   p.err = err;
   const long long q_rows = rows * a->H;
   const long long k_rows = static_cast<long long>(a->batch) * a->L;
-  if (a->H == 32) return launch_inv<InvCfg<32, DSA_INV_NSTAGE>>(p, a->q, q_rows, a->k, k_rows, w.total, st);
-  return launch_inv<InvCfg<64, DSA_INV_NSTAGE>>(p, a->q, q_rows, a->k, k_rows, w.total, st);
+  if (a->qk_dtype == DSA_FP8_E4M3) {
+    if (a->H == 32) return launch_inv<InvCfg<1, 32, 8>>(p, a->q, q_rows, a->k, k_rows, w.total, st);
+    return launch_inv<InvCfg<1, 64, 8>>(p, a->q, q_rows, a->k, k_rows, w.total, st);
+  }
+  if (a->H == 32) return launch_inv<InvCfg<2, 32, DSA_INV_NSTAGE>>(p, a->q, q_rows, a->k, k_rows, w.total, st);
+  return launch_inv<InvCfg<2, 64, DSA_INV_NSTAGE>>(p, a->q, q_rows, a->k, k_rows, w.total, st);
 }
 
 bool h_supported_bf16(int H) { return H == 8 || H == 16 || H == 32 || H == 64; }
@@ -781,7 +820,7 @@ dsa_status indexer_scores(const dsa_indexer_args* a, float* out, long long ld, v
 dsa_status indexer_score_gathered(const dsa_indexer_args* a, const int32_t* cand, int n_slots,
                                   int blk, float* out, long long ld, void* ws, size_t ws_bytes,
                                   void* stream) {
-  DSA_TRY(validate(a, true));
+  DSA_TRY(validate(a, false));
   if (!cand || !out || n_slots < 1 || blk < 1 || !aligned(cand, 4) || !aligned(out, 4))
     return DSA_ERR_ARG;
   if (static_cast<long long>(n_slots) * blk > INT_MAX / 2) return DSA_ERR_UNSUPPORTED;
@@ -793,12 +832,13 @@ dsa_status indexer_score_gathered(const dsa_indexer_args* a, const int32_t* cand
   ScoreParams pg = base_params(a, static_cast<unsigned*>(ws));
   pg.out = out;
   pg.ldo = ld;
-  pg.kg = static_cast<const __nv_bfloat16*>(a->k);
+  pg.kg = a->k;
   pg.cand = cand;
   pg.n_slots = n_slots;
   pg.blk = blk;
   pg.n_compact = n_slots * blk;
-  return run_gather(a->d, a->H, pg, a->q, static_cast<long long>(a->batch) * a->T * a->H, st);
+  return run_gather(a->d, a->H, pg, a->q, static_cast<long long>(a->batch) * a->T * a->H, st,
+                    a->qk_dtype == DSA_FP8_E4M3);
 }
 
 dsa_status indexer_topk_rows(const float* scores, long long rows, long long ld, int T,
@@ -875,9 +915,49 @@ dsa_status dsa_meanpool_keys(const void* k, int batch, int L, int d, int block, 
   if (static_cast<long long>(batch) * M > INT_MAX) return DSA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   prof::Launch pl(st, "meanpool");
-  meanpool_kernel<<<static_cast<int>(batch * M), d < 128 ? d : 128, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(k), L, d, block, static_cast<int>(M),
-      static_cast<__nv_bfloat16*>(kbar));
+  if (d % 8 == 0 && d <= 256 && aligned(k, 16))
+    meanpool_vec_kernel<false><<<static_cast<int>(batch * M), 256, 0, st>>>(
+        static_cast<const uint8_t*>(k), nullptr, L, d, block, static_cast<int>(M), static_cast<uint8_t*>(kbar),
+        nullptr);
+  else
+    meanpool_kernel<<<static_cast<int>(batch * M), d < 128 ? d : 128, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(k), L, d, block, static_cast<int>(M),
+        static_cast<__nv_bfloat16*>(kbar));
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// Pooled keys of MISA and HISA: bf16 [batch*M, d], or on an FP8 cache e4m3
+// codes [batch*M, d] plus fp32 scales [batch*M] (the cache's format).
+struct Pooled {
+  __nv_bfloat16* kbar;  // bf16
+  uint8_t* kbar8;       // FP8 codes
+  float* scale;         // FP8 scales
+};
+
+size_t pooled_bytes(const dsa_indexer_args* a, long long M) {
+  const size_t n = static_cast<size_t>(a->batch) * M;
+  return al256(n * a->d * 2) + al256(n * sizeof(float));
+}
+
+Pooled pooled_carve(Carve& c, const dsa_indexer_args* a, long long M) {
+  const size_t n = static_cast<size_t>(a->batch) * M;
+  Pooled pk{};
+  if (a->qk_dtype == DSA_FP8_E4M3) {
+    pk.kbar8 = c.take<uint8_t>(n * a->d);
+    pk.scale = c.take<float>(n);
+    c.off += al256(n * a->d * 2) - al256(n * a->d);  // keep the bf16 layout's size
+  } else {
+    pk.kbar = c.take<__nv_bfloat16>(n * a->d);
+    pk.scale = c.take<float>(n);
+  }
+  return pk;
+}
+
+dsa_status run_meanpool(const dsa_indexer_args* a, int block, long long M, const Pooled& pk, cudaStream_t st) {
+  if (a->qk_dtype != DSA_FP8_E4M3) return dsa_meanpool_keys(a->k, a->batch, a->L, a->d, block, pk.kbar, st);
+  prof::Launch pl(st, "meanpool fp8");
+  meanpool_vec_kernel<true><<<static_cast<int>(a->batch * M), 256, 0, st>>>(
+      static_cast<const uint8_t*>(a->k), a->k_scale, a->L, a->d, block, static_cast<int>(M), pk.kbar8, pk.scale);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -888,10 +968,11 @@ size_t misa_workspace_size(const dsa_indexer_args* a, int block, int h, int topk
   const size_t BT = static_cast<size_t>(a->batch) * a->T;
   const size_t M = static_cast<size_t>(blocks_of(a->L, block));
   size_t n = kHdr;
-  n += al256(a->batch * M * a->d * 2);            // pooled keys
+  n += pooled_bytes(a, static_cast<long long>(M));  // pooled keys
   n += al256(2 * BT * a->H * sizeof(float));      // router partial sums
   n += al256(BT * h * a->d * 2);                  // gathered queries of the kept heads
   n += al256(BT * h * sizeof(float));             // their weights
+  n += al256(BT * h * sizeof(float));             // their query scales (FP8)
   n += al256(BT * h * sizeof(int32_t));           // kept heads
   n += al256(BT * a->L * sizeof(float));          // routed scores
   if (kprime > 0) {
@@ -904,11 +985,12 @@ size_t misa_workspace_size(const dsa_indexer_args* a, int block, int h, int topk
 dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, int topk, int kprime,
                                  int32_t* out_idx, float* out_score, int32_t* out_heads,
                                  int32_t* out_cand, void* ws, size_t ws_bytes, void* stream) {
-  DSA_TRY(validate(a, true));
+  DSA_TRY(validate(a, false));
   if (!out_idx || block < 1 || h < 1 || h > a->H || topk < 1 || topk > (1 << 24) || kprime < 0 ||
       kprime > (1 << 24))
     return DSA_ERR_ARG;
   if (!h_supported_bf16(h) || a->H > 64) return DSA_ERR_UNSUPPORTED;
+  const bool fp8 = a->qk_dtype == DSA_FP8_E4M3;
   if (kprime > 0 && (a->d != 128 || (a->H != 32 && a->H != 64))) return DSA_ERR_UNSUPPORTED;
   DSA_TRY(check_ws(ws, ws_bytes, misa_workspace_size(a, block, h, topk, kprime)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -919,35 +1001,43 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   if (static_cast<long long>(a->batch) * M > INT_MAX) return DSA_ERR_UNSUPPORTED;
 
   Carve c{static_cast<char*>(ws), kHdr};
-  __nv_bfloat16* kbar = c.take<__nv_bfloat16>(static_cast<size_t>(a->batch) * M * a->d);
+  const Pooled pk = pooled_carve(c, a, M);
   float* part = c.take<float>(2 * static_cast<size_t>(BT) * a->H);
-  __nv_bfloat16* q_sel = c.take<__nv_bfloat16>(static_cast<size_t>(BT) * h * a->d);
+  uint8_t* q_sel = c.take<uint8_t>(static_cast<size_t>(BT) * h * a->d * 2);
   float* w_sel = c.take<float>(static_cast<size_t>(BT) * h);
+  float* qs_sel = c.take<float>(static_cast<size_t>(BT) * h);
   int32_t* heads_ws = c.take<int32_t>(static_cast<size_t>(BT) * h);
   float* routed = c.take<float>(static_cast<size_t>(BT) * a->L);
   int32_t* heads = out_heads ? out_heads : heads_ws;
 
-  // 1. pooled keys
-  DSA_TRY(dsa_meanpool_keys(a->k, a->batch, a->L, a->d, block, kbar, stream));
+  // 1. pooled keys (FP8 cache: in the cache's format)
+  DSA_TRY(run_meanpool(a, block, M, pk, st));
   // 2. router affinities (partial ReLU sums over visible pooled keys)
   prof::Stage misa_stage("router");
   ScoreParams pr = base_params(a, err);
   pr.Lk = static_cast<int>(M);
   pr.pstride = block;
   pr.out = part;
-  DSA_TRY(run_router(a->d, a->H, pr, a->q, BT * a->H, kbar, a->batch * M, st));
-  // 3. top-h heads per query; gather their query rows and weights
+  if (fp8) {
+    pr.k_scale = pk.scale;
+    DSA_TRY(run_router_fp8(a->d, a->H, pr, a->q, BT * a->H, pk.kbar8, a->batch * M, st));
+  } else {
+    DSA_TRY(run_router(a->d, a->H, pr, a->q, BT * a->H, pk.kbar, a->batch * M, st));
+  }
+  // 3. top-h heads per query; gather their query rows, weights (and query scales)
   {
     prof::Launch pl(st, "select_heads");
     select_heads_kernel<<<static_cast<int>((BT + 7) / 8), 256, 0, st>>>(
-        part, BT, a->H, h, a->w, static_cast<const __nv_bfloat16*>(a->q), a->d, heads, q_sel, w_sel);
+        part, BT, a->H, h, a->w, fp8 ? a->q_scale : nullptr, static_cast<const uint8_t*>(a->q),
+        a->d * (fp8 ? 1 : 2), heads, q_sel, w_sel, qs_sel);
   }
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   // 4. routed token scores with the kept heads only, and their top-k (or
-  // top-k' candidates), through candidate lists where that applies
+  // top-k' candidates)
   misa_stage.set("routed");
   ScoreParams ps = base_params(a, err);
   ps.w = w_sel;
+  ps.q_scale = fp8 ? qs_sel : nullptr;
   ps.out = routed;
   ps.ldo = a->L;
   const long long k_rows = static_cast<long long>(a->batch) * a->L;
@@ -961,7 +1051,8 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   const int ksel = kprime > 0 ? kprime : topk;
   int32_t* sel = kprime > 0 ? cand : out_idx;
   float* sel_score = kprime > 0 ? nullptr : out_score;
-  DSA_TRY(run_scores_bf16(a->d, h, ps, q_sel, BT * h, a->k, k_rows, st));
+  if (fp8) DSA_TRY(run_scores_fp8(a->d, h, ps, q_sel, BT * h, a->k, k_rows, st));
+  else DSA_TRY(run_scores_bf16(a->d, h, ps, q_sel, BT * h, a->k, k_rows, st));
   DSA_TRY(launch_topk(ws, topk_params(routed, BT, a->L, a->T, a->q_offset, 1, a->L, ksel, sel, sel_score, nullptr,
                                   0, 1),
                       st));
@@ -971,12 +1062,12 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   ScoreParams pg = base_params(a, err);
   pg.out = compact;
   pg.ldo = kprime;
-  pg.kg = static_cast<const __nv_bfloat16*>(a->k);
+  pg.kg = a->k;
   pg.cand = cand;
   pg.n_slots = kprime;
   pg.blk = 1;
   pg.n_compact = kprime;
-  DSA_TRY(run_gather(a->d, a->H, pg, a->q, BT * a->H, st));
+  DSA_TRY(run_gather(a->d, a->H, pg, a->q, BT * a->H, st, fp8));
   return launch_topk(ws, topk_params(compact, BT, kprime, a->T, a->q_offset, 0, kprime, topk, out_idx,
                                  out_score, cand, kprime, 1),
                      st);
@@ -988,7 +1079,7 @@ size_t hisa_workspace_size(const dsa_indexer_args* a, int block, int m, int topk
   const size_t BT = static_cast<size_t>(a->batch) * a->T;
   const size_t M = static_cast<size_t>(blocks_of(a->L, block));
   size_t n = kHdr;
-  n += al256(a->batch * M * a->d * 2);                        // pooled keys
+  n += pooled_bytes(a, static_cast<long long>(M));            // pooled keys (FP8: codes + scales)
   n += al256(BT * M * sizeof(float));                         // block scores
   n += al256(BT * m * sizeof(int32_t));                       // kept blocks
   n += al256(BT * static_cast<size_t>(m) * block * sizeof(float));  // token scores of kept blocks
@@ -1005,7 +1096,7 @@ size_t hisa_refine_workspace_size(const dsa_indexer_args* a, int m, int blk) {
 
 dsa_status hisa_refine_scores(const dsa_indexer_args* a, const int32_t* blocks, int m, int blk, float* out,
                               long long ld, void* ws, size_t ws_bytes, void* stream) {
-  DSA_TRY(validate(a, true));
+  DSA_TRY(validate(a, false));
   if (!blocks || !out || m < 1 || blk < 1 || !aligned(blocks, 4) || !aligned(out, 4)) return DSA_ERR_ARG;
   if (static_cast<long long>(m) * blk > INT_MAX / 2) return DSA_ERR_UNSUPPORTED;
   if (ld < static_cast<long long>(m) * blk) return DSA_ERR_ARG;
@@ -1023,10 +1114,12 @@ dsa_status hisa_refine_scores(const dsa_indexer_args* a, const int32_t* blocks, 
 dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, int topk,
                                   int32_t* out_idx, float* out_score, int32_t* out_blocks,
                                   void* ws, size_t ws_bytes, void* stream) {
-  DSA_TRY(validate(a, true));
+  DSA_TRY(validate(a, false));
   if (!out_idx || block < 1 || m < 1 || topk < 1 || topk > (1 << 24)) return DSA_ERR_ARG;
   if (static_cast<long long>(m) * block > INT_MAX / 2) return DSA_ERR_UNSUPPORTED;
   if (a->d != 128 || (a->H != 32 && a->H != 64)) return DSA_ERR_UNSUPPORTED;
+  const bool fp8 = a->qk_dtype == DSA_FP8_E4M3;
+  if (fp8 && block % 128 != 0) return DSA_ERR_UNSUPPORTED;  // FP8 refinement: whole key tiles only
   DSA_TRY(check_ws(ws, ws_bytes, hisa_workspace_size(a, block, m, topk)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DSA_TRY(clear_status(ws, st));
@@ -1037,14 +1130,14 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   const int ncomp = m * block;
 
   Carve c{static_cast<char*>(ws), kHdr};
-  __nv_bfloat16* kbar = c.take<__nv_bfloat16>(static_cast<size_t>(a->batch) * M * a->d);
+  const Pooled pk = pooled_carve(c, a, M);
   float* bscore = c.take<float>(static_cast<size_t>(BT) * M);
   int32_t* blocks_ws = c.take<int32_t>(static_cast<size_t>(BT) * m);
   float* compact = c.take<float>(static_cast<size_t>(BT) * ncomp);
   int32_t* blocks = out_blocks ? out_blocks : blocks_ws;
 
-  // 1. pooled keys
-  DSA_TRY(dsa_meanpool_keys(a->k, a->batch, a->L, a->d, block, kbar, stream));
+  // 1. pooled keys (FP8 cache: e4m3 codes + per-block scales)
+  DSA_TRY(run_meanpool(a, block, M, pk, st));
   // 2. block scores on the pooled keys (block m visible iff m * block <= p_t)
   prof::Stage hisa_stage("blocks");
   ScoreParams pb = base_params(a, err);
@@ -1052,7 +1145,12 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   pb.pstride = block;
   pb.out = bscore;
   pb.ldo = M;
-  DSA_TRY(run_scores_bf16(a->d, a->H, pb, a->q, BT * a->H, kbar, a->batch * M, st));
+  if (fp8) {
+    pb.k_scale = pk.scale;
+    DSA_TRY(run_scores_fp8(a->d, a->H, pb, a->q, BT * a->H, pk.kbar8, a->batch * M, st));
+  } else {
+    DSA_TRY(run_scores_bf16(a->d, a->H, pb, a->q, BT * a->H, pk.kbar, a->batch * M, st));
+  }
   // 3. top-m blocks
   DSA_TRY(launch_topk(ws, topk_params(bscore, BT, M, a->T, a->q_offset, block, static_cast<int>(M), m,
                                   blocks, nullptr, nullptr, 0, 1),
@@ -1071,12 +1169,12 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   ScoreParams pg = base_params(a, err);
   pg.out = compact;
   pg.ldo = ncomp;
-  pg.kg = static_cast<const __nv_bfloat16*>(a->k);
+  pg.kg = a->k;
   pg.cand = blocks;
   pg.n_slots = m;
   pg.blk = block;
   pg.n_compact = ncomp;
-  DSA_TRY(run_gather(a->d, a->H, pg, a->q, BT * a->H, st));
+  DSA_TRY(run_gather(a->d, a->H, pg, a->q, BT * a->H, st, fp8));
   // 5. top-k tokens
   return launch_topk(ws, topk_params(compact, BT, ncomp, a->T, a->q_offset, 0, ncomp, topk, out_idx,
                                  out_score, blocks, m, block),

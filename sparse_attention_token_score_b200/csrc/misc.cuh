@@ -2,6 +2,7 @@
 // keys and the MISA head selection.
 #pragma once
 #include "common.cuh"
+#include <cuda_fp8.h>
 
 namespace dsa {
 
@@ -27,6 +28,89 @@ __global__ void meanpool_kernel(const __nv_bfloat16* __restrict__ k, int L, int 
   }
 }
 
+// Pooled keys of an FP8 e4m3 key cache, kept in the cache's format: per
+// block the fp64 mean of the dequantised keys (code value x per-token scale),
+// a scale absmax/448 (absmax rounded to fp32, divided in fp32; 1 when the
+// mean is zero) and codes e4m3(mean / scale), rounded to nearest even with
+// saturation.
+//
+// Vectorised pooling, bf16 (the mean as above, rounded to bf16) or FP8 keys,
+// 16-byte rows, d <= 256: a CTA of 256 threads pools one block; each thread reads
+// 16-byte pieces of token rows (rows r, r + RPI, ... of the block, the same
+// 16 bytes of each), accumulates their values (times the token's scale for
+// FP8) in fp64, and the per-thread partial sums are added up per column
+// through shared memory. The products and sums are exact in fp64 here, so
+// the result does not depend on the order and equals the scalar kernels'.
+template <bool FP8>
+__global__ void __launch_bounds__(256) meanpool_vec_kernel(const uint8_t* __restrict__ k,
+                                                           const float* __restrict__ ks, int L, int d, int B,
+                                                           int M, uint8_t* __restrict__ out,
+                                                           float* __restrict__ out_scale) {
+  constexpr int EPV = FP8 ? 16 : 8;           // elements per 16-byte piece
+  __shared__ double red[32 * 128];            // [rows in flight][d]
+  __shared__ double wmax[8];
+  const long long bm = blockIdx.x;
+  const long long b = bm / M;
+  const int m = static_cast<int>(bm % M);
+  const int s0 = m * B;
+  const int s1 = min(s0 + B, L);
+  const int rb = d * (FP8 ? 1 : 2);           // bytes per key row
+  const int tpr = rb / 16;                    // threads per row
+  const int rpi = 256 / tpr;                  // rows in flight
+  const int t = threadIdx.x;
+  const int r = t / tpr, c = t % tpr;
+  double acc[EPV];
+#pragma unroll
+  for (int e = 0; e < EPV; ++e) acc[e] = 0.0;
+  if (r < rpi) {
+    for (int s = s0 + r; s < s1; s += rpi) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(k + (b * L + s) * rb) + c);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      if constexpr (FP8) {
+        const double sc = static_cast<double>(__ldg(ks + b * L + s));
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          __nv_fp8_e4m3 x;
+          x.__x = static_cast<__nv_fp8_storage_t>((w4[e >> 2] >> (8 * (e & 3))) & 0xffu);
+          acc[e] += static_cast<double>(static_cast<float>(x)) * sc;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          acc[e] += static_cast<double>(__uint_as_float(((w4[e >> 1] >> (16 * (e & 1))) & 0xffffu) << 16));
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) red[r * d + c * EPV + e] = acc[e];
+  }
+  __syncthreads();
+  double mean = 0.0;
+  if (t < d) {
+    const int nrow = min(rpi, s1 - s0);
+    double sum = 0.0;
+    for (int i = 0; i < nrow; ++i) sum += red[i * d + t];
+    mean = sum / static_cast<double>(s1 - s0);
+  }
+  if constexpr (!FP8) {
+    if (t < d) reinterpret_cast<__nv_bfloat16*>(out)[bm * d + t] = __double2bfloat16(mean);
+  } else {
+    double a = t < d ? fabs(mean) : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmax(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((t & 31) == 0) wmax[t >> 5] = a;
+    __syncthreads();
+    double amax = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) amax = fmax(amax, wmax[w]);
+    const float af = static_cast<float>(amax);
+    const float scale = af > 0.f ? af / 448.f : 1.f;
+    if (t < d)
+      out[bm * d + t] = static_cast<uint8_t>(__nv_cvt_double_to_fp8(mean / static_cast<double>(scale), __NV_SATFINITE,
+                                                                    __NV_E4M3));
+    if (t == 0) out_scale[bm] = scale;
+  }
+}
+
 // MISA routing (same page, "Methodology", step 1): per query, the head
 // affinity a[h] = |w[h]| * (part0[h] + part1[h]) (the two partial ReLU sums
 // over pooled keys from the router kernel); keep the top-hsel heads by
@@ -34,9 +118,12 @@ __global__ void meanpool_kernel(const __nv_bfloat16* __restrict__ k, int L, int 
 // their weights, and gathers their query rows into a compact [rows, hsel, d]
 // tensor for the routed scoring pass. One warp per query row; H <= 64.
 __global__ void select_heads_kernel(const float* __restrict__ part, long long rows, int H, int hsel,
-                                    const float* __restrict__ w, const __nv_bfloat16* __restrict__ q,
-                                    int d, int* __restrict__ heads, __nv_bfloat16* __restrict__ q_sel,
-                                    float* __restrict__ w_sel) {
+                                    const float* __restrict__ w, const float* __restrict__ q_scale,
+                                    const uint8_t* __restrict__ q, int row_bytes, int* __restrict__ heads,
+                                    uint8_t* __restrict__ q_sel, float* __restrict__ w_sel,
+                                    float* __restrict__ qs_sel) {
+  // part: the router's two partial sums [2][rows, H]; q_scale (FP8 queries,
+  // else null) scales the affinity like |w| and is gathered with the rows
   const int lane = threadIdx.x & 31;
   const long long r = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= rows) return;
@@ -46,7 +133,12 @@ __global__ void select_heads_kernel(const float* __restrict__ part, long long ro
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int h = lane + 32 * i;
-    a[i] = h < H ? fabsf(w[r * H + h]) * (part[r * H + h] + part[plane + r * H + h]) : -INFINITY;
+    float s = 0.f;
+    if (h < H) {
+      s = fabsf(w[r * H + h]) * (part[r * H + h] + part[plane + r * H + h]);
+      if (q_scale) s *= q_scale[r * H + h];
+    }
+    a[i] = h < H ? s : -INFINITY;
   }
   for (int j = 0; j < H; ++j) {
     const float aj = __shfl_sync(0xffffffffu, a[j >> 5], j & 31);
@@ -61,25 +153,25 @@ __global__ void select_heads_kernel(const float* __restrict__ part, long long ro
   const uint32_t m0 = __ballot_sync(0xffffffffu, sel0);
   const uint32_t m1 = __ballot_sync(0xffffffffu, sel1);
   const uint32_t below = (1u << lane) - 1u;
-  if (sel0) {
-    const int pos = __popc(m0 & below);
-    heads[r * hsel + pos] = lane;
-    w_sel[r * hsel + pos] = w[r * H + lane];
-  }
-  if (sel1) {
-    const int pos = __popc(m0) + __popc(m1 & below);
-    heads[r * hsel + pos] = lane + 32;
-    w_sel[r * hsel + pos] = w[r * H + lane + 32];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool sel = i == 0 ? sel0 : sel1;
+    if (!sel) continue;
+    const int h = lane + 32 * i;
+    const int pos = (i == 0 ? 0 : __popc(m0)) + __popc((i == 0 ? m0 : m1) & below);
+    heads[r * hsel + pos] = h;
+    w_sel[r * hsel + pos] = w[r * H + h];
+    if (q_scale) qs_sel[r * hsel + pos] = q_scale[r * H + h];
   }
   __syncwarp();
   // gather the kept query rows (16-byte chunks)
-  const int chunks = d / 8;
+  const int chunks = row_bytes / 16;
   for (int i = lane; i < hsel * chunks; i += 32) {
     const int pos = i / chunks;
     const int c = i % chunks;
     const int h = heads[r * hsel + pos];
-    const uint4 v = *reinterpret_cast<const uint4*>(q + (r * H + h) * d + c * 8);
-    *reinterpret_cast<uint4*>(q_sel + (r * hsel + pos) * d + c * 8) = v;
+    const uint4 v = *reinterpret_cast<const uint4*>(q + (r * H + h) * row_bytes + c * 16);
+    *reinterpret_cast<uint4*>(q_sel + (r * hsel + pos) * row_bytes + c * 16) = v;
   }
 }
 

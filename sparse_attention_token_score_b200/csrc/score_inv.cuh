@@ -34,6 +34,8 @@ struct InvParams {
   int m;                    // kept blocks per query (slots)
   long long q_offset;
   const float* w;           // [batch*T, H]
+  const float* q_scale;     // [batch*T, H] (FP8) or nullptr
+  const float* k_scale;     // [batch*L] (FP8) or nullptr
   float* out;               // [batch*T, ldo] compact rows: position slot * blk + i
   long long ldo;
   const int* it_tile;       // [items] key tile of item i: g * (blk / 128) + u (g = b * M + j)
@@ -42,10 +44,11 @@ struct InvParams {
   unsigned* err;
 };
 
-template <int H_, int NSTAGE_>
+template <int ELEM_, int H_, int NSTAGE_>
 struct InvCfg {
+  static constexpr int ELEM = ELEM_;                     // bytes per element: 2 = bf16, 1 = e4m3
   static constexpr int D = 128, H = H_, NSTAGE = NSTAGE_;
-  static constexpr int ROW_BYTES = D * 2;                // bf16
+  static constexpr int ROW_BYTES = D * ELEM;
   static constexpr int KBLK = ROW_BYTES / 128;           // 128-byte column blocks per row
   static constexpr int QC = 128 / H;                     // queries per item
   static constexpr int NROWS = QC * H;                   // streamed query rows per item (MMA N)
@@ -61,7 +64,7 @@ struct InvCfg {
   static constexpr int EPI_WARP0 = 2;
   static constexpr int EPIW = 8;
   static constexpr int NTHREADS = (EPI_WARP0 + EPIW) * 32;
-  static constexpr uint32_t IDESC = umma_idesc(1u, 128, NROWS);
+  static constexpr uint32_t IDESC = umma_idesc(ELEM == 2 ? 1u : 0u, 128, NROWS);
   static constexpr int SMEM_K = 0;
   static constexpr int SMEM_Q = NKBUF * K_BYTES;
   static constexpr int SMEM_COEF = SMEM_Q + NSTAGE * Q_BYTES;   // per epilogue warp: NROWS coefficients
@@ -133,9 +136,10 @@ struct ItemWalk {
     if (i + ahead >= i1) v = make_int4(-1, -1, -1, -1);
     return v;
   }
-  __device__ __forceinline__ void advance(const InvParams& p, bool with_slots) {
+  __device__ __forceinline__ void advance(const InvParams& p, bool with_slots, int step = 1) {
     prev_tile = tile;
-    if (++i - bbase == 32) {
+    i += step;
+    while (i - bbase >= 32) {
       bbase += 32;
       tile_c = tile_n;
       row_c = row_n;
@@ -225,7 +229,8 @@ score_inv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_arrive_expect_tx(kfull(kb_), C::K_BYTES);
 #pragma unroll
             for (int cb = 0; cb < C::KBLK; ++cb)
-              tma_load_2d(s_k + kb_ * C::K_BYTES + cb * C::KROWS * 128, &tm_k, kfull(kb_), cb * 64, row0);
+              tma_load_2d(s_k + kb_ * C::K_BYTES + cb * C::KROWS * 128, &tm_k, kfull(kb_), cb * (128 / C::ELEM),
+                          row0);
             ++gk;
           }
         }
@@ -243,7 +248,7 @@ score_inv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int cb = 0; cb < C::KBLK; ++cb)
               tma_load_2d(s_q + stage * C::Q_BYTES + cb * C::NROWS * 128 + i * C::H * 128, &tm_q, full(stage),
-                          cb * 64, r * C::H);
+                          cb * (128 / C::ELEM), r * C::H);
           }
         }
       }
@@ -281,7 +286,8 @@ score_inv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int inner = (ks * 32) % 128;
             const uint64_t adesc = umma_desc_sw128(s_k + kb_ * C::K_BYTES + cb * C::KROWS * 128 + inner);
             const uint64_t bdesc = umma_desc_sw128(s_q + stage * C::Q_BYTES + cb * C::NROWS * 128 + inner);
-            mma_bf16(d_tmem, adesc, bdesc, C::IDESC, ks > 0 ? 1u : 0u);
+            if (C::ELEM == 2) mma_bf16(d_tmem, adesc, bdesc, C::IDESC, ks > 0 ? 1u : 0u);
+            else mma_f8(d_tmem, adesc, bdesc, C::IDESC, ks > 0 ? 1u : 0u);
           }
           tc_commit(empty(stage));
           tc_commit(tfull(buf));
@@ -314,17 +320,25 @@ score_inv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       int r = item_row(rows, c0 / C::H);
       if (r < 0) r = rows.x;
       if (r < 0) return make_float4(0.f, 0.f, 0.f, 0.f);  // no such item
-      return __ldg(reinterpret_cast<const float4*>(p.w + static_cast<long long>(r) * C::H + (c0 % C::H)));
+      const long long ci = static_cast<long long>(r) * C::H + (c0 % C::H);
+      float4 wv = __ldg(reinterpret_cast<const float4*>(p.w + ci));
+      if (C::ELEM == 1) {  // FP8: w * q_scale
+        const float4 qs = __ldg(reinterpret_cast<const float4*>(p.q_scale + ci));
+        wv.x *= qs.x; wv.y *= qs.y; wv.z *= qs.z; wv.w *= qs.w;
+      }
+      return wv;
     };
+    // the two sets take alternate items: this set walks items i0 + set,
+    // i0 + set + 2, ...
+    if (set == 1) s.advance(p, true);
     float4 wnext = make_float4(0.f, 0.f, 0.f, 0.f);
-    {
+    if (s.i < s.i1) {
       s.cur();
-      wnext = coef_load(set == 0 ? s.rows : s.peek_rows(1));
+      wnext = coef_load(s.rows);
     }
-    uint32_t it = 0;
-    for (; s.i < s.i1; s.advance(p, true), ++it) {
+    for (; s.i < s.i1; s.advance(p, true, 2)) {
       s.cur();
-      if (static_cast<int>(it & 1u) != set) continue;
+      const uint32_t it = static_cast<uint32_t>(s.i - s.i0);
       const int buf = static_cast<int>(it % C::NACC);
       const int U = p.blk / 128;
       const int g = s.tile / U;
@@ -334,6 +348,8 @@ score_inv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       __syncwarp();
       wnext = coef_load(s.peek_rows(2));
       const int tok = j * p.blk + u * 128 + row;  // token of this lane's key in its sequence
+      float kscale = 1.f;  // FP8: this key's dequant scale
+      if (C::ELEM == 1 && tok < p.L) kscale = __ldg(p.k_scale + static_cast<long long>(g / p.M) * p.L + tok);
       if (!mbar_wait(tfull(buf), (it / C::NACC) & 1u, p.err)) break;
       tc_fence_after();
       const uint32_t taddr = lane_addr + static_cast<uint32_t>(buf * C::NROWS);
@@ -373,7 +389,7 @@ score_inv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (r < 0) continue;
         const float2 f0 = unpack2(acc2[i][0]);
         const float2 f1 = unpack2(acc2[i][1]);
-        const float score = (f0.x + f0.y) + (f1.x + f1.y);
+        const float score = ((f0.x + f0.y) + (f1.x + f1.y)) * kscale;
         const long long pos = p.q_offset + (r % p.T);
         const bool vis = tok < p.L && tok <= pos;
         p.out[static_cast<long long>(r) * p.ldo + static_cast<long long>(item_row(s.slots, i)) * p.blk + u * 128 +
@@ -415,43 +431,60 @@ __global__ void invert_count_kernel(const int* __restrict__ blocks, long long ro
 
 // One CTA: exclusive prefix sums of the counts (list starts) and of the items
 // per block (tiles x chunks); total items at ioff[nb]. Clears the cursors.
+// Each thread owns a contiguous run of blocks: it sums its run, one
+// block-wide scan of the run totals gives every run its start, and a second
+// pass over the run writes the starts.
 template <int NT>
 __global__ void __launch_bounds__(NT) invert_scan_kernel(const int* __restrict__ cnt, int nb, int tiles,
                                                           int qc, int* __restrict__ qoff, int* __restrict__ ioff,
                                                           int* __restrict__ cursor, long long* __restrict__ total) {
   __shared__ int wsum[2][NT / 32];
-  __shared__ int carry[2];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  if (threadIdx.x == 0) { carry[0] = 0; carry[1] = 0; }
+  const int E = (nb + NT - 1) / NT;
+  const int g0 = static_cast<int>(threadIdx.x) * E;
+  const int g1 = min(g0 + E, nb);
+  int sa = 0, sb = 0;
+  for (int g = g0; g < g1; ++g) {
+    const int c = cnt[g];
+    sa += c;
+    sb += tiles * ((c + qc - 1) / qc);
+  }
+  // inclusive scan of the run totals: within the warp, then over the warps
+  int a = sa, bi = sb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ya = __shfl_up_sync(0xffffffffu, a, o);
+    const int yb = __shfl_up_sync(0xffffffffu, bi, o);
+    if (lane >= o) { a += ya; bi += yb; }
+  }
+  if (lane == 31) { wsum[0][wid] = a; wsum[1][wid] = bi; }
   __syncthreads();
-  for (int base = 0; base < nb; base += NT) {
-    const int g = base + static_cast<int>(threadIdx.x);
-    const int c = g < nb ? cnt[g] : 0;
-    const int it = tiles * ((c + qc - 1) / qc);
-    int a = c, bi = it;
+  if (wid == 0) {
+    int wa = lane < NT / 32 ? wsum[0][lane] : 0;
+    int wb = lane < NT / 32 ? wsum[1][lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int ya = __shfl_up_sync(0xffffffffu, a, o);
-      const int yb = __shfl_up_sync(0xffffffffu, bi, o);
-      if (lane >= o) { a += ya; bi += yb; }
+      const int ya = __shfl_up_sync(0xffffffffu, wa, o);
+      const int yb = __shfl_up_sync(0xffffffffu, wb, o);
+      if (lane >= o) { wa += ya; wb += yb; }
     }
-    if (lane == 31) { wsum[0][wid] = a; wsum[1][wid] = bi; }
-    __syncthreads();
-    int pa = carry[0], pb = carry[1];
-    for (int w2 = 0; w2 < wid; ++w2) { pa += wsum[0][w2]; pb += wsum[1][w2]; }
-    if (g < nb) {
-      qoff[g] = pa + a - c;
-      ioff[g] = pb + bi - it;
-      cursor[g] = 0;
-    }
-    __syncthreads();
-    if (threadIdx.x == NT - 1) { carry[0] = pa + a; carry[1] = pb + bi; }
-    __syncthreads();
+    if (lane < NT / 32) { wsum[0][lane] = wa; wsum[1][lane] = wb; }
   }
-  if (threadIdx.x == 0) {
-    qoff[nb] = carry[0];
-    ioff[nb] = carry[1];
-    *total = carry[1];
+  __syncthreads();
+  int pa = (wid > 0 ? wsum[0][wid - 1] : 0) + a - sa;   // exclusive start of this run
+  int pb = (wid > 0 ? wsum[1][wid - 1] : 0) + bi - sb;
+  for (int g = g0; g < g1; ++g) {
+    const int c = cnt[g];
+    qoff[g] = pa;
+    ioff[g] = pb;
+    cursor[g] = 0;
+    pa += c;
+    pb += tiles * ((c + qc - 1) / qc);
+  }
+  if (threadIdx.x == NT - 1) {
+    qoff[nb] = wsum[0][NT / 32 - 1];
+    ioff[nb] = wsum[1][NT / 32 - 1];
+    *total = wsum[1][NT / 32 - 1];
   }
 }
 

@@ -57,7 +57,7 @@ struct ScoreParams {
   const float* k_scale; // [batch*Lk]   (FP8) or nullptr
   float* out;           // score: [batch*T, ldo]; router: 2 x [batch*T*H] partial sums
   long long ldo;
-  const __nv_bfloat16* kg;  // gather mode: keys [batch*L_tok, D]
+  const void* kg;           // gather mode: keys [batch*L_tok, D] (bf16 or e4m3)
   const int* cand;          // gather mode: [batch*T, n_slots] block / token ids, -1 = none
   int n_slots, blk, n_compact;  // compact position c -> cand[c / blk] * blk + c % blk
   int blk_tma;              // gather mode, blk % 128 == 0: a tile is one contiguous key run (TMA)
@@ -124,8 +124,7 @@ struct ScoreCfg {
   static constexpr int MMA_N = ROUTER ? KROWS : QROWS;
   static_assert(ROUTER ? QROWS == 128 : (QROWS % 16 == 0 && QROWS >= 32 && QROWS <= 256),
                 "bad tile shape");
-  static_assert(!GATHER || (QPT == 1 && ELEM == 2 && ROW_BYTES == 256),
-                "gather mode: one bf16 query per group, d = 128");
+  static_assert(!GATHER || (QPT == 1 && D == 128), "gather mode: one query per group, d = 128");
   // Gathers: the producer warps take tiles round robin. Stage s is refilled
   // for tile i only after the MMAs of tile i - NSTAGE are done, and the MMA
   // thread consumes tiles in order, so with NSTAGE >= NPROD a warp's wait on
@@ -164,8 +163,10 @@ struct ScoreCfg {
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_K = NQBUF * Q_BYTES;
   // FP8: the epilogue applies per-key dequant scales (loaded from global
-  // memory by the thread that owns the key, ahead of the tile's MMAs)
-  static constexpr bool KEY_SCALES = ELEM == 1 && !ROUTER && !GATHER;
+  // memory by the thread that owns the key, ahead of the tile's MMAs; for
+  // gathers, by the key's token). The router weights its pooled-key columns
+  // by their scales instead.
+  static constexpr bool KEY_SCALES = ELEM == 1 && !ROUTER;
   // per epilogue warp: the head weights (x query scales) of its columns for
   // the current query group, refilled when the group changes
   static constexpr int NCOL_THREAD = ROUTER ? 0 : (SPLIT_TILES ? QROWS : QROWS / NSETS);
@@ -490,9 +491,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       } else {
         // Gather 128 key rows (one per compact position) with 16-byte cp.async:
-        // a half-warp copies one 256-byte row, chunk c of row r lands at its
-        // 128-byte-swizzle slot (c ^ (r & 7)) so the tensor core sees the same
-        // layout a TMA load would have written. Rows without a visible token
+        // RCH lanes copy one row (16 for a 256-byte bf16 row, 8 for a
+        // 128-byte FP8 row), chunk c of row r lands at its 128-byte-swizzle
+        // slot (c ^ (r & 7)) of column block c / 8, so the tensor core sees the
+        // same layout a TMA load would have written. Rows without a visible token
         // are zero-filled by the same instruction (nothing is read).
         // The tile's 128 token ids are resolved first (lane l owns rows l,
         // l+32, l+64, l+96: four independent loads), then handed to the
@@ -507,22 +509,25 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int u = 0; u < 4; ++u) toks[u] = gathered_token(p, r, s.j * C::KROWS + 32 * u + lane, q_pos);
         if (!mbar_wait(empty(stage), ph ^ 1u, p.err)) ok = false;
         if (ok) {
-          const int ch = lane & 15;
+          constexpr int RCH = C::ROW_BYTES / 16;  // lanes (16-byte chunks) per row
+          constexpr int RPI = 32 / RCH;           // rows per warp instruction
+          const int ch = lane % RCH;
           const uint32_t tile = s_k + stage * C::K_BYTES + (ch >> 3) * C::KROWS * 128;
           // per lane: the global address of its four rows and which of them exist
-          const __nv_bfloat16* kseq = p.kg + static_cast<long long>(b) * p.L_tok * C::D;
+          const char* kseq = reinterpret_cast<const char*>(p.kg) +
+                             static_cast<long long>(b) * p.L_tok * C::ROW_BYTES;
           unsigned long long ga[4];
           uint32_t vm[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             vm[u] = __ballot_sync(0xffffffffu, toks[u] >= 0);
-            ga[u] = reinterpret_cast<unsigned long long>(kseq + (toks[u] >= 0 ? toks[u] : 0) * C::D);
+            ga[u] = reinterpret_cast<unsigned long long>(kseq + (toks[u] >= 0 ? toks[u] : 0) * C::ROW_BYTES);
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int rl = 2 * i + (lane >> 4);  // row 32u + rl lives in lane rl
+            for (int i = 0; i < 32 / RPI; ++i) {
+              const int rl = RPI * i + lane / RCH;  // row 32u + rl lives in lane rl
               const int row = 32 * u + rl;
               const unsigned long long a = __shfl_sync(0xffffffffu, ga[u], rl);
               const uint32_t dst = tile + row * 128 + (((ch & 7) ^ (rl & 7)) << 4);
@@ -640,7 +645,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         // FP8: this row's key dequant scale, likewise
         float ks = 1.f;
-        if constexpr (C::KEY_SCALES) {
+        if constexpr (C::KEY_SCALES && C::GATHER) {
+          if (gtok >= 0) ks = __ldg(p.k_scale + static_cast<long long>(b) * p.L_tok + gtok);
+        } else if constexpr (C::KEY_SCALES) {
           const int skey = s.j * C::KROWS + row;
           if (skey < p.Lk) ks = __ldg(p.k_scale + static_cast<long long>(b) * p.Lk + skey);
         }
@@ -676,7 +683,15 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int cc = 0; cc < C::KROWS; cc += 32) {
             float v[32];
             tmem_ld32(taddr + cc, v);
-            if (m0 + cc + 32 <= mv) {
+            if constexpr (C::ELEM == 1) {
+              // FP8 pooled keys: column m carries its dequant scale (>= 0, so
+              // it moves out of the ReLU); lane i loads column cc + i's, 0 for
+              // columns past the visible ones
+              const long long mc = m0 + cc + lane;
+              const float kl = mc < mv ? __ldg(p.k_scale + static_cast<long long>(b) * p.Lk + mc) : 0.f;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) part = fmaf(__shfl_sync(0xffffffffu, kl, i), fmaxf(v[i], 0.f), part);
+            } else if (m0 + cc + 32 <= mv) {
 #pragma unroll
               for (int i = 0; i < 32; ++i) part += fmaxf(v[i], 0.f);
             } else {
@@ -693,6 +708,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           static_assert(QH == QHT, "threshold slots");
           constexpr int NC = QH * C::H;                          // columns per thread
           constexpr int NCH = NC / 32;                           // 32-column chunks
+          static_assert(NC % 32 == 0 && NCH >= 1, "each epilogue thread takes whole 32-column chunks");
           // independent partial sums per query (breaks the FMA dependency chain)
 #if defined(DSA_NO_FFMA2)
           constexpr int NP = C::H >= 32 ? 4 : (C::H == 16 ? 2 : 1);
@@ -815,7 +831,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           if (C::GATHER) {
             const long long r = static_cast<long long>(b) * p.T + tg;
-            if (key < p.n_compact) p.out[r * p.ldo + key] = gtok >= 0 ? accq[0] : -INFINITY;
+            if (key < p.n_compact) p.out[r * p.ldo + key] = gtok >= 0 ? ks * accq[0] : -INFINITY;
           } else {
             // query q0+ql sees this key iff key * pstride <= q_offset + t0 + ql
             const int t0 = tg * C::QPT + q0;
@@ -823,8 +839,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if constexpr (C::BND) {
               // DoSA: bound >= threshold for some visible key of the warp ->
               // the tile is live for the query's refinement group
-#pragma unroll
               uint32_t lmask = 0;  // bit ql: this key is live for query ql
+#pragma unroll
               for (int ql = 0; ql < QH; ++ql) {
                 const float2 tc = *reinterpret_cast<const float2*>(cw + NC + 2 * ql);  // (thr, c_t)
                 const bool live = key < p.Lk && e <= ql && fmaf(tc.y, kn, accq[ql]) >= tc.x;

@@ -86,8 +86,10 @@ def test_variant_argument_checks(lib):
     assert lib.misa_route_score_topk(ctypes.byref(a), 64, 65, 16, 0, out, None, None, None, ws, big, None) == -1
     assert lib.misa_route_score_topk(ctypes.byref(a), 64, 12, 16, 0, out, None, None, None, ws, big, None) == -2
     assert lib.misa_route_score_topk(ctypes.byref(a), 0, 8, 16, 0, out, None, None, None, ws, big, None) == -1
-    # MISA is bf16 only
-    f = _args(qk_dtype=B.DSA_FP8_E4M3, q_scale=0x60000, k_scale=0x70000)
+    # FP8 MISA: d = 128 and H in {32, 64} only (rejected before any launch)
+    f = _args(qk_dtype=B.DSA_FP8_E4M3, q_scale=0x60000, k_scale=0x70000, H=16)
+    assert lib.misa_route_score_topk(ctypes.byref(f), 64, 8, 16, 0, out, None, None, None, ws, big, None) == -2
+    f = _args(qk_dtype=B.DSA_FP8_E4M3, q_scale=0x60000, k_scale=0x70000, d=64)
     assert lib.misa_route_score_topk(ctypes.byref(f), 64, 8, 16, 0, out, None, None, None, ws, big, None) == -2
     assert lib.hisa_block_filter_topk(ctypes.byref(a), 128, 0, 16, out, None, None, ws, big, None) == -1
     h8 = _args(H=8)
@@ -113,7 +115,7 @@ def test_stage_entry_point_checks(lib):
     assert lib.indexer_score_gathered(ctypes.byref(a), cand, 8, 128, out, 1000, ws, big, None) == -1
     assert lib.indexer_score_gathered(ctypes.byref(_args(H=16)), cand, 8, 1, out, 8, ws, big, None) == -2
     assert lib.indexer_score_gathered(ctypes.byref(_args(d=64)), cand, 8, 1, out, 8, ws, big, None) == -2
-    f = _args(qk_dtype=B.DSA_FP8_E4M3, q_scale=0x60000, k_scale=0x70000)
+    f = _args(qk_dtype=B.DSA_FP8_E4M3, q_scale=0x60000, k_scale=0x70000, H=8)
     assert lib.indexer_score_gathered(ctypes.byref(f), cand, 8, 1, out, 8, ws, big, None) == -2
     # indexer_topk_rows: pitch below the row, index map shorter than the row,
     # k out of range, negative position stride
@@ -170,6 +172,8 @@ def test_hisa_refine_checks(lib):
     assert lib.hisa_refine_scores(ctypes.byref(a), None, 4, 128, out, 512, ws, big, None) == -1
     assert lib.hisa_refine_scores(ctypes.byref(a), blocks, 4, 128, out, 511, ws, big, None) == -1  # ld < m*blk
     assert lib.hisa_refine_scores(ctypes.byref(a), blocks, 4, 96, out, 512, ws, big, None) == -2  # blk % 128
+    f8 = _args(L=1000, q_offset=996, qk_dtype=B.DSA_FP8_E4M3, q_scale=0x60000, k_scale=0x70000)
+    assert lib.hisa_block_filter_topk(ctypes.byref(f8), 96, 4, 16, out, None, None, ws, big, None) == -2
     assert lib.hisa_refine_scores(ctypes.byref(_args(H=16, L=1000, q_offset=996)), blocks, 4, 128, out, 512,
                                   ws, big, None) == -2
     assert lib.hisa_refine_scores(ctypes.byref(a), blocks, 4, 128, out, 512, ws, need - 1, None) == -3

@@ -10,7 +10,7 @@ from sparse_attention_token_score_b200 import workloads as wl
 
 
 @pytest.mark.parametrize("name", ["tiny", "dsa", "decode", "misa", "hisa", "dsa_fp8", "indexcache", "dosa",
-                                  "dosa_lownorm", "dsa_lists"])
+                                  "dosa_lownorm", "dsa_lists", "hisa_decode"])
 def test_pairs_are_the_dense_visible_pairs(name):
     c, batch, off, pairs, label = bench.workload_desc(name)
     T = c["T"]
@@ -20,7 +20,8 @@ def test_pairs_are_the_dense_visible_pairs(name):
     assert label.startswith({"tiny": "tiny_prefill", "dsa": "dsa_chunk", "decode": "decode_fp8",
                               "misa": "misa_dagger", "hisa": "hisa", "dsa_fp8": "dsa_chunk_fp8",
                               "indexcache": "indexcache_dsa_chunk", "dosa": "dosa_dsa_chunk",
-                              "dosa_lownorm": "dosa_lownorm_dsa_chunk", "dsa_lists": "dsa_chunk_lists"}[name])
+                              "dosa_lownorm": "dosa_lownorm_dsa_chunk", "dsa_lists": "dsa_chunk_lists",
+                              "hisa_decode": "hisa_decode_fp8"}[name])
 
 
 def test_dsa_chunk_size():

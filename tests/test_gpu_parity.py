@@ -413,7 +413,7 @@ def _heads_check(gpu_heads, aff, h, what):
         check_selection(gpu_heads[i], np.arange(aff.shape[1]), aff[i], aff[i], h, what=f"{what} heads {i}")
 
 
-def _misa_check(inp, block, h, topk, kprime, queries, what, batches=(0,), stats=None):
+def _misa_check(inp, block, h, topk, kprime, queries, what, batches=(0,), stats=None, rtol=RTOL_BF16):
     ix = _indexer(inp)
     IDX, SC, HEADS, CAND = ix.misa(block, h, topk, kprime, with_score=True, with_heads=True,
                                    with_cand=True)
@@ -421,10 +421,11 @@ def _misa_check(inp, block, h, topk, kprime, queries, what, batches=(0,), stats=
     for b in batches:
         _misa_check_one(inp, block, h, topk, kprime, queries, f"{what} b={b}", b,
                         IDX.cpu().numpy()[b], SC.cpu().numpy()[b], HEADS.cpu().numpy()[b],
-                        CAND.cpu().numpy()[b] if CAND is not None else None, stats)
+                        CAND.cpu().numpy()[b] if CAND is not None else None, stats, rtol)
 
 
-def _misa_check_one(inp, block, h, topk, kprime, queries, what, b, idx, sc, heads, cand, stats=None):
+def _misa_check_one(inp, block, h, topk, kprime, queries, what, b, idx, sc, heads, cand, stats=None,
+                    rtol=RTOL_BF16):
     qs = np.asarray(queries)
     free = oracle.misa(inp, block, h, topk, kprime=0, queries=qs, b=b)
     _heads_check(heads[qs], free["affinity"], h, what)
@@ -437,7 +438,7 @@ def _misa_check_one(inp, block, h, topk, kprime, queries, what, b, idx, sc, head
             s, c = cond["routed_scores"][i], cond["routed_cond"][i]
             check_selection(idx[t], np.arange(V), s, c, topk, what=f"{what} t={t}", stats=stats)
             n = min(topk, V)
-            check_scores(sc[t, :n], s[idx[t, :n]], c[idx[t, :n]], RTOL_BF16, what=f"{what} t={t}",
+            check_scores(sc[t, :n], s[idx[t, :n]], c[idx[t, :n]], rtol, what=f"{what} t={t}",
                          stats=stats)
         else:
             check_selection(cand[t], np.arange(V), cond["routed_scores"][i], cond["routed_cond"][i],
@@ -447,7 +448,7 @@ def _misa_check_one(inp, block, h, topk, kprime, queries, what, b, idx, sc, head
             check_selection(idx[t], cv, s, c, topk, what=f"{what} t={t}", stats=stats)
             n = min(topk, cv.size)
             where = np.searchsorted(cv, idx[t, :n])
-            check_scores(sc[t, :n], s[where], c[where], RTOL_BF16, what=f"{what} scores t={t}", stats=stats)
+            check_scores(sc[t, :n], s[where], c[where], rtol, what=f"{what} scores t={t}", stats=stats)
 
 
 @pytest.mark.parametrize("kprime", [0, 400])
@@ -473,6 +474,35 @@ def test_misa_h8_head_dim_64():
     # router with 16 queries x 8 heads per row tile, d = 64, plain MISA
     inp = wl.prefill_inputs(40, 1500, 8, 64, q_offset=1460, seed=27)
     _misa_check(inp, block=32, h=8, topk=64, kprime=0, queries=range(40), what="misa h8 d64")
+
+
+@pytest.mark.parametrize("kprime", [0, 500])
+def test_misa_fp8_prefill(kprime):
+    # FP8 cache: e4m3 pooled keys with per-block scales in the router, e4m3
+    # routed pass with the kept heads' query scales, FP8 token gathers
+    inp = wl.fp8_prefill_inputs(40, 3000, 64, 128, q_offset=2960, seed=131, w_std=0.125)
+    _misa_check(inp, block=64, h=8, topk=100, kprime=kprime, queries=range(40), what=f"misa fp8 k'={kprime}",
+                rtol=RTOL_FP8)
+
+
+def test_misa_fp8_decode_batch():
+    # the decode key cache (one query per sequence at L-1); H = 64 with 8
+    # routed heads, H = 32 with 16
+    for H, h in ((64, 8), (32, 16)):
+        inp = wl.decode_inputs(batch=4, L=5000, H=H, d=128, seed=140 + H, cluster_frac=0.05)
+        _misa_check(inp, block=64, h=h, topk=150, kprime=600, queries=[0], what=f"misa fp8 decode H={H}",
+                    batches=(0, 1, 2, 3), rtol=RTOL_FP8)
+
+
+def test_misa_fp8_all_heads_equals_dense_gpu():
+    inp = wl.decode_inputs(batch=3, L=3000, H=32, d=128, seed=133)
+    ix = _indexer(inp)
+    d_idx, d_sc = ix.dense(64, with_score=True)
+    m_idx, m_sc, heads, _ = ix.misa(64, 32, 64, 0, with_score=True, with_heads=True)
+    assert ix.device_status() == 0
+    assert torch.equal(heads[:, 0], torch.arange(32, dtype=torch.int32, device="cuda").expand(3, 32))
+    assert torch.equal(d_idx, m_idx)
+    assert torch.equal(d_sc, m_sc)
 
 
 def test_misa_all_heads_equals_dense_gpu():
@@ -514,16 +544,16 @@ def test_misa_plain_config_sampled():
 
 
 # ------------------------------------------------------------------ HISA
-def _hisa_check(inp, block, m, topk, queries, what, batches=(0,), stats=None):
+def _hisa_check(inp, block, m, topk, queries, what, batches=(0,), stats=None, rtol=RTOL_BF16):
     ix = _indexer(inp)
     IDX, SC, BLOCKS = ix.hisa(block, m, topk, with_score=True, with_blocks=True)
     assert ix.device_status() == 0
     for b in batches:
         _hisa_check_one(inp, block, m, topk, queries, f"{what} b={b}", b, IDX.cpu().numpy()[b],
-                        SC.cpu().numpy()[b], BLOCKS.cpu().numpy()[b], stats)
+                        SC.cpu().numpy()[b], BLOCKS.cpu().numpy()[b], stats, rtol)
 
 
-def _hisa_check_one(inp, block, m, topk, queries, what, b, idx, sc, blocks, stats=None):
+def _hisa_check_one(inp, block, m, topk, queries, what, b, idx, sc, blocks, stats=None, rtol=RTOL_BF16):
     qs = np.asarray(queries)
     free = oracle.hisa(inp, block, m, topk, queries=qs, b=b)
     for i, t in enumerate(qs):
@@ -536,7 +566,22 @@ def _hisa_check_one(inp, block, m, topk, queries, what, b, idx, sc, blocks, stat
         check_selection(idx[t], toks, s, c, topk, what=f"{what} t={t}", stats=stats)
         n = min(topk, toks.size)
         where = np.searchsorted(toks, idx[t, :n])
-        check_scores(sc[t, :n], s[where], c[where], RTOL_BF16, what=f"{what} scores t={t}", stats=stats)
+        check_scores(sc[t, :n], s[where], c[where], rtol, what=f"{what} scores t={t}", stats=stats)
+
+
+def test_hisa_fp8_prefill():
+    # FP8 cache: pooled keys in e4m3 + per-block scale, FP8 block scores,
+    # FP8 block-major refinement
+    inp = wl.fp8_prefill_inputs(30, 5000, 32, 128, q_offset=4970, seed=17)
+    _hisa_check(inp, block=128, m=8, topk=300, queries=range(30), what="hisa fp8", rtol=RTOL_FP8)
+
+
+def test_hisa_fp8_decode_batch():
+    # the decode key cache (one query per sequence at L-1), H = 64 and 32
+    for H in (64, 32):
+        inp = wl.decode_inputs(batch=4, L=6000, H=H, d=128, seed=96 + H, cluster_frac=0.05)
+        _hisa_check(inp, block=128, m=12, topk=200, queries=[0], what=f"hisa fp8 decode H={H}",
+                    batches=(0, 1, 2, 3), rtol=RTOL_FP8)
 
 
 def test_hisa_small():
@@ -598,6 +643,14 @@ def test_gathered_scores_elementwise(blk, n_slots):
             assert np.all(np.isneginf(out[r][~ok]))
             s_, c_ = oracle.score_pairs(q, k, w, np.full(ok.sum(), t), tok[ok])
             check_scores(out[r][ok], s_, c_, RTOL_BF16, what=f"gathered blk={blk} r={r}")
+
+
+def test_misa_hisa_on_a_decode_batch():
+    # decode shape: independent sequences with one query each at position L-1
+    # (bf16 key caches): the routed, dagger and hierarchical paths per sequence
+    inp = wl.prefill_inputs(1, 6000, 32, 128, q_offset=5999, seed=95, batch=4)
+    _misa_check(inp, block=64, h=8, topk=200, kprime=800, queries=[0], what="misa decode", batches=(0, 1, 2, 3))
+    _hisa_check(inp, block=128, m=12, topk=200, queries=[0], what="hisa decode", batches=(0, 1, 2, 3))
 
 
 # ------------------------------------------------------------------ HISA refinement, block major

@@ -507,3 +507,72 @@ def test_dosa_tile_planted_mistake_is_caught(monkeypatch):
     dense = oracle.dense_topk(inp, 16)
     got = oracle.dosa_tile_topk(inp, 16, 1, 16, 4)
     assert not np.array_equal(dense["idx"], got["idx"])
+
+
+# ------------------------------------------------------------ FP8 pooled keys
+def test_e4m3_encoder_is_nearest_even_and_matches_torch():
+    import torch
+    # exact midpoints go to the even code: 1.0625 between 1.0 (0x38) and 1.125 (0x39)
+    assert oracle.f64_to_e4m3(np.array([1.0625, -1.0625, 1.1875]))[:3].tolist() == [0x38, 0xB8, 0x3A]
+    assert oracle.f64_to_e4m3(np.array([1000.0, -1000.0, 0.0]))[:3].tolist() == [0x7E, 0xFE, 0x00]
+    x = np.random.default_rng(3).standard_normal(20000).astype(np.float32) * np.float32(40.0)
+    ref = torch.from_numpy(np.clip(x, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.f64_to_e4m3(x.astype(np.float64)), ref)
+    # every code decodes and re-encodes to itself
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    back = oracle.f64_to_e4m3(oracle.decode_e4m3(codes))
+    assert np.array_equal(back[codes != 0x80], codes[codes != 0x80])
+
+
+def test_meanpool_e4m3_closed_form():
+    # block of two tokens (scale 1): the mean (2, 1, -0.5, 0, ...) is representable
+    # after scaling by amax / 448 = 2 / 448, so it decodes back exactly
+    d = 16
+    k = np.zeros((4, d), dtype=np.float64)
+    k[0, :3], k[1, :3] = [1.0, 0.5, -0.25], [3.0, 1.5, -0.75]
+    k[2:] = 0.0                                       # an all-zero block: scale 1, codes 0
+    codes = oracle.f64_to_e4m3(k)
+    got, sc = oracle.meanpool_e4m3(codes, np.ones(4, dtype=np.float32), 2)
+    assert sc[0] == np.float32(2.0) / np.float32(448.0) and sc[1] == np.float32(1.0)
+    # mean / scale = (448, 224, -112) up to the fp32 rounding of the scale
+    assert got[0][:3].tolist() == oracle.f64_to_e4m3(np.array([448.0, 224.0, -112.0])).tolist()
+    mean = oracle.decode_e4m3(got[0]) * np.float64(sc[0])
+    assert np.allclose(mean[:3], [2.0, 1.0, -0.5], rtol=1e-6, atol=0) and np.all(mean[3:] == 0)
+    assert np.all(got[1] == 0)
+
+
+def test_hisa_fp8_all_blocks_is_dense():
+    inp = wl.decode_inputs(batch=2, L=900, H=32, d=128, seed=77)
+    for b in range(2):
+        dense = oracle.dense_topk(inp, 40, b=b)
+        h = oracle.hisa(inp, 128, 8, 40, b=b)   # 8 blocks of 128 cover all 900 keys
+        assert np.array_equal(dense["idx"], h["idx"])
+
+
+def test_misa_fp8_all_heads_and_all_candidates_are_dense():
+    # MISA on an FP8 cache reduces to the dense FP8 indexer when every head is
+    # routed (h = H) or every visible key is a MISA-dagger candidate (k' >= V)
+    inp = wl.decode_inputs(batch=2, L=700, H=32, d=128, seed=78)
+    for b in range(2):
+        dense = oracle.dense_topk(inp, 30, b=b)
+        m = oracle.misa(inp, 64, 32, 30, b=b)
+        assert np.array_equal(dense["idx"], m["idx"])
+        assert np.array_equal(m["routed_scores"][0], dense["scores"][0])
+        md = oracle.misa(inp, 64, 4, 30, kprime=700, b=b)
+        assert np.array_equal(dense["idx"], md["idx"])
+
+
+def test_misa_fp8_router_brute_force():
+    # affinity of every head from the decoded pooled keys, summed by hand
+    inp = wl.decode_inputs(batch=1, L=300, H=32, d=128, seed=79)
+    q, k, w = oracle.dequant(inp)
+    m = oracle.misa(inp, 64, 3, 10)
+    codes, scales = m["kbar_bits"]
+    assert codes.shape == (5, 128) and scales.shape == (5,)
+    kbar = oracle.decode_e4m3(codes) * scales.astype(np.float64)[:, None]
+    p = inp.q_offset                        # one query, at the end of the cache
+    nb = p // 64 + 1
+    aff = [abs(w[0, h]) * sum(max(0.0, float(q[0, h] @ kbar[j])) for j in range(nb)) for h in range(32)]
+    assert np.allclose(m["affinity"][0], aff, rtol=1e-12, atol=0)
+    want = sorted(range(32), key=lambda h: (-aff[h], h))[:3]
+    assert sorted(m["heads"][0].tolist()) == sorted(want)
