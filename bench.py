@@ -78,12 +78,14 @@ def workload_desc(name, queries=None, batch=None):
            "misa": "misa_dagger", "hisa": "hisa", "dsa_fp8": "dsa_chunk_fp8",
            "indexcache": "indexcache_dsa_chunk", "dosa": "dosa_dsa_chunk",
            "dosa_lownorm": "dosa_lownorm_dsa_chunk", "dsa_lists": "dsa_chunk_lists",
-           "hisa_decode": "hisa_decode_fp8"}[name]
+           "hisa_decode": "hisa_decode_fp8", "misa_decode": "misa_dagger_decode_fp8"}[name]
     label = f"{tag}_B{batch}_T{c['T']}_L{c['L']}_H{c['H']}_d{c['d']}_k{c['topk']}"
-    if name == "misa":
+    if name in ("misa", "misa_decode"):
         label += f"_blk{c['block']}_h{c['h']}_kp{c['kprime']}"
     if name in ("hisa", "hisa_decode"):
         label += f"_blk{c['block']}_m{c['m']}"
+    if name in POOLED_CACHE:  # pooled keys kept across steps, the last block re-pooled per step
+        label += "_pooledcache"
     if name == "indexcache":
         label += f"_layers{c['pattern']}"
     if name in ("dosa", "dosa_lownorm"):
@@ -94,6 +96,7 @@ def workload_desc(name, queries=None, batch=None):
 DENSE = ("tiny", "dsa", "decode", "dsa_fp8", "indexcache")  # workloads whose F layer is indexer_score_topk
 DOSA = ("dosa", "dosa_lownorm")                              # dosa_score_topk
 LISTS = ("dsa_lists",)                                       # indexer_score_topk_lists
+POOLED_CACHE = ("hisa_decode", "misa_decode")                # *_pooled calls on a pooled-key cache
 
 
 class Runner:
@@ -125,10 +128,17 @@ class Runner:
             self.live = torch.empty((self.batch, -(-c["T"] // qpt), -(-c["L"] // 128)), dtype=torch.uint8,
                                     device="cuda")
             self.live_pairs = None
-        elif name == "misa":
+        elif name in ("misa", "misa_decode"):
             self.ws = B.alloc_workspace(B.misa_workspace_size(a, c["block"], c["h"], self.topk, c["kprime"]))
         else:
             self.ws = B.alloc_workspace(B.hisa_workspace_size(a, c["block"], c["m"], self.topk))
+        if name in POOLED_CACHE:
+            # decode: the pooled keys live in a cache next to the key cache;
+            # completed blocks are pooled once (here), the last block again
+            # at every step
+            self.M = -(-c["L"] // c["block"])
+            self.kbar, self.ksc = B.pooled_cache(a, c["block"], device="cuda")
+            B.dsa_pool_keys(a, c["block"], 0, self.M, self.kbar, self.ksc)
         self.dtype = "e4m3" if inp.dtype != "bf16" else "bf16"
 
     def step(self, args=None, out=None):
@@ -145,6 +155,14 @@ class Runner:
             B.indexer_score_topk_lists(a, self.topk, o, None, self.ws)
         elif self.name in DOSA:
             B.dosa_score_topk(a, self.topk, c["n_screen"], o, None, self.live, self.ws)
+        elif self.name in POOLED_CACHE:
+            B.dsa_pool_keys(a, c["block"], self.M - 1, self.M, self.kbar, self.ksc)
+            if self.name == "misa_decode":
+                B.misa_route_score_topk_pooled(a, c["block"], c["h"], self.topk, c["kprime"], self.kbar, self.ksc,
+                                               o, None, None, None, self.ws)
+            else:
+                B.hisa_block_filter_topk_pooled(a, c["block"], c["m"], self.topk, self.kbar, self.ksc, o, None,
+                                                None, self.ws)
         elif self.name == "misa":
             B.misa_route_score_topk(a, c["block"], c["h"], self.topk, c["kprime"], o, None, None,
                                     None, self.ws)
@@ -178,18 +196,21 @@ class Runner:
                 return pairs * 2.0 * d * H, ("tensor_fp8" if self.name == "dsa_fp8" else "tensor")
             if label == "topk_rows":
                 return pairs * 4 + rows * k * 4, "hbm"    # every visible score read, k ids written
-        if self.name == "misa":
+        if self.name in ("misa", "misa_decode"):
+            fp8 = self.name == "misa_decode"
             blk, h, kp = c["block"], c["h"], c["kprime"]
             M = -(-L // blk)
             vis_blocks = int(self.batch * np.minimum(pos // blk + 1, M).sum())
             if stage == "router" and label.startswith("score_tc"):
-                return vis_blocks * 2.0 * d * H, "tensor"
+                return vis_blocks * 2.0 * d * H, "tensor_fp8" if fp8 else "tensor"
             if stage == "routed" and label.startswith("score_tc"):
+                if fp8:                                    # the key stream: one FP8 row + scale per pair
+                    return self.pairs * (d + 4), "hbm"
                 return self.pairs * 2.0 * d * h, "tensor"
             if stage == "routed" and label == "topk_rows":
                 return self.pairs * 4 + rows * kp * 4, "hbm"
             if stage == "re-score" and label.startswith("score_tc"):
-                return rows * kp * 2.0 * d * H, "tensor"
+                return rows * kp * 2.0 * d * H, "tensor_fp8" if fp8 else "tensor"
             if stage == "re-score" and label == "topk_rows":
                 return rows * kp * 4 + rows * k * 8, "hbm"
         if self.name in ("hisa", "hisa_decode"):
@@ -244,6 +265,7 @@ TRAFFIC = {
 }
 KERNEL_SOURCES = {
     "score_tc": ("score_tc.cuh", "common.cuh"),
+    "score_inv": ("score_inv.cuh", "common.cuh"),
     "topk_rows": ("topk.cuh",),  # the top-k uses none of common.cuh's helpers
 }
 
@@ -252,7 +274,9 @@ def source_hash(kernel_name):
     """Hash of the kernel's source lines, full-line comments and blank lines
     excluded (a comment edit does not invalidate a capture)."""
     import hashlib
-    fam = "topk_rows" if kernel_name.startswith("topk_rows") else "score_tc"
+    label = kernel_name.split(": ")[-1]
+    fam = "topk_rows" if label.startswith("topk_rows") else ("score_inv" if label.startswith("score_inv")
+                                                             else "score_tc")
     h = hashlib.sha1()
     for f in KERNEL_SOURCES[fam]:
         with open(os.path.join(ROOT, "sparse_attention_token_score_b200", "csrc", f)) as fh:
@@ -450,7 +474,7 @@ def oracle_sample(name, inp, budget_s=10.0, max_q=4096, with_pairs=False):
 
     def run(qs, b=0):
         t0 = time.perf_counter()
-        if name == "misa":
+        if name in ("misa", "misa_decode"):
             oracle.misa(inp, c["block"], c["h"], c["topk"], kprime=c["kprime"], queries=qs, b=b)
         elif name in ("hisa", "hisa_decode"):
             oracle.hisa(inp, c["block"], c["m"], c["topk"], queries=qs, b=b)
@@ -464,7 +488,7 @@ def oracle_sample(name, inp, budget_s=10.0, max_q=4096, with_pairs=False):
         off = inp.q_offset
         return int(sum(min(off + int(t) + 1, inp.L) for t in qs)) * len(c.get("pattern", "F"))
 
-    if name in ("decode", "hisa_decode"):
+    if name in ("decode", "hisa_decode", "misa_decode"):
         # one unit = one sequence's query; add sequences until budget_s is spent
         t, nb = 0.0, 0
         while t < budget_s and nb < inp.batch:
@@ -550,8 +574,8 @@ def make_inputs(name, seed, queries=0, batch=0):
 
 
 # ------------------------------------------------------------------ main
-SUB_WORKLOADS = ("tiny", "decode", "misa", "hisa", "hisa_decode", "dsa_fp8", "indexcache", "dsa_lists", "dosa",
-                 "dosa_lownorm")
+SUB_WORKLOADS = ("tiny", "decode", "misa", "hisa", "hisa_decode", "misa_decode", "dsa_fp8", "indexcache",
+                 "dsa_lists", "dosa", "dosa_lownorm")
 MIN_TIMED_MS = 60.0  # sub-records run enough steps that the clock sampler sees the GPU busy
 
 
@@ -673,7 +697,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="all", choices=["all", "tiny", "dsa", "decode", "misa", "hisa", "dsa_fp8", "indexcache", "dosa",
-                             "dosa_lownorm", "dsa_lists", "hisa_decode"],
+                             "dosa_lownorm", "dsa_lists", "hisa_decode", "misa_decode"],
                     help="all (default): the dsa chunk is the headline line, the other four "
                          "workloads are measured in the same run under 'workloads'")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -252,6 +252,40 @@ DSA_EXPORT dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int bloc
                                   int32_t* out_idx, float* out_score, int32_t* out_blocks,
                                   void* workspace, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------ pooled-key cache
+ * The pooled keys MISA and HISA read depend only on the key cache, and a
+ * completed block's pooled key never changes: a decode loop can keep them
+ * (pool each block once, the last, still growing block again at each step)
+ * instead of pooling the whole cache at every call.
+ *
+ * dsa_pool_keys: pools blocks m0 .. min(m1, M) - 1 of every sequence of
+ * a->k (M = ceil(L / block)) into the cache, in the form the *_pooled calls
+ * read:
+ *   bf16:  kbar [batch, M, d] bf16 (as dsa_meanpool_keys); kbar_scale unused (may be NULL)
+ *   FP8:   kbar [batch, M, d] e4m3 codes and kbar_scale [batch, M] fp32, the
+ *          format described under misa_route_score_topk (fp64 mean of the
+ *          dequantised keys, scale absmax/448, codes of mean / scale)
+ * Entries outside [m0, m1) are left untouched. kbar: 16-byte aligned.
+ * DSA_ERR_ARG for m0 < 0, m1 < m0 or a missing buffer.
+ *
+ * misa_route_score_topk_pooled / hisa_block_filter_topk_pooled: the same as
+ * misa_route_score_topk / hisa_block_filter_topk (same outputs, same
+ * workspace size), reading the pooled keys from kbar / kbar_scale (every
+ * block of every sequence, as dsa_pool_keys writes them) instead of pooling
+ * the key cache. The result equals the unpooled call's bit for bit when the
+ * cache holds the pooled keys of the current a->k. */
+DSA_EXPORT dsa_status dsa_pool_keys(const dsa_indexer_args* a, int block, int m0, int m1, void* kbar,
+                                    float* kbar_scale, void* stream);
+DSA_EXPORT dsa_status misa_route_score_topk_pooled(const dsa_indexer_args* a, int block, int h, int topk,
+                                                   int kprime, const void* kbar, const float* kbar_scale,
+                                                   int32_t* out_idx, float* out_score, int32_t* out_heads,
+                                                   int32_t* out_cand, void* workspace, size_t ws_bytes,
+                                                   void* stream);
+DSA_EXPORT dsa_status hisa_block_filter_topk_pooled(const dsa_indexer_args* a, int block, int m, int topk,
+                                                    const void* kbar, const float* kbar_scale, int32_t* out_idx,
+                                                    float* out_score, int32_t* out_blocks, void* workspace,
+                                                    size_t ws_bytes, void* stream);
+
 /* HISA token refinement alone (HISA review, section 3 and Figure 1), block
  * major: the kept blocks [batch*T, m] (block ids, -1 = empty slot) are
  * inverted into per-block lists of the queries that kept them, and each kept

@@ -75,6 +75,11 @@ _SIGS = {
     "hisa_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "hisa_block_filter_topk": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P,
                                               _P, _P, _P, ctypes.c_size_t, _P]),
+    "dsa_pool_keys": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P]),
+    "misa_route_score_topk_pooled": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                    _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "hisa_block_filter_topk_pooled": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P,
+                                                     _P, _P, _P, _P, ctypes.c_size_t, _P]),
 }
 
 
@@ -240,6 +245,44 @@ def hisa_block_filter_topk(args: IndexerArgs, block: int, m: int, topk: int, out
            lib().hisa_block_filter_topk(ctypes.byref(args), block, m, topk, _ptr(out_idx),
                                         _ptr(out_score), _ptr(out_blocks), _ptr(workspace),
                                         workspace.numel(), _stream_ptr(stream)))
+
+
+def pooled_cache(args: IndexerArgs, block: int, device=None):
+    """Empty pooled-key cache buffers for dsa_pool_keys: (kbar, kbar_scale);
+    kbar is bf16 [batch, M, d] or, for an FP8 cache, uint8 codes [batch, M, d]
+    with fp32 scales [batch, M]."""
+    M = -(-args.L // block)
+    fp8 = args.qk_dtype == DSA_FP8_E4M3
+    kbar = torch.empty((args.batch, M, args.d), dtype=torch.uint8 if fp8 else torch.bfloat16, device=device)
+    scale = torch.empty((args.batch, M), dtype=torch.float32, device=device) if fp8 else None
+    return kbar, scale
+
+
+def dsa_pool_keys(args: IndexerArgs, block: int, m0: int, m1: int, kbar: torch.Tensor,
+                  kbar_scale: Optional[torch.Tensor], stream=None):
+    _check("dsa_pool_keys", lib().dsa_pool_keys(ctypes.byref(args), block, m0, m1, _ptr(kbar), _ptr(kbar_scale),
+                                                _stream_ptr(stream)))
+
+
+def misa_route_score_topk_pooled(args: IndexerArgs, block: int, h: int, topk: int, kprime: int,
+                                 kbar: torch.Tensor, kbar_scale: Optional[torch.Tensor], out_idx: torch.Tensor,
+                                 out_score: Optional[torch.Tensor], out_heads: Optional[torch.Tensor],
+                                 out_cand: Optional[torch.Tensor], workspace: torch.Tensor, stream=None):
+    _check("misa_route_score_topk_pooled",
+           lib().misa_route_score_topk_pooled(ctypes.byref(args), block, h, topk, kprime, _ptr(kbar),
+                                              _ptr(kbar_scale), _ptr(out_idx), _ptr(out_score), _ptr(out_heads),
+                                              _ptr(out_cand), _ptr(workspace), workspace.numel(),
+                                              _stream_ptr(stream)))
+
+
+def hisa_block_filter_topk_pooled(args: IndexerArgs, block: int, m: int, topk: int, kbar: torch.Tensor,
+                                  kbar_scale: Optional[torch.Tensor], out_idx: torch.Tensor,
+                                  out_score: Optional[torch.Tensor], out_blocks: Optional[torch.Tensor],
+                                  workspace: torch.Tensor, stream=None):
+    _check("hisa_block_filter_topk_pooled",
+           lib().hisa_block_filter_topk_pooled(ctypes.byref(args), block, m, topk, _ptr(kbar), _ptr(kbar_scale),
+                                               _ptr(out_idx), _ptr(out_score), _ptr(out_blocks), _ptr(workspace),
+                                               workspace.numel(), _stream_ptr(stream)))
 
 
 def hisa_refine_workspace_size(args: IndexerArgs, m: int, blk: int) -> int:

@@ -181,12 +181,15 @@ dsa_status launch_score(const ScoreParams& p, const void* q, long long q_rows, c
 dsa_status run_scores_bf16(int D, int H, const ScoreParams& p, const void* q, long long q_rows,
                            const void* k, long long k_rows, cudaStream_t st, int epi = kEpiStore,
                            long long k_stride = 0) {
-#ifndef DSA_EPIW
-#define DSA_EPIW 8
+// Epilogue warps: 8 for 64 heads (4 queries per tile); 16 for fewer heads,
+// where a thread of an 8-warp epilogue holds 8 to 16 queries' partial sums
+// and spills (the 8-head MISA routed pass: 0.59 against 0.70-0.81 ms).
+#ifndef DSA_EPIW64
+#define DSA_EPIW64 8
 #endif
   const bool list = p.pairs != nullptr;
 #define DSA_CFG(DD, HH, EE, LL) \
-  ScoreCfg<2, DD, HH, 256 / HH, ScoreMode::kTma, (DD == 128 ? 4 : 8), DSA_EPIW, 1, EE, LL>
+  ScoreCfg<2, DD, HH, 256 / HH, ScoreMode::kTma, (DD == 128 ? 4 : 8), (HH == 64 ? DSA_EPIW64 : 16), 1, EE, LL>
 #define DSA_LAUNCH(DD, HH, EE, LL) return launch_score<DSA_CFG(DD, HH, EE, LL)>(p, q, q_rows, k, k_rows, st, k_stride);
 #define DSA_CASE(DD, HH)                                            \
   if (D == DD && H == HH) {                                         \
@@ -213,9 +216,20 @@ dsa_status run_scores_bf16(int D, int H, const ScoreParams& p, const void* q, lo
 
 // FP8 scoring (kind::f8f6f4). Decode (one query per sequence): one query per
 // group, N = H. Prefill (T > 1): 256 / H queries per group, N = 256, as the
-// bf16 path.
+// bf16 path, with sixteen epilogue warps (the FP8 MMAs take half the time of
+// bf16 ones, so the epilogue arithmetic sets the pace: 1.40 against 1.44 ms
+// with eight on the FP8 DSA chunk).
 #ifndef DSA_FP8_NSTAGE
 #define DSA_FP8_NSTAGE 8
+#endif
+#ifndef DSA_FP8_EPIW
+#define DSA_FP8_EPIW 16
+#endif
+#ifndef DSA_FP8_DEC_EPIW
+#define DSA_FP8_DEC_EPIW 8
+#endif
+#ifndef DSA_FP8_DEC_NSTAGE
+#define DSA_FP8_DEC_NSTAGE DSA_FP8_NSTAGE
 #endif
 dsa_status run_scores_fp8(int D, int H, const ScoreParams& p, const void* q, long long q_rows,
                           const void* k, long long k_rows, cudaStream_t st) {
@@ -224,17 +238,17 @@ dsa_status run_scores_fp8(int D, int H, const ScoreParams& p, const void* q, lon
   // takes at least 32 columns, so a group has 64 / H queries even in decode,
   // where only the first of them exists
   if (D == 128 && H == 16)
-    return prefill ? launch_score<ScoreCfg<1, 128, 16, 16, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st)
+    return prefill ? launch_score<ScoreCfg<1, 128, 16, 16, ScoreMode::kTma, DSA_FP8_NSTAGE, 16>>(p, q, q_rows, k, k_rows, st)
                    : launch_score<ScoreCfg<1, 128, 16, 4, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
   if (D == 128 && H == 8)
-    return prefill ? launch_score<ScoreCfg<1, 128, 8, 32, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st)
+    return prefill ? launch_score<ScoreCfg<1, 128, 8, 32, ScoreMode::kTma, DSA_FP8_NSTAGE, 16>>(p, q, q_rows, k, k_rows, st)
                    : launch_score<ScoreCfg<1, 128, 8, 8, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
   if (D == 128 && H == 64)
-    return prefill ? launch_score<ScoreCfg<1, 128, 64, 4, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st)
-                   : launch_score<ScoreCfg<1, 128, 64, 1, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
+    return prefill ? launch_score<ScoreCfg<1, 128, 64, 4, ScoreMode::kTma, DSA_FP8_NSTAGE, DSA_FP8_EPIW>>(p, q, q_rows, k, k_rows, st)
+                   : launch_score<ScoreCfg<1, 128, 64, 1, ScoreMode::kTma, DSA_FP8_DEC_NSTAGE, DSA_FP8_DEC_EPIW>>(p, q, q_rows, k, k_rows, st);
   if (D == 128 && H == 32)
-    return prefill ? launch_score<ScoreCfg<1, 128, 32, 8, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st)
-                   : launch_score<ScoreCfg<1, 128, 32, 1, ScoreMode::kTma, DSA_FP8_NSTAGE>>(p, q, q_rows, k, k_rows, st);
+    return prefill ? launch_score<ScoreCfg<1, 128, 32, 8, ScoreMode::kTma, DSA_FP8_NSTAGE, DSA_FP8_EPIW>>(p, q, q_rows, k, k_rows, st)
+                   : launch_score<ScoreCfg<1, 128, 32, 1, ScoreMode::kTma, DSA_FP8_DEC_NSTAGE, DSA_FP8_DEC_EPIW>>(p, q, q_rows, k, k_rows, st);
   return DSA_ERR_UNSUPPORTED;
 }
 
@@ -423,8 +437,8 @@ dsa_status run_refine_inverted(const dsa_indexer_args* a, const int32_t* blocks,
   }
   {
     prof::Launch pl(st, "invert_scan");
-    invert_scan_kernel<1024><<<1, 1024, 0, st>>>(w.cnt, static_cast<int>(nb), blk / 128, 128 / a->H, w.qoff,
-                                               w.ioff, w.cursor, w.total);
+    invert_scan_kernel<1024><<<static_cast<int>((nb + 4095) / 4096), 1024, 0, st>>>(
+        w.cnt, static_cast<int>(nb), blk / 128, 128 / a->H, w.qoff, w.ioff, w.cursor, w.total);
   }
   {
     prof::Launch pl(st, "invert_fill");
@@ -908,22 +922,29 @@ dsa_status indexer_score_topk_lists(const dsa_indexer_args* a, int topk, int32_t
   return fused_score_topk(a->d, a->H, p, a->q, a->k, a->L, topk, out_idx, out_score, scores, f, w, ws, st);
 }
 
+// bf16 pooling of blocks [m0, m0 + nm) of every sequence.
+dsa_status launch_meanpool_bf16(const void* k, int batch, int L, int d, int block, long long M, long long m0,
+                                long long nm, void* kbar, cudaStream_t st) {
+  if (static_cast<long long>(batch) * nm > INT_MAX) return DSA_ERR_UNSUPPORTED;
+  if (nm < 1) return DSA_OK;
+  prof::Launch pl(st, "meanpool");
+  const int grid = static_cast<int>(batch * nm);
+  if (d % 8 == 0 && d <= 256 && aligned(k, 16))
+    meanpool_vec_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k), L, d, block,
+                                              static_cast<int>(M), static_cast<int>(m0), static_cast<int>(nm),
+                                              static_cast<__nv_bfloat16*>(kbar));
+  else
+    meanpool_kernel<<<grid, d < 128 ? d : 128, 0, st>>>(static_cast<const __nv_bfloat16*>(k), L, d, block,
+                                                        static_cast<int>(M), static_cast<int>(m0),
+                                                        static_cast<int>(nm), static_cast<__nv_bfloat16*>(kbar));
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
 dsa_status dsa_meanpool_keys(const void* k, int batch, int L, int d, int block, void* kbar,
                              void* stream) {
   if (!k || !kbar || batch < 1 || L < 1 || d < 1 || d > 1024 || block < 1) return DSA_ERR_ARG;
   const long long M = blocks_of(L, block);
-  if (static_cast<long long>(batch) * M > INT_MAX) return DSA_ERR_UNSUPPORTED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  prof::Launch pl(st, "meanpool");
-  if (d % 8 == 0 && d <= 256 && aligned(k, 16))
-    meanpool_vec_kernel<false><<<static_cast<int>(batch * M), 256, 0, st>>>(
-        static_cast<const uint8_t*>(k), nullptr, L, d, block, static_cast<int>(M), static_cast<uint8_t*>(kbar),
-        nullptr);
-  else
-    meanpool_kernel<<<static_cast<int>(batch * M), d < 128 ? d : 128, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(k), L, d, block, static_cast<int>(M),
-        static_cast<__nv_bfloat16*>(kbar));
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return launch_meanpool_bf16(k, batch, L, d, block, M, 0, M, kbar, static_cast<cudaStream_t>(stream));
 }
 
 // Pooled keys of MISA and HISA: bf16 [batch*M, d], or on an FP8 cache e4m3
@@ -953,12 +974,45 @@ Pooled pooled_carve(Carve& c, const dsa_indexer_args* a, long long M) {
   return pk;
 }
 
-dsa_status run_meanpool(const dsa_indexer_args* a, int block, long long M, const Pooled& pk, cudaStream_t st) {
-  if (a->qk_dtype != DSA_FP8_E4M3) return dsa_meanpool_keys(a->k, a->batch, a->L, a->d, block, pk.kbar, st);
+// Pools blocks [m0, m1) of every sequence into pk.
+dsa_status run_meanpool(const dsa_indexer_args* a, int block, long long M, const Pooled& pk, cudaStream_t st,
+                        long long m0 = 0, long long m1 = -1) {
+  if (m1 < 0 || m1 > M) m1 = M;
+  if (m0 < 0) m0 = 0;
+  const long long nm = m1 - m0;
+  if (a->qk_dtype != DSA_FP8_E4M3)
+    return launch_meanpool_bf16(a->k, a->batch, a->L, a->d, block, M, m0, nm, pk.kbar, st);
+  if (nm < 1) return DSA_OK;
+  if (static_cast<long long>(a->batch) * nm > INT_MAX) return DSA_ERR_UNSUPPORTED;
   prof::Launch pl(st, "meanpool fp8");
-  meanpool_vec_kernel<true><<<static_cast<int>(a->batch * M), 256, 0, st>>>(
-      static_cast<const uint8_t*>(a->k), a->k_scale, a->L, a->d, block, static_cast<int>(M), pk.kbar8, pk.scale);
+  meanpool_fp8_kernel<<<static_cast<int>(a->batch * nm), 4 * a->d, 0, st>>>(
+      static_cast<const uint8_t*>(a->k), a->k_scale, a->L, a->d, block, static_cast<int>(M), static_cast<int>(m0),
+      static_cast<int>(nm), pk.kbar8, pk.scale);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// Caller-kept pooled keys (the *_pooled entry points): checked and wrapped.
+dsa_status given_pooled(const dsa_indexer_args* a, const void* kbar, const float* kbar_scale, Pooled& pk) {
+  if (!kbar || !aligned(kbar, 16)) return DSA_ERR_ARG;
+  pk = Pooled{};
+  if (a->qk_dtype == DSA_FP8_E4M3) {
+    if (!kbar_scale || !aligned(kbar_scale, 4)) return DSA_ERR_ARG;
+    pk.kbar8 = const_cast<uint8_t*>(static_cast<const uint8_t*>(kbar));
+    pk.scale = const_cast<float*>(kbar_scale);
+  } else {
+    pk.kbar = const_cast<__nv_bfloat16*>(static_cast<const __nv_bfloat16*>(kbar));
+  }
+  return DSA_OK;
+}
+
+dsa_status dsa_pool_keys(const dsa_indexer_args* a, int block, int m0, int m1, void* kbar, float* kbar_scale,
+                         void* stream) {
+  DSA_TRY(validate(a, false));
+  if (block < 1 || m0 < 0 || m1 < m0) return DSA_ERR_ARG;
+  Pooled pk{};
+  DSA_TRY(given_pooled(a, kbar, kbar_scale, pk));
+  const long long M = blocks_of(a->L, block);
+  return run_meanpool(a, block, M, pk, static_cast<cudaStream_t>(stream), m0, m1 < M ? m1 : M);
 }
 
 size_t misa_workspace_size(const dsa_indexer_args* a, int block, int h, int topk, int kprime) {
@@ -982,10 +1036,10 @@ size_t misa_workspace_size(const dsa_indexer_args* a, int block, int h, int topk
   return n;
 }
 
-dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, int topk, int kprime,
-                                 int32_t* out_idx, float* out_score, int32_t* out_heads,
-                                 int32_t* out_cand, void* ws, size_t ws_bytes, void* stream) {
-  DSA_TRY(validate(a, false));
+// given: caller-kept pooled keys (nullptr: pooled here, into the workspace)
+dsa_status misa_run(const dsa_indexer_args* a, int block, int h, int topk, int kprime, const Pooled* given,
+                    int32_t* out_idx, float* out_score, int32_t* out_heads, int32_t* out_cand, void* ws,
+                    size_t ws_bytes, void* stream) {
   if (!out_idx || block < 1 || h < 1 || h > a->H || topk < 1 || topk > (1 << 24) || kprime < 0 ||
       kprime > (1 << 24))
     return DSA_ERR_ARG;
@@ -1001,7 +1055,8 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   if (static_cast<long long>(a->batch) * M > INT_MAX) return DSA_ERR_UNSUPPORTED;
 
   Carve c{static_cast<char*>(ws), kHdr};
-  const Pooled pk = pooled_carve(c, a, M);
+  const Pooled pk_ws = pooled_carve(c, a, M);
+  const Pooled& pk = given ? *given : pk_ws;
   float* part = c.take<float>(2 * static_cast<size_t>(BT) * a->H);
   uint8_t* q_sel = c.take<uint8_t>(static_cast<size_t>(BT) * h * a->d * 2);
   float* w_sel = c.take<float>(static_cast<size_t>(BT) * h);
@@ -1010,8 +1065,8 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
   float* routed = c.take<float>(static_cast<size_t>(BT) * a->L);
   int32_t* heads = out_heads ? out_heads : heads_ws;
 
-  // 1. pooled keys (FP8 cache: in the cache's format)
-  DSA_TRY(run_meanpool(a, block, M, pk, st));
+  // 1. pooled keys (FP8 cache: in the cache's format), unless the caller keeps them
+  if (!given) DSA_TRY(run_meanpool(a, block, M, pk, st));
   // 2. router affinities (partial ReLU sums over visible pooled keys)
   prof::Stage misa_stage("router");
   ScoreParams pr = base_params(a, err);
@@ -1073,6 +1128,24 @@ dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, in
                      st);
 }
 
+dsa_status misa_route_score_topk(const dsa_indexer_args* a, int block, int h, int topk, int kprime,
+                                 int32_t* out_idx, float* out_score, int32_t* out_heads,
+                                 int32_t* out_cand, void* ws, size_t ws_bytes, void* stream) {
+  DSA_TRY(validate(a, false));
+  return misa_run(a, block, h, topk, kprime, nullptr, out_idx, out_score, out_heads, out_cand, ws, ws_bytes,
+                  stream);
+}
+
+dsa_status misa_route_score_topk_pooled(const dsa_indexer_args* a, int block, int h, int topk, int kprime,
+                                        const void* kbar, const float* kbar_scale, int32_t* out_idx,
+                                        float* out_score, int32_t* out_heads, int32_t* out_cand, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  DSA_TRY(validate(a, false));
+  Pooled pk{};
+  DSA_TRY(given_pooled(a, kbar, kbar_scale, pk));
+  return misa_run(a, block, h, topk, kprime, &pk, out_idx, out_score, out_heads, out_cand, ws, ws_bytes, stream);
+}
+
 size_t hisa_workspace_size(const dsa_indexer_args* a, int block, int m, int topk) {
   (void)topk;
   if (!a || a->batch < 1 || a->T < 1 || a->L < 1 || a->d < 1 || block < 1 || m < 1) return 0;
@@ -1111,10 +1184,9 @@ dsa_status hisa_refine_scores(const dsa_indexer_args* a, const int32_t* blocks, 
   return run_refine_inverted(a, blocks, m, blk, out, ld, w, static_cast<unsigned*>(ws), st);
 }
 
-dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, int topk,
-                                  int32_t* out_idx, float* out_score, int32_t* out_blocks,
-                                  void* ws, size_t ws_bytes, void* stream) {
-  DSA_TRY(validate(a, false));
+dsa_status hisa_run(const dsa_indexer_args* a, int block, int m, int topk, const Pooled* given,
+                    int32_t* out_idx, float* out_score, int32_t* out_blocks, void* ws, size_t ws_bytes,
+                    void* stream) {
   if (!out_idx || block < 1 || m < 1 || topk < 1 || topk > (1 << 24)) return DSA_ERR_ARG;
   if (static_cast<long long>(m) * block > INT_MAX / 2) return DSA_ERR_UNSUPPORTED;
   if (a->d != 128 || (a->H != 32 && a->H != 64)) return DSA_ERR_UNSUPPORTED;
@@ -1130,14 +1202,15 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   const int ncomp = m * block;
 
   Carve c{static_cast<char*>(ws), kHdr};
-  const Pooled pk = pooled_carve(c, a, M);
+  const Pooled pk_ws = pooled_carve(c, a, M);
+  const Pooled& pk = given ? *given : pk_ws;
   float* bscore = c.take<float>(static_cast<size_t>(BT) * M);
   int32_t* blocks_ws = c.take<int32_t>(static_cast<size_t>(BT) * m);
   float* compact = c.take<float>(static_cast<size_t>(BT) * ncomp);
   int32_t* blocks = out_blocks ? out_blocks : blocks_ws;
 
-  // 1. pooled keys (FP8 cache: e4m3 codes + per-block scales)
-  DSA_TRY(run_meanpool(a, block, M, pk, st));
+  // 1. pooled keys (FP8 cache: e4m3 codes + per-block scales), unless the caller keeps them
+  if (!given) DSA_TRY(run_meanpool(a, block, M, pk, st));
   // 2. block scores on the pooled keys (block m visible iff m * block <= p_t)
   prof::Stage hisa_stage("blocks");
   ScoreParams pb = base_params(a, err);
@@ -1179,6 +1252,22 @@ dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, i
   return launch_topk(ws, topk_params(compact, BT, ncomp, a->T, a->q_offset, 0, ncomp, topk, out_idx,
                                  out_score, blocks, m, block),
                      st);
+}
+
+dsa_status hisa_block_filter_topk(const dsa_indexer_args* a, int block, int m, int topk,
+                                  int32_t* out_idx, float* out_score, int32_t* out_blocks,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  DSA_TRY(validate(a, false));
+  return hisa_run(a, block, m, topk, nullptr, out_idx, out_score, out_blocks, ws, ws_bytes, stream);
+}
+
+dsa_status hisa_block_filter_topk_pooled(const dsa_indexer_args* a, int block, int m, int topk, const void* kbar,
+                                         const float* kbar_scale, int32_t* out_idx, float* out_score,
+                                         int32_t* out_blocks, void* ws, size_t ws_bytes, void* stream) {
+  DSA_TRY(validate(a, false));
+  Pooled pk{};
+  DSA_TRY(given_pooled(a, kbar, kbar_scale, pk));
+  return hisa_run(a, block, m, topk, &pk, out_idx, out_score, out_blocks, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------ DoSA

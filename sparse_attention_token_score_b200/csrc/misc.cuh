@@ -12,13 +12,13 @@ namespace dsa {
 // HISA review, section 3, uses the same pooled representatives):
 //     kbar[b, m, :] = bf16( mean of k[b, mB : min((m+1)B, L), :] )
 // The sum runs in fp64, which is exact for bf16 inputs at these block sizes,
-// and is rounded to bf16 once (round to nearest even).
-// Grid: batch * M blocks; threads over the d columns.
-__global__ void meanpool_kernel(const __nv_bfloat16* __restrict__ k, int L, int d, int B, int M,
+// and is rounded to bf16 once (round to nearest even). Every kernel below
+// pools blocks m0 .. m0 + nm - 1 of every sequence (grid: batch * nm CTAs).
+__global__ void meanpool_kernel(const __nv_bfloat16* __restrict__ k, int L, int d, int B, int M, int m0, int nm,
                                 __nv_bfloat16* __restrict__ kbar) {
-  const long long bm = blockIdx.x;
-  const long long b = bm / M;
-  const int m = static_cast<int>(bm % M);
+  const long long b = blockIdx.x / nm;
+  const int m = m0 + static_cast<int>(blockIdx.x % nm);
+  const long long bm = b * M + m;
   const int s0 = m * B;
   const int s1 = min(s0 + B, L);
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
@@ -28,87 +28,91 @@ __global__ void meanpool_kernel(const __nv_bfloat16* __restrict__ k, int L, int 
   }
 }
 
-// Pooled keys of an FP8 e4m3 key cache, kept in the cache's format: per
-// block the fp64 mean of the dequantised keys (code value x per-token scale),
-// a scale absmax/448 (absmax rounded to fp32, divided in fp32; 1 when the
-// mean is zero) and codes e4m3(mean / scale), rounded to nearest even with
-// saturation.
-//
-// Vectorised pooling, bf16 (the mean as above, rounded to bf16) or FP8 keys,
-// 16-byte rows, d <= 256: a CTA of 256 threads pools one block; each thread reads
-// 16-byte pieces of token rows (rows r, r + RPI, ... of the block, the same
-// 16 bytes of each), accumulates their values (times the token's scale for
-// FP8) in fp64, and the per-thread partial sums are added up per column
-// through shared memory. The products and sums are exact in fp64 here, so
-// the result does not depend on the order and equals the scalar kernels'.
-template <bool FP8>
-__global__ void __launch_bounds__(256) meanpool_vec_kernel(const uint8_t* __restrict__ k,
-                                                           const float* __restrict__ ks, int L, int d, int B,
-                                                           int M, uint8_t* __restrict__ out,
-                                                           float* __restrict__ out_scale) {
-  constexpr int EPV = FP8 ? 16 : 8;           // elements per 16-byte piece
-  __shared__ double red[32 * 128];            // [rows in flight][d]
-  __shared__ double wmax[8];
-  const long long bm = blockIdx.x;
-  const long long b = bm / M;
-  const int m = static_cast<int>(bm % M);
+// The same for bf16 rows of 16-byte multiples (d % 8 == 0, d <= 256): a CTA
+// of 256 threads pools one block; each thread reads one 16-byte piece of
+// token rows r, r + RPI, ... of the block and accumulates its 8 values in
+// fp64; the per-thread partial sums are added per column through shared
+// memory. The sums are exact, so the order does not change the result.
+__global__ void __launch_bounds__(256) meanpool_vec_kernel(const __nv_bfloat16* __restrict__ k, int L, int d,
+                                                           int B, int M, int m0, int nm,
+                                                           __nv_bfloat16* __restrict__ kbar) {
+  __shared__ double red[32 * 64];             // [rows in flight][d]: RPI * d = 2048
+  const long long b = blockIdx.x / nm;
+  const int m = m0 + static_cast<int>(blockIdx.x % nm);
+  const long long bm = b * M + m;
   const int s0 = m * B;
   const int s1 = min(s0 + B, L);
-  const int rb = d * (FP8 ? 1 : 2);           // bytes per key row
-  const int tpr = rb / 16;                    // threads per row
+  const int tpr = d / 8;                      // threads per row (16-byte pieces)
   const int rpi = 256 / tpr;                  // rows in flight
   const int t = threadIdx.x;
   const int r = t / tpr, c = t % tpr;
-  double acc[EPV];
+  double acc[8];
 #pragma unroll
-  for (int e = 0; e < EPV; ++e) acc[e] = 0.0;
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
   if (r < rpi) {
     for (int s = s0 + r; s < s1; s += rpi) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(k + (b * L + s) * rb) + c);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(k + (b * L + s) * d) + c);
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-      if constexpr (FP8) {
-        const double sc = static_cast<double>(__ldg(ks + b * L + s));
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          __nv_fp8_e4m3 x;
-          x.__x = static_cast<__nv_fp8_storage_t>((w4[e >> 2] >> (8 * (e & 3))) & 0xffu);
-          acc[e] += static_cast<double>(static_cast<float>(x)) * sc;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          acc[e] += static_cast<double>(__uint_as_float(((w4[e >> 1] >> (16 * (e & 1))) & 0xffffu) << 16));
-      }
+      for (int e = 0; e < 8; ++e)
+        acc[e] += static_cast<double>(__uint_as_float(((w4[e >> 1] >> (16 * (e & 1))) & 0xffffu) << 16));
     }
 #pragma unroll
-    for (int e = 0; e < EPV; ++e) red[r * d + c * EPV + e] = acc[e];
+    for (int e = 0; e < 8; ++e) red[r * d + c * 8 + e] = acc[e];
   }
   __syncthreads();
-  double mean = 0.0;
   if (t < d) {
     const int nrow = min(rpi, s1 - s0);
     double sum = 0.0;
     for (int i = 0; i < nrow; ++i) sum += red[i * d + t];
-    mean = sum / static_cast<double>(s1 - s0);
+    kbar[bm * d + t] = __double2bfloat16(sum / static_cast<double>(s1 - s0));
   }
-  if constexpr (!FP8) {
-    if (t < d) reinterpret_cast<__nv_bfloat16*>(out)[bm * d + t] = __double2bfloat16(mean);
-  } else {
-    double a = t < d ? fabs(mean) : 0.0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a = fmax(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if ((t & 31) == 0) wmax[t >> 5] = a;
-    __syncthreads();
-    double amax = 0.0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) amax = fmax(amax, wmax[w]);
-    const float af = static_cast<float>(amax);
-    const float scale = af > 0.f ? af / 448.f : 1.f;
-    if (t < d)
-      out[bm * d + t] = static_cast<uint8_t>(__nv_cvt_double_to_fp8(mean / static_cast<double>(scale), __NV_SATFINITE,
-                                                                    __NV_E4M3));
-    if (t == 0) out_scale[bm] = scale;
+}
+
+// Pooled keys of an FP8 e4m3 key cache, kept in the cache's format: per
+// block the fp64 mean of the dequantised keys (code value x per-token scale),
+// a scale absmax/448 (absmax rounded to fp32, divided in fp32; 1 when the
+// mean is zero) and codes e4m3(mean / scale), rounded to nearest even with
+// saturation. 4 * d threads (d <= 128): thread (g, c) sums column c over
+// tokens g, g + 4, ... of the block (independent loads, eight in flight);
+// the four partial sums of a column are added in shared memory. The fp64
+// sums are exact here, so the order does not change the result.
+__global__ void __launch_bounds__(512) meanpool_fp8_kernel(const uint8_t* __restrict__ k8,
+                                                           const float* __restrict__ ks, int L, int d, int B,
+                                                           int M, int m0, int nm, uint8_t* __restrict__ kbar8,
+                                                           float* __restrict__ kbar_scale) {
+  __shared__ double part[4 * 128];
+  __shared__ double red[32];
+  const long long b = blockIdx.x / nm;
+  const int m = m0 + static_cast<int>(blockIdx.x % nm);
+  const long long bm = b * M + m;
+  const int s0 = m * B;
+  const int s1 = min(s0 + B, L);
+  const int g = threadIdx.x / d, c = threadIdx.x % d;
+  double acc = 0.0;
+#pragma unroll 8
+  for (int s = s0 + g; s < s1; s += 4) {
+    __nv_fp8_e4m3 v;
+    v.__x = k8[(b * L + s) * d + c];
+    acc += static_cast<double>(static_cast<float>(v)) * static_cast<double>(__ldg(ks + b * L + s));
   }
+  part[g * d + c] = acc;
+  __syncthreads();
+  double mean = 0.0;
+  if (threadIdx.x < d)
+    mean = (((part[c] + part[d + c]) + part[2 * d + c]) + part[3 * d + c]) / static_cast<double>(s1 - s0);
+  double a = threadIdx.x < d ? fabs(mean) : 0.0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmax(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  double amax = 0.0;
+  for (int w = 0; w < static_cast<int>((blockDim.x + 31) >> 5); ++w) amax = fmax(amax, red[w]);
+  const float af = static_cast<float>(amax);
+  const float scale = af > 0.f ? af / 448.f : 1.f;
+  if (threadIdx.x < d)
+    kbar8[bm * d + c] = static_cast<uint8_t>(__nv_cvt_double_to_fp8(mean / static_cast<double>(scale), __NV_SATFINITE, __NV_E4M3));
+  if (threadIdx.x == 0) kbar_scale[bm] = scale;
 }
 
 // MISA routing (same page, "Methodology", step 1): per query, the head

@@ -429,27 +429,48 @@ __global__ void invert_count_kernel(const int* __restrict__ blocks, long long ro
   }
 }
 
-// One CTA: exclusive prefix sums of the counts (list starts) and of the items
-// per block (tiles x chunks); total items at ioff[nb]. Clears the cursors.
-// Each thread owns a contiguous run of blocks: it sums its run, one
-// block-wide scan of the run totals gives every run its start, and a second
-// pass over the run writes the starts.
+// Exclusive prefix sums of the counts (list starts) and of the items per
+// block (tiles x chunks); total items at ioff[nb]. Clears the cursors.
+// CTA c scans blocks [4 NT c, 4 NT (c + 1)) (each thread 4 consecutive
+// blocks, loads and stores coalesced); the sum of all blocks before its range
+// it adds up itself (a coalesced read of at most nb counts), so the CTAs need
+// no communication. The last CTA writes the totals.
 template <int NT>
 __global__ void __launch_bounds__(NT) invert_scan_kernel(const int* __restrict__ cnt, int nb, int tiles,
                                                           int qc, int* __restrict__ qoff, int* __restrict__ ioff,
                                                           int* __restrict__ cursor, long long* __restrict__ total) {
   __shared__ int wsum[2][NT / 32];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int E = (nb + NT - 1) / NT;
-  const int g0 = static_cast<int>(threadIdx.x) * E;
-  const int g1 = min(g0 + E, nb);
-  int sa = 0, sb = 0;
-  for (int g = g0; g < g1; ++g) {
+  const int base = blockIdx.x * 4 * NT;
+  // 1. sum of the blocks before this CTA's range
+  int pa = 0, pb = 0;
+  for (int g = static_cast<int>(threadIdx.x); g < base; g += NT) {
     const int c = cnt[g];
-    sa += c;
-    sb += tiles * ((c + qc - 1) / qc);
+    pa += c;
+    pb += tiles * ((c + qc - 1) / qc);
   }
-  // inclusive scan of the run totals: within the warp, then over the warps
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    pa += __shfl_xor_sync(0xffffffffu, pa, o);
+    pb += __shfl_xor_sync(0xffffffffu, pb, o);
+  }
+  if (lane == 0) { wsum[0][wid] = pa; wsum[1][wid] = pb; }
+  __syncthreads();
+  int carry_a = 0, carry_b = 0;
+#pragma unroll 4
+  for (int w = 0; w < NT / 32; ++w) { carry_a += wsum[0][w]; carry_b += wsum[1][w]; }
+  __syncthreads();  // wsum is reused below
+  // 2. this CTA's range: 4 consecutive blocks per thread
+  const int g0 = base + 4 * static_cast<int>(threadIdx.x);
+  int c[4], it[4];
+  int sa = 0, sb = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    c[u] = g0 + u < nb ? cnt[g0 + u] : 0;
+    it[u] = tiles * ((c[u] + qc - 1) / qc);
+    sa += c[u];
+    sb += it[u];
+  }
   int a = sa, bi = sb;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -471,20 +492,23 @@ __global__ void __launch_bounds__(NT) invert_scan_kernel(const int* __restrict__
     if (lane < NT / 32) { wsum[0][lane] = wa; wsum[1][lane] = wb; }
   }
   __syncthreads();
-  int pa = (wid > 0 ? wsum[0][wid - 1] : 0) + a - sa;   // exclusive start of this run
-  int pb = (wid > 0 ? wsum[1][wid - 1] : 0) + bi - sb;
-  for (int g = g0; g < g1; ++g) {
-    const int c = cnt[g];
-    qoff[g] = pa;
-    ioff[g] = pb;
-    cursor[g] = 0;
-    pa += c;
-    pb += tiles * ((c + qc - 1) / qc);
+  int xa = carry_a + (wid > 0 ? wsum[0][wid - 1] : 0) + a - sa;   // exclusive start of this thread's 4
+  int xb = carry_b + (wid > 0 ? wsum[1][wid - 1] : 0) + bi - sb;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    if (g0 + u < nb) {
+      qoff[g0 + u] = xa;
+      ioff[g0 + u] = xb;
+      cursor[g0 + u] = 0;
+    }
+    xa += c[u];
+    xb += it[u];
   }
-  if (threadIdx.x == NT - 1) {
-    qoff[nb] = wsum[0][NT / 32 - 1];
-    ioff[nb] = wsum[1][NT / 32 - 1];
-    *total = wsum[1][NT / 32 - 1];
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
+    const int ta = carry_a + wsum[0][NT / 32 - 1], tb = carry_b + wsum[1][NT / 32 - 1];
+    qoff[nb] = ta;
+    ioff[nb] = tb;
+    *total = tb;
   }
 }
 

@@ -146,12 +146,12 @@ struct ScoreCfg {
   static constexpr int MMA_WARP = NPROD;
   static constexpr int EPI_WARP0 = NPROD + 1;
   // Epilogue warps: EPIW = 4 * NSETS; each set of 4 warps covers the 128
-  // TMEM lanes. Sets take alternate tiles (router and one-query groups, 2
-  // sets), or split the queries of every tile between them.
+  // TMEM lanes. Sets take tiles round robin (router and one-query groups),
+  // or split the queries of every tile between them.
   static constexpr int EPIW = EPIW_;
   static constexpr int NSETS = EPIW / 4;
   static constexpr bool SPLIT_TILES = ROUTER || QPT == 1;
-  static_assert(EPIW == 8 || (EPIW == 16 && !SPLIT_TILES && QPT % 4 == 0), "epilogue warps");
+  static_assert(EPIW == 8 || (EPIW == 16 && !ROUTER && (SPLIT_TILES || QPT % 4 == 0)), "epilogue warps");
   static constexpr int NTHREADS = (EPI_WARP0 + EPIW) * 32;
   static constexpr int TEMPTY_ARRIVALS = SPLIT_TILES ? 4 : EPIW;
   static constexpr uint32_t IDESC = umma_idesc(ELEM == 2 ? 1u : 0u, 128, MMA_N);
@@ -633,7 +633,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       {
       const int buf = static_cast<int>(it % C::NACC);
       // split tiles: the two sets take alternate tiles (buffer b: set b & 1)
-      const bool mine = C::SPLIT_TILES ? (static_cast<int>(it & 1u) == set) : true;
+      const bool mine = C::SPLIT_TILES ? (static_cast<int>(it % C::NSETS) == set) : true;
       if (mine) {
         // gather mode: this row's token (and visibility), loaded before the
         // wait so that its latency hides behind the tile's MMAs
@@ -756,60 +756,97 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int j = 0; j < NP; ++j) acc2[i][j] = 0ull;
 #endif
-          // TMEM -> registers one 32-column chunk at a time: the next chunk's
-          // load is issued before this chunk's arithmetic, and the buffer goes
-          // back to the MMA warp as soon as the last chunk has landed, so the
-          // next tile's MMAs overlap the remaining math.
-          constexpr int PH = 1;  // chunks per phase (more would exceed the register budget)
-          constexpr int NPHASE = NCH / PH;
-          uint32_t vb[2][PH][32];
+          if constexpr (C::EPIW == 16) {
+            // Sixteen epilogue warps (four per sub-partition, 96 registers a
+            // thread): one 32-column chunk in flight per warp, the other
+            // warps hide its load latency; head weights read four at a time.
 #pragma unroll
-          for (int c = 0; c < PH; ++c) tmem_ld32_issue(taddr + q0 * C::H + c * 32, vb[0][c]);
-#pragma unroll
-          for (int c = 0; c < PH; ++c) tmem_ld_wait(vb[0][c]);
-#pragma unroll
-          for (int ph = 0; ph < NPHASE; ++ph) {
-            if (ph + 1 < NPHASE) {
-#pragma unroll
-              for (int c = 0; c < PH; ++c)
-                tmem_ld32_issue(taddr + q0 * C::H + ((ph + 1) * PH + c) * 32, vb[(ph + 1) & 1][c]);
-            } else {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(tempty(buf));
-            }
-#pragma unroll
-            for (int c = 0; c < PH; ++c) {
-              const int cc = (ph * PH + c) * 32;
-              const uint32_t (&v)[32] = vb[ph & 1][c];
-              float coef[32];
+            for (int ph = 0; ph < NCH; ++ph) {
+              uint32_t v[32];
+              tmem_ld32_issue(taddr + q0 * C::H + ph * 32, v);
+              tmem_ld_wait(v);
+              if (ph == NCH - 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty(buf));
+              }
 #pragma unroll
               for (int i = 0; i < 32; i += 4) {
-                const float4 c4 = *reinterpret_cast<const float4*>(cw + cc + i);
-                coef[i] = c4.x; coef[i + 1] = c4.y; coef[i + 2] = c4.z; coef[i + 3] = c4.w;
+                const float4 c4 = *reinterpret_cast<const float4*>(cw + ph * 32 + i);
+                const int ql = (ph * 32 + i) / C::H;
+#if defined(DSA_NO_FFMA2)
+                acc[ql][i % NP] = fmaf(c4.x, fmaxf(__uint_as_float(v[i]), 0.f), acc[ql][i % NP]);
+                acc[ql][(i + 1) % NP] = fmaf(c4.y, fmaxf(__uint_as_float(v[i + 1]), 0.f), acc[ql][(i + 1) % NP]);
+                acc[ql][(i + 2) % NP] = fmaf(c4.z, fmaxf(__uint_as_float(v[i + 2]), 0.f), acc[ql][(i + 2) % NP]);
+                acc[ql][(i + 3) % NP] = fmaf(c4.w, fmaxf(__uint_as_float(v[i + 3]), 0.f), acc[ql][(i + 3) % NP]);
+#else
+                acc2[ql][(i / 2) % NP] = ffma2(pack2(c4.x, c4.y),
+                                               pack2(fmaxf(__uint_as_float(v[i]), 0.f),
+                                                     fmaxf(__uint_as_float(v[i + 1]), 0.f)),
+                                               acc2[ql][(i / 2) % NP]);
+                acc2[ql][(i / 2 + 1) % NP] = ffma2(pack2(c4.z, c4.w),
+                                                   pack2(fmaxf(__uint_as_float(v[i + 2]), 0.f),
+                                                         fmaxf(__uint_as_float(v[i + 3]), 0.f)),
+                                                   acc2[ql][(i / 2 + 1) % NP]);
+#endif
               }
+            }
+          } else {
+            // TMEM -> registers one 32-column chunk at a time: the next chunk's
+            // load is issued before this chunk's arithmetic, and the buffer goes
+            // back to the MMA warp as soon as the last chunk has landed, so the
+            // next tile's MMAs overlap the remaining math.
+            constexpr int PH = 1;  // chunks per phase (more would exceed the register budget)
+            constexpr int NPHASE = NCH / PH;
+            uint32_t vb[2][PH][32];
+#pragma unroll
+            for (int c = 0; c < PH; ++c) tmem_ld32_issue(taddr + q0 * C::H + c * 32, vb[0][c]);
+#pragma unroll
+            for (int c = 0; c < PH; ++c) tmem_ld_wait(vb[0][c]);
+#pragma unroll
+            for (int ph = 0; ph < NPHASE; ++ph) {
+              if (ph + 1 < NPHASE) {
+#pragma unroll
+                for (int c = 0; c < PH; ++c)
+                  tmem_ld32_issue(taddr + q0 * C::H + ((ph + 1) * PH + c) * 32, vb[(ph + 1) & 1][c]);
+              } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty(buf));
+              }
+#pragma unroll
+              for (int c = 0; c < PH; ++c) {
+                const int cc = (ph * PH + c) * 32;
+                const uint32_t (&v)[32] = vb[ph & 1][c];
+                float coef[32];
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                  const float4 c4 = *reinterpret_cast<const float4*>(cw + cc + i);
+                  coef[i] = c4.x; coef[i + 1] = c4.y; coef[i + 2] = c4.z; coef[i + 3] = c4.w;
+                }
 #if defined(DSA_NO_FFMA2)
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int ql = (cc + i) / C::H;
-                const int pp = i % NP;
-                acc[ql][pp] = fmaf(coef[i], fmaxf(__uint_as_float(v[i]), 0.f), acc[ql][pp]);
-              }
+                for (int i = 0; i < 32; ++i) {
+                  const int ql = (cc + i) / C::H;
+                  const int pp = i % NP;
+                  acc[ql][pp] = fmaf(coef[i], fmaxf(__uint_as_float(v[i]), 0.f), acc[ql][pp]);
+                }
 #else
 #pragma unroll
-              for (int i = 0; i < 32; i += 2) {
-                const int ql = (cc + i) / C::H;
-                const int pp = (i / 2) % NP;
-                acc2[ql][pp] = ffma2(pack2(coef[i], coef[i + 1]),
-                                     pack2(fmaxf(__uint_as_float(v[i]), 0.f),
-                                           fmaxf(__uint_as_float(v[i + 1]), 0.f)),
-                                     acc2[ql][pp]);
-              }
+                for (int i = 0; i < 32; i += 2) {
+                  const int ql = (cc + i) / C::H;
+                  const int pp = (i / 2) % NP;
+                  acc2[ql][pp] = ffma2(pack2(coef[i], coef[i + 1]),
+                                       pack2(fmaxf(__uint_as_float(v[i]), 0.f),
+                                             fmaxf(__uint_as_float(v[i + 1]), 0.f)),
+                                       acc2[ql][pp]);
+                }
 #endif
-            }
-            if (ph + 1 < NPHASE) {
+              }
+              if (ph + 1 < NPHASE) {
 #pragma unroll
-              for (int c = 0; c < PH; ++c) tmem_ld_wait(vb[(ph + 1) & 1][c]);
+                for (int c = 0; c < PH; ++c) tmem_ld_wait(vb[(ph + 1) & 1][c]);
+              }
             }
           }
 #if !defined(DSA_NO_FFMA2)

@@ -24,6 +24,8 @@ Distributions follow the five workloads the indexer is measured on:
              FSSS: one layer runs the indexer, three reuse its indices (only
              the F layer has inputs: S layers compute no indexer projections)
 * ``hisa_decode`` HISA (block 128, top-128 blocks) on the ``decode`` FP8 cache
+* ``misa_decode`` MISA-dagger (block 64, top-8 heads, k'=8192) on the ``decode``
+             FP8 cache
 * ``dsa_lists`` the ``dsa`` chunk through the candidate-list selection
 * ``dosa``   the ``dsa`` chunk through DoSA's certified pruning (5 screened heads)
 * ``dosa_lownorm`` the ``dsa`` shape with three of every four key tiles shrunk
@@ -251,6 +253,8 @@ CONFIGS = {
     "indexcache": dict(kind="indexcache", pattern="FSSS", T=4096, L=32768, H=64, d=128, q_offset=28672,
                        topk=2048, needles=64, w_std=0.125),
     "hisa_decode": dict(kind="decode", batch=64, T=1, L=131072, H=64, d=128, topk=2048, block=128, m=128),
+    "misa_decode": dict(kind="decode", batch=64, T=1, L=131072, H=64, d=128, topk=2048, block=64, h=8,
+                        kprime=8192),
     "dsa_lists": dict(kind="dosa", T=4096, L=32768, H=64, d=128, q_offset=28672, topk=2048, needles=64,
                       w_std=0.125),
     "dosa": dict(kind="dosa", T=4096, L=32768, H=64, d=128, q_offset=28672, topk=2048, needles=64,

@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 25
+    assert len(names) == 28
     assert set(names) == set(B._SIGS)
     for n in names:
         assert getattr(lib, n) is not None
@@ -96,6 +96,22 @@ def test_variant_argument_checks(lib):
     assert lib.hisa_block_filter_topk(ctypes.byref(h8), 128, 2, 16, out, None, None, ws, big, None) == -2
     assert lib.indexer_topk_rows(None, 4, 256, 4, 0, 1, 256, 16, None, 0, 1, out, None, ws, big, None) == -1
     assert lib.dsa_meanpool_keys(None, 1, 256, 128, 64, ws, None) == -1
+    # pooled-key cache: missing buffers, bad block ranges (rejected before any launch)
+    kb = ctypes.c_void_p(0x90000)
+    assert lib.dsa_pool_keys(ctypes.byref(a), 64, 0, 4, None, None, None) == -1
+    assert lib.dsa_pool_keys(ctypes.byref(a), 64, 3, 2, kb, None, None) == -1
+    assert lib.dsa_pool_keys(ctypes.byref(a), 64, -1, 2, kb, None, None) == -1
+    assert lib.dsa_pool_keys(ctypes.byref(a), 0, 0, 2, kb, None, None) == -1
+    f = _args(qk_dtype=B.DSA_FP8_E4M3, q_scale=0x60000, k_scale=0x70000)
+    assert lib.dsa_pool_keys(ctypes.byref(f), 64, 0, 4, kb, None, None) == -1  # FP8 needs the scales
+    assert lib.misa_route_score_topk_pooled(ctypes.byref(a), 64, 8, 16, 0, None, None, out, None, None, None,
+                                            ws, big, None) == -1
+    assert lib.misa_route_score_topk_pooled(ctypes.byref(f), 64, 8, 16, 0, kb, None, out, None, None, None,
+                                            ws, big, None) == -1
+    assert lib.hisa_block_filter_topk_pooled(ctypes.byref(a), 128, 2, 16, None, None, out, None, None, ws, big,
+                                             None) == -1
+    assert lib.hisa_block_filter_topk_pooled(ctypes.byref(h8), 128, 2, 16, kb, None, out, None, None, ws, big,
+                                             None) == -2
 
 
 def test_stage_entry_point_checks(lib):

@@ -58,6 +58,15 @@ def test_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     f.write_text(f.read_text() + "\nstatic int changed_code = 1;\n")  # code does
     assert bench.traffic_for(*key) is None
     assert bench.traffic_for("dsa", "no such kernel") is None
+    # a staged name ("stage: kernel") hashes its own kernel family's sources
+    key = ("hisa", "tokens: score_inv (block-major)")
+    monkeypatch.setitem(bench.TRAFFIC, key, (7.0e6, bench.source_hash(key[1])))
+    assert bench.traffic_for(*key) == 7.0e6
+    f.write_text(f.read_text() + "\nstatic int changed_again = 2;\n")  # score_tc.cuh: not its source
+    assert bench.traffic_for(*key) == 7.0e6
+    g = dst / "score_inv.cuh"
+    g.write_text(g.read_text() + "\nstatic int changed_inv = 3;\n")
+    assert bench.traffic_for(*key) is None
 
 
 def test_reference_arm_json_line():

@@ -599,6 +599,56 @@ def test_hisa_batched_h64():
     _hisa_check(inp, block=128, m=6, topk=100, queries=range(16), what="hisa b2", batches=(0, 1))
 
 
+def _pooled_cache(ix, block):
+    """The pooled-key cache built in two pieces (all blocks but the last,
+    then the last), as a decode loop keeps it."""
+    a = ix.args
+    kbar, ksc = B.pooled_cache(a, block, device="cuda")
+    M = kbar.shape[1]
+    B.dsa_pool_keys(a, block, 0, M - 1, kbar, ksc)
+    B.dsa_pool_keys(a, block, M - 1, M + 5, kbar, ksc)   # m1 past M is clamped
+    return kbar, ksc
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_pooled_cache_calls_equal_unpooled(fp8):
+    # MISA-dagger and HISA reading a caller-kept pooled-key cache give the
+    # unpooled calls' indices and scores bit for bit
+    if fp8:
+        inp = wl.decode_inputs(batch=3, L=5000, H=64, d=128, seed=150, cluster_frac=0.05)
+    else:
+        inp = wl.prefill_inputs(24, 4000, 64, 128, q_offset=3976, seed=151, w_std=0.125, batch=2)
+    ix = _indexer(inp)
+    a = ix.args
+    for blk in (64, 128):
+        kbar, ksc = _pooled_cache(ix, blk)
+        if not fp8:
+            ref = torch.empty_like(kbar)
+            B.dsa_meanpool_keys(ix.k, blk, ref)
+            assert torch.equal(kbar, ref)
+        else:
+            for b in range(inp.batch):
+                codes, scales = oracle.meanpool_e4m3(inp.k[b], inp.k_scale[b], blk)
+                assert np.array_equal(kbar[b].cpu().numpy(), codes)
+                assert np.array_equal(ksc[b].cpu().numpy(), scales)
+        if blk == 64:
+            idx, sc, heads, cand = ix.misa(blk, 8, 100, 600, with_score=True, with_heads=True, with_cand=True)
+            i2, s2 = torch.empty_like(idx), torch.empty_like(sc)
+            h2, c2 = torch.empty_like(heads), torch.empty_like(cand)
+            ws = B.alloc_workspace(B.misa_workspace_size(a, blk, 8, 100, 600))
+            B.misa_route_score_topk_pooled(a, blk, 8, 100, 600, kbar, ksc, i2, s2, h2, c2, ws)
+            assert B.dsa_device_status(ws) == 0
+            assert torch.equal(idx, i2) and torch.equal(sc, s2) and torch.equal(heads, h2) and torch.equal(cand, c2)
+        else:
+            idx, sc, blocks = ix.hisa(blk, 10, 150, with_score=True, with_blocks=True)
+            i2, s2, b2 = torch.empty_like(idx), torch.empty_like(sc), torch.empty_like(blocks)
+            ws = B.alloc_workspace(B.hisa_workspace_size(a, blk, 10, 150))
+            B.hisa_block_filter_topk_pooled(a, blk, 10, 150, kbar, ksc, i2, s2, b2, ws)
+            assert B.dsa_device_status(ws) == 0
+            assert torch.equal(idx, i2) and torch.equal(sc, s2) and torch.equal(blocks, b2)
+        assert ix.device_status() == 0
+
+
 def test_hisa_all_blocks_equals_dense():
     inp = wl.prefill_inputs(12, 1500, 32, 128, q_offset=1488, seed=19)
     ix = _indexer(inp)
