@@ -210,7 +210,9 @@ class Runner:
             if stage == "routed" and label == "topk_rows":
                 return self.pairs * 4 + rows * kp * 4, "hbm"
             if stage == "re-score" and label.startswith("score_tc"):
-                return rows * kp * 2.0 * d * H, "tensor_fp8" if fp8 else "tensor"
+                if fp8:                                    # one query per sequence: the gathered rows + scales
+                    return rows * kp * (d + 4), "hbm"
+                return rows * kp * 2.0 * d * H, "tensor"
             if stage == "re-score" and label == "topk_rows":
                 return rows * kp * 4 + rows * k * 8, "hbm"
         if self.name in ("hisa", "hisa_decode"):
@@ -219,9 +221,13 @@ class Runner:
             M = -(-L // blk)
             vis_blocks = int(self.batch * np.minimum(pos // blk + 1, M).sum())
             if stage == "blocks" and label.startswith("score_tc"):
-                return vis_blocks * 2.0 * d * H, "tensor_fp8" if fp8 else "tensor"
+                if fp8:                                    # decode: one query per sequence, pooled rows + scales
+                    return vis_blocks * (d + 4), "hbm"
+                return vis_blocks * 2.0 * d * H, "tensor"
             if stage == "tokens" and label.startswith("score_"):
-                return rows * m * blk * 2.0 * d * H, "tensor_fp8" if fp8 else "tensor"
+                if fp8:                                    # decode: the kept blocks' key rows + scales
+                    return rows * m * blk * (d + 4), "hbm"
+                return rows * m * blk * 2.0 * d * H, "tensor"
             if stage == "tokens" and label == "topk_rows":
                 return rows * m * blk * 4 + rows * k * 8, "hbm"
         return None, None
@@ -251,17 +257,20 @@ class Runner:
 # one ncu capture of the kernel named, valid only while its sources hash to
 # the value recorded with it (None otherwise). Full-size captures unless the
 # profile summary says it was scaled from a smaller case.
-_SC, _TK = "483be90f01b3", "b877d4d6299f"   # score_tc / topk_rows sources of the captures
+_SC, _INV, _TK = "b29d8789998d", "c482859cb74d", "8749fcc51b44"   # score_tc / score_inv / topk_rows sources
 TRAFFIC = {
-    ("dsa", "score_tc<bf16>"): (86.33e6 + 448.97e6, _SC),
-    ("dsa", "topk_rows"): (504.22e6 + 28.66e6, _TK),
-    ("decode", "score_tc<fp8>"): (1.11e9 + 33.55e6, _SC),
-    ("decode", "topk_rows"): (33.62e6, _TK),
-    ("misa", "topk_rows (k'=8192 over routed rows)"): (1.98e9 + 61.00e6, _TK),
-    ("misa", "score_tc<bf16> gathered (MISA-dagger re-score)"): (138.21e6 + 54.98e6, _SC),
-    ("misa", "topk_rows (k=2048 over k' candidates)"): (134.28e6 + 8.11e6, _TK),
-    ("hisa", "score_tc<bf16> gathered (HISA kept blocks)"): (264.02e6 + 66.76e6, _SC),
-    ("hisa", "topk_rows (k=2048 over m*block tokens)"): (67.70e6 + 1.11e6, _TK),
+    ("dsa", "score_tc"): (88.40e6 + 451.43e6, _SC),
+    ("dsa", "topk_rows"): (504.69e6 + 28.58e6, _TK),
+    ("decode", "score_tc fp8"): (1108.40e6 + 33.85e6, _SC),
+    ("decode", "topk_rows"): (33.63e6, _TK),
+    ("misa", "routed: score_tc"): (279.75e6 + 1019.77e6, _SC),
+    ("misa", "routed: topk_rows"): (1986.28e6 + 60.96e6, _TK),
+    ("misa", "re-score: score_tc gathered"): (137.48e6 + 54.51e6, _SC),
+    ("hisa", "tokens: score_inv (block-major)"): (81.49e6 + 33.05e6, _INV),
+    ("hisa", "tokens: topk_rows"): (67.71e6 + 1.39e6, _TK),
+    ("dsa_fp8", "score_tc fp8"): (45.22e6 + 446.36e6, _SC),
+    ("hisa_decode", "tokens: score_inv (block-major)"): (139.33e6 + 4.57e6, _INV),
+    ("misa_decode", "routed: score_tc fp8"): (1107.75e6 + 33.49e6, _SC),
 }
 KERNEL_SOURCES = {
     "score_tc": ("score_tc.cuh", "common.cuh"),

@@ -91,6 +91,16 @@ struct TkCfg {
   static constexpr int BYTES = WORDS * 4;
   static constexpr int OUT_CAP = 2 * CAP;  // output positions staged in the key + position space
   static constexpr int MIN_CTAS = MINC_;  // CTAs per SM the register budget is sized for
+  // Sample layout. Rows of up to 32768 scores: every S-th score, which
+  // touches every 32-byte sector of the row, so the sampling read brings the
+  // row into L2 for the band pass. Longer rows: runs of 32 consecutive
+  // scores every 32 S (a few KB of the row), since the rows in flight of a
+  // long-row launch do not fit in L2 and a row sampled into L2 would be
+  // evicted before its band pass and read from HBM twice.
+#ifndef DSA_TK_RUNS
+#define DSA_TK_RUNS 1
+#endif
+  static constexpr bool RUN_SAMPLE = DSA_TK_RUNS && BMW_ > 1024;
   static_assert(MINC_ * (BYTES + 1024) <= 228 * 1024, "shared memory for MIN_CTAS CTAs per SM");
 };
 using TkShort = TkCfg<1024, 2048, 4, 256, 4>;  // rows up to 32768: 44.5 KB, 4 CTAs per SM
@@ -299,7 +309,9 @@ __device__ bool topk_row_band(const TopkParams& p, uint32_t* sm, long long r, in
   float vmin = INFINITY, vmax = -INFINITY;
 #pragma unroll 8
   for (int m = tid; m < ns; m += TK_NT) {
-    const float x = __ldcg(row + static_cast<long long>(m) * S);
+    const long long pos = C::RUN_SAMPLE ? static_cast<long long>(m >> 5) * (32 * S) + (m & 31)
+                                        : static_cast<long long>(m) * S;
+    const float x = pos < n ? __ldcg(row + pos) : -INFINITY;
     fsamp[m] = x;
     if (present(x)) { ++nsv; vmin = fminf(vmin, x); vmax = fmaxf(vmax, x); }
   }
@@ -726,6 +738,92 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) topk_rows_kernel(const Top
       if (os) os[j] = -INFINITY;
     }
     __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- short rows
+// Rows of at most TK_SMALL scores: one warp per row, the row's keys in
+// registers (position 32 j + lane in slot j). The k-th largest present key
+// tau is found bit by bit from the top (tau = the largest t with at least
+// keff keys >= t; only the bits below the common prefix of the row's
+// smallest and largest present keys are searched); then the keys > tau and
+// the lowest-positioned keys equal to tau are written in position order
+// (ballots give each selected key its output slot). No shared memory, no
+// block barriers: one warp finishes a 2048-score row in a few thousand
+// instructions.
+constexpr int TK_SMALL = 2048;
+
+__global__ void __launch_bounds__(256) topk_small_kernel(const TopkParams p) {
+  constexpr int J = TK_SMALL / 32;
+  const int lane = threadIdx.x & 31;
+  const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const uint32_t lt = (1u << lane) - 1u;
+  for (long long r = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < p.rows;
+       r += nwarps) {
+    const int n = row_length(p, r);
+    const float* row = p.scores + r * p.ld;
+    uint32_t key[J];
+    uint32_t kmin = 0xffffffffu, kmax = 0u, cnt = 0u;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int pos = 32 * j + lane;
+      key[j] = pos < n ? score_key(__ldcg(row + pos)) : 0u;
+      if (key[j] != 0u) {
+        ++cnt;
+        kmin = min(kmin, key[j]);
+        kmax = max(kmax, key[j]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    const uint32_t keff = min(static_cast<uint32_t>(p.k), cnt);
+    uint32_t tau = kmin;  // keff == cnt, or every present key equal: tau = the smallest
+    if (keff > 0u && keff < cnt && kmin != kmax) {
+      // bits of tau above the highest bit where kmin and kmax differ are theirs
+      const int hb = 31 - __clz(kmin ^ kmax);
+      tau = kmax & ~((hb >= 31) ? 0xffffffffu : ((2u << hb) - 1u));
+      for (int b = hb; b >= 0; --b) {
+        const uint32_t t = tau | (1u << b);
+        uint32_t c = 0;
+#pragma unroll
+        for (int j = 0; j < J; ++j) c += key[j] >= t ? 1u : 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if (c >= keff) tau = t;
+      }
+    }
+    // keys above tau, then as many tau-equal keys (lowest positions) as fit
+    uint32_t above = 0;
+#pragma unroll
+    for (int j = 0; j < J; ++j) above += (keff > 0u && key[j] > tau) ? 1u : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+    const uint32_t need = keff - above;
+    int32_t* oi = p.out_idx + r * p.k;
+    float* os = p.out_score ? p.out_score + r * p.k : nullptr;
+    uint32_t eq_seen = 0, out = 0;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const bool eq = keff > 0u && key[j] == tau && key[j] != 0u;
+      const uint32_t em = __ballot_sync(0xffffffffu, eq);
+      const bool sel = (keff > 0u && key[j] > tau) || (eq && eq_seen + __popc(em & lt) < need);
+      eq_seen += __popc(em);
+      const uint32_t sm = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        const uint32_t o = out + __popc(sm & lt);
+        oi[o] = map_index(p, r, 32 * j + lane);
+        if (os) os[o] = key_score(key[j]);
+      }
+      out += __popc(sm);
+    }
+    for (int j = static_cast<int>(keff) + lane; j < p.k; j += 32) {
+      oi[j] = -1;
+      if (os) os[j] = -INFINITY;
+    }
   }
 }
 

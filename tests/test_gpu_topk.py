@@ -130,3 +130,45 @@ def test_many_long_rows_mass_ties():
     s = rng.integers(-3, 4, size=(rows, n)).astype(np.float32) * np.float32(0.5)
     idx, sc = _run(s, rows, 0, 0, n, k)
     _check(s, idx, sc, _expect(s, rows, 0, 0, n, k), "long rows, mass ties")
+
+
+@pytest.mark.parametrize("n,k", [(2048, 256), (2048, 2047), (1500, 1500), (2000, 3000), (64, 7), (1, 1)])
+def test_short_rows_one_warp_each(n, k):
+    # rows of at most 2048 scores (one warp per row): random values, mass ties
+    # with signed zeros, absent entries, NaN, all-equal rows, k >= n
+    rng = np.random.default_rng(n * 7 + k)
+    rows = 40
+    s = (rng.standard_normal((rows, n)) * 0.05).astype(np.float32)
+    s[1] = rng.integers(-3, 4, size=n).astype(np.float32) * np.float32(0.25)
+    s[2] = np.where(rng.random(n) < 0.5, np.float32(-0.0), np.float32(0.0))
+    s[3, rng.random(n) < 0.6] = -np.inf
+    s[4] = -np.inf
+    s[5] = np.float32(1.5)
+    s[6, rng.random(n) < 0.2] = np.nan
+    s[7, : n // 2] = -np.inf
+    idx, sc = _run(s, rows, 0, 0, n, k)
+    exp_in = s.copy()
+    exp_in[np.isnan(exp_in)] = -np.inf  # NaN is absent too
+    exp = _expect(exp_in, rows, 0, 0, n, k)
+    _check(s, idx, sc, exp, f"short n={n} k={k}")
+    sel = exp >= 0
+    r_ = np.repeat(np.arange(rows)[:, None], k, axis=1)
+    want = exp_in[r_[sel], exp[sel]]
+    assert np.array_equal(sc[sel], np.where(want == 0, np.float32(0.0), want))
+
+
+def test_short_rows_causal_lengths_and_maps():
+    # many short rows (more than one row per warp of the grid), per-query
+    # causal lengths, pooled-block strides and a block index map
+    rng = np.random.default_rng(21)
+    T, L = 3000, 2048
+    s = rng.standard_normal((T, L)).astype(np.float32)
+    idx, sc = _run(s, T, 100, 1, L, 128)
+    _check(s, idx, sc, _expect(s, T, 100, 1, L, 128), "short causal")
+    idx, sc = _run(s[:50], 50, 5000, 4, L, 300)
+    _check(s[:50], idx, sc, _expect(s[:50], 50, 5000, 4, L, 300), "short block stride")
+    m, blk = 8, 128
+    cand = np.sort(rng.choice(4000, size=(20, m), replace=False), axis=1).astype(np.int32)
+    s2 = rng.standard_normal((20, m * blk)).astype(np.float32)
+    idx, sc = _run(s2, 20, 0, 0, m * blk, 200, cand=cand, n_slots=m, blk=blk)
+    _check(s2, idx, sc, _expect(s2, 20, 0, 0, m * blk, 200, cand=cand, blk=blk), "short block map")
