@@ -307,13 +307,22 @@ __device__ bool topk_row_band(const TopkParams& p, uint32_t* sm, long long r, in
   for (int i = tid; i < TK_BINS; i += TK_NT) hist[i] = 0;
   uint32_t nsv = 0;
   float vmin = INFINITY, vmax = -INFINITY;
-#pragma unroll 8
-  for (int m = tid; m < ns; m += TK_NT) {
-    const long long pos = C::RUN_SAMPLE ? static_cast<long long>(m >> 5) * (32 * S) + (m & 31)
-                                        : static_cast<long long>(m) * S;
-    const float x = pos < n ? __ldcg(row + pos) : -INFINITY;
-    fsamp[m] = x;
-    if (present(x)) { ++nsv; vmin = fminf(vmin, x); vmax = fmaxf(vmax, x); }
+  // eight samples per thread in flight: all loads first, then their uses
+  for (int m0 = tid; m0 < ns; m0 += 8 * TK_NT) {
+    float xs[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int m = m0 + u * TK_NT;
+      const long long pos = C::RUN_SAMPLE ? static_cast<long long>(m >> 5) * (32 * S) + (m & 31)
+                                          : static_cast<long long>(m) * S;
+      xs[u] = (m < ns && pos < n) ? __ldcg(row + pos) : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int m = m0 + u * TK_NT;
+      if (m < ns) fsamp[m] = xs[u];
+      if (present(xs[u])) { ++nsv; vmin = fminf(vmin, xs[u]); vmax = fmaxf(vmax, xs[u]); }
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -764,10 +773,18 @@ __global__ void __launch_bounds__(256) topk_small_kernel(const TopkParams p) {
     const float* row = p.scores + r * p.ld;
     uint32_t key[J];
     uint32_t kmin = 0xffffffffu, kmax = 0u, cnt = 0u;
+    // all loads first (64 in flight per lane), then the keys
 #pragma unroll
     for (int j = 0; j < J; ++j) {
       const int pos = 32 * j + lane;
-      key[j] = pos < n ? score_key(__ldcg(row + pos)) : 0u;
+      key[j] = pos < n ? __float_as_uint(__ldcg(row + pos)) : 0xff800000u;  // -inf past the row
+    }
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      key[j] = score_key(__uint_as_float(key[j]));
+      // keep the key in its register: the search below reads it many times
+      // and must not re-issue the load
+      asm volatile("" : "+r"(key[j]));
       if (key[j] != 0u) {
         ++cnt;
         kmin = min(kmin, key[j]);
@@ -786,14 +803,18 @@ __global__ void __launch_bounds__(256) topk_small_kernel(const TopkParams p) {
       // bits of tau above the highest bit where kmin and kmax differ are theirs
       const int hb = 31 - __clz(kmin ^ kmax);
       tau = kmax & ~((hb >= 31) ? 0xffffffffu : ((2u << hb) - 1u));
-      for (int b = hb; b >= 0; --b) {
+      // count(key >= tau) >= keff holds throughout; once it is exactly keff
+      // the keys >= tau are the selection and the lower bits do not matter
+      uint32_t clo = cnt;
+      for (int b = hb; b >= 0 && clo != keff; --b) {
         const uint32_t t = tau | (1u << b);
-        uint32_t c = 0;
+        uint32_t c4[4] = {0u, 0u, 0u, 0u};  // four chains of adds
 #pragma unroll
-        for (int j = 0; j < J; ++j) c += key[j] >= t ? 1u : 0u;
+        for (int j = 0; j < J; ++j) c4[j & 3] += key[j] >= t ? 1u : 0u;
+        uint32_t c = (c4[0] + c4[1]) + (c4[2] + c4[3]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-        if (c >= keff) tau = t;
+        if (c >= keff) { tau = t; clo = c; }
       }
     }
     // keys above tau, then as many tau-equal keys (lowest positions) as fit
