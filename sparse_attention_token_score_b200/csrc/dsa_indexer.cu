@@ -345,11 +345,10 @@ dsa_status launch_topk_cfg(const TopkParams& tp, cudaStream_t st) {
 dsa_status launch_topk(void* ws, TopkParams tp, cudaStream_t st) {
   tp.err = static_cast<unsigned*>(ws);
   if (tp.Lrow <= TK_SMALL && tp.cres == nullptr) {
-    // short rows: one warp per row, 8 rows per CTA
-    const long long ctas = (tp.rows + 7) / 8;
-    const long long cap = static_cast<long long>(num_sms()) * 8;
+    // short rows: one 128-thread CTA per row, up to 16 CTAs per SM
+    const long long cap = static_cast<long long>(num_sms()) * 16;
     prof::Launch pl(st, "topk_rows");
-    topk_small_kernel<<<static_cast<int>(ctas < cap ? ctas : cap), 256, 0, st>>>(tp);
+    topk_small_kernel<<<static_cast<int>(tp.rows < cap ? tp.rows : cap), TK_SNT, 0, st>>>(tp);
     return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
   }
   if (tp.Lrow <= TkShort::MAX_ROW) return launch_topk_cfg<TkShort>(tp, st);

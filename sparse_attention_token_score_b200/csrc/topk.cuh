@@ -751,52 +751,73 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) topk_rows_kernel(const Top
 }
 
 // ---------------------------------------------------------------- short rows
-// Rows of at most TK_SMALL scores: one warp per row, the row's keys in
-// registers (position 32 j + lane in slot j). The k-th largest present key
-// tau is found bit by bit from the top (tau = the largest t with at least
-// keff keys >= t; only the bits below the common prefix of the row's
-// smallest and largest present keys are searched); then the keys > tau and
-// the lowest-positioned keys equal to tau are written in position order
-// (ballots give each selected key its output slot). No shared memory, no
-// block barriers: one warp finishes a 2048-score row in a few thousand
-// instructions.
+// Rows of at most TK_SMALL scores: one 128-thread CTA per row (grid-stride
+// over rows), 16 keys per thread in registers (position tid + 128 j in slot
+// j). The keff-th largest present key tau is found bit by bit from the top
+// (tau = the largest t with at least keff keys >= t; only the bits below the
+// common prefix of the row's smallest and largest present keys are searched,
+// and the search stops once the keys >= the current prefix are exactly
+// keff). Then the keys > tau and the lowest-positioned keys equal to tau are
+// written in position order (per 128 positions: warp ballots, the four
+// warps' counts through shared memory). Every step is a few instructions per
+// thread and one CTA barrier; no histogram, no sample.
 constexpr int TK_SMALL = 2048;
+constexpr int TK_SNT = 128;                   // threads per row
+constexpr int TK_SKPT = TK_SMALL / TK_SNT;    // keys per thread
 
-__global__ void __launch_bounds__(256) topk_small_kernel(const TopkParams p) {
-  constexpr int J = TK_SMALL / 32;
-  const int lane = threadIdx.x & 31;
-  const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+__global__ void __launch_bounds__(TK_SNT) topk_small_kernel(const TopkParams p) {
+  constexpr int J = TK_SKPT, NW = TK_SNT / 32;
+  __shared__ uint32_t red[2][3][NW];          // double-buffered warp partials
+  __shared__ uint32_t wcnt[2][NW];            // emit: selected / tau-equal keys per warp
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const uint32_t lt = (1u << lane) - 1u;
-  for (long long r = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < p.rows;
-       r += nwarps) {
+  int par = 0;                                // which red buffer the next reduction uses
+  // sum (a), min (b) and max (c) over the CTA; one barrier
+  auto reduce3 = [&](uint32_t& a, uint32_t& b2, uint32_t& c) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a += __shfl_xor_sync(0xffffffffu, a, o);
+      b2 = min(b2, __shfl_xor_sync(0xffffffffu, b2, o));
+      c = max(c, __shfl_xor_sync(0xffffffffu, c, o));
+    }
+    if (lane == 0) { red[par][0][wid] = a; red[par][1][wid] = b2; red[par][2][wid] = c; }
+    __syncthreads();
+    a = 0u; b2 = 0xffffffffu; c = 0u;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) { a += red[par][0][w]; b2 = min(b2, red[par][1][w]); c = max(c, red[par][2][w]); }
+    par ^= 1;
+  };
+  auto reduce_sum = [&](uint32_t a) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) red[par][0][wid] = a;
+    __syncthreads();
+    a = 0u;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) a += red[par][0][w];
+    par ^= 1;
+    return a;
+  };
+  for (long long r = blockIdx.x; r < p.rows; r += gridDim.x) {
     const int n = row_length(p, r);
     const float* row = p.scores + r * p.ld;
     uint32_t key[J];
-    uint32_t kmin = 0xffffffffu, kmax = 0u, cnt = 0u;
-    // all loads first (64 in flight per lane), then the keys
 #pragma unroll
     for (int j = 0; j < J; ++j) {
-      const int pos = 32 * j + lane;
+      const int pos = tid + TK_SNT * j;
       key[j] = pos < n ? __float_as_uint(__ldcg(row + pos)) : 0xff800000u;  // -inf past the row
     }
+    uint32_t cnt = 0u, kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
     for (int j = 0; j < J; ++j) {
       key[j] = score_key(__uint_as_float(key[j]));
-      // keep the key in its register: the search below reads it many times
-      // and must not re-issue the load
-      asm volatile("" : "+r"(key[j]));
       if (key[j] != 0u) {
         ++cnt;
         kmin = min(kmin, key[j]);
         kmax = max(kmax, key[j]);
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-    }
+    reduce3(cnt, kmin, kmax);
     const uint32_t keff = min(static_cast<uint32_t>(p.k), cnt);
     uint32_t tau = kmin;  // keff == cnt, or every present key equal: tau = the smallest
     if (keff > 0u && keff < cnt && kmin != kmax) {
@@ -808,43 +829,59 @@ __global__ void __launch_bounds__(256) topk_small_kernel(const TopkParams p) {
       uint32_t clo = cnt;
       for (int b = hb; b >= 0 && clo != keff; --b) {
         const uint32_t t = tau | (1u << b);
-        uint32_t c4[4] = {0u, 0u, 0u, 0u};  // four chains of adds
+        uint32_t c = 0u;
 #pragma unroll
-        for (int j = 0; j < J; ++j) c4[j & 3] += key[j] >= t ? 1u : 0u;
-        uint32_t c = (c4[0] + c4[1]) + (c4[2] + c4[3]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        for (int j = 0; j < J; ++j) c += key[j] >= t ? 1u : 0u;
+        c = reduce_sum(c);
         if (c >= keff) { tau = t; clo = c; }
       }
     }
     // keys above tau, then as many tau-equal keys (lowest positions) as fit
-    uint32_t above = 0;
+    uint32_t above = 0u;
 #pragma unroll
     for (int j = 0; j < J; ++j) above += (keff > 0u && key[j] > tau) ? 1u : 0u;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+    above = reduce_sum(above);
     const uint32_t need = keff - above;
     int32_t* oi = p.out_idx + r * p.k;
     float* os = p.out_score ? p.out_score + r * p.k : nullptr;
-    uint32_t eq_seen = 0, out = 0;
+    uint32_t eq_seen = 0u, out = 0u;
 #pragma unroll
     for (int j = 0; j < J; ++j) {
+      // positions 128 j .. 128 j + 127: warp w holds 32 w .. 32 w + 31
+      const bool gt = keff > 0u && key[j] > tau;
       const bool eq = keff > 0u && key[j] == tau && key[j] != 0u;
       const uint32_t em = __ballot_sync(0xffffffffu, eq);
-      const bool sel = (keff > 0u && key[j] > tau) || (eq && eq_seen + __popc(em & lt) < need);
-      eq_seen += __popc(em);
+      const uint32_t gm = __ballot_sync(0xffffffffu, gt);
+      if (lane == 0) { wcnt[j & 1][wid] = __popc(em); red[par][0][wid] = __popc(gm); }
+      __syncthreads();
+      uint32_t eq_before = eq_seen, gt_before = 0u, eq_tot = 0u, gt_tot = 0u;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const uint32_t e = wcnt[j & 1][w], g = red[par][0][w];
+        if (w < wid) { eq_before += e; gt_before += g; }
+        eq_tot += e;
+        gt_tot += g;
+      }
+      par ^= 1;
+      // tau-equal keys taken before this warp's: min(need, eq_seen + earlier warps')
+      const uint32_t eq_rank = eq_before + __popc(em & lt);
+      const bool sel = gt || (eq && eq_rank < need);
+      const uint32_t taken_before = min(need, eq_before);
       const uint32_t sm = __ballot_sync(0xffffffffu, sel);
       if (sel) {
-        const uint32_t o = out + __popc(sm & lt);
-        oi[o] = map_index(p, r, 32 * j + lane);
+        const uint32_t o = out + gt_before + taken_before - min(need, eq_seen) + __popc(sm & lt);
+        oi[o] = map_index(p, r, tid + TK_SNT * j);
         if (os) os[o] = key_score(key[j]);
       }
-      out += __popc(sm);
+      const uint32_t taken_all = min(need, eq_seen + eq_tot) - min(need, eq_seen);
+      out += gt_tot + taken_all;
+      eq_seen += eq_tot;
     }
-    for (int j = static_cast<int>(keff) + lane; j < p.k; j += 32) {
+    for (int j = static_cast<int>(keff) + tid; j < p.k; j += TK_SNT) {
       oi[j] = -1;
       if (os) os[j] = -INFINITY;
     }
+    __syncthreads();  // the next row reuses the shared words
   }
 }
 
