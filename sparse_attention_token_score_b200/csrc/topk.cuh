@@ -751,22 +751,20 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) topk_rows_kernel(const Top
 }
 
 // ---------------------------------------------------------------- short rows
-// Rows of at most TK_SMALL scores: one 128-thread CTA per row (grid-stride
-// over rows), 16 keys per thread in registers (position tid + 128 j in slot
-// j). The keff-th largest present key tau is found bit by bit from the top
+// Rows of at most NT * KPT scores (2048: 128 threads x 16 keys): one CTA per
+// row (grid-stride over rows), KPT keys per
+// thread in registers (position tid + NT j in slot j). The keff-th largest present key tau is found bit by bit from the top
 // (tau = the largest t with at least keff keys >= t; only the bits below the
 // common prefix of the row's smallest and largest present keys are searched,
 // and the search stops once the keys >= the current prefix are exactly
 // keff). Then the keys > tau and the lowest-positioned keys equal to tau are
-// written in position order (per 128 positions: warp ballots, the four
-// warps' counts through shared memory). Every step is a few instructions per
-// thread and one CTA barrier; no histogram, no sample.
-constexpr int TK_SMALL = 2048;
-constexpr int TK_SNT = 128;                   // threads per row
-constexpr int TK_SKPT = TK_SMALL / TK_SNT;    // keys per thread
-
-__global__ void __launch_bounds__(TK_SNT) topk_small_kernel(const TopkParams p) {
-  constexpr int J = TK_SKPT, NW = TK_SNT / 32;
+// written in position order (per NT positions: warp ballots, the warps'
+// counts through shared memory). Every step is a few instructions per thread
+// and one CTA barrier; no histogram, no sample.
+template <int NT, int KPT>
+__global__ void __launch_bounds__(NT) topk_small_kernel(const TopkParams p) {
+  constexpr int J = KPT, NW = NT / 32;
+  constexpr int TK_SNT = NT;
   __shared__ uint32_t red[2][3][NW];          // double-buffered warp partials
   __shared__ uint32_t wcnt[2][NW];            // emit: selected / tau-equal keys per warp
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;

@@ -132,10 +132,12 @@ def test_many_long_rows_mass_ties():
     _check(s, idx, sc, _expect(s, rows, 0, 0, n, k), "long rows, mass ties")
 
 
-@pytest.mark.parametrize("n,k", [(2048, 256), (2048, 2047), (1500, 1500), (2000, 3000), (64, 7), (1, 1)])
-def test_short_rows_one_warp_each(n, k):
-    # rows of at most 2048 scores (one warp per row): random values, mass ties
-    # with signed zeros, absent entries, NaN, all-equal rows, k >= n
+@pytest.mark.parametrize("n,k", [(2048, 256), (2048, 2047), (1500, 1500), (2000, 3000), (64, 7), (1, 1),
+                                 (3000, 100), (8192, 2048), (12000, 13000), (16384, 2048)])
+def test_short_rows_one_cta_each(n, k):
+    # rows of at most 2048 scores take one CTA per row (keys in registers),
+    # longer ones the sampled-band CTAs: random values, mass ties with signed zeros, absent entries, NaN,
+    # all-equal rows, k >= n
     rng = np.random.default_rng(n * 7 + k)
     rows = 40
     s = (rng.standard_normal((rows, n)) * 0.05).astype(np.float32)
