@@ -257,15 +257,17 @@ class Runner:
 # one ncu capture of the kernel named, valid only while its sources hash to
 # the value recorded with it (None otherwise). Full-size captures unless the
 # profile summary says it was scaled from a smaller case.
-_SC, _INV, _TK = "b29d8789998d", "c482859cb74d", "8749fcc51b44"   # score_tc / score_inv / topk_rows sources
+_SC, _INV, _TK = "b29d8789998d", "c482859cb74d", "778ac90fa8a8"   # score_tc / score_inv / topk_rows sources
 TRAFFIC = {
     ("dsa", "score_tc"): (88.40e6 + 451.43e6, _SC),
-    ("dsa", "topk_rows"): (504.69e6 + 28.58e6, _TK),
+    ("dsa", "topk_rows"): (504.61e6 + 28.62e6, _TK),
+    ("tiny", "topk_rows"): (8.56e6, _TK),
     ("decode", "score_tc fp8"): (1108.40e6 + 33.85e6, _SC),
     ("decode", "topk_rows"): (33.63e6, _TK),
     ("misa", "routed: score_tc"): (279.75e6 + 1019.77e6, _SC),
-    ("misa", "routed: topk_rows"): (1986.28e6 + 60.96e6, _TK),
+    ("misa", "routed: topk_rows"): (1349.15e6 + 60.24e6, _TK),
     ("misa", "re-score: score_tc gathered"): (137.48e6 + 54.51e6, _SC),
+    ("hisa", "blocks: topk_rows"): (8.43e6, _TK),
     ("hisa", "tokens: score_inv (block-major)"): (81.49e6 + 33.05e6, _INV),
     ("hisa", "tokens: topk_rows"): (67.71e6 + 1.39e6, _TK),
     ("dsa_fp8", "score_tc fp8"): (45.22e6 + 446.36e6, _SC),
@@ -345,14 +347,25 @@ def run_e2e(r, inp, steps, torch, barrier):
     inputs host -> device from pinned memory, runs the call and copies its
     indices device -> host. Two buffer sets on three streams (copy in, call,
     copy out) let a step's copies overlap the previous step's call, as a
-    server streaming batches would. Returns (device ms of the `steps` steps,
-    H2D bytes per step, D2H bytes per step)."""
+    server streaming batches would. Decode workloads keep the key cache
+    resident (it is the model's cache): a step copies its queries, weights
+    and query scales and the one new key row (and scale) per sequence, which
+    it writes at the cache's last position. Returns (device ms of the `steps`
+    steps, H2D bytes per step, D2H bytes per step)."""
     from sparse_attention_token_score_b200 import binding as B
+    decode = r.c.get("kind") == "decode"
     srcs = r.dev
     host = [t.cpu().pin_memory() if t is not None else None for t in srcs]
+    L = inp.L
+    if decode:  # the cache stays on the device; only the newest row per sequence travels
+        host[1] = srcs[1][:, L - 1:L].cpu().pin_memory()
+        host[4] = srcs[4][:, L - 1:L].cpu().pin_memory()
+        cache_k, cache_ks = srcs[1].clone(), srcs[4].clone()
     sets = []
     for _ in range(2):
         dev = [torch.empty_like(t) if t is not None else None for t in srcs]
+        if decode:
+            dev[1], dev[4] = cache_k, cache_ks
         sets.append({"dev": dev, "args": B.make_args(dev[0], dev[1], dev[2], inp.q_offset, dev[3], dev[4]),
                      "idx": torch.empty_like(r.idx),
                      "out": torch.empty(r.idx.shape, dtype=torch.int32, pin_memory=True),
@@ -362,9 +375,15 @@ def run_e2e(r, inp, steps, torch, barrier):
     def issue(i):
         b = sets[i % 2]
         s_in.wait_event(b["done"])      # the call of step i - 2 has read this set's inputs
+        if decode:                       # and step i - 1's call has read the shared cache
+            s_in.wait_event(sets[(i + 1) % 2]["done"])
         with torch.cuda.stream(s_in):
-            for h, d in zip(host, b["dev"]):
-                if h is not None:
+            for j, (h, d) in enumerate(zip(host, b["dev"])):
+                if h is None:
+                    continue
+                if decode and j in (1, 4):
+                    d[:, L - 1:L].copy_(h, non_blocking=True)
+                else:
                     d.copy_(h, non_blocking=True)
             b["loaded"].record(s_in)
         s_run.wait_event(b["loaded"])
@@ -688,7 +707,9 @@ def measure_workload(name, args, torch, world, rank, local, flush, barrier, rmax
         "queries_per_s": world * r.batch * c["T"] * steps / (total_ms / 1e3),
         "roofline": roof, "kernels": per_kernel, "cpu_baseline": cpu,
         "e2e": {"value": e_pairs_per_s / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e_ms / steps, "pipeline": "2 buffer sets, copy-in / call / copy-out streams"},
+                "ms_per_step": e_ms / steps, "pipeline": "2 buffer sets, copy-in / call / copy-out streams",
+                **({"key_cache": "resident; each step copies one new key row (and scale) per sequence"}
+                   if r.c.get("kind") == "decode" else {})},
         "gpu_launches": int(round(launches_per_step * steps)), "clocks": clocks,
         "step_ms": {"min": min(times), "median": statistics.median(times), "max": max(times)},
     }
