@@ -100,7 +100,7 @@ constexpr int CCHUNK = 64;  // candidate slots reserved per warp and query at a 
 enum : int { kEpiStore = 0, kEpiCand = 1, kEpiBound = 2 };
 
 template <int ELEM_, int D_, int H_, int QPT_, ScoreMode MODE_, int NSTAGE_, int EPIW_ = 8, int NQBUF_ = 1,
-          int EPI_ = kEpiStore, bool LIST_ = false>
+          int EPI_ = kEpiStore, bool LIST_ = false, int CTAS_ = 1>
 struct ScoreCfg {
   static constexpr int ELEM = ELEM_;  // bytes per element: 2 = bf16, 1 = e4m3
   static constexpr int D = D_, H = H_, QPT = QPT_, NSTAGE = NSTAGE_;
@@ -139,7 +139,12 @@ struct ScoreCfg {
   // columns (at most DSA_NACC_MAX). Narrow tiles (one query per group) carry
   // little MMA work each, so with two buffers the MMA -> epilogue -> MMA
   // round trip would set the pace; more buffers let the MMAs run ahead.
-  static constexpr int NACC = (512 / MMA_N < DSA_NACC_MAX) ? 512 / MMA_N : DSA_NACC_MAX;
+  // CTAs per SM: 1, or 2 for streams that want more loads in flight than one
+  // CTA's shared memory holds (each then owns half of TMEM and of the SM's
+  // registers, and its epilogue keeps one TMEM chunk in flight per warp)
+  static constexpr int CTAS = CTAS_;
+  static_assert(CTAS == 1 || (CTAS == 2 && !ROUTER), "CTAs per SM");
+  static constexpr int NACC = ((512 / CTAS) / MMA_N < DSA_NACC_MAX) ? (512 / CTAS) / MMA_N : DSA_NACC_MAX;
   static_assert(NACC >= 2 && (NACC & (NACC - 1)) == 0, "accumulator buffers");
   static constexpr int TMEM_COLS = (NACC * MMA_N <= 32) ? 32 : (NACC * MMA_N <= 64) ? 64
                                  : (NACC * MMA_N <= 128) ? 128 : (NACC * MMA_N <= 256) ? 256 : 512;
@@ -178,8 +183,9 @@ struct ScoreCfg {
   static constexpr int NBAR = 2 * NSTAGE + 2 * NQBUF + 2 * NACC + 1;
   static constexpr int SMEM_USED = SMEM_BAR + NBAR * 8 + 16;
   // Pad to more than half an SM so two CTAs never share an SM's TMEM.
-  static constexpr int SMEM_BYTES = (SMEM_USED + 1024 < 120 * 1024) ? 120 * 1024 : SMEM_USED + 1024;
-  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static constexpr int SMEM_BYTES = CTAS == 2 ? SMEM_USED + 1024
+                                   : ((SMEM_USED + 1024 < 120 * 1024) ? 120 * 1024 : SMEM_USED + 1024);
+  static_assert(SMEM_BYTES <= (CTAS == 2 ? 112 * 1024 : 227 * 1024), "shared memory");
 };
 
 // Iterates this CTA's (group, tile) pairs. Every thread runs its own copy;
@@ -369,7 +375,7 @@ __global__ void pairs_build_kernel(const uint8_t* __restrict__ flags, long long 
 }
 
 template <class C>
-__global__ void __launch_bounds__(C::NTHREADS, 1)
+__global__ void __launch_bounds__(C::NTHREADS, C::CTAS)
 score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const ScoreParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -756,7 +762,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int j = 0; j < NP; ++j) acc2[i][j] = 0ull;
 #endif
-          if constexpr (C::EPIW == 16) {
+          if constexpr (C::EPIW == 16 || C::CTAS == 2) {
             // Sixteen epilogue warps (four per sub-partition, 96 registers a
             // thread): one 32-column chunk in flight per warp, the other
             // warps hide its load latency; head weights read four at a time.
