@@ -296,8 +296,14 @@ dsa_status run_router_fp8(int D, int H, const ScoreParams& p, const void* q, lon
 #ifndef DSA_GATHER_NQ
 #define DSA_GATHER_NQ 2
 #endif
+// FP8 gathers (decode MISA-dagger candidates, decode HISA kept blocks): two
+// CTAs per SM with 5 stages each (decode HISA token stage: 0.089 -> 0.080 ms
+// with the kept blocks streaming by TMA; 0.125 ms block major).
 #ifndef DSA_GATHER8_NS
-#define DSA_GATHER8_NS 8
+#define DSA_GATHER8_NS 5
+#endif
+#ifndef DSA_GATHER8_CTAS
+#define DSA_GATHER8_CTAS 2
 #endif
 dsa_status run_gather(int D, int H, ScoreParams p, const void* q, long long q_rows,
                       cudaStream_t st, bool fp8 = false) {
@@ -305,11 +311,11 @@ dsa_status run_gather(int D, int H, ScoreParams p, const void* q, long long q_ro
   const long long k_rows = static_cast<long long>(p.batch) * p.L_tok;
   if (fp8) {  // e4m3 rows of 128 bytes, per-token key scales (p.k_scale)
     if (D == 128 && H == 64)
-      return launch_score<ScoreCfg<1, 128, 64, 1, ScoreMode::kGather, DSA_GATHER8_NS, 8, DSA_GATHER_NQ>>(
-          p, q, q_rows, p.kg, k_rows, st);
+      return launch_score<ScoreCfg<1, 128, 64, 1, ScoreMode::kGather, DSA_GATHER8_NS, 8, DSA_GATHER_NQ, kEpiStore,
+                                   false, DSA_GATHER8_CTAS>>(p, q, q_rows, p.kg, k_rows, st);
     if (D == 128 && H == 32)
-      return launch_score<ScoreCfg<1, 128, 32, 1, ScoreMode::kGather, DSA_GATHER8_NS, 8, DSA_GATHER_NQ>>(
-          p, q, q_rows, p.kg, k_rows, st);
+      return launch_score<ScoreCfg<1, 128, 32, 1, ScoreMode::kGather, DSA_GATHER8_NS, 8, DSA_GATHER_NQ, kEpiStore,
+                                   false, DSA_GATHER8_CTAS>>(p, q, q_rows, p.kg, k_rows, st);
     return DSA_ERR_UNSUPPORTED;
   }
   if (D == 128 && H == 64)
@@ -1254,8 +1260,14 @@ dsa_status hisa_run(const dsa_indexer_args* a, int block, int m, int topk, const
   hisa_stage.set("tokens");
   // 4. token scores inside the kept blocks (compact rows of m * block):
   // block-major over the inverted kept-block lists when blocks are whole key
-  // tiles, else one query per tile with gathered rows
-  if (inv_supported(a, block)) {
+  // tiles and a sequence has several queries to share them; with one query
+  // per sequence (decode) nothing is shared, so its query stays stationary
+  // and its kept blocks stream through whole-tile TMA loads (the gather
+  // path); blocks that are not whole tiles are gathered row by row
+#ifndef DSA_HISA_DECODE_GATHER
+#define DSA_HISA_DECODE_GATHER 1
+#endif
+  if (inv_supported(a, block) && !(DSA_HISA_DECODE_GATHER && a->T == 1)) {
     const InvWs w = inv_carve(c, BT, m, a->batch * M, block, a->H);
     DSA_TRY(run_refine_inverted(a, blocks, m, block, compact, ncomp, w, err, st));
     return launch_topk(ws, topk_params(compact, BT, ncomp, a->T, a->q_offset, 0, ncomp, topk, out_idx,
