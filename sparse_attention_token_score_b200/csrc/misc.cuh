@@ -73,46 +73,70 @@ __global__ void __launch_bounds__(256) meanpool_vec_kernel(const __nv_bfloat16* 
 // block the fp64 mean of the dequantised keys (code value x per-token scale),
 // a scale absmax/448 (absmax rounded to fp32, divided in fp32; 1 when the
 // mean is zero) and codes e4m3(mean / scale), rounded to nearest even with
-// saturation. 4 * d threads (d <= 128): thread (g, c) sums column c over
-// tokens g, g + 4, ... of the block (independent loads, eight in flight);
-// the four partial sums of a column are added in shared memory. The fp64
-// sums are exact here, so the order does not change the result.
+// saturation. 512 threads, d % 4 == 0, d <= 128, rows 4-byte aligned: thread
+// (g, c) reads bytes 4c .. 4c + 3 of token rows g, g + G, ... of the block
+// (G = 512 / (d / 4) row groups), eight rows and their scales loaded before
+// any of them is used, so a block of up to 8 G tokens costs one round trip to
+// memory; the G partial sums of a column are added in shared memory. The
+// fp64 sums are exact here, so the order does not change the result.
 __global__ void __launch_bounds__(512) meanpool_fp8_kernel(const uint8_t* __restrict__ k8,
                                                            const float* __restrict__ ks, int L, int d, int B,
                                                            int M, int m0, int nm, uint8_t* __restrict__ kbar8,
                                                            float* __restrict__ kbar_scale) {
-  __shared__ double part[4 * 128];
-  __shared__ double red[32];
+  __shared__ double part[2048];  // [G][d]: G * d = 4 * 512
+  __shared__ double red[16];
   const long long b = blockIdx.x / nm;
   const int m = m0 + static_cast<int>(blockIdx.x % nm);
   const long long bm = b * M + m;
   const int s0 = m * B;
   const int s1 = min(s0 + B, L);
-  const int g = threadIdx.x / d, c = threadIdx.x % d;
-  double acc = 0.0;
-#pragma unroll 8
-  for (int s = s0 + g; s < s1; s += 4) {
-    __nv_fp8_e4m3 v;
-    v.__x = k8[(b * L + s) * d + c];
-    acc += static_cast<double>(static_cast<float>(v)) * static_cast<double>(__ldg(ks + b * L + s));
+  const int tpr = d / 4;  // threads per token row
+  const int G = 512 / tpr;  // row groups
+  const int g = threadIdx.x / tpr, c = threadIdx.x % tpr;
+  if (g < G) {
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int sb = s0 + g; sb < s1; sb += 8 * G) {
+      uint32_t v[8];
+      float sc[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int s = sb + u * G;
+        v[u] = s < s1 ? __ldg(reinterpret_cast<const uint32_t*>(k8 + (b * L + s) * d) + c) : 0u;
+        sc[u] = s < s1 ? __ldg(ks + b * L + s) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          __nv_fp8_e4m3 x;
+          x.__x = static_cast<__nv_fp8_storage_t>((v[u] >> (8 * e)) & 0xffu);
+          acc[e] += static_cast<double>(static_cast<float>(x)) * static_cast<double>(sc[u]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) part[g * d + 4 * c + e] = acc[e];
   }
-  part[g * d + c] = acc;
   __syncthreads();
+  const int col = threadIdx.x;
   double mean = 0.0;
-  if (threadIdx.x < d)
-    mean = (((part[c] + part[d + c]) + part[2 * d + c]) + part[3 * d + c]) / static_cast<double>(s1 - s0);
-  double a = threadIdx.x < d ? fabs(mean) : 0.0;
+  if (col < d) {
+    double sum = 0.0;
+    for (int i = 0; i < G; ++i) sum += part[i * d + col];
+    mean = sum / static_cast<double>(s1 - s0);
+  }
+  double a = col < d ? fabs(mean) : 0.0;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) a = fmax(a, __shfl_xor_sync(0xffffffffu, a, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  if ((col & 31) == 0) red[col >> 5] = a;
   __syncthreads();
   double amax = 0.0;
-  for (int w = 0; w < static_cast<int>((blockDim.x + 31) >> 5); ++w) amax = fmax(amax, red[w]);
+  for (int w = 0; w < 16; ++w) amax = fmax(amax, red[w]);
   const float af = static_cast<float>(amax);
   const float scale = af > 0.f ? af / 448.f : 1.f;
-  if (threadIdx.x < d)
-    kbar8[bm * d + c] = static_cast<uint8_t>(__nv_cvt_double_to_fp8(mean / static_cast<double>(scale), __NV_SATFINITE, __NV_E4M3));
-  if (threadIdx.x == 0) kbar_scale[bm] = scale;
+  if (col < d)
+    kbar8[bm * d + col] = static_cast<uint8_t>(
+        __nv_cvt_double_to_fp8(mean / static_cast<double>(scale), __NV_SATFINITE, __NV_E4M3));
+  if (col == 0) kbar_scale[bm] = scale;
 }
 
 // MISA routing (same page, "Methodology", step 1): per query, the head

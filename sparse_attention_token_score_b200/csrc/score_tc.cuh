@@ -172,6 +172,9 @@ struct ScoreCfg {
   // gathers, by the key's token). The router weights its pooled-key columns
   // by their scales instead.
   static constexpr bool KEY_SCALES = ELEM == 1 && !ROUTER;
+  // the plain store epilogue (bf16, eight warps, one CTA per SM) has a loop of its own
+  static constexpr bool PLAIN = EPI_ == kEpiStore && !LIST_ && ELEM == 2 && !ROUTER && !GATHER && EPIW == 8 &&
+                                CTAS_ == 1 && !SPLIT_TILES;
   // per epilogue warp: the head weights (x query scales) of its columns for
   // the current query group, refilled when the group changes
   static constexpr int NCOL_THREAD = ROUTER ? 0 : (SPLIT_TILES ? QROWS : QROWS / NSETS);
@@ -615,6 +618,108 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float racc = 0.f;                          // router partial sum
     int coef_g = -1;                           // query group of the staged head weights
     uint32_t it = 0;
+    if constexpr (C::PLAIN) {
+      // Plain bf16 scores with eight epilogue warps (the dense 64-head tile):
+      // the store path alone, without the variants' code below (with it in
+      // the loop the same work compiled to code 3 % slower on the DSA chunk).
+      for (; !s.done; s.next(p), ++it) {
+        const int b = s.b;
+        const int tg = s.tg;
+        const int buf = static_cast<int>(it % C::NACC);
+        if (!mbar_wait(tfull(buf), (it / C::NACC) & 1u, p.err)) break;
+        tc_fence_after();
+        const uint32_t taddr = lane_addr + static_cast<uint32_t>(buf * C::MMA_N);
+        {
+          constexpr int QH = C::QPT / C::NSETS;  // queries per thread
+          constexpr int NC = QH * C::H;          // columns per thread
+          constexpr int NCH = NC / 32;           // 32-column chunks
+          constexpr int NP = C::H >= 32 ? 2 : 1;  // packed partial sums per query
+          const int q0 = set * QH;               // first query (in group)
+          const int key = s.j * C::KROWS + row;  // key row
+          const long long rbase = static_cast<long long>(b) * p.T + tg * C::QPT + q0;
+          // this warp's head weights for the group (queries past T reuse the
+          // last query's weights; their outputs are never stored)
+          static_assert(NC == C::NCOL_THREAD, "coefficient slot");
+          float* cw = reinterpret_cast<float*>(smem + C::SMEM_COEF) + e * NC;
+          if (s.g != coef_g) {
+            for (int c = lane; c < NC; c += 32) {
+              const int ql = c / C::H;
+              const int h = c % C::H;
+              const int tq = tg * C::QPT + q0 + ql;
+              const long long ci = (rbase + ql - (tq < p.T ? 0 : tq - p.T + 1)) * C::H + h;
+              cw[c] = __ldg(p.w + ci);
+            }
+            __syncwarp();
+            coef_g = s.g;
+          }
+          float acc[QH][NP];
+          unsigned long long acc2[QH][NP];
+#pragma unroll
+          for (int i = 0; i < QH; ++i)
+#pragma unroll
+            for (int j = 0; j < NP; ++j) acc2[i][j] = 0ull;
+          // TMEM -> registers one 32-column chunk at a time: the next chunk's
+          // load is issued before this chunk's arithmetic, and the buffer goes
+          // back to the MMA warp as soon as the last chunk has landed, so the
+          // next tile's MMAs overlap the remaining math.
+          uint32_t vb[2][32];
+          tmem_ld32_issue(taddr + q0 * C::H, vb[0]);
+          tmem_ld_wait(vb[0]);
+#pragma unroll
+          for (int ph = 0; ph < NCH; ++ph) {
+            if (ph + 1 < NCH) {
+              tmem_ld32_issue(taddr + q0 * C::H + (ph + 1) * 32, vb[(ph + 1) & 1]);
+            } else {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(tempty(buf));
+            }
+            const int cc = ph * 32;
+            const uint32_t (&v)[32] = vb[ph & 1];
+            float coef[32];
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 c4 = *reinterpret_cast<const float4*>(cw + cc + i);
+              coef[i] = c4.x; coef[i + 1] = c4.y; coef[i + 2] = c4.z; coef[i + 3] = c4.w;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const int ql = (cc + i) / C::H;
+              const int pp = (i / 2) % NP;
+              acc2[ql][pp] = ffma2(pack2(coef[i], coef[i + 1]),
+                                   pack2(fmaxf(__uint_as_float(v[i]), 0.f),
+                                         fmaxf(__uint_as_float(v[i + 1]), 0.f)),
+                                   acc2[ql][pp]);
+            }
+            if (ph + 1 < NCH) tmem_ld_wait(vb[(ph + 1) & 1]);
+          }
+#pragma unroll
+          for (int i = 0; i < QH; ++i)
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+              const float2 f = unpack2(acc2[i][j]);
+              acc[i][j] = f.x + f.y;
+            }
+          float accq[QH];
+#pragma unroll
+          for (int i = 0; i < QH; ++i) {
+            float a = acc[i][0];
+            if (NP == 2) a = acc[i][0] + acc[i][1];
+            accq[i] = a;
+          }
+          if (key < p.Lk) {
+            // query q0+ql sees this key iff key * pstride <= q_offset + t0 + ql
+            const int t0 = tg * C::QPT + q0;
+            const long long e = static_cast<long long>(key) * p.pstride - (p.q_offset + t0);
+            float* orow = p.out + rbase * p.ldo + key;
+#pragma unroll
+            for (int ql = 0; ql < QH; ++ql) {
+              if (t0 + ql < p.T && e <= ql) orow[ql * p.ldo] = accq[ql];
+            }
+          }
+        }
+      }
+    } else {
     // candidate lists (CMP): lane ql keeps the reservation state of this
     // warp's query ql: current chunk (base, used), whether the next chunk has
     // been requested (and where it starts), and the real entries written
@@ -995,8 +1100,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         racc = 0.f;
       }
     }
+    }
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == C::MMA_WARP) {

@@ -106,6 +106,7 @@ struct TkCfg {
 using TkShort = TkCfg<1024, 2048, 4, 256, 4>;  // rows up to 32768: 44.5 KB, 4 CTAs per SM
 using TkLong = TkCfg<4096, 6144, 4, 512, 2>;   // rows up to 131072: 88.5 KB, 2 CTAs per SM
 using TkWide = TkCfg<4096, 6144, 8, 512, 1>;   // as TkLong, one wider CTA per row for launches with few rows
+using TkShortWide = TkCfg<1024, 2048, 8, 512, 1>;  // as TkShort, one wider CTA per row for launches with few rows
 
 __device__ __forceinline__ uint32_t score_key(float x) {
   if (!(x > -INFINITY)) return 0u;  // -inf (absent) and NaN

@@ -610,6 +610,21 @@ def _pooled_cache(ix, block):
     return kbar, ksc
 
 
+@pytest.mark.parametrize("blk", [1, 16, 200, 256, 1000])
+def test_fp8_pooled_keys_bit_exact(blk):
+    # FP8 pooled keys (codes and scales) of every block, the last one ragged,
+    # equal the oracle's bit for bit, for blocks shorter and longer than one
+    # pass of the pooling kernel's row groups
+    inp = wl.decode_inputs(batch=2, L=2345, H=64, d=128, seed=152, cluster_frac=0.05)
+    ix = _indexer(inp)
+    kbar, ksc = B.pooled_cache(ix.args, blk, device="cuda")
+    B.dsa_pool_keys(ix.args, blk, 0, kbar.shape[1], kbar, ksc)
+    for b in range(inp.batch):
+        codes, scales = oracle.meanpool_e4m3(inp.k[b], inp.k_scale[b], blk)
+        assert np.array_equal(kbar[b].cpu().numpy(), codes)
+        assert np.array_equal(ksc[b].cpu().numpy(), scales)
+
+
 @pytest.mark.parametrize("fp8", [False, True])
 def test_pooled_cache_calls_equal_unpooled(fp8):
     # MISA-dagger and HISA reading a caller-kept pooled-key cache give the

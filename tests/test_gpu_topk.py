@@ -122,6 +122,18 @@ def test_many_long_rows():
     _check(s, idx, sc, exp, "many long rows")
 
 
+def test_many_short_rows():
+    # more rows (of at most 32768 scores) than SMs: the 256-thread short-row
+    # layout, 4 CTAs per SM (fewer rows take one 512-thread CTA each)
+    rng = np.random.default_rng(13)
+    rows, n, k = 400, 20000, 2048
+    s = (rng.standard_normal((rows, n)) * 0.05).astype(np.float32)
+    s[::5, n // 2:] = -np.inf
+    s[3::11] = np.round(s[3::11] * 8) / 8  # rows with many ties
+    idx, sc = _run(s, rows, 0, 0, n, k)
+    _check(s, idx, sc, _expect(s, rows, 0, 0, n, k), "many short rows")
+
+
 def test_many_long_rows_mass_ties():
     # the long-row layout's fallback path: few distinct values, enough rows
     # longer than 32768 to fill the GPU
