@@ -175,6 +175,10 @@ struct ScoreCfg {
   // the plain store epilogue (bf16, eight warps, one CTA per SM) has a loop of its own
   static constexpr bool PLAIN = EPI_ == kEpiStore && !LIST_ && ELEM == 2 && !ROUTER && !GATHER && EPIW == 8 &&
                                 CTAS_ == 1 && !SPLIT_TILES;
+  // the other bf16 store kernels (16 epilogue warps) likewise: 0.585 -> 0.561 ms
+  // on the routed MISA pass; FP8 stays on the shared loop (1.41 against 1.46 ms
+  // with its own on the FP8 DSA chunk)
+  static constexpr bool PLAIN2 = EPI_ == kEpiStore && !LIST_ && ELEM == 2 && !ROUTER && !GATHER && !PLAIN;
   // per epilogue warp: the head weights (x query scales) of its columns for
   // the current query group, refilled when the group changes
   static constexpr int NCOL_THREAD = ROUTER ? 0 : (SPLIT_TILES ? QROWS : QROWS / NSETS);
@@ -715,6 +719,133 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int ql = 0; ql < QH; ++ql) {
               if (t0 + ql < p.T && e <= ql) orow[ql * p.ldo] = accq[ql];
+            }
+          }
+        }
+      }
+    } else if constexpr (C::PLAIN2) {
+      // The other bf16 store kernels (16 epilogue warps, or one query per
+      // group) likewise without the variants' code.
+      for (; !s.done; s.next(p), ++it) {
+        const int b = s.b;
+        const int tg = s.tg;
+        const int buf = static_cast<int>(it % C::NACC);
+        const bool mine = C::SPLIT_TILES ? (static_cast<int>(it % C::NSETS) == set) : true;
+        if (mine) {
+          constexpr int QH = C::SPLIT_TILES ? 1 : C::QPT / C::NSETS;  // queries per thread
+          constexpr int NC = QH * C::H;                               // columns per thread
+          constexpr int NCH = NC / 32;                                // 32-column chunks
+          constexpr int NP = C::H >= 32 ? 2 : 1;                      // packed partial sums per query
+          static_assert(NC == C::NCOL_THREAD && NC % 32 == 0 && NCH >= 1, "coefficient slot, chunks");
+          const int q0 = C::SPLIT_TILES ? 0 : set * QH;               // first query (in group)
+          const int key = s.j * C::KROWS + row;                       // key row
+          const long long rbase = static_cast<long long>(b) * p.T + tg * C::QPT + q0;
+          // FP8: this row's key dequant scale, loaded before the wait
+          float ks = 1.f;
+          if constexpr (C::KEY_SCALES) {
+            if (key < p.Lk) ks = __ldg(p.k_scale + static_cast<long long>(b) * p.Lk + key);
+          }
+          if (!mbar_wait(tfull(buf), (it / C::NACC) & 1u, p.err)) break;
+          tc_fence_after();
+          const uint32_t taddr = lane_addr + static_cast<uint32_t>(buf * C::MMA_N);
+          // this warp's head weights (x query scales) for the group
+          float* cw = reinterpret_cast<float*>(smem + C::SMEM_COEF) + e * NC;
+          if (s.g != coef_g) {
+            for (int c = lane; c < NC; c += 32) {
+              const int ql = c / C::H;
+              const int h = c % C::H;
+              const int tq = tg * C::QPT + q0 + ql;
+              const long long ci = (rbase + ql - (tq < p.T ? 0 : tq - p.T + 1)) * C::H + h;
+              float cv = __ldg(p.w + ci);
+              if (C::ELEM == 1) cv *= __ldg(p.q_scale + ci);
+              cw[c] = cv;
+            }
+            __syncwarp();
+            coef_g = s.g;
+          }
+          unsigned long long acc2[QH][NP];
+#pragma unroll
+          for (int i = 0; i < QH; ++i)
+#pragma unroll
+            for (int j = 0; j < NP; ++j) acc2[i][j] = 0ull;
+          if constexpr (C::EPIW == 16 || C::CTAS == 2) {
+            // one 32-column chunk in flight per warp; the other warps of the
+            // sub-partition hide its load latency
+#pragma unroll
+            for (int ph = 0; ph < NCH; ++ph) {
+              uint32_t v[32];
+              tmem_ld32_issue(taddr + q0 * C::H + ph * 32, v);
+              tmem_ld_wait(v);
+              if (ph == NCH - 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty(buf));
+              }
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                const float4 c4 = *reinterpret_cast<const float4*>(cw + ph * 32 + i);
+                const int ql = (ph * 32 + i) / C::H;
+                acc2[ql][(i / 2) % NP] = ffma2(pack2(c4.x, c4.y),
+                                               pack2(fmaxf(__uint_as_float(v[i]), 0.f),
+                                                     fmaxf(__uint_as_float(v[i + 1]), 0.f)),
+                                               acc2[ql][(i / 2) % NP]);
+                acc2[ql][(i / 2 + 1) % NP] = ffma2(pack2(c4.z, c4.w),
+                                                   pack2(fmaxf(__uint_as_float(v[i + 2]), 0.f),
+                                                         fmaxf(__uint_as_float(v[i + 3]), 0.f)),
+                                                   acc2[ql][(i / 2 + 1) % NP]);
+              }
+            }
+          } else {
+            // the next chunk's TMEM load issued before this chunk's arithmetic
+            uint32_t vb[2][32];
+            tmem_ld32_issue(taddr + q0 * C::H, vb[0]);
+            tmem_ld_wait(vb[0]);
+#pragma unroll
+            for (int ph = 0; ph < NCH; ++ph) {
+              if (ph + 1 < NCH) {
+                tmem_ld32_issue(taddr + q0 * C::H + (ph + 1) * 32, vb[(ph + 1) & 1]);
+              } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty(buf));
+              }
+              const int cc = ph * 32;
+              const uint32_t (&v)[32] = vb[ph & 1];
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                const float4 c4 = *reinterpret_cast<const float4*>(cw + cc + i);
+                const int ql = (cc + i) / C::H;
+                acc2[ql][(i / 2) % NP] = ffma2(pack2(c4.x, c4.y),
+                                               pack2(fmaxf(__uint_as_float(v[i]), 0.f),
+                                                     fmaxf(__uint_as_float(v[i + 1]), 0.f)),
+                                               acc2[ql][(i / 2) % NP]);
+                acc2[ql][(i / 2 + 1) % NP] = ffma2(pack2(c4.z, c4.w),
+                                                   pack2(fmaxf(__uint_as_float(v[i + 2]), 0.f),
+                                                         fmaxf(__uint_as_float(v[i + 3]), 0.f)),
+                                                   acc2[ql][(i / 2 + 1) % NP]);
+              }
+              if (ph + 1 < NCH) tmem_ld_wait(vb[(ph + 1) & 1]);
+            }
+          }
+          float accq[QH];
+#pragma unroll
+          for (int i = 0; i < QH; ++i) {
+            float a = 0.f;
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+              const float2 f = unpack2(acc2[i][j]);
+              a += f.x + f.y;
+            }
+            accq[i] = a;
+          }
+          if (key < p.Lk) {
+            // query q0+ql sees this key iff key * pstride <= q_offset + t0 + ql
+            const int t0 = tg * C::QPT + q0;
+            const long long e = static_cast<long long>(key) * p.pstride - (p.q_offset + t0);
+            float* orow = p.out + rbase * p.ldo + key;
+#pragma unroll
+            for (int ql = 0; ql < QH; ++ql) {
+              if (t0 + ql < p.T && e <= ql) orow[ql * p.ldo] = ks * accq[ql];
             }
           }
         }
