@@ -353,8 +353,9 @@ dsa_status launch_topk_cfg(const TopkParams& tp, cudaStream_t st) {
 
 // ws: the call's workspace (its first word is the device status word).
 // Rows up to 32768 scores use the short-row layout (4 CTAs of 256 threads per
-// SM, or one 512-thread CTA per row when there are fewer rows than SMs); longer rows use 2 CTAs of 512 threads per SM when there are enough rows
-// to fill the GPU, else one 512-thread CTA (with more loads in flight) per row.
+// SM, or one 512-thread CTA per row when there are fewer rows than SMs);
+// longer rows use 2 CTAs of 512 threads per SM when there are enough rows to
+// fill the GPU, else one 512-thread CTA (with more loads in flight) per row.
 // (One CTA per SM for long rows, so fewer rows in flight stay in L2 between
 // the sampling read and the band pass, measured slower: 0.72 vs 0.59 ms on
 // the MISA-dagger k' selection.)
